@@ -1,0 +1,59 @@
+"""CPU oracle for the fused pre-norm linear layer: plain, slow, fp64.
+
+TEST INFRASTRUCTURE. Only the tests, the package's smoke check and the
+benchmark's CPU-baseline / reference leg may import or call this package; the
+CUDA library and its Python binding never do, and this package imports neither
+of them. It shares no code, constant or helper with the CUDA path. Inputs come
+from the seeded generator (``synthetic.py``) as bf16 values widened to float64.
+
+What is computed, and where the pages say so:
+
+* residual add -- the graph-optimisation layer fuses "residual + LayerNorm"
+  (TensorRT-LLM 简介, "其底层架构可拆解为四个关键层次", 图优化层); the GPT-style
+  chain Input -> Add -> Bias -> LayerNorm -> GELU is the Layer Fusion figure of
+  "TRT-LLM 编译优化管线 / 构建阶段详解 / 3. Layer Fusion" (trt-llm-deep-dive).
+* LayerNorm statistics in the order mean -> variance -> rsqrt(var + eps) ->
+  gamma * (x - mean) * rsqrt + beta, then a dot with the QKV weight written to
+  separate q/k/v outputs: the fused_layernorm_qkv kernel of TensorRT-LLM 深度工程实践,
+  §2.3 跨算子融合 ("LayerNorm + QKV Projection 融合").
+* RMSNorm is named as a model-definition op (TensorRT-LLM 简介, 模型定义层); the
+  pages give no formula, so the textbook one is used (reading R3 below).
+* SwiGLU: y = SiLU(x @ gate) * (x @ up), TensorRT-LLM 深度工程实践, §2.3
+  ("GEMM + 激活融合（SwiGLU）").
+* LayerNorm + Linear + GELU into one kernel: trt-llm-deep-dive, 面试视角 answer on
+  "更激进的 kernel fusion".
+* QKV projection + reshape + GQA grouping: TensorRT-LLM 深度工程实践, §2.2 图构建与
+  算子映射; GQA/MQA head counts come from the model config (§2.1).
+
+Readings taken where the pages are silent:
+  R1 variance is the population variance (divide by K), two passes about the mean.
+  R2 eps sits inside the square root: rstd = (var + eps)^(-1/2).
+  R3 RMSNorm: a = h * gamma / sqrt(mean(h^2) + eps); no mean, no beta.
+  R4 statistics use the unrounded h = x + residual (+ bias_in), exact in fp64.
+  R5 bias_in (GELU variant) is a [K] vector added before the norm; bias_out is
+     added before GELU: out = GELU_tanh(y + bias_out).
+  R6 GELU is the tanh form 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))).
+  R7 W is [N, K] like a linear layer's weight; QKV columns are ordered
+     [Q heads | K heads | V heads], D contiguous columns per head, stored
+     head-major Q[h, m, d] = y[m, h*D + d]. SwiGLU's W stacks gate rows [0, I)
+     over up rows [I, 2I).
+  R8 residual_out is h rounded once to bf16, round-to-nearest-even.
+
+Parity pins live in tests/test_oracle_pins.py; every function here is pinned.
+"""
+from .core import (  # noqa: F401
+    bf16_round,
+    residual_add,
+    layernorm,
+    rmsnorm,
+    normalize,
+    projection,
+    split_qkv_head_major,
+    silu,
+    swiglu,
+    gelu_tanh,
+    add_norm_qkv,
+    add_norm_swiglu,
+    add_bias_norm_gelu,
+    run,
+)

@@ -1,0 +1,166 @@
+"""fp64 reference arithmetic of the fused pre-norm linear layer (test infrastructure).
+
+Each function follows one step of the pages' description in their order; the
+package docstring gives the citations and the readings R1..R8. No blocking, no
+fusion, no reordering: numpy's float64 matmul is the only library primitive.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def _f64(a) -> np.ndarray:
+    return np.asarray(a, dtype=np.float64)
+
+
+def bf16_round(v) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16, ties to even (reading R8).
+
+    bfloat16 keeps 8 significant bits. With v = m * 2**e and 0.5 <= |m| < 1,
+    m * 2**8 is an exact float64 and np.rint rounds half to even, so the result
+    is the correctly rounded bf16 value (normal range; the workloads never
+    leave it)."""
+    v = _f64(v)
+    m, e = np.frexp(v)
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
+
+
+def residual_add(x, residual, bias_in=None) -> np.ndarray:
+    """h = x + residual (+ bias_in broadcast over rows), exact in fp64 (R4, R5)."""
+    h = _f64(x) + _f64(residual)
+    if bias_in is not None:
+        h = h + _f64(bias_in)[None, :]
+    return h
+
+
+def layernorm(h, gamma, beta, eps):
+    """LayerNorm of each row of h, in the fused_layernorm_qkv order:
+    mean, then variance about it (R1), then rsqrt(var + eps) (R2), then
+    gamma * (h - mean) * rstd + beta. Returns (a, mean, rstd)."""
+    h = _f64(h)
+    K = h.shape[1]
+    mean = h.sum(axis=1) / K
+    d = h - mean[:, None]
+    var = (d * d).sum(axis=1) / K
+    rstd = 1.0 / np.sqrt(var + eps)
+    g = _f64(gamma)[None, :]
+    b = np.zeros_like(g) if beta is None else _f64(beta)[None, :]
+    a = g * d * rstd[:, None] + b
+    return a, mean, rstd
+
+
+def rmsnorm(h, gamma, eps):
+    """RMSNorm of each row (R3): a = h * rstd * gamma, rstd = (mean(h^2)+eps)^-1/2.
+    Returns (a, rstd)."""
+    h = _f64(h)
+    K = h.shape[1]
+    ms = (h * h).sum(axis=1) / K
+    rstd = 1.0 / np.sqrt(ms + eps)
+    a = h * rstd[:, None] * _f64(gamma)[None, :]
+    return a, rstd
+
+
+def normalize(h, gamma, beta, norm: str, eps: float):
+    """Dispatch on the norm kind. Returns (a, mean or None, rstd)."""
+    if norm == "layernorm":
+        return layernorm(h, gamma, beta, eps)
+    if norm == "rmsnorm":
+        a, rstd = rmsnorm(h, gamma, eps)
+        return a, None, rstd
+    raise ValueError(f"unknown norm {norm!r}")
+
+
+def projection(a, W, bias=None) -> np.ndarray:
+    """y[m, n] = sum_k a[m, k] * W[n, k] (+ bias[n]); W is [N, K] (R7)."""
+    y = _f64(a) @ _f64(W).T
+    if bias is not None:
+        y = y + _f64(bias)[None, :]
+    return y
+
+
+def split_qkv_head_major(y, Hq, Hkv, D):
+    """Columns [0, Hq*D) are Q, the next Hkv*D are K, the last Hkv*D are V;
+    each is returned head-major [H, M, D] (R7)."""
+    y = _f64(y)
+    M, N = y.shape
+    if N != (Hq + 2 * Hkv) * D:
+        raise ValueError("N must equal (Hq + 2*Hkv) * D")
+    q = y[:, : Hq * D].reshape(M, Hq, D).transpose(1, 0, 2)
+    k = y[:, Hq * D:(Hq + Hkv) * D].reshape(M, Hkv, D).transpose(1, 0, 2)
+    v = y[:, (Hq + Hkv) * D:].reshape(M, Hkv, D).transpose(1, 0, 2)
+    return np.ascontiguousarray(q), np.ascontiguousarray(k), np.ascontiguousarray(v)
+
+
+def silu(z) -> np.ndarray:
+    """SiLU(z) = z / (1 + exp(-z)) in fp64."""
+    z = _f64(z)
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def swiglu(y, I) -> np.ndarray:
+    """SiLU(gate) * up with gate = y[:, :I] and up = y[:, I:2I] (R7)."""
+    y = _f64(y)
+    return silu(y[:, :I]) * y[:, I:2 * I]
+
+
+def gelu_tanh(z) -> np.ndarray:
+    """GELU, tanh form (R6)."""
+    z = _f64(z)
+    return 0.5 * z * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (z + 0.044715 * z ** 3)))
+
+
+def _stats(out: dict, mean, rstd) -> dict:
+    if mean is not None:
+        out["mean"] = mean
+    out["rstd"] = rstd
+    return out
+
+
+def add_norm_qkv(x, residual, gamma, beta, norm, eps, W, bias, Hq, Hkv, D) -> dict:
+    """Residual add -> norm -> QKV projection -> head-major Q/K/V split."""
+    h = residual_add(x, residual)
+    a, mean, rstd = normalize(h, gamma, beta, norm, eps)
+    y = projection(a, W, bias)
+    q, k, v = split_qkv_head_major(y, Hq, Hkv, D)
+    return _stats({"residual_out": bf16_round(h), "q": q, "k": k, "v": v}, mean, rstd)
+
+
+def add_norm_swiglu(x, residual, gamma, beta, norm, eps, W, bias, I) -> dict:
+    """Residual add -> norm -> gate/up projection -> SiLU(gate) * up."""
+    h = residual_add(x, residual)
+    a, mean, rstd = normalize(h, gamma, beta, norm, eps)
+    y = projection(a, W, bias)
+    return _stats({"residual_out": bf16_round(h), "out": swiglu(y, I)}, mean, rstd)
+
+
+def add_bias_norm_gelu(x, residual, bias_in, gamma, beta, norm, eps, W, bias_out) -> dict:
+    """Residual add + bias_in -> norm -> projection + bias_out -> GELU_tanh."""
+    h = residual_add(x, residual, bias_in)
+    a, mean, rstd = normalize(h, gamma, beta, norm, eps)
+    z = projection(a, W, bias_out)
+    return _stats({"residual_out": bf16_round(h), "out": gelu_tanh(z)}, mean, rstd)
+
+
+def run(w, inputs: dict, rows=None) -> dict:
+    """Evaluate workload ``w`` (a synthetic.Workload) on ``inputs`` (tensors or
+    arrays, bf16 values), optionally on a subset of rows (the op is row-wise)."""
+    def g(name):
+        t = inputs.get(name)
+        if t is None:
+            return None
+        if hasattr(t, "detach"):
+            t = t.detach().cpu().double().numpy()
+        return _f64(t)
+
+    x, r = g("x"), g("residual")
+    if rows is not None:
+        x, r = x[rows], r[rows]
+    if w.op == "qkv":
+        return add_norm_qkv(x, r, g("gamma"), g("beta"), w.norm, w.eps, g("W"),
+                            g("bias_out"), w.Hq, w.Hkv, w.D)
+    if w.op == "swiglu":
+        return add_norm_swiglu(x, r, g("gamma"), g("beta"), w.norm, w.eps, g("W"),
+                               g("bias_out"), w.I)
+    return add_bias_norm_gelu(x, r, g("bias_in"), g("gamma"), g("beta"), w.norm, w.eps,
+                              g("W"), g("bias_out"))

@@ -1,0 +1,433 @@
+"""Pins of the fp64 CPU oracle to things other than itself.
+
+Each pin checks the oracle against an invariant, a closed form, a library
+routine on a special case, or a brute-force loop on tiny inputs. The mutation
+tests at the bottom plant plausible mistakes in the oracle (on the CPU, by
+monkeypatching one function at a time) and require that at least one pin
+fails for every planted mistake.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from oracle import core
+
+
+def _rand(shape, seed, scale=1.0, loc=0.0):
+    return np.random.default_rng(seed).normal(loc, scale, size=shape)
+
+
+def _t(a):
+    return torch.tensor(np.asarray(a, dtype=np.float64))
+
+
+# --------------------------------------------------------------------------
+# pins: each takes the oracle module so that the mutation tests can reuse them
+# --------------------------------------------------------------------------
+
+def pin_layernorm_invariants(ora):
+    """gamma=1, beta=0: every row of a has mean 0 and population variance
+    var/(var+eps); the returned statistics match numpy's mean and variance."""
+    K = 96
+    h = _rand((16, K), 1, scale=1.7, loc=0.3)
+    eps = 0.05
+    a, mean, rstd = ora.layernorm(h, np.ones(K), np.zeros(K), eps)
+    var = np.var(h, axis=1)
+    assert np.max(np.abs(a.mean(axis=1))) <= 1e-12
+    np.testing.assert_allclose(np.var(a, axis=1), var / (var + eps), rtol=1e-12, atol=0)
+    np.testing.assert_allclose(mean, np.mean(h, axis=1), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(rstd ** -2 - eps, var, rtol=1e-12)
+
+
+def pin_rmsnorm_invariant(ora):
+    """gamma=1: mean(a^2) = ms/(ms+eps) with ms = mean(h^2) (rows with a
+    non-zero mean, so a centred variant fails)."""
+    K = 96
+    h = _rand((16, K), 2, scale=1.3, loc=0.4)
+    eps = 0.05
+    a, rstd = ora.rmsnorm(h, np.ones(K), eps)
+    ms = np.mean(h * h, axis=1)
+    np.testing.assert_allclose(np.mean(a * a, axis=1), ms / (ms + eps), rtol=1e-12)
+    np.testing.assert_allclose(rstd ** -2 - eps, ms, rtol=1e-12)
+
+
+def pin_norms_match_torch(ora):
+    """Special case = library routine: torch's float64 layer_norm / rms_norm."""
+    K = 64
+    h = _rand((8, K), 3, scale=2.0, loc=-0.5)
+    g = _rand(K, 4, 0.1, 1.0)
+    b = _rand(K, 5, 0.1)
+    for eps in (1e-5, 0.3):
+        a, _, _ = ora.layernorm(h, g, b, eps)
+        ref = F.layer_norm(_t(h), (K,), _t(g), _t(b), eps).numpy()
+        assert np.max(np.abs(a - ref)) <= 1e-12
+        a2, _ = ora.rmsnorm(h, g, eps)
+        ref2 = F.rms_norm(_t(h), (K,), _t(g), eps).numpy()
+        assert np.max(np.abs(a2 - ref2)) <= 1e-12
+
+
+def pin_identity_weight(ora):
+    """W = identity (N = K): QKV is a re-indexing of the normalised rows,
+    SwiGLU with W = [I; 2I] is SiLU(a) * 2a, GELU with W = I is GELU(a + b)."""
+    Hq, Hkv, D = 2, 1, 8
+    K = (Hq + 2 * Hkv) * D
+    M = 5
+    x, r = _rand((M, K), 6), _rand((M, K), 7)
+    g, b = _rand(K, 8, 0.1, 1.0), _rand(K, 9, 0.1)
+    eps = 1e-5
+    a = F.layer_norm(_t(x) + _t(r), (K,), _t(g), _t(b), eps).numpy()
+    out = ora.add_norm_qkv(x, r, g, b, "layernorm", eps, np.eye(K), None, Hq, Hkv, D)
+    assert out["q"].shape == (Hq, M, D) and out["k"].shape == (Hkv, M, D)
+    assert out["v"].shape == (Hkv, M, D)
+    for m in range(M):
+        for d in range(D):
+            for hh in range(Hq):
+                assert abs(out["q"][hh, m, d] - a[m, hh * D + d]) <= 1e-12
+            for hh in range(Hkv):
+                assert abs(out["k"][hh, m, d] - a[m, (Hq + hh) * D + d]) <= 1e-12
+                assert abs(out["v"][hh, m, d] - a[m, (Hq + Hkv + hh) * D + d]) <= 1e-12
+
+    W2 = np.concatenate([np.eye(K), 2.0 * np.eye(K)], axis=0)
+    ar = F.rms_norm(_t(x) + _t(r), (K,), _t(g), eps)
+    sw = ora.add_norm_swiglu(x, r, g, None, "rmsnorm", eps, W2, None, K)["out"]
+    ref = (F.silu(ar) * 2.0 * ar).numpy()
+    assert np.max(np.abs(sw - ref)) <= 1e-12
+
+    bi, bo = _rand(K, 10), _rand(K, 11, 0.02)
+    al = F.layer_norm(_t(x) + _t(r) + _t(bi), (K,), _t(g), _t(b), eps)
+    ge = ora.add_bias_norm_gelu(x, r, bi, g, b, "layernorm", eps, np.eye(K), bo)["out"]
+    ref = F.gelu(al + _t(bo), approximate="tanh").numpy()
+    assert np.max(np.abs(ge - ref)) <= 1e-12
+
+
+def pin_one_hot(ora):
+    """h = s * e_j (x = s e_j - t e_i, residual = t e_i): closed forms.
+    LayerNorm: a_k = gamma_k (delta_kj - 1/K) s rstd + beta_k with
+    rstd = (s^2 (K-1)/K^2 + eps)^(-1/2). RMSNorm: y_n = W[n, j] gamma_j s /
+    sqrt(s^2/K + eps), which exposes the index order of the projection."""
+    K, N = 48, 24
+    j, i, s, t = 7, 30, 3.0, 1.25
+    x = np.zeros((1, K))
+    r = np.zeros((1, K))
+    x[0, j], x[0, i], r[0, i] = s, -t, t
+    g, b = _rand(K, 12, 0.1, 1.0), _rand(K, 13, 0.1)
+    W = _rand((N, K), 14)
+    eps = 1e-3
+    a, mean, rstd = ora.layernorm(ora.residual_add(x, r), g, b, eps)
+    rs = (s * s * (K - 1) / K ** 2 + eps) ** -0.5
+    ak = g * ((np.arange(K) == j) - 1.0 / K) * s * rs + b
+    assert abs(mean[0] - s / K) <= 1e-15
+    assert abs(rstd[0] - rs) <= 1e-12 * rs
+    assert np.max(np.abs(a[0] - ak)) <= 1e-12
+    # RMS through the whole QKV path: N = (Hq + 2 Hkv) D with Hq=2, Hkv=1, D=6
+    out = ora.add_norm_qkv(x, r, g, None, "rmsnorm", eps, W, None, 2, 1, 6)
+    yn = W[:, j] * g[j] * s / math.sqrt(s * s / K + eps)
+    y = np.concatenate([out["q"][:, 0, :].reshape(-1), out["k"][:, 0, :].reshape(-1),
+                        out["v"][:, 0, :].reshape(-1)])
+    assert np.max(np.abs(y - yn)) <= 1e-12
+
+
+def _brute(op, x, r, bias_in, g, b, norm, eps, W, bias_out, Hq=0, Hkv=0, D=0, I=0):
+    """Per-element loops, independent of the vectorised oracle."""
+    M, K = len(x), len(x[0])
+    N = len(W)
+    res = {"rows": []}
+    for m in range(M):
+        h = [x[m][k] + r[m][k] + (bias_in[k] if bias_in is not None else 0.0) for k in range(K)]
+        if norm == "layernorm":
+            mu = 0.0
+            for k in range(K):
+                mu += h[k]
+            mu /= K
+            var = 0.0
+            for k in range(K):
+                var += (h[k] - mu) * (h[k] - mu)
+            var /= K
+            rs = 1.0 / math.sqrt(var + eps)
+            a = [g[k] * (h[k] - mu) * rs + (b[k] if b is not None else 0.0) for k in range(K)]
+        else:
+            ss = 0.0
+            for k in range(K):
+                ss += h[k] * h[k]
+            rs = 1.0 / math.sqrt(ss / K + eps)
+            a = [h[k] * rs * g[k] for k in range(K)]
+        y = []
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                acc += a[k] * W[n][k]
+            if bias_out is not None:
+                acc += bias_out[n]
+            y.append(acc)
+        res["rows"].append(y)
+    return res
+
+
+def pin_brute_force(ora):
+    """Tiny shapes against per-element loops, all three epilogues."""
+    M, K = 3, 16
+    x, r = _rand((M, K), 20), _rand((M, K), 21)
+    g, b, bi = _rand(K, 22, 0.1, 1.0), _rand(K, 23, 0.1), _rand(K, 24)
+    eps = 1e-5
+    # QKV, LayerNorm, with bias
+    Hq, Hkv, D = 2, 1, 4
+    N = (Hq + 2 * Hkv) * D
+    W, bo = _rand((N, K), 25, 0.25), _rand(N, 26, 0.02)
+    out = ora.add_norm_qkv(x, r, g, b, "layernorm", eps, W, bo, Hq, Hkv, D)
+    y = _brute("qkv", x.tolist(), r.tolist(), None, g, b, "layernorm", eps, W.tolist(), bo)["rows"]
+    for m in range(M):
+        for n in range(N):
+            if n < Hq * D:
+                got = out["q"][n // D, m, n % D]
+            elif n < (Hq + Hkv) * D:
+                got = out["k"][(n - Hq * D) // D, m, n % D]
+            else:
+                got = out["v"][(n - (Hq + Hkv) * D) // D, m, n % D]
+            assert abs(got - y[m][n]) <= 1e-12
+    # SwiGLU, RMSNorm
+    I = 5
+    W = _rand((2 * I, K), 27, 0.25)
+    out = ora.add_norm_swiglu(x, r, g, None, "rmsnorm", eps, W, None, I)["out"]
+    y = _brute("swiglu", x.tolist(), r.tolist(), None, g, None, "rmsnorm", eps, W.tolist(), None)["rows"]
+    for m in range(M):
+        for j in range(I):
+            gate, up = y[m][j], y[m][I + j]
+            assert abs(out[m, j] - gate / (1.0 + math.exp(-gate)) * up) <= 1e-12
+    # Bias + LayerNorm + GELU
+    N = 6
+    W, bo = _rand((N, K), 28, 0.25), _rand(N, 29, 0.02)
+    out = ora.add_bias_norm_gelu(x, r, bi, g, b, "layernorm", eps, W, bo)
+    y = _brute("gelu", x.tolist(), r.tolist(), bi, g, b, "layernorm", eps, W.tolist(), bo)["rows"]
+    c = math.sqrt(2.0 / math.pi)
+    for m in range(M):
+        for n in range(N):
+            z = y[m][n]
+            ref = 0.5 * z * (1.0 + math.tanh(c * (z + 0.044715 * z ** 3)))
+            assert abs(out["out"][m, n] - ref) <= 1e-12
+    for m in range(M):
+        h = x[m] + r[m] + bi
+        assert np.all(out["residual_out"][m] == ora.bf16_round(h))
+
+
+def pin_epilogue_values(ora):
+    """SiLU / GELU_tanh: hand values, limits, torch float64, erf-GELU within 1e-3."""
+    assert float(ora.silu(0.0)) == 0.0 and float(ora.gelu_tanh(0.0)) == 0.0
+    assert abs(float(ora.silu(40.0)) - 40.0) <= 1e-12
+    assert abs(float(ora.silu(-40.0)) - (-40.0 * math.exp(-40.0))) <= 1e-25
+    assert abs(float(ora.gelu_tanh(10.0)) - 10.0) <= 1e-12
+    # gelu_tanh(1) = 0.5 (1 + tanh(sqrt(2/pi) * 1.044715))
+    assert abs(float(ora.gelu_tanh(1.0)) - 0.5 * (1 + math.tanh(math.sqrt(2 / math.pi) * 1.044715))) <= 1e-15
+    z = np.linspace(-8.0, 8.0, 321)
+    assert np.max(np.abs(ora.silu(z) - F.silu(_t(z)).numpy())) <= 1e-14
+    assert np.max(np.abs(ora.gelu_tanh(z) - F.gelu(_t(z), approximate="tanh").numpy())) <= 1e-14
+    erf_gelu = np.array([0.5 * v * (1.0 + math.erf(v / math.sqrt(2.0))) for v in z])
+    assert np.max(np.abs(ora.gelu_tanh(z) - erf_gelu)) <= 1e-3
+    y = np.stack([z, -z[::-1] * 0.5], axis=1)
+    sw = ora.swiglu(np.concatenate([y[:, :1], y[:, 1:]], axis=1), 1)[:, 0]
+    assert np.max(np.abs(sw - F.silu(_t(z)).numpy() * (-z[::-1] * 0.5))) <= 1e-14
+
+
+def pin_qkv_bijection(ora):
+    """Unique ids through the split: each lands exactly once, at Q[h,m,d] =
+    y[m, h*D + d] and likewise for K and V after the Q block."""
+    M, Hq, Hkv, D = 3, 4, 2, 5
+    N = (Hq + 2 * Hkv) * D
+    y = np.arange(M * N, dtype=np.float64).reshape(M, N)
+    q, k, v = ora.split_qkv_head_major(y, Hq, Hkv, D)
+    assert q.shape == (Hq, M, D) and k.shape == (Hkv, M, D) and v.shape == (Hkv, M, D)
+    ids = np.sort(np.concatenate([q.ravel(), k.ravel(), v.ravel()]))
+    assert np.array_equal(ids, np.arange(M * N, dtype=np.float64))
+    for m in range(M):
+        for d in range(D):
+            for h in range(Hq):
+                assert q[h, m, d] == m * N + h * D + d
+            for h in range(Hkv):
+                assert k[h, m, d] == m * N + (Hq + h) * D + d
+                assert v[h, m, d] == m * N + (Hq + Hkv + h) * D + d
+
+
+def pin_bf16_round(ora):
+    """Ties go to even; values representable in fp32 round as torch's
+    single-rounding fp32 -> bf16 conversion does."""
+    e = 2.0 ** -8
+    cases = {1 + e: 1.0, 1 + 3 * e: 1 + 2 ** -6, 1 + e + 2 ** -30: 1 + 2 ** -7,
+             -(1 + e): -1.0, 2 * (1 + 3 * e): 2 * (1 + 2 ** -6), 0.0: 0.0}
+    for v, want in cases.items():
+        assert float(ora.bf16_round(np.array([v]))[0]) == want, v
+    v = torch.randn(4096, generator=torch.Generator().manual_seed(3), dtype=torch.float32) * 7
+    ref = v.to(torch.bfloat16).double().numpy()
+    assert np.array_equal(ora.bf16_round(v.double().numpy()), ref)
+
+
+def pin_residual_out(ora):
+    """residual_out: x when residual = 0, 2x when residual = x (exact in bf16),
+    and torch's fp32 -> bf16 rounding of x + r wherever the fp32 sum is exact."""
+    g = torch.Generator().manual_seed(5)
+    xb = torch.randn(4, 64, generator=g).to(torch.bfloat16)
+    rb = torch.randn(4, 64, generator=g).to(torch.bfloat16)
+    x, r = xb.double().numpy(), rb.double().numpy()
+    K = 64
+    gam = np.ones(K)
+    o = ora.add_norm_swiglu(x, np.zeros_like(x), gam, None, "rmsnorm", 1e-5, np.ones((2, K)), None, 1)
+    assert np.array_equal(o["residual_out"], x)
+    o = ora.add_norm_swiglu(x, x, gam, None, "rmsnorm", 1e-5, np.ones((2, K)), None, 1)
+    assert np.array_equal(o["residual_out"], 2 * x)
+    o = ora.add_norm_swiglu(x, r, gam, None, "rmsnorm", 1e-5, np.ones((2, K)), None, 1)
+    s32 = (xb.float() + rb.float())
+    exact = s32.double().numpy() == x + r
+    assert exact.mean() > 0.9
+    assert np.array_equal(o["residual_out"][exact], s32.to(torch.bfloat16).double().numpy()[exact])
+
+
+PINS = [pin_layernorm_invariants, pin_rmsnorm_invariant, pin_norms_match_torch,
+        pin_identity_weight, pin_one_hot, pin_brute_force, pin_epilogue_values,
+        pin_qkv_bijection, pin_bf16_round, pin_residual_out]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
+def test_pin_holds(pin):
+    pin(core)
+
+
+# --------------------------------------------------------------------------
+# planted mistakes: every one must break at least one pin
+# --------------------------------------------------------------------------
+
+ORIG = {name: getattr(core, name) for name in ("layernorm", "rmsnorm", "split_qkv_head_major")}
+
+
+def _ln_unbiased(h, gamma, beta, eps):
+    h = np.asarray(h, np.float64)
+    K = h.shape[1]
+    mean = h.sum(1) / K
+    var = ((h - mean[:, None]) ** 2).sum(1) / (K - 1)
+    rstd = 1 / np.sqrt(var + eps)
+    bb = 0 if beta is None else np.asarray(beta)[None]
+    return np.asarray(gamma)[None] * (h - mean[:, None]) * rstd[:, None] + bb, mean, rstd
+
+
+def _ln_eps_outside(h, gamma, beta, eps):
+    h = np.asarray(h, np.float64)
+    K = h.shape[1]
+    mean = h.sum(1) / K
+    var = ((h - mean[:, None]) ** 2).sum(1) / K
+    rstd = 1 / (np.sqrt(var) + eps)
+    bb = 0 if beta is None else np.asarray(beta)[None]
+    return np.asarray(gamma)[None] * (h - mean[:, None]) * rstd[:, None] + bb, mean, rstd
+
+
+def _ln_no_beta(h, gamma, beta, eps):
+    return ORIG["layernorm"](h, gamma, None, eps)
+
+
+def _ln_gamma_before_centering(h, gamma, beta, eps):
+    h = np.asarray(h, np.float64)
+    K = h.shape[1]
+    mean = h.sum(1) / K
+    var = ((h - mean[:, None]) ** 2).sum(1) / K
+    rstd = 1 / np.sqrt(var + eps)
+    bb = 0 if beta is None else np.asarray(beta)[None]
+    return (np.asarray(gamma)[None] * h - mean[:, None]) * rstd[:, None] + bb, mean, rstd
+
+
+def _rms_centred(h, gamma, eps):
+    a, _, rstd = ORIG["layernorm"](h, gamma, None, eps)
+    return a, rstd
+
+
+def _rms_no_eps(h, gamma, eps):
+    return ORIG["rmsnorm"](h, gamma, 0.0)
+
+
+def _proj_transposed(a, W, bias=None):
+    y = np.asarray(a) @ np.asarray(W)
+    return y if bias is None else y + np.asarray(bias)[None]
+
+
+def _proj_no_bias(a, W, bias=None):
+    return np.asarray(a) @ np.asarray(W).T
+
+
+def _split_kv_swapped(y, Hq, Hkv, D):
+    q, k, v = ORIG["split_qkv_head_major"](y, Hq, Hkv, D)
+    return q, v, k
+
+
+def _split_token_major(y, Hq, Hkv, D):
+    q, k, v = ORIG["split_qkv_head_major"](y, Hq, Hkv, D)
+    return (np.ascontiguousarray(q.transpose(1, 0, 2)), np.ascontiguousarray(k.transpose(1, 0, 2)),
+            np.ascontiguousarray(v.transpose(1, 0, 2)))
+
+
+def _swiglu_swapped(y, I):
+    y = np.asarray(y, np.float64)
+    return core.silu(y[:, I:2 * I]) * y[:, :I]
+
+
+def _gelu_wrong_cubic(z):
+    z = np.asarray(z, np.float64)
+    return 0.5 * z * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (z + 0.0447 * z ** 3)))
+
+
+def _silu_sigmoid_only(z):
+    z = np.asarray(z, np.float64)
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+def _gelu_bias_after(x, residual, bias_in, gamma, beta, norm, eps, W, bias_out):
+    h = core.residual_add(x, residual, bias_in)
+    a, mean, rstd = core.normalize(h, gamma, beta, norm, eps)
+    out = core.gelu_tanh(core.projection(a, W)) + (0 if bias_out is None else np.asarray(bias_out)[None])
+    return {"residual_out": core.bf16_round(h), "out": out, "rstd": rstd, "mean": mean}
+
+
+def _residual_drops_bias_in(x, residual, bias_in=None):
+    return np.asarray(x, np.float64) + np.asarray(residual, np.float64)
+
+
+def _residual_ignores_residual(x, residual, bias_in=None):
+    h = np.asarray(x, np.float64)
+    return h if bias_in is None else h + np.asarray(bias_in)[None]
+
+
+def _bf16_truncate(v):
+    v = np.asarray(v, np.float64)
+    m, e = np.frexp(v)
+    return np.ldexp(np.trunc(m * 256.0) / 256.0, e)
+
+
+MUTANTS = {
+    "variance_divides_by_K_minus_1": ("layernorm", _ln_unbiased),
+    "eps_outside_sqrt": ("layernorm", _ln_eps_outside),
+    "beta_dropped": ("layernorm", _ln_no_beta),
+    "gamma_before_centering": ("layernorm", _ln_gamma_before_centering),
+    "rmsnorm_subtracts_mean": ("rmsnorm", _rms_centred),
+    "rmsnorm_without_eps": ("rmsnorm", _rms_no_eps),
+    "projection_transposed": ("projection", _proj_transposed),
+    "projection_drops_bias": ("projection", _proj_no_bias),
+    "k_and_v_swapped": ("split_qkv_head_major", _split_kv_swapped),
+    "token_major_not_head_major": ("split_qkv_head_major", _split_token_major),
+    "gate_and_up_swapped": ("swiglu", _swiglu_swapped),
+    "gelu_cubic_coefficient": ("gelu_tanh", _gelu_wrong_cubic),
+    "silu_is_sigmoid": ("silu", _silu_sigmoid_only),
+    "bias_out_after_gelu": ("add_bias_norm_gelu", _gelu_bias_after),
+    "bias_in_dropped": ("residual_add", _residual_drops_bias_in),
+    "residual_ignored": ("residual_add", _residual_ignores_residual),
+    "bf16_truncates": ("bf16_round", _bf16_truncate),
+}
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_planted_mistake_breaks_a_pin(mutant, monkeypatch):
+    attr, fn = MUTANTS[mutant]
+    monkeypatch.setattr(core, attr, fn)
+    broken = []
+    for pin in PINS:
+        try:
+            pin(core)
+        except (AssertionError, ValueError, IndexError):
+            broken.append(pin.__name__)
+    assert broken, f"planted mistake {mutant!r} passed every pin"
