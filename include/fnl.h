@@ -1,0 +1,153 @@
+/*
+ * fnl -- fused pre-norm linear layer for NVIDIA B200 (sm_100a).
+ *
+ * One call runs, on one GPU and in one pass over the weights:
+ *   residual add  ->  LayerNorm or RMSNorm  ->  bf16 projection GEMM with fp32
+ *   accumulation on the tcgen05 tensor cores  ->  a fused epilogue
+ * with the normalised activations built in shared memory only (never written
+ * to global memory). The three epilogues are the three fusions the pages
+ * describe:
+ *   fnl_add_norm_qkv        LayerNorm + QKV projection fused into one kernel,
+ *                           q/k/v written directly (TensorRT-LLM 深度工程实践,
+ *                           §2.3 跨算子融合, "LayerNorm + QKV Projection 融合"),
+ *                           with the GQA head grouping of §2.2 图构建与算子映射;
+ *   fnl_add_norm_swiglu     gate/up GEMM with SiLU(gate) * up done in registers
+ *                           and one write-back (same page, §2.3 "GEMM + 激活融合
+ *                           （SwiGLU）");
+ *   fnl_add_bias_norm_gelu  Add -> Bias -> LayerNorm -> Linear -> GELU as one
+ *                           kernel (trt-llm-deep-dive, "3. Layer Fusion" figure
+ *                           and the 面试视角 answer on kernel fusion).
+ * Residual + LayerNorm fusion and the RMSNorm op are named in TensorRT-LLM 简介
+ * (the four-layer architecture: 模型定义层, 图优化层).
+ *
+ * Notation: M tokens (rows), K hidden size, N rows of W (= output columns
+ * before the epilogue). All matrices are row-major bf16 (raw 16-bit patterns,
+ * fnl_bf16), all pointers are DEVICE pointers of the handle's device, owned by
+ * the caller and left untouched after the call returns (results are written
+ * asynchronously on `stream`).
+ *   x, residual   [M, K]
+ *   residual_out  [M, K]   = bf16_rne(x + residual (+ bias_in)); must not
+ *                          overlap x, residual or bias_in
+ *   gamma         [K]      norm scale
+ *   beta          [K]      LayerNorm shift, NULL = 0; must be NULL for RMSNorm
+ *   W             [N, K]   projection weight, row n = output column n
+ * Statistics use h = x + residual (+ bias_in) in fp32 before rounding:
+ *   LayerNorm  mean = sum(h)/K, var = sum((h-mean)^2)/K, rstd = 1/sqrt(var+eps),
+ *              a = (h - mean) * rstd * gamma + beta
+ *   RMSNorm    rstd = 1/sqrt(sum(h^2)/K + eps), a = h * rstd * gamma
+ * a is rounded to bf16 for the tensor cores; y = a W^T accumulates in fp32.
+ * mean_out / rstd_out (fp32 [M], nullable) receive the statistics; mean_out
+ * must be NULL for RMSNorm.
+ *
+ * Requirements (checked on the host before any launch):
+ *   - every bf16 pointer 16-byte aligned, fp32 outputs 4-byte aligned;
+ *   - K, N (and D, I) multiples of 8; 1 <= K <= 32768; M >= 0 (M = 0 is a no-op);
+ *   - outputs overlap neither each other nor any input;
+ *   - the handle is used by one host thread / one stream at a time (its
+ *     workspace is shared by its calls).
+ * Calls are asynchronous: they enqueue one or two kernels on `stream` and
+ * return. They never synchronise, except the first call whose shape needs more
+ * workspace than the handle holds: that call synchronises `stream`, then
+ * reallocates (create the handle with fnl_options.max_tokens / max_n to
+ * reserve it up front, e.g. before capturing the calls in a CUDA graph).
+ * Error behaviour: argument errors return FNL_ERR_* without touching the GPU;
+ * launch errors return FNL_ERR_CUDA; fnl_last_error() gives the text. Device
+ * waits inside the kernels are bounded: a wait that gives up records a code
+ * that fnl_check() reports as FNL_ERR_DEVICE_STATUS.
+ */
+#ifndef FNL_H_
+#define FNL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t fnl_bf16;                 /* raw bfloat16 bits */
+typedef struct CUstream_st* fnl_stream;    /* same type as cudaStream_t; NULL = default stream */
+typedef struct fnl_handle fnl_handle;      /* opaque: device, workspace, last error */
+
+typedef enum {
+  FNL_OK = 0,
+  FNL_ERR_INVALID_ARG = 1,    /* NULL where required, bad size, bad enum, eps < 0 */
+  FNL_ERR_ALIGNMENT = 2,      /* pointer or leading dimension not aligned */
+  FNL_ERR_ALIAS = 3,          /* an output overlaps an input or another output */
+  FNL_ERR_UNSUPPORTED = 4,    /* shape outside what the kernels handle (K > 32768, ...) */
+  FNL_ERR_CUDA = 5,           /* CUDA runtime/driver error (allocation, launch) */
+  FNL_ERR_DEVICE_STATUS = 6   /* a kernel's bounded wait gave up (see fnl_check) */
+} fnl_status;
+
+typedef enum { FNL_NORM_LAYERNORM = 0, FNL_NORM_RMSNORM = 1 } fnl_norm;
+
+typedef enum {
+  FNL_PATH_AUTO = 0,          /* M <= 128: small-M split-K kernel; else tile kernel */
+  FNL_PATH_TILE = 1,          /* force the large-M persistent tile kernel */
+  FNL_PATH_SPLITK = 2         /* force the small-M split-K kernel (requires M <= 128) */
+} fnl_path;
+
+typedef struct {
+  int max_tokens;   /* reserve workspace for M up to this (0: grow on demand) */
+  int max_n;        /* reserve workspace for N up to this (0: grow on demand) */
+  int path;         /* fnl_path */
+  int max_ctas;     /* cap on persistent CTAs (0: one per SM) -- for tests */
+} fnl_options;
+
+/* Create a handle on `device` (cudaSetDevice is called). opt may be NULL. */
+fnl_status fnl_create(fnl_handle** out, int device, const fnl_options* opt);
+
+/* Free the handle's workspace. Synchronises the device first. NULL is a no-op. */
+fnl_status fnl_destroy(fnl_handle* h);
+
+/* Static text of a status code. */
+const char* fnl_status_string(fnl_status s);
+
+/* Text of the handle's last error ("" if none). Valid until the next call. */
+const char* fnl_last_error(const fnl_handle* h);
+
+/* Synchronise `stream`, read and clear the device status word. Returns
+ * FNL_ERR_DEVICE_STATUS if a kernel since the last check gave up a wait. */
+fnl_status fnl_check(fnl_handle* h, fnl_stream stream);
+
+/* Residual add -> norm -> QKV projection -> head-major GQA split.
+ * N = (Hq + 2*Hkv) * D; W rows [0, Hq*D) are the query heads, the next Hkv*D
+ * the key heads, the last Hkv*D the value heads, D consecutive rows per head.
+ * bias: nullable [N]. Outputs q [Hq, M, D], k [Hkv, M, D], v [Hkv, M, D]
+ * with q[h, m, d] = y[m, h*D + d] (and likewise after the Q block).
+ * Hq must be a multiple of Hkv. */
+fnl_status fnl_add_norm_qkv(fnl_handle* h, fnl_stream stream,
+                            const fnl_bf16* x, const fnl_bf16* residual, fnl_bf16* residual_out,
+                            const fnl_bf16* gamma, const fnl_bf16* beta, fnl_norm norm, float eps,
+                            const fnl_bf16* W, const fnl_bf16* bias,
+                            int M, int K, int Hq, int Hkv, int D,
+                            fnl_bf16* q, fnl_bf16* k, fnl_bf16* v,
+                            float* mean_out, float* rstd_out);
+
+/* Residual add -> norm -> gate/up projection -> SiLU(gate) * up.
+ * W is [2I, K]: rows [0, I) gate, rows [I, 2I) up. bias: nullable [2I].
+ * out [M, I] = SiLU(y[:, :I]) * y[:, I:], SiLU(g) = g / (1 + exp(-g)). */
+fnl_status fnl_add_norm_swiglu(fnl_handle* h, fnl_stream stream,
+                               const fnl_bf16* x, const fnl_bf16* residual, fnl_bf16* residual_out,
+                               const fnl_bf16* gamma, const fnl_bf16* beta, fnl_norm norm, float eps,
+                               const fnl_bf16* W, const fnl_bf16* bias,
+                               int M, int K, int I,
+                               fnl_bf16* out, float* mean_out, float* rstd_out);
+
+/* Residual add + bias_in -> norm -> projection + bias_out -> GELU (tanh form).
+ * bias_in: nullable [K], added to every row before the norm (and included in
+ * residual_out). bias_out: nullable [N]. out [M, N] = GELU(y + bias_out),
+ * GELU(z) = 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))). */
+fnl_status fnl_add_bias_norm_gelu(fnl_handle* h, fnl_stream stream,
+                                  const fnl_bf16* x, const fnl_bf16* residual, const fnl_bf16* bias_in,
+                                  fnl_bf16* residual_out,
+                                  const fnl_bf16* gamma, const fnl_bf16* beta, fnl_norm norm, float eps,
+                                  const fnl_bf16* W, const fnl_bf16* bias_out,
+                                  int M, int K, int N,
+                                  fnl_bf16* out, float* mean_out, float* rstd_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FNL_H_ */

@@ -1,0 +1,169 @@
+"""GPU parity: the CUDA path (through the C-ABI) against the fp64 oracle.
+
+Every workload runs at its full size in the launch configuration the benchmark
+times; small workloads are compared on every element, large ones on a seeded
+row sample (tile boundaries, packed-sequence boundaries, random rows), with
+residual_out and the statistics compared on every row.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synthetic
+from parity import check, sample_rows
+from transformer_layer_residual_b200 import fnl
+
+pytestmark = pytest.mark.gpu
+
+WL = synthetic.workloads()
+
+
+@pytest.fixture(scope="module")
+def handle(cuda_device):
+    h = fnl.Handle(0)
+    yield h
+    h.check()
+    h.close()
+
+
+def run_and_check(h, w, inputs, rows=None, **hkw):
+    dev = {k: v.cuda() for k, v in inputs.items()}
+    got = fnl.run_workload(h, w, dev)
+    h.check()
+    res = check(w, inputs, got, rows=rows)
+    return res, got
+
+
+@pytest.mark.parametrize("name", ["c1_tiny_ln_qkv", "c2_decode_rms_qkv", "c5_70b_rms_qkv_m1",
+                                  "c5_70b_rms_qkv_m8", "c5_70b_rms_qkv_m32", "c5_70b_rms_qkv_m256"])
+def test_full_compare(handle, name):
+    w = WL[name]
+    res, _ = run_and_check(handle, w, synthetic.make_inputs(w))
+    print(name, res)
+
+
+@pytest.mark.parametrize("name", ["c3_prefill_rms_swiglu", "c4_gpt_ln_gelu", "c5_70b_rms_qkv_m2048",
+                                  "c5_70b_rms_qkv_m8192", "c5_70b_rms_qkv_ragged"])
+def test_sampled_compare(handle, name):
+    w = WL[name]
+    inputs = synthetic.make_inputs(w)
+    rows = sample_rows(w.M, w.seq_lens)
+    res, _ = run_and_check(handle, w, inputs, rows=rows)
+    print(name, res)
+
+
+TAIL_CASES = []
+for op in ("qkv", "swiglu", "gelu"):
+    for norm in ("layernorm", "rmsnorm"):
+        for M in (1, 7, 16, 129, 200):
+            TAIL_CASES.append((op, norm, M))
+
+
+def _tail_workload(op, norm, M, K=200, seed=3):
+    # K = 200: three full 64-wide k-blocks and a ragged one; N not a tile multiple
+    if op == "qkv":
+        return synthetic.make_custom(op, norm, M, K, Hq=6, Hkv=2, D=40, bias_out=True, seed=seed)
+    if op == "swiglu":
+        return synthetic.make_custom(op, norm, M, K, I=200, bias_out=True, seed=seed)
+    return synthetic.make_custom(op, norm, M, K, N=328, bias_in=True, bias_out=True, seed=seed)
+
+
+@pytest.mark.parametrize("op,norm,M", TAIL_CASES)
+def test_tile_tails(handle, op, norm, M):
+    w, inputs = _tail_workload(op, norm, M)
+    run_and_check(handle, w, inputs)
+
+
+@pytest.mark.parametrize("path", ["tile", "splitk"])
+@pytest.mark.parametrize("op", ["qkv", "swiglu", "gelu"])
+@pytest.mark.parametrize("norm", ["layernorm", "rmsnorm"])
+def test_forced_paths(cuda_device, path, op, norm):
+    """Both kernels on the same small-M problems (the dispatch threshold is a
+    performance choice, not a correctness one)."""
+    h = fnl.Handle(0, path=path)
+    for M in (5, 64, 128):
+        w, inputs = _tail_workload(op, norm, M, K=520, seed=M)
+        run_and_check(h, w, inputs)
+    h.close()
+
+
+def test_few_ctas_many_segments(cuda_device):
+    """Capping the grid forces several split-K segments and tiles per CTA."""
+    for ctas in (1, 3, 7):
+        h = fnl.Handle(0, max_ctas=ctas)
+        w, inputs = _tail_workload("qkv", "rmsnorm", 33, K=1024)
+        run_and_check(h, w, inputs)
+        w, inputs = _tail_workload("swiglu", "layernorm", 300, K=320)
+        run_and_check(h, w, inputs)
+        h.close()
+
+
+def test_deterministic(handle):
+    w = WL["c2_decode_rms_qkv"]
+    dev = {k: v.cuda() for k, v in synthetic.make_inputs(w).items()}
+    a = fnl.run_workload(handle, w, dev)
+    b = fnl.run_workload(handle, w, dev)
+    handle.check()
+    for k in ("q", "k", "v", "residual_out", "rstd"):
+        assert torch.equal(a[k], b[k]), k
+
+
+def test_m_zero_is_a_noop(handle):
+    K, Hq, Hkv, D = 64, 2, 1, 8
+    x = torch.zeros(0, K, dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros((Hq + 2 * Hkv) * D, K, dtype=torch.bfloat16, device="cuda")
+    g = torch.ones(K, dtype=torch.bfloat16, device="cuda")
+    out = fnl.add_norm_qkv(handle, x, x.clone(), g, None, W, Hq, Hkv, D, norm="rmsnorm")
+    handle.check()
+    assert out["q"].shape == (Hq, 0, D)
+
+
+def test_output_guard_bands(handle):
+    """Outputs written into the middle of larger buffers leave the sentinels alone."""
+    w, inputs = _tail_workload("qkv", "layernorm", 129)
+    dev = {k: v.cuda() for k, v in inputs.items()}
+    M, K = w.M, w.K
+    pad = 64
+    sent = torch.tensor(-12345.0, dtype=torch.bfloat16)
+
+    def guarded(n):
+        buf = torch.full((n + 2 * pad,), float(sent), dtype=torch.bfloat16, device="cuda")
+        return buf, buf[pad:pad + n]
+
+    rb, ro = guarded(M * K)
+    qb, qo = guarded(w.Hq * M * w.D)
+    kbuf, ko = guarded(w.Hkv * M * w.D)
+    vb, vo = guarded(w.Hkv * M * w.D)
+    fnl.add_norm_qkv(handle, dev["x"], dev["residual"], dev["gamma"], dev["beta"], dev["W"], w.Hq, w.Hkv, w.D,
+                     norm=w.norm, bias=dev["bias_out"], residual_out=ro.view(M, K),
+                     q=qo.view(w.Hq, M, w.D), k=ko.view(w.Hkv, M, w.D), v=vo.view(w.Hkv, M, w.D))
+    handle.check()
+    for buf in (rb, qb, kbuf, vb):
+        assert torch.all(buf[:pad] == sent) and torch.all(buf[-pad:] == sent)
+
+
+def test_argument_errors(handle):
+    K, Hq, Hkv, D, M = 64, 2, 1, 8, 4
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    x = torch.randn(M, K, **bf)
+    r = torch.randn(M, K, **bf)
+    g = torch.ones(K, **bf)
+    W = torch.randn((Hq + 2 * Hkv) * D, K, **bf)
+    with pytest.raises(fnl.FnlError) as e:   # residual_out aliases x
+        fnl.add_norm_qkv(handle, x, r, g, None, W, Hq, Hkv, D, residual_out=x)
+    assert e.value.status == 3
+    with pytest.raises(fnl.FnlError) as e:   # beta with RMSNorm
+        fnl.add_norm_qkv(handle, x, r, g, g, W, Hq, Hkv, D, norm="rmsnorm")
+    assert e.value.status == 1
+    with pytest.raises(fnl.FnlError) as e:   # Hq not a multiple of Hkv
+        fnl.add_norm_qkv(handle, x, r, g, None, torch.randn(5 * 8 + 2 * 2 * 8, K, **bf), 5, 2, 8)
+    assert e.value.status == 1
+    big = torch.randn(M * K + 8, **bf)
+    with pytest.raises(fnl.FnlError) as e:   # misaligned x (2-byte offset)
+        fnl.add_norm_qkv(handle, big[1:1 + M * K].view(M, K), r, g, None, W, Hq, Hkv, D)
+    assert e.value.status == 2
+    xs = torch.randn(M, 12, **bf)
+    with pytest.raises(fnl.FnlError) as e:   # K not a multiple of 8
+        fnl.add_norm_qkv(handle, xs, xs.clone(), torch.ones(12, **bf), None, torch.randn(32, 12, **bf), 2, 1, 8)
+    assert e.value.status == 2
+    handle.check()

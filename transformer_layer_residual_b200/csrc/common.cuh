@@ -1,0 +1,125 @@
+// Parameters and epilogue arithmetic shared by the fused-op kernels.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace fnl {
+
+typedef __nv_bfloat16 bf16;
+
+enum Epi : int { kEpiQKV = 0, kEpiSwiGLU = 1, kEpiGELU = 2 };
+enum Norm : int { kLayerNorm = 0, kRMSNorm = 1 };
+
+struct OpParams {
+  int M, K, N;       // tokens, hidden, rows of W
+  int I;             // SwiGLU intermediate size (N = 2I)
+  int Hq, Hkv, D;    // QKV heads
+  float eps;
+  const bf16* gamma;
+  const bf16* beta;      // LayerNorm shift, may be null
+  const bf16* bias_in;   // [K], may be null
+  const bf16* bias;      // [N] output bias, may be null
+  bf16* residual_out;    // written in the GEMM kernels for RMSNorm, by the stats kernel for LayerNorm
+  float* rstd_out;       // RMSNorm statistics output (GEMM kernels), may be null
+  const float2* stats;   // LayerNorm (mean, rstd) per row, written by the stats kernel
+  bf16* q;
+  bf16* k;
+  bf16* v;
+  bf16* out;
+  // small-M split-K workspace
+  float* part;           // [T][max_seg][mpad][128] fp32 partial accumulators
+  float* part_ss;        // [T][max_seg][mpad] partial sums of h^2 (RMSNorm)
+  unsigned* counters;    // [T] arrival counters, zero between launches
+  int max_seg;
+  int mpad;
+  int stages;
+  int* status;           // device status word (bounded-wait failures)
+};
+
+__device__ __forceinline__ uint4 ldg16(const void* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+__device__ __forceinline__ void load8_or_zero(const bf16* base, int k0, bool ok, float (&f)[8]) {
+  if (base != nullptr && ok) {
+    unpack8(ldg16(base + k0), f);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] = 0.f;
+  }
+}
+
+// SiLU(g) = g / (1 + e^-g).
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.f + __expf(-g)); }
+
+// GELU, tanh form: 0.5 z (1 + tanh(u)) with u = sqrt(2/pi)(z + 0.044715 z^3),
+// evaluated as z / (1 + e^(-2u)) (the same function: 0.5(1 + tanh u) is the
+// logistic function of 2u), which avoids the cancellation of 1 + tanh(u) for
+// negative z.
+__device__ __forceinline__ float gelu_tanh_f(float z) {
+  const float u2 = -1.5957691216057308f * z * fmaf(0.044715f * z, z, 1.f);   // -2u
+  return __fdividef(z, 1.f + __expf(u2));
+}
+
+// Store 8 consecutive output columns [n, n+8) of row m (QKV or GELU epilogue).
+// acc is the raw fp32 accumulator, scale the deferred RMSNorm 1/rms (1 for LN).
+template <int EPI>
+__device__ __forceinline__ void store_out8(const OpParams& p, int m, int n, const float (&acc)[8], float scale) {
+  float y[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) y[e] = acc[e] * scale;
+  if (p.bias != nullptr) {
+    float b[8];
+    unpack8(ldg16(p.bias + n), b);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] += b[e];
+  }
+  bf16* dst;
+  if (EPI == kEpiGELU) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] = gelu_tanh_f(y[e]);
+    dst = p.out + static_cast<size_t>(m) * p.N + n;
+  } else {
+    const int D = p.D;
+    const int nq = p.Hq * D;
+    const int nk = nq + p.Hkv * D;
+    if (n < nq) {
+      const int h = n / D;
+      dst = p.q + (static_cast<size_t>(h) * p.M + m) * D + (n - h * D);
+    } else if (n < nk) {
+      const int n2 = n - nq, h = n2 / D;
+      dst = p.k + (static_cast<size_t>(h) * p.M + m) * D + (n2 - h * D);
+    } else {
+      const int n2 = n - nk, h = n2 / D;
+      dst = p.v + (static_cast<size_t>(h) * p.M + m) * D + (n2 - h * D);
+    }
+  }
+  *reinterpret_cast<uint4*>(dst) = pack8(y);
+}
+
+// SwiGLU epilogue for output columns [j, j+8) of row m.
+__device__ __forceinline__ void store_swiglu8(const OpParams& p, int m, int j, const float (&gate)[8],
+                                              const float (&up)[8], float scale) {
+  float g[8], u[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    g[e] = gate[e] * scale;
+    u[e] = up[e] * scale;
+  }
+  if (p.bias != nullptr) {
+    float bg[8], bu[8];
+    unpack8(ldg16(p.bias + j), bg);
+    unpack8(ldg16(p.bias + p.I + j), bu);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      g[e] += bg[e];
+      u[e] += bu[e];
+    }
+  }
+  float y[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) y[e] = silu_f(g[e]) * u[e];
+  *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(m) * p.I + j) = pack8(y);
+}
+
+}  // namespace fnl

@@ -1,0 +1,488 @@
+// C-ABI host library for the fused pre-norm linear layer (include/fnl.h).
+//
+// Host responsibilities: argument validation (alignment, sizes, aliasing),
+// the handle's device workspace (status word, split-K arrival counters,
+// LayerNorm statistics, split-K partials), TMA tensor-map encoding, the M
+// regime choice (small-M split-K kernel vs large-M tile kernel) and the
+// launches (the LayerNorm statistics kernel chained to the GEMM kernel by
+// programmatic dependent launch).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "fnl.h"
+#include "k1_stats.cuh"
+#include "k2_tile.cuh"
+#include "k3_splitk.cuh"
+
+using fnl::bf16;
+using fnl::OpParams;
+
+struct fnl_handle {
+  int device = 0;
+  int num_sms = 148;
+  fnl_options opt{};
+  uint8_t* ws = nullptr;     // device workspace
+  size_t ws_bytes = 0;
+  std::string err;
+};
+
+namespace {
+
+// ------------------------------------------------------------------ workspace
+// [status 256 B][counters kMaxTiles * 4 B][stats][part_ss][part]
+constexpr size_t kStatusBytes = 256;
+constexpr int kMaxTiles = 65536;
+constexpr size_t kCountersBytes = static_cast<size_t>(kMaxTiles) * 4;
+constexpr size_t kFixedBytes = kStatusBytes + kCountersBytes;
+
+size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+fnl_status fail(fnl_handle* h, fnl_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  if (h) h->err = buf;
+  return s;
+}
+
+fnl_status cuda_fail(fnl_handle* h, cudaError_t e, const char* what) {
+  return fail(h, FNL_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+fnl_status ensure_workspace(fnl_handle* h, cudaStream_t stream, size_t need) {
+  if (need <= h->ws_bytes) return FNL_OK;
+  cudaError_t e;
+  if (h->ws) {
+    if ((e = cudaStreamSynchronize(stream)) != cudaSuccess) return cuda_fail(h, e, "cudaStreamSynchronize");
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(h, e, "cudaDeviceSynchronize");
+    cudaFree(h->ws);
+    h->ws = nullptr;
+    h->ws_bytes = 0;
+  }
+  const size_t bytes = align256(need + need / 4);
+  if ((e = cudaMalloc(&h->ws, bytes)) != cudaSuccess) return cuda_fail(h, e, "cudaMalloc(workspace)");
+  if ((e = cudaMemset(h->ws, 0, bytes)) != cudaSuccess) return cuda_fail(h, e, "cudaMemset(workspace)");
+  h->ws_bytes = bytes;
+  return FNL_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+fnl_status get_encoder(fnl_handle* h) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return fail(h, FNL_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+  return FNL_OK;
+}
+
+// Row-major bf16 [rows, cols] (cols contiguous), box [box_rows, 64] with the
+// 128-byte swizzle the UMMA descriptors expect; out-of-range elements read 0.
+fnl_status make_map(fnl_handle* h, CUtensorMap* m, const void* ptr, long long rows, long long cols,
+                    int box_rows) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(h, FNL_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return FNL_OK;
+}
+
+// ------------------------------------------------------------------ validation
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+bool al4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0; }
+
+struct Range {
+  const void* p;
+  size_t bytes;
+  const char* name;
+};
+bool overlap(const Range& a, const Range& b) {
+  if (!a.p || !b.p || a.bytes == 0 || b.bytes == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a.p), b0 = reinterpret_cast<uintptr_t>(b.p);
+  return a0 < b0 + b.bytes && b0 < a0 + a.bytes;
+}
+
+enum class Op { QKV, SwiGLU, GELU };
+
+struct Call {
+  Op op;
+  cudaStream_t stream;
+  const bf16 *x, *residual, *bias_in, *gamma, *beta, *W, *bias;
+  bf16* residual_out;
+  fnl_norm norm;
+  float eps;
+  int M, K, N, I, Hq, Hkv, D;
+  bf16 *q, *k, *v, *out;
+  float *mean_out, *rstd_out;
+};
+
+fnl_status validate(fnl_handle* h, const Call& c) {
+  if (!h) return FNL_ERR_INVALID_ARG;
+  if (c.norm != FNL_NORM_LAYERNORM && c.norm != FNL_NORM_RMSNORM)
+    return fail(h, FNL_ERR_INVALID_ARG, "norm must be FNL_NORM_LAYERNORM or FNL_NORM_RMSNORM");
+  if (!(c.eps >= 0.f) || c.eps != c.eps || c.eps > 1e30f)
+    return fail(h, FNL_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (c.M < 0 || c.K <= 0 || c.N <= 0) return fail(h, FNL_ERR_INVALID_ARG, "need M >= 0, K > 0, N > 0");
+  if (c.K % 8 || c.N % 8) return fail(h, FNL_ERR_ALIGNMENT, "K and N must be multiples of 8 (K=%d N=%d)", c.K, c.N);
+  if (c.K > 32768) return fail(h, FNL_ERR_UNSUPPORTED, "K=%d exceeds 32768", c.K);
+  if (c.op == Op::QKV) {
+    if (c.Hq <= 0 || c.Hkv <= 0 || c.D <= 0) return fail(h, FNL_ERR_INVALID_ARG, "Hq, Hkv, D must be > 0");
+    if (c.Hq % c.Hkv) return fail(h, FNL_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", c.Hq, c.Hkv);
+    if (c.D % 8) return fail(h, FNL_ERR_ALIGNMENT, "D must be a multiple of 8 (D=%d)", c.D);
+  }
+  if (c.op == Op::SwiGLU && (c.I <= 0 || c.I % 8))
+    return fail(h, FNL_ERR_ALIGNMENT, "I must be a positive multiple of 8 (I=%d)", c.I);
+  if (c.N / 128 + 1 > kMaxTiles) return fail(h, FNL_ERR_UNSUPPORTED, "N=%d too large", c.N);
+  if (c.norm == FNL_NORM_RMSNORM && c.beta)
+    return fail(h, FNL_ERR_INVALID_ARG, "beta must be NULL for RMSNorm");
+  if (c.norm == FNL_NORM_RMSNORM && c.mean_out)
+    return fail(h, FNL_ERR_INVALID_ARG, "mean_out must be NULL for RMSNorm (no mean is computed)");
+  if (h->opt.path == FNL_PATH_SPLITK && c.M > fnl::k3::MAX_MPAD)
+    return fail(h, FNL_ERR_UNSUPPORTED, "forced split-K path needs M <= %d", fnl::k3::MAX_MPAD);
+  if (c.M == 0) return FNL_OK;
+  // required pointers
+  if (!c.x || !c.residual || !c.residual_out || !c.gamma || !c.W)
+    return fail(h, FNL_ERR_INVALID_ARG, "x, residual, residual_out, gamma and W are required");
+  if (c.op == Op::QKV && (!c.q || !c.k || !c.v)) return fail(h, FNL_ERR_INVALID_ARG, "q, k, v are required");
+  if (c.op != Op::QKV && !c.out) return fail(h, FNL_ERR_INVALID_ARG, "out is required");
+  const void* p16[] = {c.x, c.residual, c.bias_in, c.gamma, c.beta, c.W, c.bias, c.residual_out,
+                       c.q, c.k, c.v, c.out};
+  for (const void* p : p16)
+    if (p && !al16(p)) return fail(h, FNL_ERR_ALIGNMENT, "a bf16 pointer is not 16-byte aligned");
+  if ((c.mean_out && !al4(c.mean_out)) || (c.rstd_out && !al4(c.rstd_out)))
+    return fail(h, FNL_ERR_ALIGNMENT, "mean_out / rstd_out must be 4-byte aligned");
+  // aliasing: outputs vs inputs and vs each other
+  const size_t MK = static_cast<size_t>(c.M) * c.K * 2;
+  const size_t n_out = c.op == Op::SwiGLU ? static_cast<size_t>(c.I) : static_cast<size_t>(c.N);
+  std::vector<Range> ins = {{c.x, MK, "x"},
+                            {c.residual, MK, "residual"},
+                            {c.bias_in, static_cast<size_t>(c.K) * 2, "bias_in"},
+                            {c.gamma, static_cast<size_t>(c.K) * 2, "gamma"},
+                            {c.beta, static_cast<size_t>(c.K) * 2, "beta"},
+                            {c.W, static_cast<size_t>(c.N) * c.K * 2, "W"},
+                            {c.bias, static_cast<size_t>(c.N) * 2, "bias"}};
+  std::vector<Range> outs = {{c.residual_out, MK, "residual_out"},
+                             {c.mean_out, static_cast<size_t>(c.M) * 4, "mean_out"},
+                             {c.rstd_out, static_cast<size_t>(c.M) * 4, "rstd_out"}};
+  if (c.op == Op::QKV) {
+    outs.push_back({c.q, static_cast<size_t>(c.Hq) * c.M * c.D * 2, "q"});
+    outs.push_back({c.k, static_cast<size_t>(c.Hkv) * c.M * c.D * 2, "k"});
+    outs.push_back({c.v, static_cast<size_t>(c.Hkv) * c.M * c.D * 2, "v"});
+  } else {
+    outs.push_back({c.out, static_cast<size_t>(c.M) * n_out * 2, "out"});
+  }
+  for (size_t i = 0; i < outs.size(); ++i) {
+    for (const Range& in : ins)
+      if (overlap(outs[i], in))
+        return fail(h, FNL_ERR_ALIAS, "output %s overlaps input %s", outs[i].name, in.name);
+    for (size_t j = i + 1; j < outs.size(); ++j)
+      if (overlap(outs[i], outs[j]))
+        return fail(h, FNL_ERR_ALIAS, "outputs %s and %s overlap", outs[i].name, outs[j].name);
+  }
+  return FNL_OK;
+}
+
+// ------------------------------------------------------------------ launches
+template <typename Kern>
+fnl_status set_smem(fnl_handle* h, Kern kern, int bytes) {
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaFuncSetAttribute");
+  return FNL_OK;
+}
+
+template <typename Kern>
+fnl_status launch_gemm(fnl_handle* h, Kern kern, int grid, int threads, int smem, bool pdl, cudaStream_t stream,
+                       const CUtensorMap& mx, const CUtensorMap& mr, const CUtensorMap& mw, const OpParams& p) {
+  fnl_status st = set_smem(h, kern, smem);
+  if (st != FNL_OK) return st;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mx, mr, mw, p);
+  if (e != cudaSuccess) return cuda_fail(h, e, "launch of the fused GEMM kernel");
+  return FNL_OK;
+}
+
+template <int EPI>
+fnl_status dispatch_gemm(fnl_handle* h, bool small, bool rms, int grid, int threads, int smem, bool pdl,
+                         cudaStream_t stream, const CUtensorMap& mx, const CUtensorMap& mr, const CUtensorMap& mw,
+                         const OpParams& p) {
+  if (small) {
+    if (rms)
+      return launch_gemm(h, fnl::k3_splitk_kernel<EPI, fnl::kRMSNorm>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
+    return launch_gemm(h, fnl::k3_splitk_kernel<EPI, fnl::kLayerNorm>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
+  }
+  if (rms)
+    return launch_gemm(h, fnl::k2_tile_kernel<EPI, fnl::kRMSNorm>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
+  return launch_gemm(h, fnl::k2_tile_kernel<EPI, fnl::kLayerNorm>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
+}
+
+fnl_status launch_k1(fnl_handle* h, const Call& c, float2* stats, cudaStream_t stream) {
+  const int nvec = c.K / 8;
+  const int v = (nvec + fnl::kK1Threads - 1) / fnl::kK1Threads;
+  dim3 grid(c.M), block(fnl::kK1Threads);
+#define FNL_K1(MAXV)                                                                                     \
+  fnl::k1_layernorm_stats<MAXV><<<grid, block, 0, stream>>>(c.x, c.residual, c.bias_in, c.residual_out, \
+                                                            stats, c.mean_out, c.rstd_out, c.M, c.K, c.eps)
+  if (v <= 1) FNL_K1(1);
+  else if (v <= 2) FNL_K1(2);
+  else if (v <= 4) FNL_K1(4);
+  else if (v <= 8) FNL_K1(8);
+  else FNL_K1(16);
+#undef FNL_K1
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(h, e, "launch of the LayerNorm statistics kernel");
+  return FNL_OK;
+}
+
+int round_up(int a, int b) { return (a + b - 1) / b * b; }
+
+fnl_status run(fnl_handle* h, const Call& c) {
+  fnl_status st = validate(h, c);
+  if (st != FNL_OK || c.M == 0) return st;
+  if ((st = get_encoder(h)) != FNL_OK) return st;
+  cudaError_t e = cudaSetDevice(h->device);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaSetDevice");
+
+  const bool rms = c.norm == FNL_NORM_RMSNORM;
+  const int epi = c.op == Op::QKV ? fnl::kEpiQKV : (c.op == Op::SwiGLU ? fnl::kEpiSwiGLU : fnl::kEpiGELU);
+  bool small = c.M <= fnl::k3::MAX_MPAD;
+  if (h->opt.path == FNL_PATH_TILE) small = false;
+  if (h->opt.path == FNL_PATH_SPLITK) small = true;
+  const int max_ctas = h->opt.max_ctas > 0 ? std::min(h->opt.max_ctas, h->num_sms) : h->num_sms;
+  const int nkb = (c.K + 63) / 64;
+
+  // plan
+  int grid = 1, threads = 0, smem = 0, mpad = 0, stages = 0, max_seg = 1, T = 0;
+  if (small) {
+    mpad = round_up(std::max(c.M, 1), 16);
+    T = c.op == Op::SwiGLU ? (c.I + 63) / 64 : (c.N + 127) / 128;
+    const long long U = static_cast<long long>(T) * nkb;
+    grid = static_cast<int>(std::min<long long>(max_ctas, U));
+    stages = std::min(fnl::k3::MAX_STAGES, (200 * 1024) / fnl::k3::stage_bytes(mpad));
+    smem = fnl::k3::smem_bytes(mpad, stages);
+    threads = fnl::k3::NUM_THREADS;
+    for (int t = 0; t < T; ++t) {
+      const int first = fnl::k3::unit_owner(static_cast<long long>(t) * nkb, grid, U);
+      const int last = fnl::k3::unit_owner(static_cast<long long>(t + 1) * nkb - 1, grid, U);
+      max_seg = std::max(max_seg, last - first + 1);
+    }
+    if (T > kMaxTiles) return fail(h, FNL_ERR_UNSUPPORTED, "too many W tiles");
+  } else {
+    const int num_m = (c.M + fnl::k2::BM - 1) / fnl::k2::BM;
+    const int num_n = c.op == Op::SwiGLU ? (c.I + 127) / 128 : (c.N + fnl::k2::BN - 1) / fnl::k2::BN;
+    const long long tiles = static_cast<long long>(num_m) * num_n;
+    grid = static_cast<int>(std::min<long long>(max_ctas, tiles));
+    smem = fnl::k2::SMEM_BYTES;
+    threads = fnl::k2::NUM_THREADS;
+  }
+
+  // workspace
+  const size_t stats_bytes = rms ? 0 : align256(static_cast<size_t>(c.M) * 8);
+  const size_t ss_bytes = small ? align256(static_cast<size_t>(T) * max_seg * mpad * 4) : 0;
+  const size_t part_bytes = small ? align256(static_cast<size_t>(T) * max_seg * mpad * 128 * 4) : 0;
+  const size_t need = kFixedBytes + stats_bytes + ss_bytes + part_bytes;
+  if ((st = ensure_workspace(h, c.stream, need)) != FNL_OK) return st;
+  uint8_t* ws = h->ws;
+  int* status = reinterpret_cast<int*>(ws);
+  unsigned* counters = reinterpret_cast<unsigned*>(ws + kStatusBytes);
+  float2* stats = reinterpret_cast<float2*>(ws + kFixedBytes);
+  float* part_ss = reinterpret_cast<float*>(ws + kFixedBytes + stats_bytes);
+  float* part = reinterpret_cast<float*>(ws + kFixedBytes + stats_bytes + ss_bytes);
+
+  OpParams p{};
+  p.M = c.M; p.K = c.K; p.N = c.N; p.I = c.I; p.Hq = c.Hq; p.Hkv = c.Hkv; p.D = c.D; p.eps = c.eps;
+  p.gamma = c.gamma; p.beta = c.beta; p.bias_in = c.bias_in; p.bias = c.bias;
+  p.residual_out = c.residual_out; p.rstd_out = rms ? c.rstd_out : nullptr; p.stats = stats;
+  p.q = c.q; p.k = c.k; p.v = c.v; p.out = c.out;
+  p.part = part; p.part_ss = part_ss; p.counters = counters; p.max_seg = max_seg; p.mpad = mpad;
+  p.stages = stages; p.status = status;
+
+  // tensor maps: x and residual tiles are [rows x 64], W tiles [rows x 64]
+  CUtensorMap mx, mr, mw;
+  const int act_rows = small ? mpad : fnl::k2::BM;
+  int w_rows;
+  if (small) w_rows = c.op == Op::SwiGLU ? 64 : fnl::k3::BW;
+  else w_rows = c.op == Op::SwiGLU ? 128 : fnl::k2::BN;
+  if ((st = make_map(h, &mx, c.x, c.M, c.K, act_rows)) != FNL_OK) return st;
+  if ((st = make_map(h, &mr, c.residual, c.M, c.K, act_rows)) != FNL_OK) return st;
+  if ((st = make_map(h, &mw, c.W, c.N, c.K, w_rows)) != FNL_OK) return st;
+
+  if (!rms) {
+    if ((st = launch_k1(h, c, stats, c.stream)) != FNL_OK) return st;
+  }
+  const bool pdl = !rms;
+  switch (epi) {
+    case fnl::kEpiQKV:
+      return dispatch_gemm<fnl::kEpiQKV>(h, small, rms, grid, threads, smem, pdl, c.stream, mx, mr, mw, p);
+    case fnl::kEpiSwiGLU:
+      return dispatch_gemm<fnl::kEpiSwiGLU>(h, small, rms, grid, threads, smem, pdl, c.stream, mx, mr, mw, p);
+    default:
+      return dispatch_gemm<fnl::kEpiGELU>(h, small, rms, grid, threads, smem, pdl, c.stream, mx, mr, mw, p);
+  }
+}
+
+const bf16* B(const fnl_bf16* p) { return reinterpret_cast<const bf16*>(p); }
+bf16* Bm(fnl_bf16* p) { return reinterpret_cast<bf16*>(p); }
+
+}  // namespace
+
+extern "C" {
+
+fnl_status fnl_create(fnl_handle** out, int device, const fnl_options* opt) {
+  if (!out) return FNL_ERR_INVALID_ARG;
+  *out = nullptr;
+  fnl_handle* h = new fnl_handle();
+  if (opt) h->opt = *opt;
+  if (h->opt.path < FNL_PATH_AUTO || h->opt.path > FNL_PATH_SPLITK || h->opt.max_tokens < 0 || h->opt.max_n < 0) {
+    delete h;
+    return FNL_ERR_INVALID_ARG;
+  }
+  h->device = device;
+  cudaError_t e = cudaSetDevice(device);
+  if (e != cudaSuccess) {
+    delete h;
+    return FNL_ERR_CUDA;
+  }
+  int sms = 0, major = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device);
+  if (major != 10) {
+    delete h;
+    return FNL_ERR_UNSUPPORTED;   // the kernels are built for sm_100a only
+  }
+  h->num_sms = sms > 0 ? sms : 148;
+  // reserve workspace for the declared maxima (small-M partials dominate)
+  size_t need = kFixedBytes;
+  if (h->opt.max_tokens > 0) need += align256(static_cast<size_t>(h->opt.max_tokens) * 8);
+  if (h->opt.max_n > 0) {
+    const size_t T = static_cast<size_t>(h->opt.max_n) / 64 + 1;
+    const size_t seg = static_cast<size_t>(h->num_sms) / std::max<size_t>(T, 1) + 2;
+    need += align256(T * seg * fnl::k3::MAX_MPAD * 4) + align256(T * seg * fnl::k3::MAX_MPAD * 128 * 4);
+  }
+  fnl_status st = ensure_workspace(h, nullptr, need);
+  if (st != FNL_OK) {
+    delete h;
+    return st;
+  }
+  *out = h;
+  return FNL_OK;
+}
+
+fnl_status fnl_destroy(fnl_handle* h) {
+  if (!h) return FNL_OK;
+  cudaSetDevice(h->device);
+  cudaDeviceSynchronize();
+  if (h->ws) cudaFree(h->ws);
+  delete h;
+  return FNL_OK;
+}
+
+const char* fnl_status_string(fnl_status s) {
+  switch (s) {
+    case FNL_OK: return "FNL_OK";
+    case FNL_ERR_INVALID_ARG: return "FNL_ERR_INVALID_ARG";
+    case FNL_ERR_ALIGNMENT: return "FNL_ERR_ALIGNMENT";
+    case FNL_ERR_ALIAS: return "FNL_ERR_ALIAS";
+    case FNL_ERR_UNSUPPORTED: return "FNL_ERR_UNSUPPORTED";
+    case FNL_ERR_CUDA: return "FNL_ERR_CUDA";
+    case FNL_ERR_DEVICE_STATUS: return "FNL_ERR_DEVICE_STATUS";
+  }
+  return "FNL_ERR_UNKNOWN";
+}
+
+const char* fnl_last_error(const fnl_handle* h) { return h ? h->err.c_str() : ""; }
+
+fnl_status fnl_check(fnl_handle* h, fnl_stream stream) {
+  if (!h) return FNL_ERR_INVALID_ARG;
+  cudaSetDevice(h->device);
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaStreamSynchronize");
+  int status = 0;
+  e = cudaMemcpy(&status, h->ws, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemcpy(status)");
+  if (status != 0) {
+    cudaMemset(h->ws, 0, sizeof(int));
+    return fail(h, FNL_ERR_DEVICE_STATUS, "a kernel gave up a bounded wait (code %d)", status);
+  }
+  return FNL_OK;
+}
+
+fnl_status fnl_add_norm_qkv(fnl_handle* h, fnl_stream stream, const fnl_bf16* x, const fnl_bf16* residual,
+                            fnl_bf16* residual_out, const fnl_bf16* gamma, const fnl_bf16* beta, fnl_norm norm,
+                            float eps, const fnl_bf16* W, const fnl_bf16* bias, int M, int K, int Hq, int Hkv,
+                            int D, fnl_bf16* q, fnl_bf16* k, fnl_bf16* v, float* mean_out, float* rstd_out) {
+  Call c{};
+  c.op = Op::QKV;
+  c.stream = reinterpret_cast<cudaStream_t>(stream);
+  c.x = B(x); c.residual = B(residual); c.bias_in = nullptr; c.gamma = B(gamma); c.beta = B(beta);
+  c.W = B(W); c.bias = B(bias); c.residual_out = Bm(residual_out);
+  c.norm = norm; c.eps = eps; c.M = M; c.K = K; c.Hq = Hq; c.Hkv = Hkv; c.D = D;
+  c.N = (Hq > 0 && Hkv > 0 && D > 0) ? (Hq + 2 * Hkv) * D : 0;
+  c.q = Bm(q); c.k = Bm(k); c.v = Bm(v); c.out = nullptr;
+  c.mean_out = mean_out; c.rstd_out = rstd_out;
+  if (c.N <= 0 && h) return fail(h, FNL_ERR_INVALID_ARG, "Hq, Hkv, D must be > 0");
+  return run(h, c);
+}
+
+fnl_status fnl_add_norm_swiglu(fnl_handle* h, fnl_stream stream, const fnl_bf16* x, const fnl_bf16* residual,
+                               fnl_bf16* residual_out, const fnl_bf16* gamma, const fnl_bf16* beta, fnl_norm norm,
+                               float eps, const fnl_bf16* W, const fnl_bf16* bias, int M, int K, int I,
+                               fnl_bf16* out, float* mean_out, float* rstd_out) {
+  Call c{};
+  c.op = Op::SwiGLU;
+  c.stream = reinterpret_cast<cudaStream_t>(stream);
+  c.x = B(x); c.residual = B(residual); c.bias_in = nullptr; c.gamma = B(gamma); c.beta = B(beta);
+  c.W = B(W); c.bias = B(bias); c.residual_out = Bm(residual_out);
+  c.norm = norm; c.eps = eps; c.M = M; c.K = K; c.I = I; c.N = I > 0 ? 2 * I : 0;
+  c.out = Bm(out);
+  c.mean_out = mean_out; c.rstd_out = rstd_out;
+  if (c.N <= 0 && h) return fail(h, FNL_ERR_INVALID_ARG, "I must be > 0");
+  return run(h, c);
+}
+
+fnl_status fnl_add_bias_norm_gelu(fnl_handle* h, fnl_stream stream, const fnl_bf16* x, const fnl_bf16* residual,
+                                  const fnl_bf16* bias_in, fnl_bf16* residual_out, const fnl_bf16* gamma,
+                                  const fnl_bf16* beta, fnl_norm norm, float eps, const fnl_bf16* W,
+                                  const fnl_bf16* bias_out, int M, int K, int N, fnl_bf16* out, float* mean_out,
+                                  float* rstd_out) {
+  Call c{};
+  c.op = Op::GELU;
+  c.stream = reinterpret_cast<cudaStream_t>(stream);
+  c.x = B(x); c.residual = B(residual); c.bias_in = B(bias_in); c.gamma = B(gamma); c.beta = B(beta);
+  c.W = B(W); c.bias = B(bias_out); c.residual_out = Bm(residual_out);
+  c.norm = norm; c.eps = eps; c.M = M; c.K = K; c.N = N;
+  c.out = Bm(out);
+  c.mean_out = mean_out; c.rstd_out = rstd_out;
+  return run(h, c);
+}
+
+}  // extern "C"

@@ -1,0 +1,374 @@
+// K2: large-M fused norm + GEMM + epilogue, persistent, one CTA per SM.
+//
+// Tile: 128 tokens x 256 W rows (SwiGLU: 128 gate rows + the matching 128 up
+// rows), K in blocks of 64. Warp roles (14 warps):
+//   warp 0      TMA producer: per k-block, x and residual tiles [128 x 64] and
+//               the W tile [256 x 64], 128-byte swizzled, into one of 3 stages;
+//   warp 1      TMEM owner and UMMA issuer (one thread): 4 x
+//               tcgen05.mma M=128 N=256 K=16 per k-block into one of two
+//               256-column fp32 accumulators;
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator (lane = token row),
+//               deferred RMSNorm scale, bias, QKV head-major split / SwiGLU /
+//               GELU, bf16 stores straight to the outputs;
+//   warps 6-13  converters: in place in shared memory, turn the x tile into the
+//               normalised bf16 A operand a = norm(x + r (+ bias_in)) using the
+//               residual tile, so the normalised activations never touch global
+//               memory (the "shared memory caching of normalised values /
+//               eliminating the intermediate write-back" of TensorRT-LLM
+//               深度工程实践, §2.3).
+// LayerNorm: (mean, rstd) per row come from the statistics kernel (K1).
+// RMSNorm: deferred scaling. The converters write a' = bf16(gamma * h) and sum
+// h^2 per row over the K loop; 1/rms is applied per accumulator row in the
+// epilogue (y = rstd * sum_k a'_k W_nk is the same product). Tiles in the first
+// N column also write residual_out and rstd_out, so RMSNorm needs no extra pass.
+#pragma once
+
+#include "common.cuh"
+
+namespace fnl {
+namespace k2 {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 3;
+constexpr int X_BYTES = BM * BK * 2;                 // 16 KB
+constexpr int W_BYTES = BN * BK * 2;                 // 32 KB
+constexpr int STAGE_BYTES = 2 * X_BYTES + W_BYTES;   // 64 KB
+constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_EPI0 = 2, NUM_EPI_WARPS = 4;
+constexpr int WARP_CONV0 = 6, NUM_CONV_WARPS = 8;
+constexpr int NUM_THREADS = (WARP_CONV0 + NUM_CONV_WARPS) * 32;   // 448
+constexpr int TMEM_COLS = 2 * BN;                                  // 512
+constexpr int GROUP_M = 16;  // tile raster: 16 M-blocks share each W tile while it is hot in L2
+
+struct Ctrl {
+  uint64_t full[STAGES], conv[STAGES], empty[STAGES];
+  uint64_t tfull[2], tempty[2], sfull[2], drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  float rs[2][BM];
+};
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + static_cast<int>(sizeof(Ctrl)) + 1024;
+
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
+  const int per_group = GROUP_M * num_n;
+  const int group = t / per_group;
+  const int first_m = group * GROUP_M;
+  const int gm = min(GROUP_M, num_m - first_m);
+  const int r = t - group * per_group;
+  mb = first_m + r % gm;
+  nb = r / gm;
+}
+
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > FNL_WAIT_NS) return false;
+  }
+  return true;
+}
+
+}  // namespace k2
+
+template <int EPI, int NORM>
+__global__ void __launch_bounds__(k2::NUM_THREADS, 1)
+    k2_tile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_r,
+                   const __grid_constant__ CUtensorMap tm_w, const OpParams p) {
+  using namespace k2;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + STAGES * STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int M = p.M, K = p.K;
+  const int num_m = (M + BM - 1) / BM;
+  const int num_n = (EPI == kEpiSwiGLU) ? (p.I + 127) / 128 : (p.N + BN - 1) / BN;
+  const int tiles = num_m * num_n;
+  const int nkb = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&ctrl->full[s], 1);
+      mbar_init(&ctrl->conv[s], NUM_CONV_WARPS);
+      mbar_init(&ctrl->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctrl->tfull[b], 1);
+      mbar_init(&ctrl->tempty[b], NUM_EPI_WARPS);
+      mbar_init(&ctrl->sfull[b], NUM_CONV_WARPS);
+    }
+    mbar_init(&ctrl->drain, 1);
+    ctrl->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == WARP_TMA && lane == 0) {
+    prefetch_tmap(&tm_x);
+    prefetch_tmap(&tm_r);
+    prefetch_tmap(&tm_w);
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(&ctrl->tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+  volatile int* abortf = &ctrl->abort_flag;
+
+  if (warp == WARP_TMA) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t s = 0, ph = 0;
+      uint32_t armed = 0;   // stages armed at least once (bitmask) for the abort drain
+      uint32_t last_par = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        int mb, nb;
+        tile_coords(t, num_m, num_n, mb, nb);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&ctrl->empty[s], ph ^ 1, abortf, p.status, kStatusWaitEmpty)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * STAGE_BYTES;
+          mbar_arrive_expect_tx(&ctrl->full[s], STAGE_BYTES);
+          tma_load_2d(st, &tm_x, &ctrl->full[s], kb * BK, mb * BM);
+          tma_load_2d(st + X_BYTES, &tm_r, &ctrl->full[s], kb * BK, mb * BM);
+          if (EPI == kEpiSwiGLU) {
+            tma_load_2d(st + 2 * X_BYTES, &tm_w, &ctrl->full[s], kb * BK, nb * 128);
+            tma_load_2d(st + 2 * X_BYTES + W_BYTES / 2, &tm_w, &ctrl->full[s], kb * BK, p.I + nb * 128);
+          } else {
+            tma_load_2d(st + 2 * X_BYTES, &tm_w, &ctrl->full[s], kb * BK, nb * BN);
+          }
+          armed |= 1u << s;
+          last_par = (last_par & ~(1u << s)) | (ph << s);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+      }
+      if (!ok) {   // let every issued copy land before the CTA can exit
+        for (int i = 0; i < STAGES; ++i)
+          if (armed & (1u << i)) drain_wait(&ctrl->full[i], (last_par >> i) & 1);
+      }
+    }
+  } else if (warp == WARP_MMA) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      uint32_t s = 0, ph = 0;
+      bool ok = true;
+      const uint32_t idesc = idesc_bf16(BM, BN);
+      int i = 0;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++i) {
+        const int b = i & 1;
+        const uint32_t use = static_cast<uint32_t>(i >> 1);
+        if (!mbar_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + b * BN;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&ctrl->conv[s], ph, abortf, p.status, kStatusWaitConv) ||
+              !mbar_wait(&ctrl->full[s], ph, abortf, p.status, kStatusWaitFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t xa = smem_u32(smem + s * STAGE_BYTES);
+          const uint64_t ad = sw128_desc(xa);
+          const uint64_t bd = sw128_desc(xa + 2 * X_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+          umma_commit(&ctrl->empty[s]);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&ctrl->tfull[b]);
+      }
+      umma_commit(&ctrl->drain);   // every issued UMMA done before TMEM is freed
+      drain_wait(&ctrl->drain, 0);
+    }
+  } else if (warp < WARP_CONV0) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;   // TMEM lane quadrant this warp may read
+    const int row_local = q * 32 + lane;
+    int i = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+      const int b = i & 1;
+      const uint32_t use = static_cast<uint32_t>(i >> 1);
+      if (!warp_wait(&ctrl->tfull[b], use & 1, abortf, p.status, kStatusWaitTmemFull)) break;
+      float scale = 1.f;
+      if (NORM == kRMSNorm) {
+        if (!warp_wait(&ctrl->sfull[b], use & 1, abortf, p.status, kStatusWaitStats)) break;
+        scale = ctrl->rs[b][row_local];
+      }
+      tc_fence_after();
+      int mb, nb;
+      tile_coords(t, num_m, num_n, mb, nb);
+      const int m = mb * BM + row_local;
+      const bool row_ok = m < M;
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
+      if (EPI == kEpiSwiGLU) {
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t g0[16], g1[16], u0[16], u1[16];
+          tmem_ld16(tbase + cc * 32, g0);
+          tmem_ld16(tbase + cc * 32 + 16, g1);
+          tmem_ld16(tbase + 128 + cc * 32, u0);
+          tmem_ld16(tbase + 128 + cc * 32 + 16, u1);
+          tmem_ld_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) {
+              const int j = nb * 128 + cc * 32 + g8 * 8;
+              if (j < p.I) {
+                float gv[8], uv[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const int c = g8 * 8 + e;
+                  gv[e] = __uint_as_float(c < 16 ? g0[c] : g1[c - 16]);
+                  uv[e] = __uint_as_float(c < 16 ? u0[c] : u1[c - 16]);
+                }
+                store_swiglu8(p, m, j, gv, uv, scale);
+              }
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          uint32_t a0[16], a1[16];
+          tmem_ld16(tbase + cc * 32, a0);
+          tmem_ld16(tbase + cc * 32 + 16, a1);
+          tmem_ld_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) {
+              const int n = nb * BN + cc * 32 + g8 * 8;
+              if (n < p.N) {
+                float av[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const int c = g8 * 8 + e;
+                  av[e] = __uint_as_float(c < 16 ? a0[c] : a1[c - 16]);
+                }
+                store_out8<EPI>(p, m, n, av, scale);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctrl->tempty[b]);
+    }
+  } else {
+    // ------------------------------------------------------------ converters
+    const int ct = threadIdx.x - WARP_CONV0 * 32;   // 0..255
+    const int c = ct & 7;                            // 16-byte chunk of the 128-byte row
+    const int rbase = ct >> 3;                       // rows rbase + 32 j
+    if (NORM == kLayerNorm) pdl_wait();              // statistics come from the previous kernel
+    uint32_t s = 0, ph = 0;
+    int i = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++i) {
+      int mb, nb;
+      tile_coords(t, num_m, num_n, mb, nb);
+      float mu[4], rs[4], ss[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int gm = mb * BM + rbase + 32 * j;
+        ss[j] = 0.f;
+        mu[j] = 0.f;
+        rs[j] = 0.f;
+        if (NORM == kLayerNorm && gm < M) {
+          const float2 st = p.stats[gm];
+          mu[j] = st.x;
+          rs[j] = st.y;
+        }
+      }
+      const bool write_res = (NORM == kRMSNorm) && nb == 0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!warp_wait(&ctrl->full[s], ph, abortf, p.status, kStatusWaitFull)) {
+          ok = false;
+          break;
+        }
+        const int k0 = kb * BK + c * 8;
+        const bool kin = k0 < K;
+        float g[8], be[8], bi[8];
+        load8_or_zero(p.gamma, k0, kin, g);
+        load8_or_zero(NORM == kLayerNorm ? p.beta : nullptr, k0, kin, be);
+        load8_or_zero(p.bias_in, k0, kin, bi);
+        const uint32_t xs = smem_u32(smem + s * STAGE_BYTES);
+        const uint32_t rsm = xs + X_BYTES;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int row = rbase + 32 * j;
+          const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
+          float h[8], rr[8], a[8];
+          unpack8(ld_shared_v4(xs + off), h);
+          unpack8(ld_shared_v4(rsm + off), rr);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) h[e] = (h[e] + rr[e]) + bi[e];
+          if (NORM == kLayerNorm) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) a[e] = fmaf((h[e] - mu[j]) * rs[j], g[e], be[e]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              a[e] = h[e] * g[e];
+              ss[j] = fmaf(h[e], h[e], ss[j]);
+            }
+          }
+          st_shared_v4(xs + off, pack8(a));
+          if (write_res) {
+            const int gm = mb * BM + row;
+            if (gm < M && kin)
+              *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(gm) * K + k0) = pack8(h);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->conv[s]);
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
+      if (!ok) break;
+      if (NORM == kRMSNorm) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], 1);
+          ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], 2);
+          ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], 4);
+        }
+        const int b = i & 1;
+        const uint32_t use = static_cast<uint32_t>(i >> 1);
+        if (!warp_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty)) break;
+        if (c == 0) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int row = rbase + 32 * j;
+            const float r = 1.f / sqrtf(ss[j] / static_cast<float>(K) + p.eps);
+            ctrl->rs[b][row] = r;
+            const int gm = mb * BM + row;
+            if (write_res && p.rstd_out != nullptr && gm < M) p.rstd_out[gm] = r;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->sfull[b]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace fnl

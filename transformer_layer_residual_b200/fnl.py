@@ -1,0 +1,222 @@
+"""ctypes binding of libfnl.so (include/fnl.h), same names as the C entry points.
+
+Argument marshalling only: the functions take torch CUDA tensors, check their
+dtype/device/contiguity, allocate missing outputs with torch, and pass raw
+pointers plus the current CUDA stream to the C library. Every step of the fused
+op runs in the library's kernels. There is no fallback: if the library is
+missing or the device is not sm_100, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfnl.so")
+_lib = None
+
+FNL_OK = 0
+STATUS_NAMES = {0: "FNL_OK", 1: "FNL_ERR_INVALID_ARG", 2: "FNL_ERR_ALIGNMENT", 3: "FNL_ERR_ALIAS",
+                4: "FNL_ERR_UNSUPPORTED", 5: "FNL_ERR_CUDA", 6: "FNL_ERR_DEVICE_STATUS"}
+NORMS = {"layernorm": 0, "rmsnorm": 1}
+PATHS = {"auto": 0, "tile": 1, "splitk": 2}
+
+EXPORTED = ("fnl_create", "fnl_destroy", "fnl_status_string", "fnl_last_error", "fnl_check",
+            "fnl_add_norm_qkv", "fnl_add_norm_swiglu", "fnl_add_bias_norm_gelu")
+
+
+class FnlError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+class _Options(ctypes.Structure):
+    _fields_ = [("max_tokens", ctypes.c_int), ("max_n", ctypes.c_int), ("path", ctypes.c_int),
+                ("max_ctas", ctypes.c_int)]
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfnl.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                           "`python -m transformer_layer_residual_b200.build`")
+    L = ctypes.CDLL(_LIB_PATH)
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    L.fnl_create.argtypes = [ctypes.POINTER(P), I, ctypes.POINTER(_Options)]
+    L.fnl_destroy.argtypes = [P]
+    L.fnl_status_string.argtypes = [I]
+    L.fnl_status_string.restype = ctypes.c_char_p
+    L.fnl_last_error.argtypes = [P]
+    L.fnl_last_error.restype = ctypes.c_char_p
+    L.fnl_check.argtypes = [P, P]
+    L.fnl_add_norm_qkv.argtypes = [P, P, P, P, P, P, P, I, F, P, P, I, I, I, I, I, P, P, P, P, P]
+    L.fnl_add_norm_swiglu.argtypes = [P, P, P, P, P, P, P, I, F, P, P, I, I, I, P, P, P]
+    L.fnl_add_bias_norm_gelu.argtypes = [P, P, P, P, P, P, P, P, I, F, P, P, I, I, I, P, P, P]
+    for name in EXPORTED:
+        if getattr(L, name).restype is None and name not in ("fnl_status_string", "fnl_last_error"):
+            getattr(L, name).restype = I
+    _lib = L
+    return L
+
+
+class Handle:
+    """Owns an fnl_handle (device workspace). One stream / thread at a time."""
+
+    def __init__(self, device: int = 0, max_tokens: int = 0, max_n: int = 0, path: str = "auto",
+                 max_ctas: int = 0):
+        L = lib()
+        self._h = ctypes.c_void_p()
+        opt = _Options(max_tokens, max_n, PATHS[path], max_ctas)
+        st = L.fnl_create(ctypes.byref(self._h), device, ctypes.byref(opt))
+        if st != FNL_OK:
+            raise FnlError(st, f"fnl_create(device={device}) failed")
+        self.device = device
+
+    def close(self):
+        if getattr(self, "_h", None) and self._h.value:
+            lib().fnl_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def ptr(self):
+        return self._h
+
+    def _raise(self, st: int, what: str):
+        msg = lib().fnl_last_error(self._h)
+        raise FnlError(st, f"{what}: {msg.decode() if msg else ''}")
+
+    def check(self, stream: Optional[torch.cuda.Stream] = None):
+        """Synchronise the stream and raise if a kernel gave up a bounded wait."""
+        st = lib().fnl_check(self._h, _stream_ptr(stream))
+        if st != FNL_OK:
+            self._raise(st, "fnl_check")
+
+
+def _stream_ptr(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, name, shape=None, dtype=torch.bfloat16):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _common(x, residual, gamma, beta, norm, residual_out, mean_out, rstd_out, W, bias):
+    M, K = x.shape
+    _need(x, "x", (M, K))
+    _need(residual, "residual", (M, K))
+    _need(gamma, "gamma", (K,))
+    _need(beta, "beta", (K,))
+    _need(W, "W")
+    if W.dim() != 2 or W.shape[1] != K:
+        raise ValueError("W must be [N, K]")
+    _need(bias, "bias", (W.shape[0],))
+    if residual_out is None:
+        residual_out = torch.empty_like(x)
+    _need(residual_out, "residual_out", (M, K))
+    if norm not in NORMS:
+        raise ValueError(f"norm must be one of {list(NORMS)}")
+    if rstd_out is not None:
+        _need(rstd_out, "rstd_out", (M,), torch.float32)
+    if mean_out is not None:
+        _need(mean_out, "mean_out", (M,), torch.float32)
+    return M, K, residual_out
+
+
+def add_norm_qkv(h: Handle, x, residual, gamma, beta, W, Hq, Hkv, D, norm="rmsnorm", eps=1e-5, bias=None,
+                 residual_out=None, q=None, k=None, v=None, mean_out=None, rstd_out=None, stream=None):
+    """fnl_add_norm_qkv. Returns dict(residual_out, q [Hq,M,D], k, v, mean, rstd)."""
+    M, K, residual_out = _common(x, residual, gamma, beta, norm, residual_out, mean_out, rstd_out, W, bias)
+    q = torch.empty(Hq, M, D, dtype=torch.bfloat16, device=x.device) if q is None else q
+    k = torch.empty(Hkv, M, D, dtype=torch.bfloat16, device=x.device) if k is None else k
+    v = torch.empty(Hkv, M, D, dtype=torch.bfloat16, device=x.device) if v is None else v
+    _need(q, "q", (Hq, M, D)); _need(k, "k", (Hkv, M, D)); _need(v, "v", (Hkv, M, D))
+    st = lib().fnl_add_norm_qkv(h.ptr, _stream_ptr(stream), _p(x), _p(residual), _p(residual_out), _p(gamma),
+                                _p(beta), NORMS[norm], float(eps), _p(W), _p(bias), M, K, Hq, Hkv, D,
+                                _p(q), _p(k), _p(v), _p(mean_out), _p(rstd_out))
+    if st != FNL_OK:
+        h._raise(st, "fnl_add_norm_qkv")
+    return {"residual_out": residual_out, "q": q, "k": k, "v": v, "mean": mean_out, "rstd": rstd_out}
+
+
+def add_norm_swiglu(h: Handle, x, residual, gamma, beta, W, I, norm="rmsnorm", eps=1e-5, bias=None,
+                    residual_out=None, out=None, mean_out=None, rstd_out=None, stream=None):
+    """fnl_add_norm_swiglu. W is [2I, K] (gate rows then up rows). Returns dict."""
+    M, K, residual_out = _common(x, residual, gamma, beta, norm, residual_out, mean_out, rstd_out, W, bias)
+    out = torch.empty(M, I, dtype=torch.bfloat16, device=x.device) if out is None else out
+    _need(out, "out", (M, I))
+    st = lib().fnl_add_norm_swiglu(h.ptr, _stream_ptr(stream), _p(x), _p(residual), _p(residual_out),
+                                   _p(gamma), _p(beta), NORMS[norm], float(eps), _p(W), _p(bias), M, K, I,
+                                   _p(out), _p(mean_out), _p(rstd_out))
+    if st != FNL_OK:
+        h._raise(st, "fnl_add_norm_swiglu")
+    return {"residual_out": residual_out, "out": out, "mean": mean_out, "rstd": rstd_out}
+
+
+def add_bias_norm_gelu(h: Handle, x, residual, gamma, beta, W, bias_in=None, bias_out=None, norm="layernorm",
+                       eps=1e-5, residual_out=None, out=None, mean_out=None, rstd_out=None, stream=None):
+    """fnl_add_bias_norm_gelu. Returns dict(residual_out, out [M,N], mean, rstd)."""
+    M, K, residual_out = _common(x, residual, gamma, beta, norm, residual_out, mean_out, rstd_out, W,
+                                 bias_out)
+    _need(bias_in, "bias_in", (K,))
+    N = W.shape[0]
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
+    _need(out, "out", (M, N))
+    st = lib().fnl_add_bias_norm_gelu(h.ptr, _stream_ptr(stream), _p(x), _p(residual), _p(bias_in),
+                                      _p(residual_out), _p(gamma), _p(beta), NORMS[norm], float(eps), _p(W),
+                                      _p(bias_out), M, K, N, _p(out), _p(mean_out), _p(rstd_out))
+    if st != FNL_OK:
+        h._raise(st, "fnl_add_bias_norm_gelu")
+    return {"residual_out": residual_out, "out": out, "mean": mean_out, "rstd": rstd_out}
+
+
+def run_workload(h: Handle, w, dev: dict, stats: bool = True, stream=None) -> dict:
+    """Run a synthetic.Workload on device tensors `dev` (same keys as
+    synthetic.make_inputs). Allocates the outputs and statistics buffers."""
+    M = dev["x"].shape[0]
+    rstd = torch.empty(M, dtype=torch.float32, device=dev["x"].device) if stats else None
+    mean = (torch.empty(M, dtype=torch.float32, device=dev["x"].device)
+            if stats and w.norm == "layernorm" else None)
+    if w.op == "qkv":
+        return add_norm_qkv(h, dev["x"], dev["residual"], dev["gamma"], dev.get("beta"), dev["W"], w.Hq, w.Hkv,
+                            w.D, norm=w.norm, eps=w.eps, bias=dev.get("bias_out"), mean_out=mean,
+                            rstd_out=rstd, stream=stream)
+    if w.op == "swiglu":
+        return add_norm_swiglu(h, dev["x"], dev["residual"], dev["gamma"], dev.get("beta"), dev["W"], w.I,
+                               norm=w.norm, eps=w.eps, bias=dev.get("bias_out"), mean_out=mean, rstd_out=rstd,
+                               stream=stream)
+    return add_bias_norm_gelu(h, dev["x"], dev["residual"], dev["gamma"], dev.get("beta"), dev["W"],
+                              bias_in=dev.get("bias_in"), bias_out=dev.get("bias_out"), norm=w.norm, eps=w.eps,
+                              mean_out=mean, rstd_out=rstd, stream=stream)
