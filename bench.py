@@ -1,0 +1,444 @@
+"""Benchmark of the fused pre-norm linear layer (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fnl|reference]
+                    [--workload NAME] [--sweep]
+
+A step is one fused call (residual add -> norm -> projection -> epilogue) over
+one batch of seeded synthetic inputs of the chosen workload (default: the
+Llama-3-8B-shaped decode QKV, M=32, K=4096, N=6144, RMSNorm). Inputs are
+resident in HBM before timing; the calls of the timed region are replayed from
+a CUDA graph (the host cost of a Python call is larger than a decode kernel),
+rotating over enough copies of W / x / residual to exceed 3x the L2 size so
+that every step streams its weights from HBM. `value` is the algorithmic HBM
+traffic (or FLOP) rate of the whole job; `e2e` times the same calls through the
+Python binding with the inputs copied from pinned host memory and the outputs
+copied back inside the timed region. Multi-GPU runs are independent replicas
+(the op has no exchange step): value = all ranks' work / max rank time.
+
+--impl reference times the fp64 CPU oracle (the only reference this op has) on
+the same workload; --sweep prints one line per workload to stderr after the
+main line (the main line stays the only stdout line).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synthetic  # noqa: E402
+
+METRIC = json.load(open(os.path.join(ROOT, "BASELINE.json")))["metric"]
+DEFAULT_WORKLOAD = "c2_decode_rms_qkv"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+HBM_BOUND_AI = 250.0   # FLOP/byte below which a workload is HBM-bound on B200 (measured ridge)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "transformer_layer_residual_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """dram bytes per launch of the dominant kernel from the committed ncu
+    summary, only if it was taken on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(workload)
+    if not d or d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons every 50 ms in a background process."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu: int):
+        self.gpu = gpu
+        self.proc = None
+        self.lines = []
+        self.marks = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, name):
+        self.marks.append((name, time.time()))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        def parse(rows):
+            sm, mx, reasons = [], [], set()
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for _, l in rows:
+                f = [x.strip() for x in l.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm.append(float(f[1]))
+                    mx.append(float(f[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, f[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+            return sm, mx, reasons
+        inside = [r for r in self.lines if t0 <= r[0] <= t1]
+        sm, mx, reasons = parse(inside)
+        where = "timed region"
+        if len(sm) < 3:   # region shorter than a few samples: use the sustain loop that follows it
+            sm, mx, reasons = parse([r for r in self.lines if r[0] >= t0])
+            where = "timed region + same step loop sustained right after it"
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
+                "samples": len(sm), "sampled_over": where}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl" if torch.cuda.is_available() else "gloo",
+                                             timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def units(w):
+    """(metric unit, algorithmic units per step, bound) for workload w."""
+    ai = w.flops() / w.algorithmic_bytes()
+    if ai < HBM_BOUND_AI:
+        return "GB/s", w.algorithmic_bytes() / 1e9, "hbm"
+    return "TFLOP/s", w.flops() / 1e12, "tensor"
+
+
+# ------------------------------------------------------------------------- fnl arm
+def bench_fnl(w, steps, warmup, world, rank, local, sweep_line=False):
+    from transformer_layer_residual_b200 import fnl
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    inputs = synthetic.make_inputs(w, seed=0)
+    per_copy = sum(t.numel() * t.element_size() for k, t in inputs.items() if k in ("x", "residual", "W"))
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = max(1, min(16, -(-3 * l2 // per_copy)))
+    copies = []
+    for i in range(R):
+        c = {k: v.to(dev) for k, v in inputs.items()}
+        copies.append(c)
+    M = w.M
+    h = fnl.Handle(local, max_tokens=M, max_n=w.N)
+    outs = []
+    for c in copies:   # pre-allocate outputs per copy so the graph holds fixed pointers
+        o = fnl.run_workload(h, w, c, stats=True)
+        outs.append(o)
+    h.check()
+
+    def call(i):
+        c, o = copies[i], outs[i]
+        if w.op == "qkv":
+            fnl.add_norm_qkv(h, c["x"], c["residual"], c["gamma"], c.get("beta"), c["W"], w.Hq, w.Hkv, w.D,
+                             norm=w.norm, eps=w.eps, bias=c.get("bias_out"), residual_out=o["residual_out"],
+                             q=o["q"], k=o["k"], v=o["v"], mean_out=o["mean"], rstd_out=o["rstd"])
+        elif w.op == "swiglu":
+            fnl.add_norm_swiglu(h, c["x"], c["residual"], c["gamma"], c.get("beta"), c["W"], w.I, norm=w.norm,
+                                eps=w.eps, bias=c.get("bias_out"), residual_out=o["residual_out"], out=o["out"],
+                                mean_out=o["mean"], rstd_out=o["rstd"])
+        else:
+            fnl.add_bias_norm_gelu(h, c["x"], c["residual"], c["gamma"], c.get("beta"), c["W"],
+                                   bias_in=c.get("bias_in"), bias_out=c.get("bias_out"), norm=w.norm, eps=w.eps,
+                                   residual_out=o["residual_out"], out=o["out"], mean_out=o["mean"],
+                                   rstd_out=o["rstd"])
+
+    stream = torch.cuda.Stream(dev)
+    # graphs: one of R calls (copy 0..R-1), one of the remainder
+    def capture(n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            for i in range(n):   # eager pass on the capture stream first
+                call(i % R)
+        stream.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                call(i % R)
+        return g
+    g_full = capture(R)
+    rem = steps % R
+    g_rem = capture(rem) if rem else None
+    n_full = steps // R
+
+    def run_steps():
+        for _ in range(n_full):
+            g_full.replay()
+        if g_rem is not None:
+            g_rem.replay()
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, -(-warmup // R))):
+            g_full.replay()
+    stream.synchronize()
+    h.check()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        run_steps()
+        ev1.record(stream)
+    ev1.synchronize()
+    t_wall1 = time.time()
+    barrier(world)
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    # keep the same loop running ~1.5 s for the clock record if the timed region was short
+    if t_wall1 - t_wall0 < 1.0:
+        t_end = time.time() + 1.5
+        with torch.cuda.stream(stream):
+            while time.time() < t_end:
+                run_steps()
+                stream.synchronize()
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+    h.check()
+    ms_max = max_over_ranks(ms, world)
+
+    unit, per_step, bound = units(w)
+    value = per_step * steps * world / (ms_max / 1e3)
+    launches_per_step = 2 if w.norm == "layernorm" else 1
+
+    # e2e: through the public binding, host buffers, copies inside the timed region
+    x_h = inputs["x"].pin_memory()
+    r_h = inputs["residual"].pin_memory()
+    c0, o0 = copies[0], outs[0]
+    out_keys = ("q", "k", "v") if w.op == "qkv" else ("out",)
+    host_out = {k: torch.empty(o0[k].shape, dtype=o0[k].dtype, pin_memory=True) for k in out_keys}
+    host_res = torch.empty(o0["residual_out"].shape, dtype=torch.bfloat16, pin_memory=True)
+    e2e_steps = max(3, min(steps, 200))
+    with torch.cuda.stream(stream):
+        for i in range(e2e_steps + 3):
+            if i == 3:
+                torch.cuda.synchronize()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            c0["x"].copy_(x_h, non_blocking=True)
+            c0["residual"].copy_(r_h, non_blocking=True)
+            call(0)
+            for k in out_keys:
+                host_out[k].copy_(o0[k], non_blocking=True)
+            host_res.copy_(o0["residual_out"], non_blocking=True)
+        e1.record(stream)
+    e1.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    h2d = x_h.numel() * 2 + r_h.numel() * 2
+    d2h = sum(t.numel() * 2 for t in host_out.values()) + host_res.numel() * 2
+    e2e_value = per_step * e2e_steps * world / (e2e_ms / 1e3)
+
+    pk, pk_src = peaks()
+    per_launch_ms = ms / steps
+    if bound == "hbm":
+        achieved = w.algorithmic_bytes() / (per_launch_ms / 1e3) / 1e9
+        peak = pk["hbm_gbs"]
+        runit = "GB/s"
+    else:
+        achieved = w.flops() / (per_launch_ms / 1e3) / 1e12
+        peak = pk["bf16_tflops"]
+        runit = "TFLOP/s"
+    line = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": unit,
+        "n_gpus": world,
+        "steps": steps,
+        "warmup": warmup,
+        "ms_per_step": round(ms_max / steps, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded normal draws rounded to bf16; random-init weights)",
+        "config": {"workload": w.name, "op": w.op, "norm": w.norm, "M": w.M, "K": w.K, "N": w.N,
+                   **({"Hq": w.Hq, "Hkv": w.Hkv, "D": w.D} if w.op == "qkv" else {}),
+                   **({"I": w.I} if w.op == "swiglu" else {}),
+                   "l2": f"inputs larger than L2: {R} rotating copies of W/x/residual "
+                         f"({R * per_copy / 1e6:.0f} MB vs L2 {l2 / 1e6:.0f} MB)",
+                   "timing": f"CUDA graph replays of {R} calls, CUDA events on the launch stream",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "tflops": round(w.flops() * steps * world / (ms_max / 1e3) / 1e12, 3),
+        "gbps": round(w.algorithmic_bytes() * steps * world / (ms_max / 1e3) / 1e9, 3),
+        "tokens_per_s_layer": round(w.M * steps * world / (ms_max / 1e3), 1),
+        "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": runit,
+                     "frac": round(achieved / peak, 4), "peak_source": f"{pk_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops burst'})",
+                     "traffic": recorded_traffic(w.name),
+                     "algorithmic_per_launch": w.algorithmic_bytes() if bound == "hbm" else w.flops(),
+                     "kernel": "fused GEMM kernel" + (" + LayerNorm stats kernel (PDL)" if w.norm == "layernorm" else "")},
+        "e2e": {"value": round(e2e_value, 3), "unit": unit, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": launches_per_step * steps,
+        "clocks": clocks,
+    }
+    h.close()
+    return line
+
+
+# ------------------------------------------------------------------------- oracle
+def oracle_rate(w, budget_s=10.0, max_steps=None, rows=None):
+    """Time the fp64 oracle (as it stands) on a bounded row sample of w.
+    Returns (units per second in the workload's unit, sample description, cores,
+    passes, seconds). Work is counted as proportional to rows (the oracle's cost
+    is the M x N x K product)."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    cores = len(os.sched_getaffinity(0))
+    rows = min(w.M, 256) if rows is None else rows
+    inputs = synthetic.make_inputs(w, rows=rows)
+    ws = synthetic.Workload(**{**w.__dict__, "M": rows, "seq_lens": None})
+    unit, per_step, _ = units(w)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.run(ws, inputs)
+        n += 1
+        el = time.perf_counter() - t0
+        if (n >= max_steps) if max_steps else (el >= budget_s):
+            break
+    # units scale linearly with rows (the op is row-wise; W traffic scales per pass)
+    frac = rows / w.M
+    rate = per_step * frac * n / el
+    sample = (f"{rows} of {w.M} rows x all N per pass, {n} passes in {el:.1f} s, scaled by M/{rows}"
+              if rows < w.M else f"full workload, {n} passes in {el:.1f} s")
+    return rate, sample, min(cores, threads), n, el
+
+
+def bench_reference(w, steps, warmup, world, rank, budget_s=120.0):
+    """The oracle as it stands, timed for exactly `steps` passes after `warmup`
+    untimed ones; each pass covers as many rows as keeps the whole run within
+    about `budget_s` seconds."""
+    if rank != 0:
+        return None
+    unit, per_step, _ = units(w)
+    _, _, _, _, t1 = oracle_rate(w, budget_s=0.0, max_steps=1)          # one pass of up to 256 rows
+    rows0 = min(w.M, 256)
+    rows = max(1, min(rows0, int(rows0 * budget_s / (max(1, steps + warmup) * max(t1, 1e-6)))))
+    for _ in range(max(0, warmup)):
+        oracle_rate(w, budget_s=0.0, max_steps=1, rows=rows)
+    rate, sample, cores, n, el = oracle_rate(w, budget_s=0.0, max_steps=max(1, steps), rows=rows)
+    return {
+        "metric": METRIC, "value": round(rate, 6), "unit": unit, "n_gpus": world, "steps": n, "warmup": warmup,
+        "ms_per_step": round(el / n * 1e3, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": w.name, "op": w.op, "norm": w.norm, "M": w.M, "K": w.K, "N": w.N},
+        "cpu_baseline": {"value": round(rate, 6), "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(rate, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="fnl", choices=["fnl", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--sweep", action="store_true", help="also bench every workload (lines to stderr)")
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
+    a = ap.parse_args()
+    if a.warmup < 3:
+        a.warmup = 3
+    world, rank, local = dist_setup(a.gpus)
+    w = synthetic.workloads()[a.workload]
+
+    if a.impl == "reference":
+        line = bench_reference(w, a.steps, a.warmup, world, rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    line = bench_fnl(w, a.steps, a.warmup, world, rank, local)
+    if rank == 0 and world == 1:
+        rate, sample, cores, _, _ = oracle_rate(w, budget_s=a.cpu_budget)
+        line["cpu_baseline"] = {"value": round(rate, 6), "unit": line["unit"], "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if a.sweep:
+        for name, ws in synthetic.workloads().items():
+            if name == a.workload:
+                continue
+            st = max(3, min(a.steps, int(2e4 / max(1.0, ws.flops() / 2e11))))
+            l2 = bench_fnl(ws, st, 3, world, rank, local)
+            if rank == 0:
+                print(json.dumps(l2), file=sys.stderr, flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

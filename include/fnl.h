@@ -35,7 +35,8 @@
  *   LayerNorm  mean = sum(h)/K, var = sum((h-mean)^2)/K, rstd = 1/sqrt(var+eps),
  *              a = (h - mean) * rstd * gamma + beta
  *   RMSNorm    rstd = 1/sqrt(sum(h^2)/K + eps), a = h * rstd * gamma
- * a is rounded to bf16 for the tensor cores; y = a W^T accumulates in fp32.
+ * a is rounded to bf16 for the tensor cores (see fnl_precision); y = a W^T
+ * accumulates in fp32.
  * mean_out / rstd_out (fp32 [M], nullable) receive the statistics; mean_out
  * must be NULL for RMSNorm.
  *
@@ -87,11 +88,24 @@ typedef enum {
   FNL_PATH_SPLITK = 2         /* force the small-M split-K kernel (requires M <= 128) */
 } fnl_path;
 
+/* How the normalised activation a is rounded for the bf16 tensor cores.
+ * A single bf16 rounding of a perturbs each output by ~2^-9 |a| |W_n|; SwiGLU
+ * multiplies that error by SiLU(gate) (up to ~5x at |gate| ~ 5), which exceeds
+ * 1e-2 + 1e-2 |out| on Llama-sized MLPs. SPLIT writes a = hi + lo (both bf16)
+ * and accumulates hi W^T + lo W^T in the same fp32 accumulator (twice the
+ * tensor-core work, no extra memory traffic). */
+typedef enum {
+  FNL_PRECISION_DEFAULT = 0,  /* SPLIT for SwiGLU, SINGLE for QKV and GELU */
+  FNL_PRECISION_SPLIT = 1,    /* hi + lo operand for every epilogue */
+  FNL_PRECISION_SINGLE = 2    /* one bf16 rounding for every epilogue */
+} fnl_precision;
+
 typedef struct {
   int max_tokens;   /* reserve workspace for M up to this (0: grow on demand) */
   int max_n;        /* reserve workspace for N up to this (0: grow on demand) */
   int path;         /* fnl_path */
   int max_ctas;     /* cap on persistent CTAs (0: one per SM) -- for tests */
+  int precision;    /* fnl_precision */
 } fnl_options;
 
 /* Create a handle on `device` (cudaSetDevice is called). opt may be NULL. */

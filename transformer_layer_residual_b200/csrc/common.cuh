@@ -33,11 +33,24 @@ struct OpParams {
   int max_seg;
   int mpad;
   int stages;
+  int split;             // 1: operand = bf16 hi + bf16 lo (two UMMAs), 0: single bf16 rounding
   int* status;           // device status word (bounded-wait failures)
 };
 
 __device__ __forceinline__ uint4 ldg16(const void* p) {
   return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// Round a[8] to bf16 (hi) and, if `split`, also the remainder a - hi to bf16 (lo).
+__device__ __forceinline__ void round_split8(const float (&a)[8], bool split, uint4& hi, uint4& lo) {
+  hi = pack8(a);
+  if (split) {
+    float h[8], r[8];
+    unpack8(hi, h);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) r[e] = a[e] - h[e];
+    lo = pack8(r);
+  }
 }
 
 __device__ __forceinline__ void load8_or_zero(const bf16* base, int k0, bool ok, float (&f)[8]) {

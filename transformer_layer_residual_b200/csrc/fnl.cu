@@ -325,6 +325,8 @@ fnl_status run(fnl_handle* h, const Call& c) {
   p.q = c.q; p.k = c.k; p.v = c.v; p.out = c.out;
   p.part = part; p.part_ss = part_ss; p.counters = counters; p.max_seg = max_seg; p.mpad = mpad;
   p.stages = stages; p.status = status;
+  p.split = h->opt.precision == FNL_PRECISION_SPLIT ||
+            (h->opt.precision == FNL_PRECISION_DEFAULT && c.op == Op::SwiGLU);
 
   // tensor maps: x and residual tiles are [rows x 64], W tiles [rows x 64]
   CUtensorMap mx, mr, mw;
@@ -362,7 +364,8 @@ fnl_status fnl_create(fnl_handle** out, int device, const fnl_options* opt) {
   *out = nullptr;
   fnl_handle* h = new fnl_handle();
   if (opt) h->opt = *opt;
-  if (h->opt.path < FNL_PATH_AUTO || h->opt.path > FNL_PATH_SPLITK || h->opt.max_tokens < 0 || h->opt.max_n < 0) {
+  if (h->opt.path < FNL_PATH_AUTO || h->opt.path > FNL_PATH_SPLITK || h->opt.max_tokens < 0 || h->opt.max_n < 0 ||
+      h->opt.precision < FNL_PRECISION_DEFAULT || h->opt.precision > FNL_PRECISION_SINGLE) {
     delete h;
     return FNL_ERR_INVALID_ARG;
   }

@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
   const int num_n = (EPI == kEpiSwiGLU) ? (p.I + 127) / 128 : (p.N + BN - 1) / BN;
   const int tiles = num_m * num_n;
   const int nkb = (K + BK - 1) / BK;
+  const bool split = p.split != 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -177,6 +178,11 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
             umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+          if (split) {   // + lo(a) W^T into the same accumulator
+            const uint64_t ld = sw128_desc(xa + X_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) umma_bf16(d, ld + 2 * kk, bd + 2 * kk, idesc, 1u);
+          }
           umma_commit(&ctrl->empty[s]);
           if (++s == STAGES) {
             s = 0;
@@ -321,7 +327,10 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
               ss[j] = fmaf(h[e], h[e], ss[j]);
             }
           }
-          st_shared_v4(xs + off, pack8(a));
+          uint4 hi, lo;
+          round_split8(a, split, hi, lo);
+          st_shared_v4(xs + off, hi);
+          if (split) st_shared_v4(rsm + off, lo);   // residual chunk already consumed by this thread
           if (write_res) {
             const int gm = mb * BM + row;
             if (gm < M && kin)

@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
   const int T = (EPI == kEpiSwiGLU) ? (p.I + 63) / 64 : (p.N + BW - 1) / BW;
   const int nkb = (K + BK - 1) / BK;
   const uint32_t ncols = tmem_cols(mpad);
+  const bool split = p.split != 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -203,6 +204,11 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
             umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+          if (split) {
+            const uint64_t ld = sw128_desc(wa + W_BYTES + XB);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) umma_bf16(d, ad + 2 * kk, ld + 2 * kk, idesc, 1u);
+          }
           umma_commit(&ctrl->empty[s]);
           if (++s == static_cast<uint32_t>(S)) {
             s = 0;
@@ -375,7 +381,10 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
                 ss[j] = fmaf(h[e], h[e], ss[j]);
               }
             }
-            st_shared_v4(xs + off, pack8(a));
+            uint4 hi, lo;
+            round_split8(a, split, hi, lo);
+            st_shared_v4(xs + off, hi);
+            if (split) st_shared_v4(rsm + off, lo);
             if (write_res && row < M && kin)
               *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(row) * K + k0) = pack8(h);
           }

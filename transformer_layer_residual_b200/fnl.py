@@ -22,6 +22,7 @@ STATUS_NAMES = {0: "FNL_OK", 1: "FNL_ERR_INVALID_ARG", 2: "FNL_ERR_ALIGNMENT", 3
                 4: "FNL_ERR_UNSUPPORTED", 5: "FNL_ERR_CUDA", 6: "FNL_ERR_DEVICE_STATUS"}
 NORMS = {"layernorm": 0, "rmsnorm": 1}
 PATHS = {"auto": 0, "tile": 1, "splitk": 2}
+PRECISIONS = {"default": 0, "split": 1, "single": 2}
 
 EXPORTED = ("fnl_create", "fnl_destroy", "fnl_status_string", "fnl_last_error", "fnl_check",
             "fnl_add_norm_qkv", "fnl_add_norm_swiglu", "fnl_add_bias_norm_gelu")
@@ -35,7 +36,7 @@ class FnlError(RuntimeError):
 
 class _Options(ctypes.Structure):
     _fields_ = [("max_tokens", ctypes.c_int), ("max_n", ctypes.c_int), ("path", ctypes.c_int),
-                ("max_ctas", ctypes.c_int)]
+                ("max_ctas", ctypes.c_int), ("precision", ctypes.c_int)]
 
 
 def lib_path() -> str:
@@ -73,10 +74,10 @@ class Handle:
     """Owns an fnl_handle (device workspace). One stream / thread at a time."""
 
     def __init__(self, device: int = 0, max_tokens: int = 0, max_n: int = 0, path: str = "auto",
-                 max_ctas: int = 0):
+                 max_ctas: int = 0, precision: str = "default"):
         L = lib()
         self._h = ctypes.c_void_p()
-        opt = _Options(max_tokens, max_n, PATHS[path], max_ctas)
+        opt = _Options(max_tokens, max_n, PATHS[path], max_ctas, PRECISIONS[precision])
         st = L.fnl_create(ctypes.byref(self._h), device, ctypes.byref(opt))
         if st != FNL_OK:
             raise FnlError(st, f"fnl_create(device={device}) failed")
