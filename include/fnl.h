@@ -160,6 +160,38 @@ fnl_status fnl_add_bias_norm_gelu(fnl_handle* h, fnl_stream stream,
                                   int M, int K, int N,
                                   fnl_bf16* out, float* mean_out, float* rstd_out);
 
+/* Allocation-free variant of fnl_add_norm_qkv for decode-sized batches.
+ * The pages have no counterpart to this entry point: it exists for callers
+ * that may not allocate device memory on the call path -- work recorded into
+ * a CUDA graph (cudaMalloc cannot be captured), latency-critical decode loops
+ * that must never hit cudaMalloc/cudaFree's implicit device synchronisation,
+ * and plugins inside an inference engine that owns all device memory through
+ * its own static memory plan. fnl_create allocates a workspace, so this entry
+ * point takes no handle; it computes exactly what fnl_add_norm_qkv computes
+ * (same arguments, same meaning, same layouts) on the calling thread's current
+ * device, with the small-M split-K kernel.
+ * Scratch: a file-scope device array of 16 MiB inside the library, held by
+ * every GPU that loads it until the process exits. Calls allocate nothing and
+ * share that array: it keeps the last call's contents, and the call clears the
+ * parts that must start at zero (status word, arrival counters) on `stream`
+ * first. Calls that overlap on one GPU (several streams or host threads at
+ * once) race on the array and must be serialised by the caller.
+ * Limits: M <= 128 (FNL_ERR_UNSUPPORTED otherwise), and the split-K partial
+ * sums must fit the array (about T * segments * roundup16(M) * 516 bytes with
+ * T = ceil(N/128); e.g. N = 10240, M = 128 fits, N = 65536, M = 128 does not:
+ * FNL_ERR_UNSUPPORTED). Other errors as for fnl_add_norm_qkv (status code only:
+ * there is no handle to hold the text or the device status word).
+ * The first call on each device resolves the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture. */
+fnl_status fnl_add_norm_qkv_static(fnl_stream stream,
+                                   const fnl_bf16* x, const fnl_bf16* residual, fnl_bf16* residual_out,
+                                   const fnl_bf16* gamma, const fnl_bf16* beta, fnl_norm norm, float eps,
+                                   const fnl_bf16* W, const fnl_bf16* bias,
+                                   int M, int K, int Hq, int Hkv, int D,
+                                   fnl_bf16* q, fnl_bf16* k, fnl_bf16* v,
+                                   float* mean_out, float* rstd_out);
+
 #ifdef __cplusplus
 }
 #endif

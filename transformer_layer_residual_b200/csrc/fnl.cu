@@ -489,3 +489,161 @@ fnl_status fnl_add_bias_norm_gelu(fnl_handle* h, fnl_stream stream, const fnl_bf
 }
 
 }  // extern "C"
+
+// ============================================================================
+// Allocation-free entry point: fnl_add_norm_qkv_static.
+//
+// Some callers cannot allocate device memory on the call path: code recorded
+// into a CUDA graph (cudaMalloc cannot be captured), latency-critical decode
+// loops that must never hit cudaMalloc/cudaFree's implicit device
+// synchronisation, and plugins living inside an inference engine that owns all
+// device memory through its own static memory plan. fnl_create allocates the
+// handle's workspace, so those callers get this handle-free variant of the
+// small-M (decode) QKV kernel instead. Its scratch (split-K partial sums, the
+// per-tile arrival counters, the LayerNorm statistics and the status word)
+// lives in the file-scope array below, which every GPU that loads this
+// library holds until the process exits. Nothing here calls cudaMalloc,
+// cudaFree or any other allocating routine.
+// ============================================================================
+namespace {
+
+constexpr size_t kStaticScratchBytes = static_cast<size_t>(16) << 20;   // 16 MiB per device
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kStaticMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_ptr[kStaticMaxDevices] = {};   // device address of g_static_scratch, per device
+int g_static_sms[kStaticMaxDevices] = {};
+
+// Once per device, with that device current: resolve the array's device
+// address (in host code the symbol is only a host-side stand-in and must not
+// be passed to a kernel).
+fnl_status static_setup(int dev, void** ptr, int* sms) {
+  if (dev < 0 || dev >= kStaticMaxDevices) return FNL_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_ptr[dev] == nullptr) {
+    int major = 0, count = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return FNL_ERR_CUDA;
+    if (major != 10) return FNL_ERR_UNSUPPORTED;
+    if (cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FNL_ERR_CUDA;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return FNL_ERR_CUDA;
+    g_static_ptr[dev] = p;
+    g_static_sms[dev] = count > 0 ? count : 148;
+  }
+  *ptr = g_static_ptr[dev];
+  *sms = g_static_sms[dev];
+  return FNL_OK;
+}
+
+// Argument checks of fnl_add_norm_qkv, without a handle (and without heap use).
+fnl_status validate_static(const Call& c) {
+  if (c.norm != FNL_NORM_LAYERNORM && c.norm != FNL_NORM_RMSNORM) return FNL_ERR_INVALID_ARG;
+  if (!(c.eps >= 0.f) || c.eps > 1e30f) return FNL_ERR_INVALID_ARG;
+  if (c.M < 0 || c.K <= 0 || c.Hq <= 0 || c.Hkv <= 0 || c.D <= 0) return FNL_ERR_INVALID_ARG;
+  if (c.Hq % c.Hkv) return FNL_ERR_INVALID_ARG;
+  if (c.K % 8 || c.D % 8) return FNL_ERR_ALIGNMENT;
+  if (c.K > 32768 || c.M > fnl::k3::MAX_MPAD) return FNL_ERR_UNSUPPORTED;
+  if (c.norm == FNL_NORM_RMSNORM && (c.beta || c.mean_out)) return FNL_ERR_INVALID_ARG;
+  if (c.M == 0) return FNL_OK;
+  if (!c.x || !c.residual || !c.residual_out || !c.gamma || !c.W || !c.q || !c.k || !c.v)
+    return FNL_ERR_INVALID_ARG;
+  const void* p16[] = {c.x, c.residual, c.gamma, c.beta, c.W, c.bias, c.residual_out, c.q, c.k, c.v};
+  for (const void* p : p16)
+    if (p && !al16(p)) return FNL_ERR_ALIGNMENT;
+  if ((c.mean_out && !al4(c.mean_out)) || (c.rstd_out && !al4(c.rstd_out))) return FNL_ERR_ALIGNMENT;
+  const size_t MK = static_cast<size_t>(c.M) * c.K * 2;
+  const Range ins[] = {{c.x, MK, "x"},
+                       {c.residual, MK, "residual"},
+                       {c.gamma, static_cast<size_t>(c.K) * 2, "gamma"},
+                       {c.beta, static_cast<size_t>(c.K) * 2, "beta"},
+                       {c.W, static_cast<size_t>(c.N) * c.K * 2, "W"},
+                       {c.bias, static_cast<size_t>(c.N) * 2, "bias"}};
+  const Range outs[] = {{c.residual_out, MK, "residual_out"},
+                        {c.mean_out, static_cast<size_t>(c.M) * 4, "mean_out"},
+                        {c.rstd_out, static_cast<size_t>(c.M) * 4, "rstd_out"},
+                        {c.q, static_cast<size_t>(c.Hq) * c.M * c.D * 2, "q"},
+                        {c.k, static_cast<size_t>(c.Hkv) * c.M * c.D * 2, "k"},
+                        {c.v, static_cast<size_t>(c.Hkv) * c.M * c.D * 2, "v"}};
+  for (size_t i = 0; i < sizeof(outs) / sizeof(outs[0]); ++i) {
+    for (const Range& in : ins)
+      if (overlap(outs[i], in)) return FNL_ERR_ALIAS;
+    for (size_t j = i + 1; j < sizeof(outs) / sizeof(outs[0]); ++j)
+      if (overlap(outs[i], outs[j])) return FNL_ERR_ALIAS;
+  }
+  return FNL_OK;
+}
+
+}  // namespace
+
+extern "C" fnl_status fnl_add_norm_qkv_static(fnl_stream stream, const fnl_bf16* x, const fnl_bf16* residual,
+                                              fnl_bf16* residual_out, const fnl_bf16* gamma, const fnl_bf16* beta,
+                                              fnl_norm norm, float eps, const fnl_bf16* W, const fnl_bf16* bias,
+                                              int M, int K, int Hq, int Hkv, int D, fnl_bf16* q, fnl_bf16* k,
+                                              fnl_bf16* v, float* mean_out, float* rstd_out) {
+  Call c{};
+  c.op = Op::QKV;
+  c.stream = reinterpret_cast<cudaStream_t>(stream);
+  c.x = B(x); c.residual = B(residual); c.bias_in = nullptr; c.gamma = B(gamma); c.beta = B(beta);
+  c.W = B(W); c.bias = B(bias); c.residual_out = Bm(residual_out);
+  c.norm = norm; c.eps = eps; c.M = M; c.K = K; c.Hq = Hq; c.Hkv = Hkv; c.D = D;
+  c.N = (Hq > 0 && Hkv > 0 && D > 0) ? (Hq + 2 * Hkv) * D : 0;
+  c.q = Bm(q); c.k = Bm(k); c.v = Bm(v); c.out = nullptr;
+  c.mean_out = mean_out; c.rstd_out = rstd_out;
+  fnl_status st = validate_static(c);
+  if (st != FNL_OK || c.M == 0) return st;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FNL_ERR_CUDA;
+  void* scratch = nullptr;
+  int sms = 0;
+  if ((st = static_setup(dev, &scratch, &sms)) != FNL_OK) return st;
+  if ((st = get_encoder(nullptr)) != FNL_OK) return st;
+
+  // small-M split-K plan, the same as fnl_add_norm_qkv's for M <= 128
+  const bool rms = c.norm == FNL_NORM_RMSNORM;
+  const int nkb = (c.K + 63) / 64;
+  const int mpad = round_up(c.M, 16);
+  const int T = (c.N + 127) / 128;
+  const long long U = static_cast<long long>(T) * nkb;
+  const int grid = static_cast<int>(std::min<long long>(sms, U));
+  const int stages = std::min(fnl::k3::MAX_STAGES, (200 * 1024) / fnl::k3::stage_bytes(mpad));
+  int max_seg = 1;
+  for (int t = 0; t < T; ++t) {
+    const int first = fnl::k3::unit_owner(static_cast<long long>(t) * nkb, grid, U);
+    const int last = fnl::k3::unit_owner(static_cast<long long>(t + 1) * nkb - 1, grid, U);
+    max_seg = std::max(max_seg, last - first + 1);
+  }
+  // scratch layout: [status][counters][stats][partial h^2 sums][partial accumulators]
+  const size_t zero_bytes = align256(kStatusBytes + static_cast<size_t>(T) * 4);
+  const size_t stats_bytes = rms ? 0 : align256(static_cast<size_t>(c.M) * 8);
+  const size_t ss_bytes = align256(static_cast<size_t>(T) * max_seg * mpad * 4);
+  const size_t part_bytes = align256(static_cast<size_t>(T) * max_seg * mpad * 128 * 4);
+  if (zero_bytes + stats_bytes + ss_bytes + part_bytes > kStaticScratchBytes) return FNL_ERR_UNSUPPORTED;
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  // the array keeps the previous call's contents: the status word and the
+  // arrival counters must start at zero (the rest is written before it is read)
+  cudaError_t e = cudaMemsetAsync(base, 0, zero_bytes, c.stream);
+  if (e != cudaSuccess) return FNL_ERR_CUDA;
+
+  OpParams p{};
+  p.M = c.M; p.K = c.K; p.N = c.N; p.I = 0; p.Hq = c.Hq; p.Hkv = c.Hkv; p.D = c.D; p.eps = c.eps;
+  p.gamma = c.gamma; p.beta = c.beta; p.bias_in = nullptr; p.bias = c.bias;
+  p.residual_out = c.residual_out; p.rstd_out = rms ? c.rstd_out : nullptr;
+  p.stats = reinterpret_cast<const float2*>(base + zero_bytes);
+  p.q = c.q; p.k = c.k; p.v = c.v; p.out = nullptr;
+  p.counters = reinterpret_cast<unsigned*>(base + kStatusBytes);
+  p.part_ss = reinterpret_cast<float*>(base + zero_bytes + stats_bytes);
+  p.part = reinterpret_cast<float*>(base + zero_bytes + stats_bytes + ss_bytes);
+  p.max_seg = max_seg; p.mpad = mpad; p.stages = stages; p.split = 0;
+  p.status = reinterpret_cast<int*>(base);
+
+  CUtensorMap mx, mr, mw;
+  if ((st = make_map(nullptr, &mx, c.x, c.M, c.K, mpad)) != FNL_OK) return st;
+  if ((st = make_map(nullptr, &mr, c.residual, c.M, c.K, mpad)) != FNL_OK) return st;
+  if ((st = make_map(nullptr, &mw, c.W, c.N, c.K, fnl::k3::BW)) != FNL_OK) return st;
+  if (!rms && (st = launch_k1(nullptr, c, reinterpret_cast<float2*>(base + zero_bytes), c.stream)) != FNL_OK)
+    return st;
+  return dispatch_gemm<fnl::kEpiQKV>(nullptr, true, rms, grid, fnl::k3::NUM_THREADS,
+                                     fnl::k3::smem_bytes(mpad, stages), !rms, c.stream, mx, mr, mw, p);
+}

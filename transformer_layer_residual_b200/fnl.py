@@ -25,7 +25,7 @@ PATHS = {"auto": 0, "tile": 1, "splitk": 2}
 PRECISIONS = {"default": 0, "split": 1, "single": 2}
 
 EXPORTED = ("fnl_create", "fnl_destroy", "fnl_status_string", "fnl_last_error", "fnl_check",
-            "fnl_add_norm_qkv", "fnl_add_norm_swiglu", "fnl_add_bias_norm_gelu")
+            "fnl_add_norm_qkv", "fnl_add_norm_swiglu", "fnl_add_bias_norm_gelu", "fnl_add_norm_qkv_static")
 
 
 class FnlError(RuntimeError):
@@ -63,6 +63,7 @@ def lib() -> ctypes.CDLL:
     L.fnl_add_norm_qkv.argtypes = [P, P, P, P, P, P, P, I, F, P, P, I, I, I, I, I, P, P, P, P, P]
     L.fnl_add_norm_swiglu.argtypes = [P, P, P, P, P, P, P, I, F, P, P, I, I, I, P, P, P]
     L.fnl_add_bias_norm_gelu.argtypes = [P, P, P, P, P, P, P, P, I, F, P, P, I, I, I, P, P, P]
+    L.fnl_add_norm_qkv_static.argtypes = [P, P, P, P, P, P, I, F, P, P, I, I, I, I, I, P, P, P, P, P]
     for name in EXPORTED:
         if getattr(L, name).restype is None and name not in ("fnl_status_string", "fnl_last_error"):
             getattr(L, name).restype = I
@@ -221,3 +222,22 @@ def run_workload(h: Handle, w, dev: dict, stats: bool = True, stream=None) -> di
     return add_bias_norm_gelu(h, dev["x"], dev["residual"], dev["gamma"], dev.get("beta"), dev["W"],
                               bias_in=dev.get("bias_in"), bias_out=dev.get("bias_out"), norm=w.norm, eps=w.eps,
                               mean_out=mean, rstd_out=rstd, stream=stream)
+
+
+def add_norm_qkv_static(x, residual, gamma, beta, W, Hq, Hkv, D, norm="rmsnorm", eps=1e-5, bias=None,
+                        residual_out=None, q=None, k=None, v=None, mean_out=None, rstd_out=None, stream=None):
+    """fnl_add_norm_qkv_static: fnl_add_norm_qkv without a handle and without
+    any device allocation inside the library (its scratch is a static device
+    array of the library; M <= 128). Output tensors not given are allocated
+    here by torch, before the call. Returns the same dict as add_norm_qkv."""
+    M, K, residual_out = _common(x, residual, gamma, beta, norm, residual_out, mean_out, rstd_out, W, bias)
+    q = torch.empty(Hq, M, D, dtype=torch.bfloat16, device=x.device) if q is None else q
+    k = torch.empty(Hkv, M, D, dtype=torch.bfloat16, device=x.device) if k is None else k
+    v = torch.empty(Hkv, M, D, dtype=torch.bfloat16, device=x.device) if v is None else v
+    _need(q, "q", (Hq, M, D)); _need(k, "k", (Hkv, M, D)); _need(v, "v", (Hkv, M, D))
+    st = lib().fnl_add_norm_qkv_static(_stream_ptr(stream), _p(x), _p(residual), _p(residual_out), _p(gamma),
+                                       _p(beta), NORMS[norm], float(eps), _p(W), _p(bias), M, K, Hq, Hkv, D,
+                                       _p(q), _p(k), _p(v), _p(mean_out), _p(rstd_out))
+    if st != FNL_OK:
+        raise FnlError(st, "fnl_add_norm_qkv_static")
+    return {"residual_out": residual_out, "q": q, "k": k, "v": v, "mean": mean_out, "rstd": rstd_out}
