@@ -53,6 +53,47 @@ __device__ __forceinline__ void round_split8(const float (&a)[8], bool split, ui
   }
 }
 
+// Per-stage copies of the k-block's slices of gamma, beta and bias_in
+// (64 bf16 each), brought in by the producer with the stage's tiles.
+constexpr int kVecElems = 64;
+constexpr int kVecStageBytes = 3 * kVecElems * 2;   // 384
+
+// Bytes of the k-block's vector slices; the producer adds them to the stage's
+// expected transaction count.
+__device__ __forceinline__ uint32_t issue_vec_loads(const OpParams& p, bool has_beta, bool has_bias_in, int kb,
+                                                    bf16* vec, uint64_t* bar) {
+  const int k0 = kb * kVecElems;
+  const int kvalid = min(kVecElems, p.K - k0);
+  const uint32_t vb = static_cast<uint32_t>(kvalid) * 2;
+  bulk_load(vec, p.gamma + k0, vb, bar);
+  uint32_t n = vb;
+  if (has_beta) {
+    bulk_load(vec + kVecElems, p.beta + k0, vb, bar);
+    n += vb;
+  }
+  if (has_bias_in) {
+    bulk_load(vec + 2 * kVecElems, p.bias_in + k0, vb, bar);
+    n += vb;
+  }
+  return n;
+}
+
+__device__ __forceinline__ uint32_t vec_bytes(const OpParams& p, bool has_beta, bool has_bias_in, int kb) {
+  const int kvalid = min(kVecElems, p.K - kb * kVecElems);
+  return static_cast<uint32_t>(kvalid) * 2 * (1 + (has_beta ? 1 : 0) + (has_bias_in ? 1 : 0));
+}
+
+// The converter's 8 gamma / beta / bias_in values of chunk c from the stage copy.
+__device__ __forceinline__ void stage_vec8(const bf16* vec, int which, bool present, int c, bool kin,
+                                           float (&f)[8]) {
+  if (present && kin) {
+    unpack8(ld_shared_v4(smem_u32(vec + which * kVecElems + c * 8)), f);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] = 0.f;
+  }
+}
+
 __device__ __forceinline__ void load8_or_zero(const bf16* base, int k0, bool ok, float (&f)[8]) {
   if (base != nullptr && ok) {
     unpack8(ldg16(base + k0), f);

@@ -341,7 +341,10 @@ fnl_status run(fnl_handle* h, const Call& c) {
   if (!rms) {
     if ((st = launch_k1(h, c, stats, c.stream)) != FNL_OK) return st;
   }
-  const bool pdl = !rms;
+  // Every GEMM kernel is a programmatic dependent of its predecessor: it
+  // streams its first weight tiles before griddepcontrol.wait and touches
+  // activations, statistics, workspace and outputs only after it.
+  const bool pdl = true;
   switch (epi) {
     case fnl::kEpiQKV:
       return dispatch_gemm<fnl::kEpiQKV>(h, small, rms, grid, threads, smem, pdl, c.stream, mx, mr, mw, p);

@@ -21,6 +21,9 @@
 // h^2 per row over the K loop; 1/rms is applied per accumulator row in the
 // epilogue (y = rstd * sum_k a'_k W_nk is the same product). Tiles in the first
 // N column also write residual_out and rstd_out, so RMSNorm needs no extra pass.
+// Each stage has a weight barrier (full_w) and an activation barrier (full_x);
+// the kernel is a programmatic dependent of the previous kernel on the stream
+// (first weight tiles before griddepcontrol.wait, everything else after it).
 #pragma once
 
 #include "common.cuh"
@@ -39,13 +42,14 @@ constexpr int TMEM_COLS = 2 * BN;                                  // 512
 constexpr int GROUP_M = 16;  // tile raster: 16 M-blocks share each W tile while it is hot in L2
 
 struct Ctrl {
-  uint64_t full[STAGES], conv[STAGES], empty[STAGES];
+  uint64_t full_w[STAGES], full_x[STAGES], conv[STAGES], empty[STAGES];
   uint64_t tfull[2], tempty[2], sfull[2], drain;
   uint32_t tmem_base;
   int abort_flag;
   float rs[2][BM];
 };
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + static_cast<int>(sizeof(Ctrl)) + 1024;
+constexpr int VEC_BYTES = (STAGES * kVecStageBytes + 127) / 128 * 128;   // [STAGES][3][64] bf16
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + VEC_BYTES + static_cast<int>(sizeof(Ctrl)) + 1024;
 
 __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
   const int per_group = GROUP_M * num_n;
@@ -74,8 +78,11 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
   using namespace k2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + STAGES * STAGE_BYTES);
+  bf16* vecs = reinterpret_cast<bf16*>(smem + STAGES * STAGE_BYTES);   // [STAGES][3][64]
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + STAGES * STAGE_BYTES + VEC_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool has_beta = NORM == kLayerNorm && p.beta != nullptr;
+  const bool has_bias_in = p.bias_in != nullptr;
 
   const int M = p.M, K = p.K;
   const int num_m = (M + BM - 1) / BM;
@@ -85,8 +92,10 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
   const bool split = p.split != 0;
 
   if (threadIdx.x == 0) {
+    pdl_launch_dependents();   // the next call's CTAs may take SMs as ours retire
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&ctrl->full[s], 1);
+      mbar_init(&ctrl->full_w[s], 1);
+      mbar_init(&ctrl->full_x[s], 1);
       mbar_init(&ctrl->conv[s], NUM_CONV_WARPS);
       mbar_init(&ctrl->empty[s], 1);
     }
@@ -117,39 +126,75 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
   if (warp == WARP_TMA) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t s = 0, ph = 0;
-      uint32_t armed = 0;   // stages armed at least once (bitmask) for the abort drain
-      uint32_t last_par = 0;
+      // positions q = (local tile index) * nkb + k-block, stage q % STAGES
+      const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+      const int P = my_tiles * nkb;
+      const int npre = P < STAGES ? P : STAGES;
+      uint32_t armed_w = 0, armed_x = 0, par_w = 0, par_x = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-        int mb, nb;
-        tile_coords(t, num_m, num_n, mb, nb);
-        for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&ctrl->empty[s], ph ^ 1, abortf, p.status, kStatusWaitEmpty)) {
+      struct Cur {
+        int t, mb, nb, kb, s;
+        uint32_t ph;
+      };
+      Cur cw{static_cast<int>(blockIdx.x), 0, 0, 0, 0, 0u};
+      if (P > 0) tile_coords(cw.t, num_m, num_n, cw.mb, cw.nb);
+      Cur cx = cw;
+      auto step = [&](Cur& c) {
+        if (++c.kb == nkb) {
+          c.kb = 0;
+          c.t += gridDim.x;
+          if (c.t < tiles) tile_coords(c.t, num_m, num_n, c.mb, c.nb);
+        }
+        if (++c.s == STAGES) {
+          c.s = 0;
+          c.ph ^= 1u;
+        }
+      };
+      auto issue_w = [&](const Cur& c) {
+        uint8_t* st = smem + c.s * STAGE_BYTES;
+        mbar_arrive_expect_tx(&ctrl->full_w[c.s], W_BYTES);
+        if (EPI == kEpiSwiGLU) {
+          tma_load_2d(st + 2 * X_BYTES, &tm_w, &ctrl->full_w[c.s], c.kb * BK, c.nb * 128);
+          tma_load_2d(st + 2 * X_BYTES + W_BYTES / 2, &tm_w, &ctrl->full_w[c.s], c.kb * BK, p.I + c.nb * 128);
+        } else {
+          tma_load_2d(st + 2 * X_BYTES, &tm_w, &ctrl->full_w[c.s], c.kb * BK, c.nb * BN);
+        }
+        armed_w |= 1u << c.s;
+        par_w = (par_w & ~(1u << c.s)) | (c.ph << c.s);
+      };
+      auto issue_x = [&](const Cur& c) {
+        uint8_t* st = smem + c.s * STAGE_BYTES;
+        mbar_arrive_expect_tx(&ctrl->full_x[c.s], 2 * X_BYTES + vec_bytes(p, has_beta, has_bias_in, c.kb));
+        issue_vec_loads(p, has_beta, has_bias_in, c.kb, vecs + c.s * 3 * kVecElems, &ctrl->full_x[c.s]);
+        tma_load_2d(st, &tm_x, &ctrl->full_x[c.s], c.kb * BK, c.mb * BM);
+        tma_load_2d(st + X_BYTES, &tm_r, &ctrl->full_x[c.s], c.kb * BK, c.mb * BM);
+        armed_x |= 1u << c.s;
+        par_x = (par_x & ~(1u << c.s)) | (c.ph << c.s);
+      };
+      // Weights of the first stages stream while the previous kernel finishes
+      // (they are never written by it); activations only after it is done.
+      for (int q = 0; q < npre; ++q) {
+        issue_w(cw);
+        step(cw);
+      }
+      pdl_wait();
+      for (int q = 0; q < P; ++q) {
+        if (q >= npre) {
+          if (!mbar_wait(&ctrl->empty[cw.s], cw.ph ^ 1, abortf, p.status, kStatusWaitEmpty)) {
             ok = false;
             break;
           }
-          uint8_t* st = smem + s * STAGE_BYTES;
-          mbar_arrive_expect_tx(&ctrl->full[s], STAGE_BYTES);
-          tma_load_2d(st, &tm_x, &ctrl->full[s], kb * BK, mb * BM);
-          tma_load_2d(st + X_BYTES, &tm_r, &ctrl->full[s], kb * BK, mb * BM);
-          if (EPI == kEpiSwiGLU) {
-            tma_load_2d(st + 2 * X_BYTES, &tm_w, &ctrl->full[s], kb * BK, nb * 128);
-            tma_load_2d(st + 2 * X_BYTES + W_BYTES / 2, &tm_w, &ctrl->full[s], kb * BK, p.I + nb * 128);
-          } else {
-            tma_load_2d(st + 2 * X_BYTES, &tm_w, &ctrl->full[s], kb * BK, nb * BN);
-          }
-          armed |= 1u << s;
-          last_par = (last_par & ~(1u << s)) | (ph << s);
-          if (++s == STAGES) {
-            s = 0;
-            ph ^= 1;
-          }
+          issue_w(cw);
+          step(cw);
         }
+        issue_x(cx);
+        step(cx);
       }
       if (!ok) {   // let every issued copy land before the CTA can exit
-        for (int i = 0; i < STAGES; ++i)
-          if (armed & (1u << i)) drain_wait(&ctrl->full[i], (last_par >> i) & 1);
+        for (int i = 0; i < STAGES; ++i) {
+          if (armed_w & (1u << i)) drain_wait(&ctrl->full_w[i], (par_w >> i) & 1);
+          if (armed_x & (1u << i)) drain_wait(&ctrl->full_x[i], (par_x >> i) & 1);
+        }
       }
     }
   } else if (warp == WARP_MMA) {
@@ -167,7 +212,7 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
         const uint32_t d = tmem + b * BN;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&ctrl->conv[s], ph, abortf, p.status, kStatusWaitConv) ||
-              !mbar_wait(&ctrl->full[s], ph, abortf, p.status, kStatusWaitFull)) {
+              !mbar_wait(&ctrl->full_w[s], ph, abortf, p.status, kStatusWaitFull)) {
             ok = false;
             break;
           }
@@ -199,6 +244,7 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;   // TMEM lane quadrant this warp may read
     const int row_local = q * 32 + lane;
+    pdl_wait();   // outputs may still be in use by the previous kernel
     int i = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
       const int b = i & 1;
@@ -296,16 +342,17 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
       }
       const bool write_res = (NORM == kRMSNorm) && nb == 0;
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!warp_wait(&ctrl->full[s], ph, abortf, p.status, kStatusWaitFull)) {
+        if (!warp_wait(&ctrl->full_x[s], ph, abortf, p.status, kStatusWaitFull)) {
           ok = false;
           break;
         }
         const int k0 = kb * BK + c * 8;
         const bool kin = k0 < K;
         float g[8], be[8], bi[8];
-        load8_or_zero(p.gamma, k0, kin, g);
-        load8_or_zero(NORM == kLayerNorm ? p.beta : nullptr, k0, kin, be);
-        load8_or_zero(p.bias_in, k0, kin, bi);
+        const bf16* vec = vecs + s * 3 * kVecElems;
+        stage_vec8(vec, 0, true, c, kin, g);
+        stage_vec8(vec, 1, has_beta, c, kin, be);
+        stage_vec8(vec, 2, has_bias_in, c, kin, bi);
         const uint32_t xs = smem_u32(smem + s * STAGE_BYTES);
         const uint32_t rsm = xs + X_BYTES;
 #pragma unroll

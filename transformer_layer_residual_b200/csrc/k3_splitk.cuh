@@ -14,6 +14,14 @@
 // Warp roles (10 warps): 0 TMA producer (W tile + x/residual tiles), 1 TMEM
 // owner and UMMA issuer, 2-5 epilogue / split-K reduction, 6-9 converters
 // (normalised bf16 operand built in place in shared memory, as in K2).
+//
+// Each stage has two barriers: full_w (the W tile, from HBM) and full_x (the
+// x / residual tiles and the gamma / beta / bias_in slices, from L2), so the
+// converters start on a stage as soon as its activations land instead of
+// waiting for its weights. The kernel is launched as a programmatic dependent
+// of the previous kernel on the stream: the producer streams the first stages
+// of W before griddepcontrol.wait and touches activations, workspace and
+// outputs only after it.
 #pragma once
 
 #include "common.cuh"
@@ -31,17 +39,20 @@ constexpr int NUM_THREADS = (WARP_CONV0 + NUM_CONV_WARPS) * 32;   // 320
 constexpr int MAX_MPAD = 128;
 
 struct Ctrl {
-  uint64_t full[MAX_STAGES], conv[MAX_STAGES], empty[MAX_STAGES];
+  uint64_t full_w[MAX_STAGES], full_x[MAX_STAGES], conv[MAX_STAGES], empty[MAX_STAGES];
   uint64_t tfull[2], tempty[2], sfull[2], drain, esync;
+  long long u0, u1;   // this CTA's unit range
   uint32_t tmem_base;
   int abort_flag;
   int last_flag;
-  float ss[2][MAX_MPAD];
+  float ssw[2][NUM_CONV_WARPS][MAX_MPAD];   // per converter warp partial sums of h^2 (RMSNorm)
+  float2 stw[NUM_CONV_WARPS][MAX_MPAD];     // per converter warp copy of (mean, rstd) (LayerNorm)
 };
 
 __host__ __device__ inline int stage_bytes(int mpad) { return W_BYTES + 2 * mpad * BK * 2; }
+constexpr int VEC_BYTES = MAX_STAGES * kVecStageBytes;   // 3 KB
 __host__ __device__ inline int smem_bytes(int mpad, int stages) {
-  return stages * stage_bytes(mpad) + static_cast<int>(sizeof(Ctrl)) + 1024;
+  return stages * stage_bytes(mpad) + VEC_BYTES + static_cast<int>(sizeof(Ctrl)) + 1024;
 }
 __host__ __device__ inline uint32_t tmem_cols(int mpad) {
   uint32_t c = 32;
@@ -51,6 +62,11 @@ __host__ __device__ inline uint32_t tmem_cols(int mpad) {
 // Index of the CTA whose unit range contains unit u (units split as g*U/G).
 __host__ __device__ inline int unit_owner(long long u, int G, long long U) {
   return static_cast<int>(((u + 1) * G - 1) / U);
+}
+// The same in double precision (exact: every operand is an integer below 2^53
+// and a quotient that is not an integer is at least 1/U away from one).
+__device__ __forceinline__ int unit_owner_fast(long long u, int G, long long U) {
+  return static_cast<int>((static_cast<double>(u + 1) * G - 1.0) / static_cast<double>(U));
 }
 
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
@@ -65,11 +81,8 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
 struct SegIter {
   long long u, u1, U;
   int G, g, nkb;
-  __device__ SegIter(int T, int nkb_, int G_, int g_) : nkb(nkb_), G(G_), g(g_) {
-    U = static_cast<long long>(T) * nkb_;
-    u = static_cast<long long>(g_) * U / G_;
-    u1 = static_cast<long long>(g_ + 1) * U / G_;
-  }
+  __device__ SegIter(long long u0_, long long u1_, long long U_, int nkb_, int G_, int g_)
+      : u(u0_), u1(u1_), U(U_), G(G_), g(g_), nkb(nkb_) {}
   __device__ bool next(int& t, int& kb0, int& nk, int& slot, int& nseg) {
     if (u >= u1) return false;
     t = static_cast<int>(u / nkb);
@@ -77,8 +90,8 @@ struct SegIter {
     const long long tile_end = static_cast<long long>(t + 1) * nkb;
     const long long e = tile_end < u1 ? tile_end : u1;
     nk = static_cast<int>(e - u);
-    const int first = unit_owner(static_cast<long long>(t) * nkb, G, U);
-    const int last = unit_owner(tile_end - 1, G, U);
+    const int first = unit_owner_fast(static_cast<long long>(t) * nkb, G, U);
+    const int last = unit_owner_fast(tile_end - 1, G, U);
     slot = g - first;
     nseg = last - first + 1;
     u = e;
@@ -87,6 +100,92 @@ struct SegIter {
 };
 
 }  // namespace k3
+
+// Last-arriving CTA of tile t: out = epilogue(sum over slots 0..nseg-1 of the
+// fp32 partials), summed in slot order so the result does not depend on which
+// CTA arrives last. Each thread takes ITEMS (row, 8-column) items at a time and
+// issues the loads of up to 4 slots of all of them before adding, so the
+// reduction costs about one L2 round trip per 4 slots instead of one per slot.
+template <int EPI, int NORM>
+__device__ __forceinline__ void k3_reduce_tile(const OpParams& p, int t, int nseg, int et) {
+  using namespace k3;
+  constexpr int ITEMS = (EPI == kEpiSwiGLU) ? 1 : 2;
+  constexpr int NT = NUM_EPI_WARPS * 32;
+  const int mpad = p.mpad;
+  const size_t slot_stride = static_cast<size_t>(mpad) * BW;
+  const float* tp = p.part + static_cast<size_t>(t) * p.max_seg * slot_stride;
+  const float* tss = p.part_ss + static_cast<size_t>(t) * p.max_seg * mpad;
+  const int G8 = (EPI == kEpiSwiGLU) ? 8 : 16;
+  const int n_items = p.M * G8;
+  for (int it0 = et; it0 < n_items; it0 += ITEMS * NT) {
+    float acc[ITEMS][8], up[ITEMS][8], ssum[ITEMS];
+    int mi[ITEMS], gi[ITEMS];
+    bool ok[ITEMS];
+#pragma unroll
+    for (int q = 0; q < ITEMS; ++q) {
+      const int item = it0 + q * NT;
+      ok[q] = item < n_items;
+      mi[q] = ok[q] ? item / G8 : 0;
+      gi[q] = ok[q] ? item - mi[q] * G8 : 0;
+      ssum[q] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[q][e] = up[q][e] = 0.f;
+    }
+    for (int base = 0; base < nseg; base += 4) {
+      float4 va[ITEMS][4][2], vu[ITEMS][4][2];
+      float vs[ITEMS][4];
+#pragma unroll
+      for (int q = 0; q < ITEMS; ++q) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int sl = base + j;
+          if (ok[q] && sl < nseg) {
+            const float* row = tp + sl * slot_stride + static_cast<size_t>(mi[q]) * BW + gi[q] * 8;
+            va[q][j][0] = __ldcg(reinterpret_cast<const float4*>(row));
+            va[q][j][1] = __ldcg(reinterpret_cast<const float4*>(row + 4));
+            if (EPI == kEpiSwiGLU) {
+              vu[q][j][0] = __ldcg(reinterpret_cast<const float4*>(row + 64));
+              vu[q][j][1] = __ldcg(reinterpret_cast<const float4*>(row + 68));
+            }
+            if (NORM == kRMSNorm) vs[q][j] = __ldcg(tss + static_cast<size_t>(sl) * mpad + mi[q]);
+          }
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < ITEMS; ++q) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (ok[q] && base + j < nseg) {
+            acc[q][0] += va[q][j][0].x; acc[q][1] += va[q][j][0].y; acc[q][2] += va[q][j][0].z; acc[q][3] += va[q][j][0].w;
+            acc[q][4] += va[q][j][1].x; acc[q][5] += va[q][j][1].y; acc[q][6] += va[q][j][1].z; acc[q][7] += va[q][j][1].w;
+            if (EPI == kEpiSwiGLU) {
+              up[q][0] += vu[q][j][0].x; up[q][1] += vu[q][j][0].y; up[q][2] += vu[q][j][0].z; up[q][3] += vu[q][j][0].w;
+              up[q][4] += vu[q][j][1].x; up[q][5] += vu[q][j][1].y; up[q][6] += vu[q][j][1].z; up[q][7] += vu[q][j][1].w;
+            }
+            if (NORM == kRMSNorm) ssum[q] += vs[q][j];
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < ITEMS; ++q) {
+      if (!ok[q]) continue;
+      const int m = mi[q], g = gi[q];
+      float scale = 1.f;
+      if (NORM == kRMSNorm) {
+        scale = 1.f / sqrtf(ssum[q] / static_cast<float>(p.K) + p.eps);
+        if (t == 0 && g == 0 && p.rstd_out != nullptr) p.rstd_out[m] = scale;
+      }
+      if (EPI == kEpiSwiGLU) {
+        const int j = t * 64 + g * 8;
+        if (j < p.I) store_swiglu8(p, m, j, acc[q], up[q], scale);
+      } else {
+        const int n = t * BW + g * 8;
+        if (n < p.N) store_out8<EPI>(p, m, n, acc[q], scale);
+      }
+    }
+  }
+}
 
 template <int EPI, int NORM>
 __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
@@ -98,8 +197,11 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
   const int mpad = p.mpad, S = p.stages;
   const int SB = stage_bytes(mpad);
   const int XB = mpad * BK * 2;
-  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + S * SB);
+  bf16* vecs = reinterpret_cast<bf16*>(smem + S * SB);   // [S][3][64]
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + S * SB + VEC_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool has_beta = NORM == kLayerNorm && p.beta != nullptr;
+  const bool has_bias_in = p.bias_in != nullptr;
 
   const int M = p.M, K = p.K;
   const int T = (EPI == kEpiSwiGLU) ? (p.I + 63) / 64 : (p.N + BW - 1) / BW;
@@ -107,10 +209,15 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
   const uint32_t ncols = tmem_cols(mpad);
   const bool split = p.split != 0;
 
+  const long long U = static_cast<long long>(T) * nkb;
   if (threadIdx.x == 0) {
+    pdl_launch_dependents();   // the next call's CTAs may take SMs as ours retire
+    ctrl->u0 = static_cast<long long>(blockIdx.x) * U / gridDim.x;
+    ctrl->u1 = static_cast<long long>(blockIdx.x + 1) * U / gridDim.x;
     for (int s = 0; s < S; ++s) {
-      mbar_init(&ctrl->full[s], 1);
-      mbar_init(&ctrl->conv[s], NUM_CONV_WARPS);
+      mbar_init(&ctrl->full_w[s], 1);
+      mbar_init(&ctrl->full_x[s], 1);
+      mbar_init(&ctrl->conv[s], 1);   // one converter warp per stage
       mbar_init(&ctrl->empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -138,48 +245,85 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = ctrl->tmem_base;
   volatile int* abortf = &ctrl->abort_flag;
+  const long long u0 = ctrl->u0, u1 = ctrl->u1;
 
   if (warp == WARP_TMA) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      SegIter it(T, nkb, gridDim.x, blockIdx.x);
-      int t, kb0, nk, slot, nseg;
-      uint32_t s = 0, ph = 0, armed = 0, last_par = 0;
+      const int P = static_cast<int>(u1 - u0);   // positions (units) of this CTA
+      const int npre = P < S ? P : S;
+      uint32_t armed_w = 0, armed_x = 0, par_w = 0, par_x = 0;
       bool ok = true;
       const uint64_t pol_w = policy_evict_first();   // W is streamed exactly once
-      while (ok && it.next(t, kb0, nk, slot, nseg)) {
-        for (int kb = kb0; kb < kb0 + nk; ++kb) {
-          if (!mbar_wait(&ctrl->empty[s], ph ^ 1, abortf, p.status, kStatusWaitEmpty)) {
+      // two cursors over the unit sequence (tile t, k-block kb, stage s, parity)
+      struct Cur {
+        int t, kb, s;
+        uint32_t ph;
+      };
+      const int t0 = static_cast<int>(u0 / nkb);
+      Cur cw{t0, static_cast<int>(u0 - static_cast<long long>(t0) * nkb), 0, 0u};
+      Cur cx = cw;
+      auto step = [&](Cur& c) {
+        if (++c.kb == nkb) {
+          c.kb = 0;
+          ++c.t;
+        }
+        if (++c.s == S) {
+          c.s = 0;
+          c.ph ^= 1u;
+        }
+      };
+      auto issue_w = [&](const Cur& c) {
+        uint8_t* st = smem + c.s * SB;
+        mbar_arrive_expect_tx(&ctrl->full_w[c.s], W_BYTES);
+        if (EPI == kEpiSwiGLU) {
+          tma_load_2d_hint(st, &tm_w, &ctrl->full_w[c.s], c.kb * BK, c.t * 64, pol_w);
+          tma_load_2d_hint(st + W_BYTES / 2, &tm_w, &ctrl->full_w[c.s], c.kb * BK, p.I + c.t * 64, pol_w);
+        } else {
+          tma_load_2d_hint(st, &tm_w, &ctrl->full_w[c.s], c.kb * BK, c.t * BW, pol_w);
+        }
+        armed_w |= 1u << c.s;
+        par_w = (par_w & ~(1u << c.s)) | (c.ph << c.s);
+      };
+      auto issue_x = [&](const Cur& c) {
+        uint8_t* st = smem + c.s * SB;
+        mbar_arrive_expect_tx(&ctrl->full_x[c.s], 2 * XB + vec_bytes(p, has_beta, has_bias_in, c.kb));
+        issue_vec_loads(p, has_beta, has_bias_in, c.kb, vecs + c.s * 3 * kVecElems, &ctrl->full_x[c.s]);
+        tma_load_2d(st + W_BYTES, &tm_x, &ctrl->full_x[c.s], c.kb * BK, 0);
+        tma_load_2d(st + W_BYTES + XB, &tm_r, &ctrl->full_x[c.s], c.kb * BK, 0);
+        armed_x |= 1u << c.s;
+        par_x = (par_x & ~(1u << c.s)) | (c.ph << c.s);
+      };
+      // Weights of the first stages stream while the previous kernel finishes
+      // (they are never written by it); activations only after it is done.
+      for (int q = 0; q < npre; ++q) {
+        issue_w(cw);
+        step(cw);
+      }
+      pdl_wait();
+      for (int q = 0; q < P; ++q) {
+        if (q >= npre) {
+          if (!mbar_wait(&ctrl->empty[cw.s], cw.ph ^ 1, abortf, p.status, kStatusWaitEmpty)) {
             ok = false;
             break;
           }
-          uint8_t* st = smem + s * SB;
-          mbar_arrive_expect_tx(&ctrl->full[s], SB);
-          if (EPI == kEpiSwiGLU) {
-            tma_load_2d_hint(st, &tm_w, &ctrl->full[s], kb * BK, t * 64, pol_w);
-            tma_load_2d_hint(st + W_BYTES / 2, &tm_w, &ctrl->full[s], kb * BK, p.I + t * 64, pol_w);
-          } else {
-            tma_load_2d_hint(st, &tm_w, &ctrl->full[s], kb * BK, t * BW, pol_w);
-          }
-          tma_load_2d(st + W_BYTES, &tm_x, &ctrl->full[s], kb * BK, 0);
-          tma_load_2d(st + W_BYTES + XB, &tm_r, &ctrl->full[s], kb * BK, 0);
-          armed |= 1u << s;
-          last_par = (last_par & ~(1u << s)) | (ph << s);
-          if (++s == static_cast<uint32_t>(S)) {
-            s = 0;
-            ph ^= 1;
-          }
+          issue_w(cw);
+          step(cw);
         }
+        issue_x(cx);
+        step(cx);
       }
-      if (!ok) {
-        for (int i = 0; i < S; ++i)
-          if (armed & (1u << i)) drain_wait(&ctrl->full[i], (last_par >> i) & 1);
+      if (!ok) {   // let every issued copy land before the CTA can exit
+        for (int i = 0; i < S; ++i) {
+          if (armed_w & (1u << i)) drain_wait(&ctrl->full_w[i], (par_w >> i) & 1);
+          if (armed_x & (1u << i)) drain_wait(&ctrl->full_x[i], (par_x >> i) & 1);
+        }
       }
     }
   } else if (warp == WARP_MMA) {
     // ------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
-      SegIter it(T, nkb, gridDim.x, blockIdx.x);
+      SegIter it(u0, u1, U, nkb, gridDim.x, blockIdx.x);
       int t, kb0, nk, slot, nseg;
       uint32_t s = 0, ph = 0;
       bool ok = true;
@@ -193,7 +337,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
         const uint32_t d = tmem + b * mpad;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&ctrl->conv[s], ph, abortf, p.status, kStatusWaitConv) ||
-              !mbar_wait(&ctrl->full[s], ph, abortf, p.status, kStatusWaitFull)) {
+              !mbar_wait(&ctrl->full_w[s], ph, abortf, p.status, kStatusWaitFull)) {
             ok = false;
             break;
           }
@@ -227,7 +371,8 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     const int q = warp & 3;
     const int et = threadIdx.x - WARP_EPI0 * 32;   // 0..127
     const int nl = q * 32 + lane;                  // W row within the tile = TMEM lane
-    SegIter it(T, nkb, gridDim.x, blockIdx.x);
+    pdl_wait();   // workspace and outputs may still be in use by the previous kernel
+    SegIter it(u0, u1, U, nkb, gridDim.x, blockIdx.x);
     int t, kb0, nk, slot, nseg;
     int i = 0;
     uint32_t eph = 0;
@@ -250,7 +395,12 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
         for (int e = 0; e < 16; ++e)
           if (mc + e < M) part[static_cast<size_t>(mc + e) * BW + nl] = __uint_as_float(v[e]);
       }
-      if (NORM == kRMSNorm && et < M) p.part_ss[base * mpad + et] = ctrl->ss[b][et];
+      if (NORM == kRMSNorm && et < M) {
+        float ssum = 0.f;
+#pragma unroll
+        for (int w = 0; w < NUM_CONV_WARPS; ++w) ssum += ctrl->ssw[b][w][et];   // fixed order
+        p.part_ss[base * mpad + et] = ssum;
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctrl->tempty[b]);
@@ -275,96 +425,72 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
       eph ^= 1;
       if (ctrl->last_flag) {
         __threadfence();
-        const float* tp = p.part + static_cast<size_t>(t) * p.max_seg * mpad * BW;
-        const float* tss = p.part_ss + static_cast<size_t>(t) * p.max_seg * mpad;
-        const int G8 = (EPI == kEpiSwiGLU) ? 8 : 16;
-        for (int item = et; item < M * G8; item += NUM_EPI_WARPS * 32) {
-          const int m = item / G8, g = item - (item / G8) * G8;
-          float scale = 1.f;
-          if (NORM == kRMSNorm) {
-            float ssum = 0.f;
-            for (int sl = 0; sl < nseg; ++sl) ssum += __ldcg(tss + static_cast<size_t>(sl) * mpad + m);
-            scale = 1.f / sqrtf(ssum / static_cast<float>(K) + p.eps);
-            if (t == 0 && g == 0 && p.rstd_out != nullptr) p.rstd_out[m] = scale;
-          }
-          if (EPI == kEpiSwiGLU) {
-            const int j = t * 64 + g * 8;
-            if (j >= p.I) continue;
-            float ga[8] = {0, 0, 0, 0, 0, 0, 0, 0}, ua[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            for (int sl = 0; sl < nseg; ++sl) {
-              const float* row = tp + (static_cast<size_t>(sl) * mpad + m) * BW;
-              const float4 a0 = __ldcg(reinterpret_cast<const float4*>(row + g * 8));
-              const float4 a1 = __ldcg(reinterpret_cast<const float4*>(row + g * 8 + 4));
-              const float4 b0 = __ldcg(reinterpret_cast<const float4*>(row + 64 + g * 8));
-              const float4 b1 = __ldcg(reinterpret_cast<const float4*>(row + 64 + g * 8 + 4));
-              ga[0] += a0.x; ga[1] += a0.y; ga[2] += a0.z; ga[3] += a0.w;
-              ga[4] += a1.x; ga[5] += a1.y; ga[6] += a1.z; ga[7] += a1.w;
-              ua[0] += b0.x; ua[1] += b0.y; ua[2] += b0.z; ua[3] += b0.w;
-              ua[4] += b1.x; ua[5] += b1.y; ua[6] += b1.z; ua[7] += b1.w;
-            }
-            store_swiglu8(p, m, j, ga, ua, scale);
-          } else {
-            const int n = t * BW + g * 8;
-            if (n >= p.N) continue;
-            float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            for (int sl = 0; sl < nseg; ++sl) {
-              const float* row = tp + (static_cast<size_t>(sl) * mpad + m) * BW;
-              const float4 a0 = __ldcg(reinterpret_cast<const float4*>(row + g * 8));
-              const float4 a1 = __ldcg(reinterpret_cast<const float4*>(row + g * 8 + 4));
-              acc[0] += a0.x; acc[1] += a0.y; acc[2] += a0.z; acc[3] += a0.w;
-              acc[4] += a1.x; acc[5] += a1.y; acc[6] += a1.z; acc[7] += a1.w;
-            }
-            store_out8<EPI>(p, m, n, acc, scale);
-          }
-        }
+        k3_reduce_tile<EPI, NORM>(p, t, nseg, et);
         if (et == 0) p.counters[t] = 0u;
       }
     }
   } else {
     // ------------------------------------------------------------ converters
-    const int ct = threadIdx.x - WARP_CONV0 * 32;   // 0..127
-    const int c = ct & 7;
-    const int rg = ct >> 3;                          // rows rg + 16 j
-    const int nj = mpad / 16;
-    float mu[8], rs[8], ss[8];
-    if (NORM == kLayerNorm) pdl_wait();
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int row = rg + 16 * j;
-      mu[j] = 0.f;
-      rs[j] = 0.f;
-      if (NORM == kLayerNorm && j < nj && row < M) {
-        const float2 st = p.stats[row];
-        mu[j] = st.x;
-        rs[j] = st.y;
-      }
+    // Converter warp cw owns pipeline positions cw, cw + 4, cw + 8, ... of this
+    // CTA's unit sequence, so up to four stages are converted at once. Lane:
+    // 16-byte chunk c of the 128-byte row, rows r0 + 4 j.
+    const int cw = warp - WARP_CONV0;
+    const int c = lane & 7;
+    const int r0 = lane >> 3;
+    const int nrow = mpad / 4;   // rows per lane, 4..32
+    if (NORM == kLayerNorm) {
+      pdl_wait();   // statistics come from the previous kernel
+      for (int r = lane; r < mpad; r += 32)
+        ctrl->stw[cw][r] = r < M ? p.stats[r] : make_float2(0.f, 0.f);
+      __syncwarp();
     }
-    SegIter it(T, nkb, gridDim.x, blockIdx.x);
+    SegIter it(u0, u1, U, nkb, gridDim.x, blockIdx.x);
     int t, kb0, nk, slot, nseg;
-    uint32_t s = 0, ph = 0;
-    int i = 0;
+    int pos = 0;   // first position of the current segment
+    int i = 0;     // segment index
+    int cq = cw, cs = cw;   // this warp's next position and its stage (S >= NUM_CONV_WARPS)
+    uint32_t cph = 0;
     bool ok = true;
     while (ok && it.next(t, kb0, nk, slot, nseg)) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) ss[j] = 0.f;
+      const int b = i & 1;
+      if (NORM == kRMSNorm) {
+        // this warp's slot of the segment's sum(h^2) per row; free once the
+        // epilogue has read the segment that used it two segments ago
+        const uint32_t use = static_cast<uint32_t>(i >> 1);
+        if (!warp_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty)) break;
+        for (int r = lane; r < mpad; r += 32) ctrl->ssw[b][cw][r] = 0.f;
+        __syncwarp();
+      }
       const bool write_res = (NORM == kRMSNorm) && t == 0;
-      for (int kb = kb0; kb < kb0 + nk; ++kb) {
-        if (!warp_wait(&ctrl->full[s], ph, abortf, p.status, kStatusWaitFull)) {
+      // positions of this segment owned by this warp (cq: next owned position,
+      // with its stage cs and parity cph, advanced by NUM_CONV_WARPS at a time)
+      for (; cq < pos + nk; cq += NUM_CONV_WARPS) {
+        const int q = cq;
+        const int s = cs;
+        const uint32_t ph = cph;
+        cs += NUM_CONV_WARPS;
+        if (cs >= S) {
+          cs -= S;
+          cph ^= 1u;
+        }
+        const int kb = kb0 + (q - pos);
+        if (!warp_wait(&ctrl->full_x[s], ph, abortf, p.status, kStatusWaitFull)) {
           ok = false;
           break;
         }
         const int k0 = kb * BK + c * 8;
         const bool kin = k0 < K;
         float g[8], be[8], bi[8];
-        load8_or_zero(p.gamma, k0, kin, g);
-        load8_or_zero(NORM == kLayerNorm ? p.beta : nullptr, k0, kin, be);
-        load8_or_zero(p.bias_in, k0, kin, bi);
+        const bf16* vec = vecs + s * 3 * kVecElems;
+        stage_vec8(vec, 0, true, c, kin, g);
+        stage_vec8(vec, 1, has_beta, c, kin, be);
+        stage_vec8(vec, 2, has_bias_in, c, kin, bi);
         const uint32_t xs = smem_u32(smem + s * SB) + W_BYTES;
         const uint32_t rsm = xs + XB;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j < nj) {
-            const int row = rg + 16 * j;
+#pragma unroll 4
+        for (int j = 0; j < nrow; ++j) {
+          {
+            const int row = r0 + 4 * j;
             const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
             float h[8], rr[8], a[8];
             unpack8(ld_shared_v4(xs + off), h);
@@ -372,14 +498,20 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) h[e] = (h[e] + rr[e]) + bi[e];
             if (NORM == kLayerNorm) {
+              const float2 st = ctrl->stw[cw][row];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) a[e] = fmaf((h[e] - mu[j]) * rs[j], g[e], be[e]);
+              for (int e = 0; e < 8; ++e) a[e] = fmaf((h[e] - st.x) * st.y, g[e], be[e]);
             } else {
+              float sq = 0.f;
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
                 a[e] = h[e] * g[e];
-                ss[j] = fmaf(h[e], h[e], ss[j]);
+                sq = fmaf(h[e], h[e], sq);
               }
+              sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+              sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+              sq += __shfl_xor_sync(0xffffffffu, sq, 4);
+              if (c == 0) ctrl->ssw[b][cw][row] += sq;
             }
             uint4 hi, lo;
             round_split8(a, split, hi, lo);
@@ -392,30 +524,13 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->conv[s]);
-        if (++s == static_cast<uint32_t>(S)) {
-          s = 0;
-          ph ^= 1;
-        }
       }
       if (!ok) break;
       if (NORM == kRMSNorm) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], 1);
-          ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], 2);
-          ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], 4);
-        }
-        const int b = i & 1;
-        const uint32_t use = static_cast<uint32_t>(i >> 1);
-        if (!warp_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty)) break;
-        if (c == 0) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (j < nj) ctrl->ss[b][rg + 16 * j] = ss[j];
-        }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ctrl->sfull[b]);
+        if (lane == 0) mbar_arrive(&ctrl->sfull[b]);   // this warp's share of the segment is in
       }
+      pos += nk;
       ++i;
     }
   }
