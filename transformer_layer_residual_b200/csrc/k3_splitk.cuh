@@ -46,7 +46,6 @@ struct Ctrl {
   int abort_flag;
   int last_flag;
   float ssw[2][NUM_CONV_WARPS][MAX_MPAD];   // per converter warp partial sums of h^2 (RMSNorm)
-  float2 stw[NUM_CONV_WARPS][MAX_MPAD];     // per converter warp copy of (mean, rstd) (LayerNorm)
 };
 
 __host__ __device__ inline int stage_bytes(int mpad) { return W_BYTES + 2 * mpad * BK * 2; }
@@ -432,17 +431,31 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
   } else {
     // ------------------------------------------------------------ converters
     // Converter warp cw owns pipeline positions cw, cw + 4, cw + 8, ... of this
-    // CTA's unit sequence, so up to four stages are converted at once. Lane:
-    // 16-byte chunk c of the 128-byte row, rows r0 + 4 j.
+    // CTA's unit sequence, so up to four stages are converted at once. Lanes
+    // are split into groups of L lanes per token row (L = 8 for M <= 4 down to
+    // 1 for M > 16): lane = (row slot, first chunk); a lane walks chunks
+    // cf, cf + L, ... of rows rb, rb + 32/L, ... (< M; padding rows keep the
+    // zeros TMA filled in, a valid operand whose columns are never read).
+    // sum(h^2) stays in registers and is reduced over the L lanes once per segment.
     const int cw = warp - WARP_CONV0;
-    const int c = lane & 7;
-    const int r0 = lane >> 3;
-    const int nrow = mpad / 4;   // rows per lane, 4..32
+    const int L = M <= 4 ? 8 : (M <= 8 ? 4 : (M <= 16 ? 2 : 1));
+    const int rpp = 32 / L;              // rows per pass of the warp
+    const int rb = lane / L, cf = lane - rb * L;
+    const int npass = (M + rpp - 1) / rpp;   // 1..4
+    float mu[4], rs[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) mu[j] = rs[j] = 0.f;
     if (NORM == kLayerNorm) {
       pdl_wait();   // statistics come from the previous kernel
-      for (int r = lane; r < mpad; r += 32)
-        ctrl->stw[cw][r] = r < M ? p.stats[r] : make_float2(0.f, 0.f);
-      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int row = rb + rpp * j;
+        if (j < npass && row < M) {
+          const float2 st = p.stats[row];
+          mu[j] = st.x;
+          rs[j] = st.y;
+        }
+      }
     }
     SegIter it(u0, u1, U, nkb, gridDim.x, blockIdx.x);
     int t, kb0, nk, slot, nseg;
@@ -453,17 +466,8 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     bool ok = true;
     while (ok && it.next(t, kb0, nk, slot, nseg)) {
       const int b = i & 1;
-      if (NORM == kRMSNorm) {
-        // this warp's slot of the segment's sum(h^2) per row; free once the
-        // epilogue has read the segment that used it two segments ago
-        const uint32_t use = static_cast<uint32_t>(i >> 1);
-        if (!warp_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty)) break;
-        for (int r = lane; r < mpad; r += 32) ctrl->ssw[b][cw][r] = 0.f;
-        __syncwarp();
-      }
+      float sq[4] = {0.f, 0.f, 0.f, 0.f};   // this warp's share of the segment's sum(h^2) per row
       const bool write_res = (NORM == kRMSNorm) && t == 0;
-      // positions of this segment owned by this warp (cq: next owned position,
-      // with its stage cs and parity cph, advanced by NUM_CONV_WARPS at a time)
       for (; cq < pos + nk; cq += NUM_CONV_WARPS) {
         const int q = cq;
         const int s = cs;
@@ -478,47 +482,44 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
           ok = false;
           break;
         }
-        const int k0 = kb * BK + c * 8;
-        const bool kin = k0 < K;
-        float g[8], be[8], bi[8];
-        const bf16* vec = vecs + s * 3 * kVecElems;
-        stage_vec8(vec, 0, true, c, kin, g);
-        stage_vec8(vec, 1, has_beta, c, kin, be);
-        stage_vec8(vec, 2, has_bias_in, c, kin, bi);
         const uint32_t xs = smem_u32(smem + s * SB) + W_BYTES;
         const uint32_t rsm = xs + XB;
-#pragma unroll 4
-        for (int j = 0; j < nrow; ++j) {
-          {
-            const int row = r0 + 4 * j;
-            const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
-            float h[8], rr[8], a[8];
-            unpack8(ld_shared_v4(xs + off), h);
-            unpack8(ld_shared_v4(rsm + off), rr);
+        const bf16* vec = vecs + s * 3 * kVecElems;
+#pragma unroll 2
+        for (int c = cf; c < 8; c += L) {
+          const int k0 = kb * BK + c * 8;
+          const bool kin = k0 < K;
+          float g[8], be[8], bi[8];
+          stage_vec8(vec, 0, true, c, kin, g);
+          stage_vec8(vec, 1, has_beta, c, kin, be);
+          stage_vec8(vec, 2, has_bias_in, c, kin, bi);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) h[e] = (h[e] + rr[e]) + bi[e];
-            if (NORM == kLayerNorm) {
-              const float2 st = ctrl->stw[cw][row];
+          for (int j = 0; j < 4; ++j) {
+            const int row = rb + rpp * j;
+            if (j < npass && row < M) {
+              const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
+              float h[8], rr[8], a[8];
+              unpack8(ld_shared_v4(xs + off), h);
+              unpack8(ld_shared_v4(rsm + off), rr);
 #pragma unroll
-              for (int e = 0; e < 8; ++e) a[e] = fmaf((h[e] - st.x) * st.y, g[e], be[e]);
-            } else {
-              float sq = 0.f;
+              for (int e = 0; e < 8; ++e) h[e] = (h[e] + rr[e]) + bi[e];
+              if (NORM == kLayerNorm) {
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                a[e] = h[e] * g[e];
-                sq = fmaf(h[e], h[e], sq);
+                for (int e = 0; e < 8; ++e) a[e] = fmaf((h[e] - mu[j]) * rs[j], g[e], be[e]);
+              } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  a[e] = h[e] * g[e];
+                  sq[j] = fmaf(h[e], h[e], sq[j]);
+                }
               }
-              sq += __shfl_xor_sync(0xffffffffu, sq, 1);
-              sq += __shfl_xor_sync(0xffffffffu, sq, 2);
-              sq += __shfl_xor_sync(0xffffffffu, sq, 4);
-              if (c == 0) ctrl->ssw[b][cw][row] += sq;
+              uint4 hi, lo;
+              round_split8(a, split, hi, lo);
+              st_shared_v4(xs + off, hi);
+              if (split) st_shared_v4(rsm + off, lo);
+              if (write_res && kin)
+                *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(row) * K + k0) = pack8(h);
             }
-            uint4 hi, lo;
-            round_split8(a, split, hi, lo);
-            st_shared_v4(xs + off, hi);
-            if (split) st_shared_v4(rsm + off, lo);
-            if (write_res && row < M && kin)
-              *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(row) * K + k0) = pack8(h);
           }
         }
         fence_proxy_async_smem();
@@ -527,8 +528,18 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
       }
       if (!ok) break;
       if (NORM == kRMSNorm) {
+        // publish this warp's share once the epilogue has read the segment
+        // that used this buffer two segments ago
+        const uint32_t use = static_cast<uint32_t>(i >> 1);
+        if (!warp_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty)) break;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          for (int o = 1; o < L; o <<= 1) sq[j] += __shfl_xor_sync(0xffffffffu, sq[j], o);
+          const int row = rb + rpp * j;
+          if (cf == 0 && j < npass && row < M) ctrl->ssw[b][cw][row] = sq[j];
+        }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&ctrl->sfull[b]);   // this warp's share of the segment is in
+        if (lane == 0) mbar_arrive(&ctrl->sfull[b]);
       }
       pos += nk;
       ++i;
