@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + STAGES * STAGE_BYTES + VEC_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool has_beta = NORM == kLayerNorm && p.beta != nullptr;
-  const bool has_bias_in = p.bias_in != nullptr;
+  const bool has_bias_in = EPI == kEpiGELU && p.bias_in != nullptr;   // only the GELU entry point has one
 
   const int M = p.M, K = p.K;
   const int num_m = (M + BM - 1) / BM;
@@ -355,13 +355,23 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
         stage_vec8(vec, 2, has_bias_in, c, kin, bi);
         const uint32_t xs = smem_u32(smem + s * STAGE_BYTES);
         const uint32_t rsm = xs + X_BYTES;
+        // loads of all four rows first, then arithmetic and stores, so the
+        // four chunks overlap instead of running in series
+        uint4 xv[4], rv[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int row = rbase + 32 * j;
+          const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
+          xv[j] = ld_shared_v4(xs + off);
+          rv[j] = ld_shared_v4(rsm + off);
+        }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int row = rbase + 32 * j;
           const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
           float h[8], rr[8], a[8];
-          unpack8(ld_shared_v4(xs + off), h);
-          unpack8(ld_shared_v4(rsm + off), rr);
+          unpack8(xv[j], h);
+          unpack8(rv[j], rr);
 #pragma unroll
           for (int e = 0; e < 8; ++e) h[e] = (h[e] + rr[e]) + bi[e];
           if (NORM == kLayerNorm) {

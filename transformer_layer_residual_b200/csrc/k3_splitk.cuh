@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + S * SB + VEC_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool has_beta = NORM == kLayerNorm && p.beta != nullptr;
-  const bool has_bias_in = p.bias_in != nullptr;
+  const bool has_bias_in = EPI == kEpiGELU && p.bias_in != nullptr;   // only the GELU entry point has one
 
   const int M = p.M, K = p.K;
   const int T = (EPI == kEpiSwiGLU) ? (p.I + 63) / 64 : (p.N + BW - 1) / BW;
@@ -442,6 +442,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     const int rpp = 32 / L;              // rows per pass of the warp
     const int rb = lane / L, cf = lane - rb * L;
     const int npass = (M + rpp - 1) / rpp;   // 1..4
+    const int cpl = 8 / L;                   // chunks per lane per row
     float mu[4], rs[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) mu[j] = rs[j] = 0.f;
@@ -485,40 +486,65 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
         const uint32_t xs = smem_u32(smem + s * SB) + W_BYTES;
         const uint32_t rsm = xs + XB;
         const bf16* vec = vecs + s * 3 * kVecElems;
-#pragma unroll 2
-        for (int c = cf; c < 8; c += L) {
-          const int k0 = kb * BK + c * 8;
-          const bool kin = k0 < K;
-          float g[8], be[8], bi[8];
-          stage_vec8(vec, 0, true, c, kin, g);
-          stage_vec8(vec, 1, has_beta, c, kin, be);
-          stage_vec8(vec, 2, has_bias_in, c, kin, bi);
+        // For each row slot j of this lane, the lane's chunks of that row in
+        // batches of 4: all shared-memory loads of a batch are issued before its
+        // arithmetic and stores, so chunks overlap instead of running in series.
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int row = rb + rpp * j;
-            if (j < npass && row < M) {
-              const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
-              float h[8], rr[8], a[8];
-              unpack8(ld_shared_v4(xs + off), h);
-              unpack8(ld_shared_v4(rsm + off), rr);
+        for (int j = 0; j < 4; ++j) {
+          const int row = rb + rpp * j;
+          if (j < npass && row < M) {
+            for (int c0 = 0; c0 < cpl; c0 += 4) {
+              uint4 xv[4], rv[4], gv[4], bev[4], biv[4];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) h[e] = (h[e] + rr[e]) + bi[e];
-              if (NORM == kLayerNorm) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) a[e] = fmaf((h[e] - mu[j]) * rs[j], g[e], be[e]);
-              } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  a[e] = h[e] * g[e];
-                  sq[j] = fmaf(h[e], h[e], sq[j]);
+              for (int u = 0; u < 4; ++u) {
+                if (c0 + u < cpl) {
+                  const int c = cf + L * (c0 + u);
+                  const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
+                  xv[u] = ld_shared_v4(xs + off);
+                  rv[u] = ld_shared_v4(rsm + off);
+                  gv[u] = ld_shared_v4(smem_u32(vec + c * 8));
+                  if (has_beta) bev[u] = ld_shared_v4(smem_u32(vec + kVecElems + c * 8));
+                  if (has_bias_in) biv[u] = ld_shared_v4(smem_u32(vec + 2 * kVecElems + c * 8));
                 }
               }
-              uint4 hi, lo;
-              round_split8(a, split, hi, lo);
-              st_shared_v4(xs + off, hi);
-              if (split) st_shared_v4(rsm + off, lo);
-              if (write_res && kin)
-                *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(row) * K + k0) = pack8(h);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                if (c0 + u < cpl) {
+                  const int c = cf + L * (c0 + u);
+                  const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
+                  const int kk0 = kb * BK + c * 8;
+                  const bool kin = kk0 < K;
+                  float h[8], rr[8], g[8], be[8], bi[8], a[8];
+                  unpack8(xv[u], h);
+                  unpack8(rv[u], rr);
+                  unpack8(gv[u], g);
+                  if (has_beta) unpack8(bev[u], be);
+                  if (has_bias_in) unpack8(biv[u], bi);
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) {
+                    if (!kin) g[e] = 0.f;
+                    if (!has_beta || !kin) be[e] = 0.f;
+                    if (!has_bias_in || !kin) bi[e] = 0.f;
+                    h[e] = (h[e] + rr[e]) + bi[e];
+                  }
+                  if (NORM == kLayerNorm) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) a[e] = fmaf((h[e] - mu[j]) * rs[j], g[e], be[e]);
+                  } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                      a[e] = h[e] * g[e];
+                      sq[j] = fmaf(h[e], h[e], sq[j]);
+                    }
+                  }
+                  uint4 hi, lo;
+                  round_split8(a, split, hi, lo);
+                  st_shared_v4(xs + off, hi);
+                  if (split) st_shared_v4(rsm + off, lo);
+                  if (write_res && kin)
+                    *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(row) * K + kk0) = pack8(h);
+                }
+              }
             }
           }
         }
