@@ -74,7 +74,7 @@ def test_tile_tails(handle, op, norm, M):
     run_and_check(handle, w, inputs)
 
 
-@pytest.mark.parametrize("path", ["tile", "splitk"])
+@pytest.mark.parametrize("path", ["tile", "wide", "splitk"])
 @pytest.mark.parametrize("op", ["qkv", "swiglu", "gelu"])
 @pytest.mark.parametrize("norm", ["layernorm", "rmsnorm"])
 def test_forced_paths(cuda_device, path, op, norm):

@@ -94,6 +94,56 @@ __device__ __forceinline__ void stage_vec8(const bf16* vec, int which, bool pres
   }
 }
 
+// 8 consecutive elements of one token row: h = x + r (+ bias_in) in fp32,
+// a = normalise(h) rounded to bf16 (hi) and, if split, the bf16 remainder (lo).
+// LayerNorm: a = (h - mean) * rstd * gamma + beta. RMSNorm (deferred scale):
+// a = h * gamma and sq += h^2 (even and odd elements in the two lanes).
+// g, be, bi: the chunk's gamma / beta / bias_in as four fp32 pairs.
+template <int NORM>
+__device__ __forceinline__ void convert8(const uint4& xv, const uint4& rv, const f32x2 (&g)[4], const f32x2 (&be)[4],
+                                         const f32x2 (&bi)[4], bool has_beta, bool has_bias_in, float mean,
+                                         float rstd, bool split, bool want_h, f32x2& sq, uint4& hi, uint4& lo,
+                                         uint4& hres) {
+  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+  const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
+  uint32_t ho[4], lw[4], hw[4];
+  const f32x2 mu2 = pk2(mean, mean), rs2 = pk2(rstd, rstd);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f32x2 h = add2(bf2_to_f2(xw[i]), bf2_to_f2(rw[i]));
+    if (has_bias_in) h = add2(h, bi[i]);
+    f32x2 a;
+    if (NORM == kLayerNorm) {
+      a = mul2(sub2(h, mu2), rs2);
+      a = has_beta ? fma2(a, g[i], be[i]) : mul2(a, g[i]);
+    } else {
+      a = mul2(h, g[i]);
+      sq = fma2(h, h, sq);
+    }
+    ho[i] = f2_to_bf2(a);
+    if (split) lw[i] = f2_to_bf2(sub2(a, bf2_to_f2(ho[i])));
+    if (want_h) hw[i] = f2_to_bf2(h);
+  }
+  hi = make_uint4(ho[0], ho[1], ho[2], ho[3]);
+  if (split) lo = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  if (want_h) hres = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+}
+
+// A 16-byte vector of 8 bf16 as four fp32 pairs (zeros when absent).
+__device__ __forceinline__ void vec_pairs(const bf16* vec, int which, bool present, int c, bool kin,
+                                          f32x2 (&f)[4]) {
+  if (present && kin) {
+    const uint4 v = ld_shared_v4(smem_u32(vec + which * kVecElems + c * 8));
+    f[0] = bf2_to_f2(v.x);
+    f[1] = bf2_to_f2(v.y);
+    f[2] = bf2_to_f2(v.z);
+    f[3] = bf2_to_f2(v.w);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = 0ull;
+  }
+}
+
 __device__ __forceinline__ void load8_or_zero(const bf16* base, int k0, bool ok, float (&f)[8]) {
   if (base != nullptr && ok) {
     unpack8(ldg16(base + k0), f);

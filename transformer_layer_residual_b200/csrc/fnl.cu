@@ -21,6 +21,7 @@
 #include "fnl.h"
 #include "k1_stats.cuh"
 #include "k2_tile.cuh"
+#include "k2_wide.cuh"
 #include "k3_splitk.cuh"
 
 using fnl::bf16;
@@ -93,17 +94,19 @@ fnl_status get_encoder(fnl_handle* h) {
   return FNL_OK;
 }
 
-// Row-major bf16 [rows, cols] (cols contiguous), box [box_rows, 64] with the
-// 128-byte swizzle the UMMA descriptors expect; out-of-range elements read 0.
+// Row-major bf16 [rows, cols] (cols contiguous), box [box_rows, box_cols] with
+// the swizzle the UMMA descriptors expect: 128-byte swizzle for 64-wide boxes,
+// 64-byte swizzle for 32-wide boxes; out-of-range elements read 0.
 fnl_status make_map(fnl_handle* h, CUtensorMap* m, const void* ptr, long long rows, long long cols,
-                    int box_rows) {
+                    int box_rows, int box_cols = 64) {
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(h, FNL_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
   return FNL_OK;
 }
@@ -234,7 +237,12 @@ fnl_status launch_gemm(fnl_handle* h, Kern kern, int grid, int threads, int smem
 template <int EPI>
 fnl_status dispatch_gemm(fnl_handle* h, bool small, bool rms, int grid, int threads, int smem, bool pdl,
                          cudaStream_t stream, const CUtensorMap& mx, const CUtensorMap& mr, const CUtensorMap& mw,
-                         const OpParams& p) {
+                         const OpParams& p, bool wide = false) {
+  if (wide) {
+    if (rms)
+      return launch_gemm(h, fnl::k2w_tile_kernel<EPI, fnl::kRMSNorm>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
+    return launch_gemm(h, fnl::k2w_tile_kernel<EPI, fnl::kLayerNorm>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
+  }
   if (small) {
     if (rms)
       return launch_gemm(h, fnl::k3_splitk_kernel<EPI, fnl::kRMSNorm>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
@@ -275,13 +283,14 @@ fnl_status run(fnl_handle* h, const Call& c) {
   const bool rms = c.norm == FNL_NORM_RMSNORM;
   const int epi = c.op == Op::QKV ? fnl::kEpiQKV : (c.op == Op::SwiGLU ? fnl::kEpiSwiGLU : fnl::kEpiGELU);
   bool small = c.M <= fnl::k3::MAX_MPAD;
-  if (h->opt.path == FNL_PATH_TILE) small = false;
+  if (h->opt.path == FNL_PATH_TILE || h->opt.path == FNL_PATH_TILE_WIDE) small = false;
   if (h->opt.path == FNL_PATH_SPLITK) small = true;
   const int max_ctas = h->opt.max_ctas > 0 ? std::min(h->opt.max_ctas, h->num_sms) : h->num_sms;
   const int nkb = (c.K + 63) / 64;
 
   // plan
   int grid = 1, threads = 0, smem = 0, mpad = 0, stages = 0, max_seg = 1, T = 0;
+  bool wide = false;
   if (small) {
     mpad = round_up(std::max(c.M, 1), 16);
     T = c.op == Op::SwiGLU ? (c.I + 63) / 64 : (c.N + 127) / 128;
@@ -297,12 +306,27 @@ fnl_status run(fnl_handle* h, const Call& c) {
     }
     if (T > kMaxTiles) return fail(h, FNL_ERR_UNSUPPORTED, "too many W tiles");
   } else {
-    const int num_m = (c.M + fnl::k2::BM - 1) / fnl::k2::BM;
-    const int num_n = c.op == Op::SwiGLU ? (c.I + 127) / 128 : (c.N + fnl::k2::BN - 1) / fnl::k2::BN;
-    const long long tiles = static_cast<long long>(num_m) * num_n;
+    // two tile shapes: 128 x 512 (less traffic and conversion per FLOP, the
+    // default) and 128 x 256 (finer), picked by how well the tiles fill whole
+    // waves of CTAs
+    const int num_m = (c.M + 127) / 128;
+    const long long tiles_n = static_cast<long long>(num_m) *
+                              (c.op == Op::SwiGLU ? (c.I + 127) / 128 : (c.N + fnl::k2::BN - 1) / fnl::k2::BN);
+    const long long tiles_w = static_cast<long long>(num_m) *
+                              (c.op == Op::SwiGLU ? (c.I + 255) / 256 : (c.N + fnl::k2w::BN - 1) / fnl::k2w::BN);
+    // estimated time = waves x time of one tile; a 128 x 512 tile takes about
+    // 1.6x a 128 x 256 tile (measured on B200 across the prefill shapes)
+    auto waves = [&](long long tiles) {
+      const long long g = std::min<long long>(max_ctas, tiles);
+      return static_cast<double>((tiles + g - 1) / g);
+    };
+    wide = waves(tiles_w) * 1.6 <= waves(tiles_n);
+    if (h->opt.path == FNL_PATH_TILE) wide = false;
+    if (h->opt.path == FNL_PATH_TILE_WIDE) wide = true;
+    const long long tiles = wide ? tiles_w : tiles_n;
     grid = static_cast<int>(std::min<long long>(max_ctas, tiles));
-    smem = fnl::k2::SMEM_BYTES;
-    threads = fnl::k2::NUM_THREADS;
+    smem = wide ? fnl::k2w::SMEM_BYTES : fnl::k2::SMEM_BYTES;
+    threads = wide ? fnl::k2w::NUM_THREADS : fnl::k2::NUM_THREADS;
   }
 
   // workspace
@@ -333,10 +357,12 @@ fnl_status run(fnl_handle* h, const Call& c) {
   const int act_rows = small ? mpad : fnl::k2::BM;
   int w_rows;
   if (small) w_rows = c.op == Op::SwiGLU ? 64 : fnl::k3::BW;
+  else if (wide) w_rows = 256;
   else w_rows = c.op == Op::SwiGLU ? 128 : fnl::k2::BN;
-  if ((st = make_map(h, &mx, c.x, c.M, c.K, act_rows)) != FNL_OK) return st;
-  if ((st = make_map(h, &mr, c.residual, c.M, c.K, act_rows)) != FNL_OK) return st;
-  if ((st = make_map(h, &mw, c.W, c.N, c.K, w_rows)) != FNL_OK) return st;
+  const int box_cols = wide ? fnl::k2w::BK : 64;
+  if ((st = make_map(h, &mx, c.x, c.M, c.K, act_rows, box_cols)) != FNL_OK) return st;
+  if ((st = make_map(h, &mr, c.residual, c.M, c.K, act_rows, box_cols)) != FNL_OK) return st;
+  if ((st = make_map(h, &mw, c.W, c.N, c.K, w_rows, box_cols)) != FNL_OK) return st;
 
   if (!rms) {
     if ((st = launch_k1(h, c, stats, c.stream)) != FNL_OK) return st;
@@ -347,11 +373,11 @@ fnl_status run(fnl_handle* h, const Call& c) {
   const bool pdl = true;
   switch (epi) {
     case fnl::kEpiQKV:
-      return dispatch_gemm<fnl::kEpiQKV>(h, small, rms, grid, threads, smem, pdl, c.stream, mx, mr, mw, p);
+      return dispatch_gemm<fnl::kEpiQKV>(h, small, rms, grid, threads, smem, pdl, c.stream, mx, mr, mw, p, wide);
     case fnl::kEpiSwiGLU:
-      return dispatch_gemm<fnl::kEpiSwiGLU>(h, small, rms, grid, threads, smem, pdl, c.stream, mx, mr, mw, p);
+      return dispatch_gemm<fnl::kEpiSwiGLU>(h, small, rms, grid, threads, smem, pdl, c.stream, mx, mr, mw, p, wide);
     default:
-      return dispatch_gemm<fnl::kEpiGELU>(h, small, rms, grid, threads, smem, pdl, c.stream, mx, mr, mw, p);
+      return dispatch_gemm<fnl::kEpiGELU>(h, small, rms, grid, threads, smem, pdl, c.stream, mx, mr, mw, p, wide);
   }
 }
 
@@ -367,7 +393,7 @@ fnl_status fnl_create(fnl_handle** out, int device, const fnl_options* opt) {
   *out = nullptr;
   fnl_handle* h = new fnl_handle();
   if (opt) h->opt = *opt;
-  if (h->opt.path < FNL_PATH_AUTO || h->opt.path > FNL_PATH_SPLITK || h->opt.max_tokens < 0 || h->opt.max_n < 0 ||
+  if (h->opt.path < FNL_PATH_AUTO || h->opt.path > FNL_PATH_TILE_WIDE || h->opt.max_tokens < 0 || h->opt.max_n < 0 ||
       h->opt.precision < FNL_PRECISION_DEFAULT || h->opt.precision > FNL_PRECISION_SINGLE) {
     delete h;
     return FNL_ERR_INVALID_ARG;

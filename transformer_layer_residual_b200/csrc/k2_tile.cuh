@@ -1,7 +1,7 @@
 // K2: large-M fused norm + GEMM + epilogue, persistent, one CTA per SM.
 //
 // Tile: 128 tokens x 256 W rows (SwiGLU: 128 gate rows + the matching 128 up
-// rows), K in blocks of 64. Warp roles (14 warps):
+// rows), K in blocks of 64. Warp roles (18 warps):
 //   warp 0      TMA producer: per k-block, x and residual tiles [128 x 64] and
 //               the W tile [256 x 64], 128-byte swizzled, into one of 3 stages;
 //   warp 1      TMEM owner and UMMA issuer (one thread): 4 x
@@ -10,7 +10,7 @@
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator (lane = token row),
 //               deferred RMSNorm scale, bias, QKV head-major split / SwiGLU /
 //               GELU, bf16 stores straight to the outputs;
-//   warps 6-13  converters: in place in shared memory, turn the x tile into the
+//   warps 6-17  converters: in place in shared memory, turn the x tile into the
 //               normalised bf16 A operand a = norm(x + r (+ bias_in)) using the
 //               residual tile, so the normalised activations never touch global
 //               memory (the "shared memory caching of normalised values /
@@ -36,8 +36,10 @@ constexpr int X_BYTES = BM * BK * 2;                 // 16 KB
 constexpr int W_BYTES = BN * BK * 2;                 // 32 KB
 constexpr int STAGE_BYTES = 2 * X_BYTES + W_BYTES;   // 64 KB
 constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_EPI0 = 2, NUM_EPI_WARPS = 4;
-constexpr int WARP_CONV0 = 6, NUM_CONV_WARPS = 8;
-constexpr int NUM_THREADS = (WARP_CONV0 + NUM_CONV_WARPS) * 32;   // 448
+constexpr int WARP_CONV0 = 6, NUM_CONV_WARPS = 12;
+constexpr int ROW_STRIDE = NUM_CONV_WARPS * 32 / 8;              // rows between a thread's rows
+constexpr int ROWS_PER_THREAD = (BM + ROW_STRIDE - 1) / ROW_STRIDE;   // 3
+constexpr int NUM_THREADS = (WARP_CONV0 + NUM_CONV_WARPS) * 32;   // 576
 constexpr int TMEM_COLS = 2 * BN;                                  // 512
 constexpr int GROUP_M = 16;  // tile raster: 16 M-blocks share each W tile while it is hot in L2
 
@@ -317,9 +319,10 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ converters
-    const int ct = threadIdx.x - WARP_CONV0 * 32;   // 0..255
+    const int ct = threadIdx.x - WARP_CONV0 * 32;   // 0 .. NUM_CONV_WARPS*32-1
     const int c = ct & 7;                            // 16-byte chunk of the 128-byte row
-    const int rbase = ct >> 3;                       // rows rbase + 32 j
+    const int rbase = ct >> 3;                       // rows rbase + ROW_STRIDE j (< BM)
+    constexpr int RPT = ROWS_PER_THREAD;
     if (NORM == kLayerNorm) pdl_wait();              // statistics come from the previous kernel
     uint32_t s = 0, ph = 0;
     int i = 0;
@@ -327,11 +330,12 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
     for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++i) {
       int mb, nb;
       tile_coords(t, num_m, num_n, mb, nb);
-      float mu[4], rs[4], ss[4];
+      float mu[RPT], rs[RPT];
+      f32x2 ss[RPT];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int gm = mb * BM + rbase + 32 * j;
-        ss[j] = 0.f;
+      for (int j = 0; j < RPT; ++j) {
+        const int gm = mb * BM + rbase + ROW_STRIDE * j;
+        ss[j] = 0ull;
         mu[j] = 0.f;
         rs[j] = 0.f;
         if (NORM == kLayerNorm && gm < M) {
@@ -348,50 +352,39 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
         }
         const int k0 = kb * BK + c * 8;
         const bool kin = k0 < K;
-        float g[8], be[8], bi[8];
+        f32x2 g2[4], be2[4], bi2[4];
         const bf16* vec = vecs + s * 3 * kVecElems;
-        stage_vec8(vec, 0, true, c, kin, g);
-        stage_vec8(vec, 1, has_beta, c, kin, be);
-        stage_vec8(vec, 2, has_bias_in, c, kin, bi);
+        vec_pairs(vec, 0, true, c, kin, g2);
+        vec_pairs(vec, 1, has_beta, c, kin, be2);
+        vec_pairs(vec, 2, has_bias_in, c, kin, bi2);
         const uint32_t xs = smem_u32(smem + s * STAGE_BYTES);
         const uint32_t rsm = xs + X_BYTES;
-        // loads of all four rows first, then arithmetic and stores, so the
-        // four chunks overlap instead of running in series
-        uint4 xv[4], rv[4];
+        // loads of all of this thread's rows first, then arithmetic and stores,
+        // so the chunks overlap instead of running in series
+        uint4 xv[RPT], rv[RPT];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int row = rbase + 32 * j;
-          const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
-          xv[j] = ld_shared_v4(xs + off);
-          rv[j] = ld_shared_v4(rsm + off);
+        for (int j = 0; j < RPT; ++j) {
+          const int row = rbase + ROW_STRIDE * j;
+          if (row < BM) {
+            const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
+            xv[j] = ld_shared_v4(xs + off);
+            rv[j] = ld_shared_v4(rsm + off);
+          }
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int row = rbase + 32 * j;
+        for (int j = 0; j < RPT; ++j) {
+          const int row = rbase + ROW_STRIDE * j;
+          if (row >= BM) continue;
           const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
-          float h[8], rr[8], a[8];
-          unpack8(xv[j], h);
-          unpack8(rv[j], rr);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) h[e] = (h[e] + rr[e]) + bi[e];
-          if (NORM == kLayerNorm) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) a[e] = fmaf((h[e] - mu[j]) * rs[j], g[e], be[e]);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              a[e] = h[e] * g[e];
-              ss[j] = fmaf(h[e], h[e], ss[j]);
-            }
-          }
-          uint4 hi, lo;
-          round_split8(a, split, hi, lo);
+          uint4 hi, lo, hres;
+          convert8<NORM>(xv[j], rv[j], g2, be2, bi2, has_beta, has_bias_in, mu[j], rs[j], split, write_res, ss[j], hi, lo,
+                         hres);
           st_shared_v4(xs + off, hi);
           if (split) st_shared_v4(rsm + off, lo);   // residual chunk already consumed by this thread
           if (write_res) {
             const int gm = mb * BM + row;
             if (gm < M && kin)
-              *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(gm) * K + k0) = pack8(h);
+              *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(gm) * K + k0) = hres;
           }
         }
         fence_proxy_async_smem();
@@ -404,20 +397,25 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
       }
       if (!ok) break;
       if (NORM == kRMSNorm) {
+        float sst[RPT];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], 1);
-          ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], 2);
-          ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], 4);
+        for (int j = 0; j < RPT; ++j) {
+          float lo_, hi_;
+          unpk2(ss[j], lo_, hi_);
+          sst[j] = lo_ + hi_;
+          sst[j] += __shfl_xor_sync(0xffffffffu, sst[j], 1);
+          sst[j] += __shfl_xor_sync(0xffffffffu, sst[j], 2);
+          sst[j] += __shfl_xor_sync(0xffffffffu, sst[j], 4);
         }
         const int b = i & 1;
         const uint32_t use = static_cast<uint32_t>(i >> 1);
         if (!warp_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty)) break;
         if (c == 0) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int row = rbase + 32 * j;
-            const float r = 1.f / sqrtf(ss[j] / static_cast<float>(K) + p.eps);
+          for (int j = 0; j < RPT; ++j) {
+            const int row = rbase + ROW_STRIDE * j;
+            if (row >= BM) continue;
+            const float r = 1.f / sqrtf(sst[j] / static_cast<float>(K) + p.eps);
             ctrl->rs[b][row] = r;
             const int gm = mb * BM + row;
             if (write_res && p.rstd_out != nullptr && gm < M) p.rstd_out[gm] = r;

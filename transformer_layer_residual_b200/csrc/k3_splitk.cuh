@@ -467,7 +467,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     bool ok = true;
     while (ok && it.next(t, kb0, nk, slot, nseg)) {
       const int b = i & 1;
-      float sq[4] = {0.f, 0.f, 0.f, 0.f};   // this warp's share of the segment's sum(h^2) per row
+      f32x2 sq[4] = {0ull, 0ull, 0ull, 0ull};   // this warp's share of the segment's sum(h^2) per row
       const bool write_res = (NORM == kRMSNorm) && t == 0;
       for (; cq < pos + nk; cq += NUM_CONV_WARPS) {
         const int q = cq;
@@ -494,7 +494,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
           const int row = rb + rpp * j;
           if (j < npass && row < M) {
             for (int c0 = 0; c0 < cpl; c0 += 4) {
-              uint4 xv[4], rv[4], gv[4], bev[4], biv[4];
+              uint4 xv[4], rv[4];
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
                 if (c0 + u < cpl) {
@@ -502,9 +502,6 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
                   const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
                   xv[u] = ld_shared_v4(xs + off);
                   rv[u] = ld_shared_v4(rsm + off);
-                  gv[u] = ld_shared_v4(smem_u32(vec + c * 8));
-                  if (has_beta) bev[u] = ld_shared_v4(smem_u32(vec + kVecElems + c * 8));
-                  if (has_bias_in) biv[u] = ld_shared_v4(smem_u32(vec + 2 * kVecElems + c * 8));
                 }
               }
 #pragma unroll
@@ -514,35 +511,17 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
                   const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
                   const int kk0 = kb * BK + c * 8;
                   const bool kin = kk0 < K;
-                  float h[8], rr[8], g[8], be[8], bi[8], a[8];
-                  unpack8(xv[u], h);
-                  unpack8(rv[u], rr);
-                  unpack8(gv[u], g);
-                  if (has_beta) unpack8(bev[u], be);
-                  if (has_bias_in) unpack8(biv[u], bi);
-#pragma unroll
-                  for (int e = 0; e < 8; ++e) {
-                    if (!kin) g[e] = 0.f;
-                    if (!has_beta || !kin) be[e] = 0.f;
-                    if (!has_bias_in || !kin) bi[e] = 0.f;
-                    h[e] = (h[e] + rr[e]) + bi[e];
-                  }
-                  if (NORM == kLayerNorm) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) a[e] = fmaf((h[e] - mu[j]) * rs[j], g[e], be[e]);
-                  } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                      a[e] = h[e] * g[e];
-                      sq[j] = fmaf(h[e], h[e], sq[j]);
-                    }
-                  }
-                  uint4 hi, lo;
-                  round_split8(a, split, hi, lo);
+                  f32x2 g2[4], be2[4], bi2[4];
+                  vec_pairs(vec, 0, true, c, kin, g2);
+                  vec_pairs(vec, 1, has_beta, c, kin, be2);
+                  vec_pairs(vec, 2, has_bias_in, c, kin, bi2);
+                  uint4 hi, lo, hres;
+                  convert8<NORM>(xv[u], rv[u], g2, be2, bi2, has_beta, has_bias_in, mu[j], rs[j], split, write_res, sq[j], hi,
+                                 lo, hres);
                   st_shared_v4(xs + off, hi);
                   if (split) st_shared_v4(rsm + off, lo);
                   if (write_res && kin)
-                    *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(row) * K + kk0) = pack8(h);
+                    *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(row) * K + kk0) = hres;
                 }
               }
             }
@@ -560,9 +539,12 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
         if (!warp_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty)) break;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          for (int o = 1; o < L; o <<= 1) sq[j] += __shfl_xor_sync(0xffffffffu, sq[j], o);
+          float lo_, hi_;
+          unpk2(sq[j], lo_, hi_);
+          float t = lo_ + hi_;
+          for (int o = 1; o < L; o <<= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
           const int row = rb + rpp * j;
-          if (cf == 0 && j < npass && row < M) ctrl->ssw[b][cw][row] = sq[j];
+          if (cf == 0 && j < npass && row < M) ctrl->ssw[b][cw][row] = t;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->sfull[b]);
