@@ -84,13 +84,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
-// One lane waits, the warp agrees on the outcome.
+// The whole warp waits: every lane polls the barrier in the same warp-wide
+// instruction and each decision is a warp vote, so the warp leaves the wait
+// converged. (Had one lane spun while the others parked on a shuffle, the warp
+// could stay split into two groups that the scheduler runs one after the other,
+// which doubles the cost of all the warp-wide work that follows the wait.)
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           int* status, int code) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, status, code) ? 1 : 0;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  return ok != 0;
+  constexpr unsigned kAll = 0xffffffffu;
+  if (__any_sync(kAll, mbar_try_wait(bar, parity))) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (__any_sync(kAll, mbar_try_wait(bar, parity))) return true;
+    if (__any_sync(kAll, *abort_flag != 0)) return false;
+    if (__any_sync(kAll, globaltimer() - t0 > FNL_WAIT_NS)) {
+      if ((threadIdx.x & 31) == 0) {
+        *abort_flag = 1;
+        if (status) atomicCAS(status, 0, code);
+      }
+      __syncwarp();
+      return false;
+    }
+  }
 }
 
 // ---------------------------------------------------------------- TMA
