@@ -15,11 +15,13 @@ struct OpParams {
   int I;             // SwiGLU intermediate size (N = 2I)
   int Hq, Hkv, D;    // QKV heads
   float eps;
+  const bf16* x_in;      // x and residual [M][K] (read directly by the small-M kernel's
+  const bf16* r_in;      // residual_out writers; the GEMM operands come through tensor maps)
   const bf16* gamma;
   const bf16* beta;      // LayerNorm shift, may be null
   const bf16* bias_in;   // [K], may be null
   const bf16* bias;      // [N] output bias, may be null
-  bf16* residual_out;    // written in the GEMM kernels for RMSNorm, by the stats kernel for LayerNorm
+  bf16* residual_out;    // written in the GEMM kernels for RMSNorm, by the statistics kernel for LayerNorm
   float* rstd_out;       // RMSNorm statistics output (GEMM kernels), may be null
   const float2* stats;   // LayerNorm (mean, rstd) per row, written by the stats kernel
   bf16* q;
@@ -39,18 +41,6 @@ struct OpParams {
 
 __device__ __forceinline__ uint4 ldg16(const void* p) {
   return __ldg(reinterpret_cast<const uint4*>(p));
-}
-
-// Round a[8] to bf16 (hi) and, if `split`, also the remainder a - hi to bf16 (lo).
-__device__ __forceinline__ void round_split8(const float (&a)[8], bool split, uint4& hi, uint4& lo) {
-  hi = pack8(a);
-  if (split) {
-    float h[8], r[8];
-    unpack8(hi, h);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) r[e] = a[e] - h[e];
-    lo = pack8(r);
-  }
 }
 
 // Per-stage copies of the k-block's slices of gamma, beta and bias_in
@@ -83,27 +73,52 @@ __device__ __forceinline__ uint32_t vec_bytes(const OpParams& p, bool has_beta, 
   return static_cast<uint32_t>(kvalid) * 2 * (1 + (has_beta ? 1 : 0) + (has_bias_in ? 1 : 0));
 }
 
-// The converter's 8 gamma / beta / bias_in values of chunk c from the stage copy.
-__device__ __forceinline__ void stage_vec8(const bf16* vec, int which, bool present, int c, bool kin,
-                                           float (&f)[8]) {
-  if (present && kin) {
-    unpack8(ld_shared_v4(smem_u32(vec + which * kVecElems + c * 8)), f);
-  } else {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) f[e] = 0.f;
+// Compile-time flag for code specialised on a condition that is uniform over a
+// stage (a generic lambda takes it as its argument type).
+template <bool B>
+struct BoolC {
+  static constexpr bool value = B;
+};
+
+// Set elements [from, n) of the three per-stage vector slices (gamma, beta,
+// bias_in; n elements apart) to zero. Called by a converter warp on the last
+// k-block when K is not a multiple of the k-block: the slices' loads covered only
+// the first K - k0 elements, and with zeros there the columns past K (whose x,
+// residual and W entries the tensor copies fill with zeros) give exactly a = 0
+// and h = 0, so the chunk loops need no bounds test.
+__device__ __forceinline__ void zero_vec_tails(bf16* vec, int n, int from) {
+  uint16_t* v = reinterpret_cast<uint16_t*>(vec);
+  for (int i = from + static_cast<int>(threadIdx.x & 31); i < n; i += 32) {
+    v[i] = 0;
+    v[n + i] = 0;
+    v[2 * n + i] = 0;
   }
+  __syncwarp();
+}
+
+// Zero all per-stage vector slices once, before the first copy into them, so a
+// slice whose vector the call does not have (beta, bias_in) reads as zeros.
+// All threads of the block; the proxy fence orders these stores before the
+// tensor-copy engine's later writes to the same words.
+__device__ __forceinline__ void zero_vec_slices(bf16* vecs, int elems) {
+  uint16_t* v = reinterpret_cast<uint16_t*>(vecs);
+  for (int i = threadIdx.x; i < elems; i += blockDim.x) v[i] = 0;
+  fence_proxy_async_smem();
 }
 
 // 8 consecutive elements of one token row: h = x + r (+ bias_in) in fp32,
-// a = normalise(h) rounded to bf16 (hi) and, if split, the bf16 remainder (lo).
-// LayerNorm: a = (h - mean) * rstd * gamma + beta. RMSNorm (deferred scale):
-// a = h * gamma and sq += h^2 (even and odd elements in the two lanes).
+// a = normalise(h) rounded to bf16 (hi) and, with SPLIT, the bf16 remainder a - hi
+// (lo); with WANT_H also bf16(h) for residual_out.
+// LayerNorm: a = (h - mean) * rstd * gamma + beta (beta = 0 when absent).
+// RMSNorm (deferred scale): a = h * gamma and sq += h^2 (even and odd elements
+// in the two lanes of the pair).
 // g, be, bi: the chunk's gamma / beta / bias_in as four fp32 pairs.
-template <int NORM>
+// Every choice is a template parameter, so the converter loops carry no
+// per-element branches.
+template <int NORM, bool BIAS_IN, bool SPLIT, bool WANT_H>
 __device__ __forceinline__ void convert8(const uint4& xv, const uint4& rv, const f32x2 (&g)[4], const f32x2 (&be)[4],
-                                         const f32x2 (&bi)[4], bool has_beta, bool has_bias_in, float mean,
-                                         float rstd, bool split, bool want_h, f32x2& sq, uint4& hi, uint4& lo,
-                                         uint4& hres) {
+                                         const f32x2 (&bi)[4], float mean, float rstd, f32x2& sq, uint4& hi,
+                                         uint4& lo, uint4& hres) {
   const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
   const uint32_t rw[4] = {rv.x, rv.y, rv.z, rv.w};
   uint32_t ho[4], lw[4], hw[4];
@@ -111,37 +126,30 @@ __device__ __forceinline__ void convert8(const uint4& xv, const uint4& rv, const
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     f32x2 h = add2(bf2_to_f2(xw[i]), bf2_to_f2(rw[i]));
-    if (has_bias_in) h = add2(h, bi[i]);
+    if (BIAS_IN) h = add2(h, bi[i]);
     f32x2 a;
     if (NORM == kLayerNorm) {
-      a = mul2(sub2(h, mu2), rs2);
-      a = has_beta ? fma2(a, g[i], be[i]) : mul2(a, g[i]);
+      a = fma2(mul2(sub2(h, mu2), rs2), g[i], be[i]);
     } else {
       a = mul2(h, g[i]);
       sq = fma2(h, h, sq);
     }
     ho[i] = f2_to_bf2(a);
-    if (split) lw[i] = f2_to_bf2(sub2(a, bf2_to_f2(ho[i])));
-    if (want_h) hw[i] = f2_to_bf2(h);
+    if (SPLIT) lw[i] = f2_to_bf2(sub2(a, bf2_to_f2(ho[i])));
+    if (WANT_H) hw[i] = f2_to_bf2(h);
   }
   hi = make_uint4(ho[0], ho[1], ho[2], ho[3]);
-  if (split) lo = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-  if (want_h) hres = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  if (SPLIT) lo = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  if (WANT_H) hres = make_uint4(hw[0], hw[1], hw[2], hw[3]);
 }
 
-// A 16-byte vector of 8 bf16 as four fp32 pairs (zeros when absent).
-__device__ __forceinline__ void vec_pairs(const bf16* vec, int which, bool present, int c, bool kin,
-                                          f32x2 (&f)[4]) {
-  if (present && kin) {
-    const uint4 v = ld_shared_v4(smem_u32(vec + which * kVecElems + c * 8));
-    f[0] = bf2_to_f2(v.x);
-    f[1] = bf2_to_f2(v.y);
-    f[2] = bf2_to_f2(v.z);
-    f[3] = bf2_to_f2(v.w);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) f[i] = 0ull;
-  }
+// The 8 bf16 at a 16-byte aligned shared-memory address as four fp32 pairs.
+__device__ __forceinline__ void vec_pairs(uint32_t addr, f32x2 (&f)[4]) {
+  const uint4 v = ld_shared_v4(addr);
+  f[0] = bf2_to_f2(v.x);
+  f[1] = bf2_to_f2(v.y);
+  f[2] = bf2_to_f2(v.z);
+  f[3] = bf2_to_f2(v.w);
 }
 
 __device__ __forceinline__ void load8_or_zero(const bf16* base, int k0, bool ok, float (&f)[8]) {

@@ -234,23 +234,37 @@ fnl_status launch_gemm(fnl_handle* h, Kern kern, int grid, int threads, int smem
   return FNL_OK;
 }
 
+template <int EPI, bool SPLIT>
+fnl_status dispatch_gemm_p(fnl_handle* h, bool small, bool rms, int grid, int threads, int smem, bool pdl,
+                           cudaStream_t stream, const CUtensorMap& mx, const CUtensorMap& mr, const CUtensorMap& mw,
+                           const OpParams& p, bool wide) {
+  using fnl::kLayerNorm;
+  using fnl::kRMSNorm;
+  if (wide) {
+    if (rms)
+      return launch_gemm(h, fnl::k2w_tile_kernel<EPI, kRMSNorm, SPLIT>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
+    return launch_gemm(h, fnl::k2w_tile_kernel<EPI, kLayerNorm, SPLIT>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
+  }
+  if (small) {
+    if (rms)
+      return launch_gemm(h, fnl::k3_splitk_kernel<EPI, kRMSNorm, SPLIT>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
+    return launch_gemm(h, fnl::k3_splitk_kernel<EPI, kLayerNorm, SPLIT>, grid, threads, smem, pdl, stream, mx, mr, mw,
+                       p);
+  }
+  if (rms)
+    return launch_gemm(h, fnl::k2_tile_kernel<EPI, kRMSNorm, SPLIT>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
+  return launch_gemm(h, fnl::k2_tile_kernel<EPI, kLayerNorm, SPLIT>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
+}
+
+// The operand precision (p.split) selects the kernel instantiation: the hi/lo
+// split is a template parameter of every GEMM kernel, so their converter loops
+// carry no branch on it.
 template <int EPI>
 fnl_status dispatch_gemm(fnl_handle* h, bool small, bool rms, int grid, int threads, int smem, bool pdl,
                          cudaStream_t stream, const CUtensorMap& mx, const CUtensorMap& mr, const CUtensorMap& mw,
                          const OpParams& p, bool wide = false) {
-  if (wide) {
-    if (rms)
-      return launch_gemm(h, fnl::k2w_tile_kernel<EPI, fnl::kRMSNorm>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
-    return launch_gemm(h, fnl::k2w_tile_kernel<EPI, fnl::kLayerNorm>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
-  }
-  if (small) {
-    if (rms)
-      return launch_gemm(h, fnl::k3_splitk_kernel<EPI, fnl::kRMSNorm>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
-    return launch_gemm(h, fnl::k3_splitk_kernel<EPI, fnl::kLayerNorm>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
-  }
-  if (rms)
-    return launch_gemm(h, fnl::k2_tile_kernel<EPI, fnl::kRMSNorm>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
-  return launch_gemm(h, fnl::k2_tile_kernel<EPI, fnl::kLayerNorm>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
+  if (p.split) return dispatch_gemm_p<EPI, true>(h, small, rms, grid, threads, smem, pdl, stream, mx, mr, mw, p, wide);
+  return dispatch_gemm_p<EPI, false>(h, small, rms, grid, threads, smem, pdl, stream, mx, mr, mw, p, wide);
 }
 
 fnl_status launch_k1(fnl_handle* h, const Call& c, float2* stats, cudaStream_t stream) {
@@ -344,6 +358,7 @@ fnl_status run(fnl_handle* h, const Call& c) {
 
   OpParams p{};
   p.M = c.M; p.K = c.K; p.N = c.N; p.I = c.I; p.Hq = c.Hq; p.Hkv = c.Hkv; p.D = c.D; p.eps = c.eps;
+  p.x_in = c.x; p.r_in = c.residual;
   p.gamma = c.gamma; p.beta = c.beta; p.bias_in = c.bias_in; p.bias = c.bias;
   p.residual_out = c.residual_out; p.rstd_out = rms ? c.rstd_out : nullptr; p.stats = stats;
   p.q = c.q; p.k = c.k; p.v = c.v; p.out = c.out;
@@ -657,6 +672,7 @@ extern "C" fnl_status fnl_add_norm_qkv_static(fnl_stream stream, const fnl_bf16*
 
   OpParams p{};
   p.M = c.M; p.K = c.K; p.N = c.N; p.I = 0; p.Hq = c.Hq; p.Hkv = c.Hkv; p.D = c.D; p.eps = c.eps;
+  p.x_in = c.x; p.r_in = c.residual;
   p.gamma = c.gamma; p.beta = c.beta; p.bias_in = nullptr; p.bias = c.bias;
   p.residual_out = c.residual_out; p.rstd_out = rms ? c.rstd_out : nullptr;
   p.stats = reinterpret_cast<const float2*>(base + zero_bytes);

@@ -73,7 +73,7 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
 
 }  // namespace k2
 
-template <int EPI, int NORM>
+template <int EPI, int NORM, bool SPLIT>
 __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
     k2_tile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_r,
                    const __grid_constant__ CUtensorMap tm_w, const OpParams p) {
@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
   const int num_n = (EPI == kEpiSwiGLU) ? (p.I + 127) / 128 : (p.N + BN - 1) / BN;
   const int tiles = num_m * num_n;
   const int nkb = (K + BK - 1) / BK;
-  const bool split = p.split != 0;
+  constexpr bool BIAS_IN = EPI == kEpiGELU;   // only the GELU entry point has a bias_in
 
   if (threadIdx.x == 0) {
     pdl_launch_dependents();   // the next call's CTAs may take SMs as ours retire
@@ -119,6 +119,7 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
     tmem_alloc(&ctrl->tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
+  zero_vec_slices(vecs, STAGES * 3 * kVecElems);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -225,7 +226,7 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
             umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
-          if (split) {   // + lo(a) W^T into the same accumulator
+          if (SPLIT) {   // + lo(a) W^T into the same accumulator
             const uint64_t ld = sw128_desc(xa + X_BYTES);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) umma_bf16(d, ld + 2 * kk, bd + 2 * kk, idesc, 1u);
@@ -350,13 +351,13 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
           ok = false;
           break;
         }
-        const int k0 = kb * BK + c * 8;
-        const bool kin = k0 < K;
-        f32x2 g2[4], be2[4], bi2[4];
-        const bf16* vec = vecs + s * 3 * kVecElems;
-        vec_pairs(vec, 0, true, c, kin, g2);
-        vec_pairs(vec, 1, has_beta, c, kin, be2);
-        vec_pairs(vec, 2, has_bias_in, c, kin, bi2);
+        bf16* vec = vecs + s * 3 * kVecElems;
+        if (K - kb * BK < BK) zero_vec_tails(vec, kVecElems, K - kb * BK);
+        const uint32_t vaddr = smem_u32(vec) + c * 16;
+        f32x2 g2[4], be2[4] = {}, bi2[4] = {};
+        vec_pairs(vaddr, g2);
+        if (NORM == kLayerNorm) vec_pairs(vaddr + 2 * kVecElems, be2);
+        if (BIAS_IN) vec_pairs(vaddr + 4 * kVecElems, bi2);
         const uint32_t xs = smem_u32(smem + s * STAGE_BYTES);
         const uint32_t rsm = xs + X_BYTES;
         // loads of all of this thread's rows first, then arithmetic and stores,
@@ -371,22 +372,28 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
             rv[j] = ld_shared_v4(rsm + off);
           }
         }
+        // instantiated with and without the residual_out store (first N column)
+        auto convert_stage = [&](auto wres_tag) {
+          constexpr bool WRES = decltype(wres_tag)::value;
 #pragma unroll
-        for (int j = 0; j < RPT; ++j) {
-          const int row = rbase + ROW_STRIDE * j;
-          if (row >= BM) continue;
-          const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
-          uint4 hi, lo, hres;
-          convert8<NORM>(xv[j], rv[j], g2, be2, bi2, has_beta, has_bias_in, mu[j], rs[j], split, write_res, ss[j], hi, lo,
-                         hres);
-          st_shared_v4(xs + off, hi);
-          if (split) st_shared_v4(rsm + off, lo);   // residual chunk already consumed by this thread
-          if (write_res) {
-            const int gm = mb * BM + row;
-            if (gm < M && kin)
-              *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(gm) * K + k0) = hres;
+          for (int j = 0; j < RPT; ++j) {
+            const int row = rbase + ROW_STRIDE * j;
+            if (row >= BM) continue;
+            const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
+            uint4 hi, lo, hres;
+            convert8<NORM, BIAS_IN, SPLIT, WRES>(xv[j], rv[j], g2, be2, bi2, mu[j], rs[j], ss[j], hi, lo, hres);
+            st_shared_v4(xs + off, hi);
+            if (SPLIT) st_shared_v4(rsm + off, lo);   // residual chunk already consumed by this thread
+            if (WRES) {
+              const int gm = mb * BM + row;
+              const int k0 = kb * BK + c * 8;
+              if (gm < M && k0 < K)
+                *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(gm) * K + k0) = hres;
+            }
           }
-        }
+        };
+        if (write_res) convert_stage(BoolC<true>{});
+        else convert_stage(BoolC<false>{});
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->conv[s]);

@@ -77,7 +77,7 @@ __device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr) {
 
 }  // namespace k2w
 
-template <int EPI, int NORM>
+template <int EPI, int NORM, bool SPLIT>
 __global__ void __launch_bounds__(k2w::NUM_THREADS, 1)
     k2w_tile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_r,
                     const __grid_constant__ CUtensorMap tm_w, const OpParams p) {
@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(k2w::NUM_THREADS, 1)
   const int num_n = (EPI == kEpiSwiGLU) ? (p.I + 255) / 256 : (p.N + BN - 1) / BN;
   const int tiles = num_m * num_n;
   const int nkb = (K + BK - 1) / BK;
-  const bool split = p.split != 0;
+  constexpr bool BIAS_IN = EPI == kEpiGELU;   // only the GELU entry point has a bias_in
 
   if (threadIdx.x == 0) {
     pdl_launch_dependents();
@@ -121,6 +121,7 @@ __global__ void __launch_bounds__(k2w::NUM_THREADS, 1)
     tmem_alloc(&ctrl->tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
+  zero_vec_slices(vecs, STAGES * 3 * VEC);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -233,7 +234,7 @@ __global__ void __launch_bounds__(k2w::NUM_THREADS, 1)
             const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
             umma_bf16(tmem, ad + 2 * kk, bd0 + 2 * kk, idesc, acc);
             umma_bf16(tmem + 256, ad + 2 * kk, bd1 + 2 * kk, idesc, acc);
-            if (split) {   // + lo(a) W^T into the same accumulators
+            if (SPLIT) {   // + lo(a) W^T into the same accumulators
               umma_bf16(tmem, ld + 2 * kk, bd0 + 2 * kk, idesc, 1u);
               umma_bf16(tmem + 256, ld + 2 * kk, bd1 + 2 * kk, idesc, 1u);
             }
@@ -358,25 +359,13 @@ __global__ void __launch_bounds__(k2w::NUM_THREADS, 1)
           ok = false;
           break;
         }
-        const int k0 = kb * BK + c * 8;
-        const bool kin = k0 < K;
-        const bf16* vec = vecs + s * 3 * VEC;
-        f32x2 g2[4], be2[4], bi2[4];
-        auto pairs = [&](int which, bool present, f32x2 (&f)[4]) {
-          if (present && kin) {
-            const uint4 v = ld_shared_v4(smem_u32(vec + which * VEC + c * 8));
-            f[0] = bf2_to_f2(v.x);
-            f[1] = bf2_to_f2(v.y);
-            f[2] = bf2_to_f2(v.z);
-            f[3] = bf2_to_f2(v.w);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) f[e] = 0ull;
-          }
-        };
-        pairs(0, true, g2);
-        pairs(1, has_beta, be2);
-        pairs(2, has_bias_in, bi2);
+        bf16* vec = vecs + s * 3 * VEC;
+        if (K - kb * BK < BK) zero_vec_tails(vec, VEC, K - kb * BK);
+        const uint32_t vaddr = smem_u32(vec) + c * 16;
+        f32x2 g2[4], be2[4] = {}, bi2[4] = {};
+        vec_pairs(vaddr, g2);
+        if (NORM == kLayerNorm) vec_pairs(vaddr + 2 * VEC, be2);
+        if (BIAS_IN) vec_pairs(vaddr + 4 * VEC, bi2);
         const uint32_t xs = smem_u32(smem + s * STAGE_BYTES);
         const uint32_t rsm = xs + X_BYTES;
         uint4 xv[2], rv[2];
@@ -387,21 +376,27 @@ __global__ void __launch_bounds__(k2w::NUM_THREADS, 1)
           xv[j] = ld_shared_v4(xs + off);
           rv[j] = ld_shared_v4(rsm + off);
         }
+        // instantiated with and without the residual_out store (first N column)
+        auto convert_stage = [&](auto wres_tag) {
+          constexpr bool WRES = decltype(wres_tag)::value;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int row = rbase + 64 * j;
-          const uint32_t off = row * 64 + ((c ^ ((row >> 1) & 3)) << 4);
-          uint4 hi, lo, hres;
-          convert8<NORM>(xv[j], rv[j], g2, be2, bi2, has_beta, has_bias_in, mu[j], rs[j], split, write_res, ss[j],
-                         hi, lo, hres);
-          st_shared_v4(xs + off, hi);
-          if (split) st_shared_v4(rsm + off, lo);
-          if (write_res) {
-            const int gm = mb * BM + row;
-            if (gm < M && kin)
-              *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(gm) * K + k0) = hres;
+          for (int j = 0; j < 2; ++j) {
+            const int row = rbase + 64 * j;
+            const uint32_t off = row * 64 + ((c ^ ((row >> 1) & 3)) << 4);
+            uint4 hi, lo, hres;
+            convert8<NORM, BIAS_IN, SPLIT, WRES>(xv[j], rv[j], g2, be2, bi2, mu[j], rs[j], ss[j], hi, lo, hres);
+            st_shared_v4(xs + off, hi);
+            if (SPLIT) st_shared_v4(rsm + off, lo);
+            if (WRES) {
+              const int gm = mb * BM + row;
+              const int k0 = kb * BK + c * 8;
+              if (gm < M && k0 < K)
+                *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(gm) * K + k0) = hres;
+            }
           }
-        }
+        };
+        if (write_res) convert_stage(BoolC<true>{});
+        else convert_stage(BoolC<false>{});
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->conv[s]);

@@ -186,7 +186,7 @@ __device__ __forceinline__ void k3_reduce_tile(const OpParams& p, int t, int nse
   }
 }
 
-template <int EPI, int NORM>
+template <int EPI, int NORM, bool SPLIT>
 __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     k3_splitk_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_r,
                      const __grid_constant__ CUtensorMap tm_w, const OpParams p) {
@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
   const int T = (EPI == kEpiSwiGLU) ? (p.I + 63) / 64 : (p.N + BW - 1) / BW;
   const int nkb = (K + BK - 1) / BK;
   const uint32_t ncols = tmem_cols(mpad);
-  const bool split = p.split != 0;
+  constexpr bool BIAS_IN = EPI == kEpiGELU;   // only the GELU entry point has a bias_in
 
   const long long U = static_cast<long long>(T) * nkb;
   if (threadIdx.x == 0) {
@@ -239,6 +239,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     tmem_alloc(&ctrl->tmem_base, ncols);
     tmem_relinquish();
   }
+  zero_vec_slices(vecs, S * 3 * kVecElems);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -347,7 +348,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
             umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
-          if (split) {
+          if (SPLIT) {
             const uint64_t ld = sw128_desc(wa + W_BYTES + XB);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) umma_bf16(d, ad + 2 * kk, ld + 2 * kk, idesc, 1u);
@@ -371,6 +372,31 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     const int et = threadIdx.x - WARP_EPI0 * 32;   // 0..127
     const int nl = q * 32 + lane;                  // W row within the tile = TMEM lane
     pdl_wait();   // workspace and outputs may still be in use by the previous kernel
+    if (NORM == kRMSNorm) {
+      // residual_out = bf16(x + r (+ bias_in)), fp32 sum as in the converters:
+      // this CTA's share of the M x K/8 16-byte chunks, written while the
+      // mainloop runs (LayerNorm's comes from the statistics kernel).
+      const int kc = K / 8;
+      const long long nch = static_cast<long long>(M) * kc;
+      const long long ch1 = nch * (blockIdx.x + 1) / gridDim.x;
+      for (long long ch = nch * blockIdx.x / gridDim.x + et; ch < ch1; ch += NUM_EPI_WARPS * 32) {
+        const int m = static_cast<int>(ch / kc);
+        const int k0 = static_cast<int>(ch - static_cast<long long>(m) * kc) * 8;
+        const size_t off = static_cast<size_t>(m) * K + k0;
+        const uint4 xv = ldg16(p.x_in + off), rv = ldg16(p.r_in + off);
+        const uint4 bv = (BIAS_IN && p.bias_in != nullptr) ? ldg16(p.bias_in + k0) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, rw[4] = {rv.x, rv.y, rv.z, rv.w};
+        const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+        uint32_t hw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          f32x2 h = add2(bf2_to_f2(xw[e]), bf2_to_f2(rw[e]));
+          if (BIAS_IN) h = add2(h, bf2_to_f2(bw[e]));
+          hw[e] = f2_to_bf2(h);
+        }
+        *reinterpret_cast<uint4*>(p.residual_out + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      }
+    }
     SegIter it(u0, u1, U, nkb, gridDim.x, blockIdx.x);
     int t, kb0, nk, slot, nseg;
     int i = 0;
@@ -468,7 +494,6 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     while (ok && it.next(t, kb0, nk, slot, nseg)) {
       const int b = i & 1;
       f32x2 sq[4] = {0ull, 0ull, 0ull, 0ull};   // this warp's share of the segment's sum(h^2) per row
-      const bool write_res = (NORM == kRMSNorm) && t == 0;
       for (; cq < pos + nk; cq += NUM_CONV_WARPS) {
         const int q = cq;
         const int s = cs;
@@ -485,7 +510,9 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
         }
         const uint32_t xs = smem_u32(smem + s * SB) + W_BYTES;
         const uint32_t rsm = xs + XB;
-        const bf16* vec = vecs + s * 3 * kVecElems;
+        bf16* vec = vecs + s * 3 * kVecElems;
+        if (K - kb * BK < BK) zero_vec_tails(vec, kVecElems, K - kb * BK);
+        const uint32_t vaddr = smem_u32(vec);
         // For each row slot j of this lane, the lane's chunks of that row in
         // batches of 4: all shared-memory loads of a batch are issued before its
         // arithmetic and stores, so chunks overlap instead of running in series.
@@ -509,19 +536,14 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
                 if (c0 + u < cpl) {
                   const int c = cf + L * (c0 + u);
                   const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
-                  const int kk0 = kb * BK + c * 8;
-                  const bool kin = kk0 < K;
-                  f32x2 g2[4], be2[4], bi2[4];
-                  vec_pairs(vec, 0, true, c, kin, g2);
-                  vec_pairs(vec, 1, has_beta, c, kin, be2);
-                  vec_pairs(vec, 2, has_bias_in, c, kin, bi2);
+                  f32x2 g2[4], be2[4] = {}, bi2[4] = {};
+                  vec_pairs(vaddr + c * 16, g2);
+                  if (NORM == kLayerNorm) vec_pairs(vaddr + 2 * kVecElems + c * 16, be2);
+                  if (BIAS_IN) vec_pairs(vaddr + 4 * kVecElems + c * 16, bi2);
                   uint4 hi, lo, hres;
-                  convert8<NORM>(xv[u], rv[u], g2, be2, bi2, has_beta, has_bias_in, mu[j], rs[j], split, write_res, sq[j], hi,
-                                 lo, hres);
+                  convert8<NORM, BIAS_IN, SPLIT, false>(xv[u], rv[u], g2, be2, bi2, mu[j], rs[j], sq[j], hi, lo, hres);
                   st_shared_v4(xs + off, hi);
-                  if (split) st_shared_v4(rsm + off, lo);
-                  if (write_res && kin)
-                    *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(row) * K + kk0) = hres;
+                  if (SPLIT) st_shared_v4(rsm + off, lo);
                 }
               }
             }
