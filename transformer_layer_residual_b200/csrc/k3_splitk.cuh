@@ -45,6 +45,7 @@ struct Ctrl {
   uint32_t tmem_base;
   int abort_flag;
   int last_flag;
+  int fin_go, fin_t, fin_nseg;   // the CTA's last segment completes its tile: reduced by all warps
   float ssw[2][NUM_CONV_WARPS][MAX_MPAD];   // per converter warp partial sums of h^2 (RMSNorm)
 };
 
@@ -102,14 +103,15 @@ struct SegIter {
 
 // Last-arriving CTA of tile t: out = epilogue(sum over slots 0..nseg-1 of the
 // fp32 partials), summed in slot order so the result does not depend on which
-// CTA arrives last. Each thread takes ITEMS (row, 8-column) items at a time and
+// CTA arrives last. Run by NT threads (et = 0..NT-1): the epilogue warps for a
+// tile that is not the CTA's last, the whole CTA for its last one (nothing else
+// is left to do then). Each thread takes ITEMS (row, 8-column) items at a time and
 // issues the loads of up to 4 slots of all of them before adding, so the
 // reduction costs about one L2 round trip per 4 slots instead of one per slot.
-template <int EPI, int NORM>
+template <int EPI, int NORM, int NT>
 __device__ __forceinline__ void k3_reduce_tile(const OpParams& p, int t, int nseg, int et) {
   using namespace k3;
   constexpr int ITEMS = (EPI == kEpiSwiGLU) ? 1 : 2;
-  constexpr int NT = NUM_EPI_WARPS * 32;
   const int mpad = p.mpad;
   const size_t slot_stride = static_cast<size_t>(mpad) * BW;
   const float* tp = p.part + static_cast<size_t>(t) * p.max_seg * slot_stride;
@@ -228,6 +230,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     mbar_init(&ctrl->esync, NUM_EPI_WARPS);
     ctrl->abort_flag = 0;
     ctrl->last_flag = 0;
+    ctrl->fin_go = 0;
     fence_mbar_init();
   }
   if (warp == WARP_TMA && lane == 0) {
@@ -449,9 +452,17 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
       if (!warp_wait(&ctrl->esync, eph, abortf, p.status, kStatusWaitDrain)) break;
       eph ^= 1;
       if (ctrl->last_flag) {
-        __threadfence();
-        k3_reduce_tile<EPI, NORM>(p, t, nseg, et);
-        if (et == 0) p.counters[t] = 0u;
+        if (it.u >= it.u1) {   // the CTA's last segment: handed to all warps below
+          if (et == 0) {
+            ctrl->fin_t = t;
+            ctrl->fin_nseg = nseg;
+            ctrl->fin_go = 1;
+          }
+        } else {
+          __threadfence();
+          k3_reduce_tile<EPI, NORM, NUM_EPI_WARPS * 32>(p, t, nseg, et);
+          if (et == 0) p.counters[t] = 0u;
+        }
       }
     }
   } else {
@@ -576,6 +587,14 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     }
   }
 
+  // Every role's loop is over (each bounded wait returns), so all warps meet
+  // here; the tile completed by this CTA's last segment is summed by all of them.
+  __syncthreads();
+  if (ctrl->fin_go && *abortf == 0) {
+    __threadfence();
+    k3_reduce_tile<EPI, NORM, NUM_THREADS>(p, ctrl->fin_t, ctrl->fin_nseg, threadIdx.x);
+    if (threadIdx.x == 0) p.counters[ctrl->fin_t] = 0u;
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == WARP_MMA) {
