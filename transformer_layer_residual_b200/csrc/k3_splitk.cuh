@@ -19,9 +19,9 @@
 // x / residual tiles and the gamma / beta / bias_in slices, from L2), so the
 // converters start on a stage as soon as its activations land instead of
 // waiting for its weights. The kernel is launched as a programmatic dependent
-// of the previous kernel on the stream: the producer streams the first stages
-// of W before griddepcontrol.wait and touches activations, workspace and
-// outputs only after it.
+// of the previous kernel on the stream, so its CTAs are resident and set up
+// (barriers, TMEM, tensor maps) when that kernel completes; every global access
+// except the tensor-map prefetch comes after griddepcontrol.wait.
 #pragma once
 
 #include "common.cuh"
@@ -37,6 +37,12 @@ constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_EPI0 = 2, NUM_EPI_WARPS = 4;
 constexpr int WARP_CONV0 = 6, NUM_CONV_WARPS = 4;
 constexpr int NUM_THREADS = (WARP_CONV0 + NUM_CONV_WARPS) * 32;   // 320
 constexpr int MAX_MPAD = 128;
+// Weight stages fetched before griddepcontrol.wait. Zero: back to back, the
+// previous call's tail (partial-sum stores, arrival atomics, the last CTA's
+// reduction) is a chain of dependent L2 round trips, and weight traffic issued
+// during it lengthens the chain by more than it saves (decode 32 x 6144 x 4096:
+// 18.7 us per call with 8 stages, 18.2 with 2, 17.7 with none).
+constexpr int PREWAIT_STAGES = 0;
 
 struct Ctrl {
   uint64_t full_w[MAX_STAGES], full_x[MAX_STAGES], conv[MAX_STAGES], empty[MAX_STAGES];
@@ -297,15 +303,19 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
         armed_x |= 1u << c.s;
         par_x = (par_x & ~(1u << c.s)) | (c.ph << c.s);
       };
-      // Weights of the first stages stream while the previous kernel finishes
-      // (they are never written by it); activations only after it is done.
-      for (int q = 0; q < npre; ++q) {
+      // Weight stages that may stream before griddepcontrol.wait (weights are
+      // never written by the previous kernel; activations are read only after it).
+      const int npre0 = npre < PREWAIT_STAGES ? npre : PREWAIT_STAGES;
+      for (int q = 0; q < npre0; ++q) {
         issue_w(cw);
         step(cw);
       }
       pdl_wait();
       for (int q = 0; q < P; ++q) {
-        if (q >= npre) {
+        if (q >= npre0 && q < npre) {   // the rest of the first ring
+          issue_w(cw);
+          step(cw);
+        } else if (q >= npre) {
           if (!mbar_wait(&ctrl->empty[cw.s], cw.ph ^ 1, abortf, p.status, kStatusWaitEmpty)) {
             ok = false;
             break;
@@ -437,14 +447,18 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
       // arrival: the last CTA of this tile reduces all slots in slot order.
       // The epilogue warps meet on an mbarrier (bounded wait), not bar.sync,
       // so a warp that gave up a wait can never leave the others blocked.
-      __threadfence();
+      // Ordering needs no fence of its own: the mbarrier orders this CTA's
+      // slot stores before thread et 0's arrival, whose acquire-release atomic
+      // publishes them at GPU scope (release is cumulative over what the
+      // barrier ordered before it) and, for the last arrival, makes the other
+      // CTAs' slots visible (acquire); the next barrier passes that on to the
+      // threads that read the slots (L2 loads).
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctrl->esync);
       if (!warp_wait(&ctrl->esync, eph, abortf, p.status, kStatusWaitDrain)) break;
       eph ^= 1;
       if (et == 0) {
-        __threadfence();
-        const unsigned old = atomicAdd(&p.counters[t], 1u);
+        const unsigned old = atom_add_acq_rel_gpu(&p.counters[t], 1u);
         ctrl->last_flag = (old == static_cast<unsigned>(nseg - 1)) ? 1 : 0;
       }
       __syncwarp();
@@ -459,7 +473,6 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
             ctrl->fin_go = 1;
           }
         } else {
-          __threadfence();
           k3_reduce_tile<EPI, NORM, NUM_EPI_WARPS * 32>(p, t, nseg, et);
           if (et == 0) p.counters[t] = 0u;
         }
@@ -591,7 +604,6 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
   // here; the tile completed by this CTA's last segment is summed by all of them.
   __syncthreads();
   if (ctrl->fin_go && *abortf == 0) {
-    __threadfence();
     k3_reduce_tile<EPI, NORM, NUM_THREADS>(p, ctrl->fin_t, ctrl->fin_nseg, threadIdx.x);
     if (threadIdx.x == 0) p.counters[ctrl->fin_t] = 0u;
   }
