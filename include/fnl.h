@@ -83,10 +83,12 @@ typedef enum {
 typedef enum { FNL_NORM_LAYERNORM = 0, FNL_NORM_RMSNORM = 1 } fnl_norm;
 
 typedef enum {
-  FNL_PATH_AUTO = 0,          /* M <= 128: small-M split-K kernel; else a tile kernel */
+  FNL_PATH_AUTO = 0,          /* M <= 128: small-M split-K kernel (cluster form when it fits); else a tile kernel */
   FNL_PATH_TILE = 1,          /* force the large-M persistent kernel, 128 x 256 tiles */
-  FNL_PATH_SPLITK = 2,        /* force the small-M split-K kernel (requires M <= 128) */
-  FNL_PATH_TILE_WIDE = 3      /* force the large-M persistent kernel, 128 x 512 tiles */
+  FNL_PATH_SPLITK = 2,        /* force the small-M split-K kernel, stream-K form (requires M <= 128) */
+  FNL_PATH_TILE_WIDE = 3,     /* force the large-M persistent kernel, 128 x 512 tiles */
+  FNL_PATH_SPLITK_CLUSTER = 4 /* force the small-M kernel's cluster form (M <= 128; FNL_ERR_UNSUPPORTED when
+                                 the tiles cannot all run at once as clusters of 2..8 CTAs) */
 } fnl_path;
 
 /* How the normalised activation a is rounded for the bf16 tensor cores.

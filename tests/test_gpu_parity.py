@@ -74,7 +74,7 @@ def test_tile_tails(handle, op, norm, M):
     run_and_check(handle, w, inputs)
 
 
-@pytest.mark.parametrize("path", ["tile", "wide", "splitk"])
+@pytest.mark.parametrize("path", ["tile", "wide", "splitk", "cluster"])
 @pytest.mark.parametrize("op", ["qkv", "swiglu", "gelu"])
 @pytest.mark.parametrize("norm", ["layernorm", "rmsnorm"])
 def test_forced_paths(cuda_device, path, op, norm):
@@ -84,6 +84,17 @@ def test_forced_paths(cuda_device, path, op, norm):
     for M in (5, 64, 128):
         w, inputs = _tail_workload(op, norm, M, K=520, seed=M)
         run_and_check(h, w, inputs)
+    h.close()
+
+
+@pytest.mark.parametrize("path", ["splitk", "cluster"])
+@pytest.mark.parametrize("name", ["c2_decode_rms_qkv", "c1_tiny_ln_qkv"])
+def test_small_m_forms(cuda_device, path, name):
+    """The small-M kernel's stream-K and cluster forms, each at full size (the
+    automatic choice takes the cluster form for these shapes when it fits)."""
+    w = WL[name]
+    h = fnl.Handle(0, path=path)
+    run_and_check(h, w, synthetic.make_inputs(w))
     h.close()
 
 

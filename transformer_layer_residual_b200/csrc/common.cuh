@@ -35,6 +35,7 @@ struct OpParams {
   int max_seg;
   int mpad;
   int stages;
+  int cls;               // small-M kernel: CTAs per cluster (one W tile per cluster), 0 = stream-K form
   int split;             // 1: operand = bf16 hi + bf16 lo (two UMMAs), 0: single bf16 rounding
   int* status;           // device status word (bounded-wait failures)
 };

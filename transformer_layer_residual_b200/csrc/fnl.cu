@@ -34,6 +34,10 @@ struct fnl_handle {
   uint8_t* ws = nullptr;     // device workspace
   size_t ws_bytes = 0;
   std::string err;
+  struct Occ {
+    int smem, cls, clusters;
+  };
+  std::vector<Occ> occ;      // resident clusters of the small-M kernel per (shared memory, cluster size)
 };
 
 namespace {
@@ -224,11 +228,22 @@ fnl_status launch_gemm(fnl_handle* h, Kern kern, int grid, int threads, int smem
   cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (p.cls > 0) {   // the small-M kernel's cluster form
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = static_cast<unsigned>(p.cls);
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = na;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mx, mr, mw, p);
   if (e != cudaSuccess) return cuda_fail(h, e, "launch of the fused GEMM kernel");
   return FNL_OK;
@@ -287,6 +302,33 @@ fnl_status launch_k1(fnl_handle* h, const Call& c, float2* stats, cudaStream_t s
 
 int round_up(int a, int b) { return (a + b - 1) / b * b; }
 
+// How many clusters of `cls` CTAs of the small-M kernel (with `smem` bytes of
+// shared memory each) the GPU runs at once; cached per handle. Every
+// instantiation has one CTA per SM, so one stands for all.
+int resident_clusters(fnl_handle* h, int smem, int cls) {
+  for (const auto& o : h->occ)
+    if (o.smem == smem && o.cls == cls) return o.clusters;
+  auto kern = fnl::k3_splitk_kernel<fnl::kEpiQKV, fnl::kRMSNorm, false>;
+  int n = 0;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(cls);
+    cfg.blockDim = dim3(fnl::k3::NUM_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute a[1];
+    a[0].id = cudaLaunchAttributeClusterDimension;
+    a[0].val.clusterDim.x = static_cast<unsigned>(cls);
+    a[0].val.clusterDim.y = 1;
+    a[0].val.clusterDim.z = 1;
+    cfg.attrs = a;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();   // a refused query leaves no sticky error behind
+  h->occ.push_back({smem, cls, n});
+  return n;
+}
+
 fnl_status run(fnl_handle* h, const Call& c) {
   fnl_status st = validate(h, c);
   if (st != FNL_OK || c.M == 0) return st;
@@ -298,12 +340,12 @@ fnl_status run(fnl_handle* h, const Call& c) {
   const int epi = c.op == Op::QKV ? fnl::kEpiQKV : (c.op == Op::SwiGLU ? fnl::kEpiSwiGLU : fnl::kEpiGELU);
   bool small = c.M <= fnl::k3::MAX_MPAD;
   if (h->opt.path == FNL_PATH_TILE || h->opt.path == FNL_PATH_TILE_WIDE) small = false;
-  if (h->opt.path == FNL_PATH_SPLITK) small = true;
+  if (h->opt.path == FNL_PATH_SPLITK || h->opt.path == FNL_PATH_SPLITK_CLUSTER) small = true;
   const int max_ctas = h->opt.max_ctas > 0 ? std::min(h->opt.max_ctas, h->num_sms) : h->num_sms;
   const int nkb = (c.K + 63) / 64;
 
   // plan
-  int grid = 1, threads = 0, smem = 0, mpad = 0, stages = 0, max_seg = 1, T = 0;
+  int grid = 1, threads = 0, smem = 0, mpad = 0, stages = 0, max_seg = 1, T = 0, cls = 0;
   bool wide = false;
   if (small) {
     mpad = round_up(std::max(c.M, 1), 16);
@@ -313,7 +355,20 @@ fnl_status run(fnl_handle* h, const Call& c) {
     stages = std::min(fnl::k3::MAX_STAGES, (200 * 1024) / fnl::k3::stage_bytes(mpad));
     smem = fnl::k3::smem_bytes(mpad, stages);
     threads = fnl::k3::NUM_THREADS;
-    for (int t = 0; t < T; ++t) {
+    // Cluster form: one W tile per cluster of cls CTAs, each taking 1/cls of
+    // its k-blocks, partial sums reduced on chip. Used when the clusters cover
+    // the GPU (or every unit of work) and all of them are resident at once.
+    if (h->opt.path == FNL_PATH_SPLITK_CLUSTER || (h->opt.path != FNL_PATH_SPLITK && h->opt.max_ctas == 0)) {
+      // the largest cluster size (<= 8, <= the k-blocks) whose T clusters are all resident
+      for (int c_ = std::min({8, h->num_sms / std::max(T, 1), nkb}); c_ >= 2 && cls == 0; --c_) {
+        const bool covers = static_cast<long long>(T) * c_ >= std::min<long long>(U, (h->num_sms * 9) / 10);
+        if ((covers || h->opt.path == FNL_PATH_SPLITK_CLUSTER) && resident_clusters(h, smem, c_) >= T) cls = c_;
+      }
+    }
+    if (h->opt.path == FNL_PATH_SPLITK_CLUSTER && cls == 0)
+      return fail(h, FNL_ERR_UNSUPPORTED, "the %d W tiles cannot run at once as clusters of 2..8 CTAs", T);
+    if (cls > 0) grid = T * cls;
+    for (int t = 0; t < T && cls == 0; ++t) {
       const int first = fnl::k3::unit_owner(static_cast<long long>(t) * nkb, grid, U);
       const int last = fnl::k3::unit_owner(static_cast<long long>(t + 1) * nkb - 1, grid, U);
       max_seg = std::max(max_seg, last - first + 1);
@@ -345,8 +400,8 @@ fnl_status run(fnl_handle* h, const Call& c) {
 
   // workspace
   const size_t stats_bytes = rms ? 0 : align256(static_cast<size_t>(c.M) * 8);
-  const size_t ss_bytes = small ? align256(static_cast<size_t>(T) * max_seg * mpad * 4) : 0;
-  const size_t part_bytes = small ? align256(static_cast<size_t>(T) * max_seg * mpad * 128 * 4) : 0;
+  const size_t ss_bytes = small && cls == 0 ? align256(static_cast<size_t>(T) * max_seg * mpad * 4) : 0;
+  const size_t part_bytes = small && cls == 0 ? align256(static_cast<size_t>(T) * max_seg * mpad * 128 * 4) : 0;
   const size_t need = kFixedBytes + stats_bytes + ss_bytes + part_bytes;
   if ((st = ensure_workspace(h, c.stream, need)) != FNL_OK) return st;
   uint8_t* ws = h->ws;
@@ -363,7 +418,7 @@ fnl_status run(fnl_handle* h, const Call& c) {
   p.residual_out = c.residual_out; p.rstd_out = rms ? c.rstd_out : nullptr; p.stats = stats;
   p.q = c.q; p.k = c.k; p.v = c.v; p.out = c.out;
   p.part = part; p.part_ss = part_ss; p.counters = counters; p.max_seg = max_seg; p.mpad = mpad;
-  p.stages = stages; p.status = status;
+  p.stages = stages; p.status = status; p.cls = cls;
   p.split = h->opt.precision == FNL_PRECISION_SPLIT ||
             (h->opt.precision == FNL_PRECISION_DEFAULT && c.op == Op::SwiGLU);
 
@@ -408,7 +463,7 @@ fnl_status fnl_create(fnl_handle** out, int device, const fnl_options* opt) {
   *out = nullptr;
   fnl_handle* h = new fnl_handle();
   if (opt) h->opt = *opt;
-  if (h->opt.path < FNL_PATH_AUTO || h->opt.path > FNL_PATH_TILE_WIDE || h->opt.max_tokens < 0 || h->opt.max_n < 0 ||
+  if (h->opt.path < FNL_PATH_AUTO || h->opt.path > FNL_PATH_SPLITK_CLUSTER || h->opt.max_tokens < 0 || h->opt.max_n < 0 ||
       h->opt.precision < FNL_PRECISION_DEFAULT || h->opt.precision > FNL_PRECISION_SINGLE) {
     delete h;
     return FNL_ERR_INVALID_ARG;

@@ -53,6 +53,7 @@ struct Ctrl {
   int last_flag;
   int fin_go, fin_t, fin_nseg;   // the CTA's last segment completes its tile: reduced by all warps
   float ssw[2][NUM_CONV_WARPS][MAX_MPAD];   // per converter warp partial sums of h^2 (RMSNorm)
+  float css[MAX_MPAD];                      // cluster form: this CTA's sum of h^2 per token
 };
 
 __host__ __device__ inline int stage_bytes(int mpad) { return W_BYTES + 2 * mpad * BK * 2; }
@@ -194,6 +195,53 @@ __device__ __forceinline__ void k3_reduce_tile(const OpParams& p, int t, int nse
   }
 }
 
+// Cluster form of the small-M kernel: CTA r of the cluster (rank order 0..cls-1)
+// sums items [r n / cls, (r + 1) n / cls) of the tile's n (row, 8-column) items
+// over the partial sums that the cluster's CTAs hold in shared memory, in rank
+// order (the same sum on every run), and runs the epilogue on them.
+template <int EPI, int NORM>
+__device__ __forceinline__ void k3_cluster_reduce(const OpParams& p, uint32_t part_local, uint32_t css_local, int t,
+                                                  int r, int cls) {
+  using namespace k3;
+  const int G8 = (EPI == kEpiSwiGLU) ? 8 : 16;
+  const int n_items = p.M * G8;
+  const int i1 = (r + 1) * n_items / cls;
+  for (int item = r * n_items / cls + static_cast<int>(threadIdx.x); item < i1; item += NUM_THREADS) {
+    const int m = item / G8, g = item - m * G8;
+    const uint32_t off = static_cast<uint32_t>(m * BW + g * 8) * 4;
+    float acc[8], up[8], ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = up[e] = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (q < cls) {
+        const uint32_t a = dsmem_addr(part_local + off, q);
+        const float4 v0 = ld_dsmem_f4(a), v1 = ld_dsmem_f4(a + 16);
+        acc[0] += v0.x; acc[1] += v0.y; acc[2] += v0.z; acc[3] += v0.w;
+        acc[4] += v1.x; acc[5] += v1.y; acc[6] += v1.z; acc[7] += v1.w;
+        if (EPI == kEpiSwiGLU) {   // the up rows are rows 64..127 of the tile
+          const float4 u0 = ld_dsmem_f4(a + 256), u1 = ld_dsmem_f4(a + 272);
+          up[0] += u0.x; up[1] += u0.y; up[2] += u0.z; up[3] += u0.w;
+          up[4] += u1.x; up[5] += u1.y; up[6] += u1.z; up[7] += u1.w;
+        }
+        if (NORM == kRMSNorm) ss += ld_dsmem_f32(dsmem_addr(css_local + m * 4, q));
+      }
+    }
+    float scale = 1.f;
+    if (NORM == kRMSNorm) {
+      scale = 1.f / sqrtf(ss / static_cast<float>(p.K) + p.eps);
+      if (t == 0 && g == 0 && p.rstd_out != nullptr) p.rstd_out[m] = scale;
+    }
+    if (EPI == kEpiSwiGLU) {
+      const int j = t * 64 + g * 8;
+      if (j < p.I) store_swiglu8(p, m, j, acc, up, scale);
+    } else {
+      const int n = t * BW + g * 8;
+      if (n < p.N) store_out8<EPI>(p, m, n, acc, scale);
+    }
+  }
+}
+
 template <int EPI, int NORM, bool SPLIT>
 __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     k3_splitk_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_r,
@@ -214,13 +262,20 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
   const int T = (EPI == kEpiSwiGLU) ? (p.I + 63) / 64 : (p.N + BW - 1) / BW;
   const int nkb = (K + BK - 1) / BK;
   const uint32_t ncols = tmem_cols(mpad);
+  const bool cl = p.cls > 0;
   constexpr bool BIAS_IN = EPI == kEpiGELU;   // only the GELU entry point has a bias_in
 
   const long long U = static_cast<long long>(T) * nkb;
   if (threadIdx.x == 0) {
     pdl_launch_dependents();   // the next call's CTAs may take SMs as ours retire
-    ctrl->u0 = static_cast<long long>(blockIdx.x) * U / gridDim.x;
-    ctrl->u1 = static_cast<long long>(blockIdx.x + 1) * U / gridDim.x;
+    if (p.cls > 0) {   // cluster form: CTA r of cluster t takes k-blocks [r nkb / cls, (r + 1) nkb / cls) of tile t
+      const long long t0 = blockIdx.x / p.cls, r = blockIdx.x % p.cls;
+      ctrl->u0 = t0 * nkb + r * nkb / p.cls;
+      ctrl->u1 = t0 * nkb + (r + 1) * nkb / p.cls;
+    } else {
+      ctrl->u0 = static_cast<long long>(blockIdx.x) * U / gridDim.x;
+      ctrl->u1 = static_cast<long long>(blockIdx.x + 1) * U / gridDim.x;
+    }
     for (int s = 0; s < S; ++s) {
       mbar_init(&ctrl->full_w[s], 1);
       mbar_init(&ctrl->full_x[s], 1);
@@ -422,8 +477,11 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
         if (!warp_wait(&ctrl->sfull[b], use & 1, abortf, p.status, kStatusWaitStats)) break;
       }
       tc_fence_after();
+      // stream-K form: the partial goes to the tile's workspace slot; cluster
+      // form: to this CTA's own shared memory (the stage buffers, all consumed
+      // once the last UMMA has completed), [mpad][128] fp32
       const size_t base = static_cast<size_t>(t) * p.max_seg + slot;
-      float* part = p.part + base * mpad * BW;
+      float* part = cl ? reinterpret_cast<float*>(smem) : p.part + base * mpad * BW;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * mpad;
       for (int mc = 0; mc < mpad; mc += 16) {
         uint32_t v[16];
@@ -437,12 +495,14 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
         float ssum = 0.f;
 #pragma unroll
         for (int w = 0; w < NUM_CONV_WARPS; ++w) ssum += ctrl->ssw[b][w][et];   // fixed order
-        p.part_ss[base * mpad + et] = ssum;
+        if (cl) ctrl->css[et] = ssum;
+        else p.part_ss[base * mpad + et] = ssum;
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctrl->tempty[b]);
       ++i;
+      if (cl) continue;   // the cluster sums its tile after the role loops
 
       // arrival: the last CTA of this tile reduces all slots in slot order.
       // The epilogue warps meet on an mbarrier (bounded wait), not bar.sync,
@@ -603,7 +663,16 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
   // Every role's loop is over (each bounded wait returns), so all warps meet
   // here; the tile completed by this CTA's last segment is summed by all of them.
   __syncthreads();
-  if (ctrl->fin_go && *abortf == 0) {
+  if (cl) {
+    // Cluster form: every CTA of the cluster holds its partial sums of the
+    // cluster's tile in its shared memory; each sums its share of the tile's
+    // items over the cluster (distributed shared memory, rank order).
+    cluster_sync();
+    if (*abortf == 0)
+      k3_cluster_reduce<EPI, NORM>(p, smem_u32(smem), smem_u32(ctrl->css), blockIdx.x / p.cls, blockIdx.x % p.cls,
+                                   p.cls);
+    cluster_sync();   // no CTA leaves while the others still read its shared memory
+  } else if (ctrl->fin_go && *abortf == 0) {
     k3_reduce_tile<EPI, NORM, NUM_THREADS>(p, ctrl->fin_t, ctrl->fin_nseg, threadIdx.x);
     if (threadIdx.x == 0) p.counters[ctrl->fin_t] = 0u;
   }
