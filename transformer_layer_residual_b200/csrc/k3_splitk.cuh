@@ -46,7 +46,7 @@ constexpr int PREWAIT_STAGES = 0;
 
 struct Ctrl {
   uint64_t full_w[MAX_STAGES], full_x[MAX_STAGES], conv[MAX_STAGES], empty[MAX_STAGES];
-  uint64_t tfull[2], tempty[2], sfull[2], drain, esync;
+  uint64_t tfull[2], tempty[2], sfull[2], drain, esync, rbar;
   long long u0, u1;   // this CTA's unit range
   uint32_t tmem_base;
   int abort_flag;
@@ -195,6 +195,53 @@ __device__ __forceinline__ void k3_reduce_tile(const OpParams& p, int t, int nse
   }
 }
 
+// The last segment's tile reduced from shared memory: slot sl's rows [0, M) of
+// partial sums at part + sl M 128 (fp32 [M][128]), its sum(h^2) per token at
+// ss + sl mpad; summed in slot order like k3_reduce_tile. All the CTA's threads.
+template <int EPI, int NORM>
+__device__ __forceinline__ void k3_reduce_tile_smem(const OpParams& p, int t, int nseg, const float* part,
+                                                    const float* ss) {
+  using namespace k3;
+  const int G8 = (EPI == kEpiSwiGLU) ? 8 : 16;
+  const int n_items = p.M * G8;
+  const int slot = p.M * BW;
+  for (int item = threadIdx.x; item < n_items; item += NUM_THREADS) {
+    const int m = item / G8, g = item - m * G8;
+    const uint32_t base = smem_u32(part + m * BW + g * 8);
+    float acc[8], up[8], ssum = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = up[e] = 0.f;
+    for (int sl = 0; sl < nseg; ++sl) {
+      const uint32_t a = base + static_cast<uint32_t>(sl * slot) * 4;
+      const uint4 v0 = ld_shared_v4(a), v1 = ld_shared_v4(a + 16);
+      acc[0] += __uint_as_float(v0.x); acc[1] += __uint_as_float(v0.y);
+      acc[2] += __uint_as_float(v0.z); acc[3] += __uint_as_float(v0.w);
+      acc[4] += __uint_as_float(v1.x); acc[5] += __uint_as_float(v1.y);
+      acc[6] += __uint_as_float(v1.z); acc[7] += __uint_as_float(v1.w);
+      if (EPI == kEpiSwiGLU) {   // the up rows are rows 64..127 of the tile
+        const uint4 u0 = ld_shared_v4(a + 256), u1 = ld_shared_v4(a + 272);
+        up[0] += __uint_as_float(u0.x); up[1] += __uint_as_float(u0.y);
+        up[2] += __uint_as_float(u0.z); up[3] += __uint_as_float(u0.w);
+        up[4] += __uint_as_float(u1.x); up[5] += __uint_as_float(u1.y);
+        up[6] += __uint_as_float(u1.z); up[7] += __uint_as_float(u1.w);
+      }
+      if (NORM == kRMSNorm) ssum += ss[sl * p.mpad + m];
+    }
+    float scale = 1.f;
+    if (NORM == kRMSNorm) {
+      scale = 1.f / sqrtf(ssum / static_cast<float>(p.K) + p.eps);
+      if (t == 0 && g == 0 && p.rstd_out != nullptr) p.rstd_out[m] = scale;
+    }
+    if (EPI == kEpiSwiGLU) {
+      const int j = t * 64 + g * 8;
+      if (j < p.I) store_swiglu8(p, m, j, acc, up, scale);
+    } else {
+      const int n = t * BW + g * 8;
+      if (n < p.N) store_out8<EPI>(p, m, n, acc, scale);
+    }
+  }
+}
+
 // Cluster form of the small-M kernel: CTA r of the cluster (rank order 0..cls-1)
 // sums items [r n / cls, (r + 1) n / cls) of the tile's n (row, 8-column) items
 // over the partial sums that the cluster's CTAs hold in shared memory, in rank
@@ -289,6 +336,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     }
     mbar_init(&ctrl->drain, 1);
     mbar_init(&ctrl->esync, NUM_EPI_WARPS);
+    mbar_init(&ctrl->rbar, 1);
     ctrl->abort_flag = 0;
     ctrl->last_flag = 0;
     ctrl->fin_go = 0;
@@ -673,8 +721,36 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
                                    p.cls);
     cluster_sync();   // no CTA leaves while the others still read its shared memory
   } else if (ctrl->fin_go && *abortf == 0) {
-    k3_reduce_tile<EPI, NORM, NUM_THREADS>(p, ctrl->fin_t, ctrl->fin_nseg, threadIdx.x);
-    if (threadIdx.x == 0) p.counters[ctrl->fin_t] = 0u;
+    // The tile's slots are bulk-copied into the (idle) stage buffers and summed
+    // there: one deep stream of copies instead of every thread's scattered L2
+    // loads. Falls back to direct loads when they do not fit.
+    const int t = ctrl->fin_t, nseg = ctrl->fin_nseg;
+    const uint32_t slot_bytes = static_cast<uint32_t>(M) * BW * 4;
+    const uint32_t ss_bytes = NORM == kRMSNorm ? static_cast<uint32_t>(mpad) * 4 : 0u;
+    if (static_cast<long long>(nseg) * (slot_bytes + ss_bytes) <= static_cast<long long>(S) * SB) {
+      if (threadIdx.x == 0) {
+        fence_proxy_async_global();
+        mbar_arrive_expect_tx(&ctrl->rbar, static_cast<uint32_t>(nseg) * (slot_bytes + ss_bytes));
+        const size_t slot_stride = static_cast<size_t>(mpad) * BW;
+        const float* tp = p.part + static_cast<size_t>(t) * p.max_seg * slot_stride;
+        const float* tss = p.part_ss + static_cast<size_t>(t) * p.max_seg * mpad;
+        for (int sl = 0; sl < nseg; ++sl) {
+          bulk_load(smem + sl * slot_bytes, tp + sl * slot_stride, slot_bytes, &ctrl->rbar);
+          if (NORM == kRMSNorm)
+            bulk_load(smem + nseg * slot_bytes + sl * ss_bytes, tss + static_cast<size_t>(sl) * mpad, ss_bytes,
+                      &ctrl->rbar);
+        }
+      }
+      if (warp_wait(&ctrl->rbar, 0, abortf, p.status, kStatusWaitFull)) {
+        k3_reduce_tile_smem<EPI, NORM>(p, t, nseg, reinterpret_cast<const float*>(smem),
+                                       reinterpret_cast<const float*>(smem + nseg * slot_bytes));
+      } else if (threadIdx.x == 0) {
+        drain_wait(&ctrl->rbar, 0);   // the copies land before the CTA can exit
+      }
+    } else {
+      k3_reduce_tile<EPI, NORM, NUM_THREADS>(p, t, nseg, threadIdx.x);
+    }
+    if (threadIdx.x == 0) p.counters[t] = 0u;
   }
   tc_fence_before();
   __syncthreads();
