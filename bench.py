@@ -303,8 +303,10 @@ def bench_fnl(w, steps, warmup, world, rank, local, sweep_line=False):
         peak = pk["hbm_gbs"]
         runit = "GB/s"
     else:
+        # a tensor-bound step runs back to back for the whole timed region, so
+        # its denominator is the GEMM throughput sustained under the power cap
         achieved = w.flops() / (per_launch_ms / 1e3) / 1e12
-        peak = pk["bf16_tflops"]
+        peak = pk["bf16_tflops_sustained"]
         runit = "TFLOP/s"
     line = {
         "metric": METRIC,
@@ -330,7 +332,7 @@ def bench_fnl(w, steps, warmup, world, rank, local, sweep_line=False):
         "gbps": round(w.algorithmic_bytes() * steps * world / (ms_max / 1e3) / 1e9, 3),
         "tokens_per_s_layer": round(w.M * steps * world / (ms_max / 1e3), 1),
         "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": runit,
-                     "frac": round(achieved / peak, 4), "peak_source": f"{pk_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops burst'})",
+                     "frac": round(achieved / peak, 4), "peak_source": f"{pk_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops_sustained'})",
                      "traffic": recorded_traffic(w.name),
                      "algorithmic_per_launch": w.algorithmic_bytes() if bound == "hbm" else w.flops(),
                      "kernel": "fused GEMM kernel" + (" + LayerNorm stats kernel (PDL)" if w.norm == "layernorm" else "")},
