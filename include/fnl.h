@@ -45,7 +45,13 @@
  *   - K, N (and D, I) multiples of 8; 1 <= K <= 32768; M >= 0 (M = 0 is a no-op);
  *   - outputs overlap neither each other nor any input;
  *   - the handle is used by one host thread / one stream at a time (its
- *     workspace is shared by its calls).
+ *     workspace is shared by its calls);
+ *   - W is not written by the kernel enqueued on `stream` immediately before
+ *     the call: the GEMM kernel is a programmatic dependent of that kernel and
+ *     the large-M kernels fetch their first weight tiles before waiting for it
+ *     (activations, statistics, workspace and outputs are touched only after
+ *     the wait). Not checkable on the host; a weight produced by the previous
+ *     kernel needs any other stream operation in between.
  * Calls are asynchronous: they enqueue one or two kernels on `stream` and
  * return. They never synchronise, except the first call whose shape needs more
  * workspace than the handle holds: that call synchronises `stream`, then

@@ -1,19 +1,28 @@
-// K3: small-M (decode) fused norm + GEMM + epilogue, stream-K over all SMs.
+// K3: small-M (decode) fused norm + GEMM + epilogue, split-K over all SMs.
 //
 // With M <= 128 tokens the op is bound by streaming W from HBM once. The
 // product is computed transposed ("swap AB"): the W tile is the UMMA M=128
 // operand and the (padded) tokens are the N operand, so a tcgen05.mma
-// M=128 x N=mpad x K=16 does useful work even for one token. The work units
-// (128-row W tile, 64-wide k-block) are split evenly over the grid (stream-K):
-// CTA g takes units [g*U/G, (g+1)*U/G), cutting at tile boundaries into
-// segments. Each segment's fp32 partial goes to a workspace slot; an arrival
-// counter per tile elects the last-arriving CTA, which sums the slots in a
-// fixed order (deterministic), applies the deferred RMSNorm scale and the
-// epilogue, and resets the counter. Nothing spins on another CTA.
+// M=128 x N=mpad x K=16 does useful work even for one token. Work units are
+// (128-row W tile, 64-wide k-block) pairs, in one of two forms:
+// - stream-K: the units are split evenly over the grid, CTA g taking
+//   [g*U/G, (g+1)*U/G), cut at tile boundaries into segments. Each segment's
+//   fp32 partial goes to a workspace slot; an arrival counter per tile (one
+//   acquire-release atomic per segment) elects the last-arriving CTA, which
+//   sums the slots in slot order (deterministic), applies the deferred RMSNorm
+//   scale and the epilogue, and resets the counter. A CTA's last segment is
+//   summed by all its warps from shared memory, after bulk copies of the slots.
+// - cluster: one W tile per cluster of cls CTAs, CTA r taking k-blocks
+//   [r nkb / cls, (r+1) nkb / cls); partials stay in shared memory and each CTA
+//   sums its share of the tile over distributed shared memory, in rank order,
+//   between two cluster barriers. Used when the clusters fill the GPU.
+// Nothing spins on another CTA except the cluster barriers, which every thread
+// of every CTA reaches after its role loop.
 //
 // Warp roles (10 warps): 0 TMA producer (W tile + x/residual tiles), 1 TMEM
-// owner and UMMA issuer, 2-5 epilogue / split-K reduction, 6-9 converters
-// (normalised bf16 operand built in place in shared memory, as in K2).
+// owner and UMMA issuer, 2-5 epilogue / split-K reduction (and, for RMSNorm,
+// residual_out while the main loop runs), 6-9 converters (normalised bf16
+// operand built in place in shared memory, as in K2).
 //
 // Each stage has two barriers: full_w (the W tile, from HBM) and full_x (the
 // x / residual tiles and the gamma / beta / bias_in slices, from L2), so the
