@@ -10,6 +10,7 @@ from .fnl import (  # noqa: F401
     Handle,
     add_bias_norm_gelu,
     add_norm_qkv,
+    add_norm_qkv_static,
     add_norm_swiglu,
     lib,
     lib_path,

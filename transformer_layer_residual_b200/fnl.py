@@ -72,7 +72,14 @@ def lib() -> ctypes.CDLL:
 
 
 class Handle:
-    """Owns an fnl_handle (device workspace). One stream / thread at a time."""
+    """Owns an fnl_handle (device workspace). One stream / thread at a time.
+
+    max_tokens / max_n reserve the workspace up front (no reallocation, and so
+    no stream synchronisation, on later calls up to that size). path forces a
+    kernel: "auto" (by M), "splitk" (small-M kernel, stream-K form), "cluster"
+    (small-M kernel, cluster form), "tile" (128x256 tiles), "wide" (128x512
+    tiles). max_ctas caps the grid (0 = all SMs). precision: "default" (split
+    hi + lo operand for SwiGLU only), "split", "single"."""
 
     def __init__(self, device: int = 0, max_tokens: int = 0, max_n: int = 0, path: str = "auto",
                  max_ctas: int = 0, precision: str = "default"):
