@@ -36,6 +36,7 @@ struct OpParams {
   int mpad;
   int stages;
   int cls;               // small-M kernel: CTAs per cluster (one W tile per cluster), 0 = stream-K form
+  int sk;                // 128x256 tile kernel: 1 = stream-K over (tile, k-block) units, 0 = whole tiles
   int split;             // 1: operand = bf16 hi + bf16 lo (two UMMAs), 0: single bf16 rounding
   int* status;           // device status word (bounded-wait failures)
 };
@@ -72,6 +73,18 @@ __device__ __forceinline__ uint32_t issue_vec_loads(const OpParams& p, bool has_
 __device__ __forceinline__ uint32_t vec_bytes(const OpParams& p, bool has_beta, bool has_bias_in, int kb) {
   const int kvalid = min(kVecElems, p.K - kb * kVecElems);
   return static_cast<uint32_t>(kvalid) * 2 * (1 + (has_beta ? 1 : 0) + (has_bias_in ? 1 : 0));
+}
+
+// Split-K work units (W tile, k-block) dealt evenly over G CTAs: CTA g takes
+// units [g U / G, (g + 1) U / G).
+// Index of the CTA whose unit range contains unit u (units split as g*U/G).
+__host__ __device__ inline int unit_owner(long long u, int G, long long U) {
+  return static_cast<int>(((u + 1) * G - 1) / U);
+}
+// The same in double precision (exact: every operand is an integer below 2^53
+// and a quotient that is not an integer is at least 1/U away from one).
+__device__ __forceinline__ int unit_owner_fast(long long u, int G, long long U) {
+  return static_cast<int>((static_cast<double>(u + 1) * G - 1.0) / static_cast<double>(U));
 }
 
 // Compile-time flag for code specialised on a condition that is uniform over a

@@ -345,7 +345,7 @@ fnl_status run(fnl_handle* h, const Call& c) {
   const int nkb = (c.K + 63) / 64;
 
   // plan
-  int grid = 1, threads = 0, smem = 0, mpad = 0, stages = 0, max_seg = 1, T = 0, cls = 0;
+  int grid = 1, threads = 0, smem = 0, mpad = 0, stages = 0, max_seg = 1, T = 0, cls = 0, sk = 0;
   bool wide = false;
   if (small) {
     mpad = round_up(std::max(c.M, 1), 16);
@@ -369,8 +369,8 @@ fnl_status run(fnl_handle* h, const Call& c) {
       return fail(h, FNL_ERR_UNSUPPORTED, "the %d W tiles cannot run at once as clusters of 2..8 CTAs", T);
     if (cls > 0) grid = T * cls;
     for (int t = 0; t < T && cls == 0; ++t) {
-      const int first = fnl::k3::unit_owner(static_cast<long long>(t) * nkb, grid, U);
-      const int last = fnl::k3::unit_owner(static_cast<long long>(t + 1) * nkb - 1, grid, U);
+      const int first = fnl::unit_owner(static_cast<long long>(t) * nkb, grid, U);
+      const int last = fnl::unit_owner(static_cast<long long>(t + 1) * nkb - 1, grid, U);
       max_seg = std::max(max_seg, last - first + 1);
     }
     if (T > kMaxTiles) return fail(h, FNL_ERR_UNSUPPORTED, "too many W tiles");
@@ -394,6 +394,21 @@ fnl_status run(fnl_handle* h, const Call& c) {
     if (h->opt.path == FNL_PATH_TILE_WIDE) wide = true;
     const long long tiles = wide ? tiles_w : tiles_n;
     grid = static_cast<int>(std::min<long long>(max_ctas, tiles));
+    // Fewer 128x256 tiles than CTAs by a fifth or more (e.g. 70B QKV at
+    // M = 256: 80 tiles, 148 SMs): stream-K over (tile, k-block) units, so
+    // every SM streams weights; partial tiles are summed by their last CTA.
+    if (!wide && tiles * 5 <= static_cast<long long>(max_ctas) * 4) {
+      sk = 1;
+      T = static_cast<int>(tiles);
+      const long long U = tiles * nkb;
+      grid = static_cast<int>(std::min<long long>(max_ctas, U));
+      for (int t = 0; t < T; ++t) {
+        const int first = fnl::unit_owner(static_cast<long long>(t) * nkb, grid, U);
+        const int last = fnl::unit_owner(static_cast<long long>(t + 1) * nkb - 1, grid, U);
+        max_seg = std::max(max_seg, last - first + 1);
+      }
+      if (T > kMaxTiles) return fail(h, FNL_ERR_UNSUPPORTED, "too many W tiles");
+    }
     smem = wide ? fnl::k2w::SMEM_BYTES : fnl::k2::SMEM_BYTES;
     threads = wide ? fnl::k2w::NUM_THREADS : fnl::k2::NUM_THREADS;
   }
@@ -401,7 +416,8 @@ fnl_status run(fnl_handle* h, const Call& c) {
   // workspace
   const size_t stats_bytes = rms ? 0 : align256(static_cast<size_t>(c.M) * 8);
   const size_t ss_bytes = small && cls == 0 ? align256(static_cast<size_t>(T) * max_seg * mpad * 4) : 0;
-  const size_t part_bytes = small && cls == 0 ? align256(static_cast<size_t>(T) * max_seg * mpad * 128 * 4) : 0;
+  size_t part_bytes = small && cls == 0 ? align256(static_cast<size_t>(T) * max_seg * mpad * 128 * 4) : 0;
+  if (sk) part_bytes = align256(static_cast<size_t>(T) * max_seg * fnl::k2::SLOT_FLOATS * 4);
   const size_t need = kFixedBytes + stats_bytes + ss_bytes + part_bytes;
   if ((st = ensure_workspace(h, c.stream, need)) != FNL_OK) return st;
   uint8_t* ws = h->ws;
@@ -418,7 +434,7 @@ fnl_status run(fnl_handle* h, const Call& c) {
   p.residual_out = c.residual_out; p.rstd_out = rms ? c.rstd_out : nullptr; p.stats = stats;
   p.q = c.q; p.k = c.k; p.v = c.v; p.out = c.out;
   p.part = part; p.part_ss = part_ss; p.counters = counters; p.max_seg = max_seg; p.mpad = mpad;
-  p.stages = stages; p.status = status; p.cls = cls;
+  p.stages = stages; p.status = status; p.cls = cls; p.sk = sk;
   p.split = h->opt.precision == FNL_PRECISION_SPLIT ||
             (h->opt.precision == FNL_PRECISION_DEFAULT && c.op == Op::SwiGLU);
 
@@ -709,8 +725,8 @@ extern "C" fnl_status fnl_add_norm_qkv_static(fnl_stream stream, const fnl_bf16*
   const int stages = std::min(fnl::k3::MAX_STAGES, (200 * 1024) / fnl::k3::stage_bytes(mpad));
   int max_seg = 1;
   for (int t = 0; t < T; ++t) {
-    const int first = fnl::k3::unit_owner(static_cast<long long>(t) * nkb, grid, U);
-    const int last = fnl::k3::unit_owner(static_cast<long long>(t + 1) * nkb - 1, grid, U);
+    const int first = fnl::unit_owner(static_cast<long long>(t) * nkb, grid, U);
+    const int last = fnl::unit_owner(static_cast<long long>(t + 1) * nkb - 1, grid, U);
     max_seg = std::max(max_seg, last - first + 1);
   }
   // scratch layout: [status][counters][stats][partial h^2 sums][partial accumulators]

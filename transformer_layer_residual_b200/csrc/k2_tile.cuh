@@ -45,11 +45,64 @@ constexpr int GROUP_M = 16;  // tile raster: 16 M-blocks share each W tile while
 
 struct Ctrl {
   uint64_t full_w[STAGES], full_x[STAGES], conv[STAGES], empty[STAGES];
-  uint64_t tfull[2], tempty[2], sfull[2], drain;
+  uint64_t tfull[2], tempty[2], sfull[2], drain, esync;
   uint32_t tmem_base;
   int abort_flag;
-  float rs[2][BM];
+  int last_flag;
+  int fin_go, fin_t, fin_nseg;   // stream-K: the CTA's last segment completes its tile (summed by all warps)
+  float rs[2][BM];               // RMSNorm: sum(h^2) per row of the segment, from the converters
 };
+// Stream-K partial of one segment: fp32 [BN / 8][BM][8] (8-column chunks, rows
+// contiguous, so a warp's 32 rows read and write 1 KB runs) and sum(h^2) [BM].
+constexpr int SLOT_FLOATS = BM * BN + BM;
+
+// The CTA's segments. Tile mode (p.sk == 0): whole tiles g, g + G, ...
+// Stream-K (p.sk != 0, used when there are fewer tiles than CTAs): the
+// (tile, k-block) units [g U / G, (g + 1) U / G), cut at tile ends; slot /
+// nseg locate the segment among the tile's CTAs.
+struct Segs {
+  long long u, u1, U;
+  int t_next, tiles, nkb, G, g;
+  bool sk;
+  __device__ bool next(int& t, int& kb0, int& nk, int& slot, int& nseg) {
+    if (!sk) {
+      if (t_next >= tiles) return false;
+      t = t_next;
+      t_next += G;
+      kb0 = 0;
+      nk = nkb;
+      slot = 0;
+      nseg = 1;
+      return true;
+    }
+    if (u >= u1) return false;
+    t = static_cast<int>(u / nkb);
+    kb0 = static_cast<int>(u - static_cast<long long>(t) * nkb);
+    const long long te = static_cast<long long>(t + 1) * nkb;
+    const long long e = te < u1 ? te : u1;
+    nk = static_cast<int>(e - u);
+    const int first = unit_owner_fast(static_cast<long long>(t) * nkb, G, U);
+    const int last = unit_owner_fast(te - 1, G, U);
+    slot = g - first;
+    nseg = last - first + 1;
+    u = e;
+    return true;
+  }
+  __device__ bool done() const { return sk ? u >= u1 : t_next >= tiles; }
+};
+__device__ __forceinline__ Segs make_segs(bool sk, int tiles, int nkb) {
+  Segs it;
+  it.sk = sk;
+  it.tiles = tiles;
+  it.nkb = nkb;
+  it.G = gridDim.x;
+  it.g = blockIdx.x;
+  it.t_next = blockIdx.x;
+  it.U = static_cast<long long>(tiles) * nkb;
+  it.u = it.U * blockIdx.x / gridDim.x;
+  it.u1 = it.U * (blockIdx.x + 1) / gridDim.x;
+  return it;
+}
 constexpr int VEC_BYTES = (STAGES * kVecStageBytes + 127) / 128 * 128;   // [STAGES][3][64] bf16
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + VEC_BYTES + static_cast<int>(sizeof(Ctrl)) + 1024;
 
@@ -73,6 +126,83 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
 
 }  // namespace k2
 
+// Stream-K fix-up of tile t by the CTA that arrived last: sum the nseg slots in
+// slot order (the same sum on every run) and run the epilogue, NT threads
+// (et = 0..NT-1). Item = (row, 8-column chunk), rows fastest so that a warp
+// reads 1 KB runs; each thread loads ITEMS items' slots before adding.
+template <int EPI, int NORM, int NT>
+__device__ __forceinline__ void k2_reduce_tile(const OpParams& p, int t, int nseg, int et, int num_m, int num_n) {
+  using namespace k2;
+  int mb, nb;
+  tile_coords(t, num_m, num_n, mb, nb);
+  const float* tp = p.part + static_cast<size_t>(t) * p.max_seg * SLOT_FLOATS;
+  constexpr int CH = (EPI == kEpiSwiGLU) ? BN / 16 : BN / 8;   // SwiGLU: gate chunks (up = chunk + BN / 16)
+  constexpr int ITEMS = (EPI == kEpiSwiGLU) ? 1 : 2;   // SwiGLU carries gate and up sums
+  const int n_items = BM * CH;
+  for (int it0 = et; it0 < n_items; it0 += ITEMS * NT) {
+    float acc[ITEMS][8], up[ITEMS][8], ssum[ITEMS];
+#pragma unroll
+    for (int q = 0; q < ITEMS; ++q) {
+      ssum[q] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[q][e] = up[q][e] = 0.f;
+    }
+    for (int sl = 0; sl < nseg; ++sl) {
+      const float* sp = tp + static_cast<size_t>(sl) * SLOT_FLOATS;
+      float4 va[ITEMS][2], vu[ITEMS][2];
+      float vs[ITEMS];
+#pragma unroll
+      for (int q = 0; q < ITEMS; ++q) {
+        const int item = it0 + q * NT;
+        if (item < n_items) {
+          const int row = item % BM, c8 = item / BM;
+          const float* a = sp + (static_cast<size_t>(c8) * BM + row) * 8;
+          va[q][0] = __ldcg(reinterpret_cast<const float4*>(a));
+          va[q][1] = __ldcg(reinterpret_cast<const float4*>(a + 4));
+          if (EPI == kEpiSwiGLU) {
+            const float* u = a + static_cast<size_t>(CH) * BM * 8;
+            vu[q][0] = __ldcg(reinterpret_cast<const float4*>(u));
+            vu[q][1] = __ldcg(reinterpret_cast<const float4*>(u + 4));
+          }
+          if (NORM == kRMSNorm) vs[q] = __ldcg(sp + BM * BN + row);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < ITEMS; ++q) {
+        if (it0 + q * NT < n_items) {
+          acc[q][0] += va[q][0].x; acc[q][1] += va[q][0].y; acc[q][2] += va[q][0].z; acc[q][3] += va[q][0].w;
+          acc[q][4] += va[q][1].x; acc[q][5] += va[q][1].y; acc[q][6] += va[q][1].z; acc[q][7] += va[q][1].w;
+          if (EPI == kEpiSwiGLU) {
+            up[q][0] += vu[q][0].x; up[q][1] += vu[q][0].y; up[q][2] += vu[q][0].z; up[q][3] += vu[q][0].w;
+            up[q][4] += vu[q][1].x; up[q][5] += vu[q][1].y; up[q][6] += vu[q][1].z; up[q][7] += vu[q][1].w;
+          }
+          if (NORM == kRMSNorm) ssum[q] += vs[q];
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < ITEMS; ++q) {
+      const int item = it0 + q * NT;
+      if (item >= n_items) continue;
+      const int row = item % BM, c8 = item / BM;
+      const int m = mb * BM + row;
+      if (m >= p.M) continue;
+      float scale = 1.f;
+      if (NORM == kRMSNorm) {
+        scale = 1.f / sqrtf(ssum[q] / static_cast<float>(p.K) + p.eps);
+        if (nb == 0 && c8 == 0 && p.rstd_out != nullptr) p.rstd_out[m] = scale;
+      }
+      if (EPI == kEpiSwiGLU) {
+        const int j = nb * (BN / 2) + c8 * 8;
+        if (j < p.I) store_swiglu8(p, m, j, acc[q], up[q], scale);
+      } else {
+        const int n = nb * BN + c8 * 8;
+        if (n < p.N) store_out8<EPI>(p, m, n, acc[q], scale);
+      }
+    }
+  }
+}
+
 template <int EPI, int NORM, bool SPLIT>
 __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
     k2_tile_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_r,
@@ -92,6 +222,7 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
   const int tiles = num_m * num_n;
   const int nkb = (K + BK - 1) / BK;
   constexpr bool BIAS_IN = EPI == kEpiGELU;   // only the GELU entry point has a bias_in
+  const bool sk = p.sk != 0;
 
   if (threadIdx.x == 0) {
     pdl_launch_dependents();   // the next call's CTAs may take SMs as ours retire
@@ -107,7 +238,10 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
       mbar_init(&ctrl->sfull[b], NUM_CONV_WARPS);
     }
     mbar_init(&ctrl->drain, 1);
+    mbar_init(&ctrl->esync, NUM_EPI_WARPS);
     ctrl->abort_flag = 0;
+    ctrl->last_flag = 0;
+    ctrl->fin_go = 0;
     fence_mbar_init();
   }
   if (warp == WARP_TMA && lane == 0) {
@@ -130,8 +264,9 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       // positions q = (local tile index) * nkb + k-block, stage q % STAGES
+      const Segs segs = make_segs(sk, tiles, nkb);
       const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-      const int P = my_tiles * nkb;
+      const int P = sk ? static_cast<int>(segs.u1 - segs.u) : my_tiles * nkb;
       const int npre = P < STAGES ? P : STAGES;
       uint32_t armed_w = 0, armed_x = 0, par_w = 0, par_x = 0;
       bool ok = true;
@@ -140,12 +275,16 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
         uint32_t ph;
       };
       Cur cw{static_cast<int>(blockIdx.x), 0, 0, 0, 0, 0u};
+      if (sk) {
+        cw.t = static_cast<int>(segs.u / nkb);
+        cw.kb = static_cast<int>(segs.u - static_cast<long long>(cw.t) * nkb);
+      }
       if (P > 0) tile_coords(cw.t, num_m, num_n, cw.mb, cw.nb);
       Cur cx = cw;
       auto step = [&](Cur& c) {
         if (++c.kb == nkb) {
           c.kb = 0;
-          c.t += gridDim.x;
+          c.t += sk ? 1 : static_cast<int>(gridDim.x);
           if (c.t < tiles) tile_coords(c.t, num_m, num_n, c.mb, c.nb);
         }
         if (++c.s == STAGES) {
@@ -207,13 +346,16 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
       bool ok = true;
       const uint32_t idesc = idesc_bf16(BM, BN);
       int i = 0;
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++i) {
+      Segs segs = make_segs(sk, tiles, nkb);
+      int t, kb0, nk, slot, nseg;
+      while (ok && segs.next(t, kb0, nk, slot, nseg)) {
         const int b = i & 1;
         const uint32_t use = static_cast<uint32_t>(i >> 1);
+        ++i;
         if (!mbar_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty)) break;
         tc_fence_after();
         const uint32_t d = tmem + b * BN;
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = 0; kb < nk; ++kb) {   // kb counts the segment's k-blocks
           if (!mbar_wait(&ctrl->conv[s], ph, abortf, p.status, kStatusWaitConv) ||
               !mbar_wait(&ctrl->full_w[s], ph, abortf, p.status, kStatusWaitFull)) {
             ok = false;
@@ -247,16 +389,21 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;   // TMEM lane quadrant this warp may read
     const int row_local = q * 32 + lane;
-    pdl_wait();   // outputs may still be in use by the previous kernel
+    pdl_wait();   // outputs and workspace may still be in use by the previous kernel
+    const int et = threadIdx.x - WARP_EPI0 * 32;   // 0..127
     int i = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+    uint32_t eph = 0;
+    Segs segs = make_segs(sk, tiles, nkb);
+    int t, kb0, nk, slot, nseg;
+    while (segs.next(t, kb0, nk, slot, nseg)) {
       const int b = i & 1;
       const uint32_t use = static_cast<uint32_t>(i >> 1);
+      ++i;
       if (!warp_wait(&ctrl->tfull[b], use & 1, abortf, p.status, kStatusWaitTmemFull)) break;
-      float scale = 1.f;
+      float ssq = 0.f;
       if (NORM == kRMSNorm) {
         if (!warp_wait(&ctrl->sfull[b], use & 1, abortf, p.status, kStatusWaitStats)) break;
-        scale = ctrl->rs[b][row_local];
+        ssq = ctrl->rs[b][row_local];
       }
       tc_fence_after();
       int mb, nb;
@@ -264,6 +411,65 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
       const int m = mb * BM + row_local;
       const bool row_ok = m < M;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * BN;
+      if (nk < nkb) {
+        // stream-K: a part of the tile's K. The fp32 partial and sum(h^2) go to
+        // the tile's slot; the last CTA to arrive sums the slots.
+        float* sp = p.part + (static_cast<size_t>(t) * p.max_seg + slot) * SLOT_FLOATS;
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          uint32_t a0[16], a1[16];
+          tmem_ld16(tbase + cc * 32, a0);
+          tmem_ld16(tbase + cc * 32 + 16, a1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int g8 = 0; g8 < 4; ++g8) {
+            float* dst = sp + (static_cast<size_t>(cc * 4 + g8) * BM + row_local) * 8;
+            float4 lo4, hi4;
+            const uint32_t* src = g8 < 2 ? a0 + g8 * 8 : a1 + (g8 - 2) * 8;
+            lo4.x = __uint_as_float(src[0]); lo4.y = __uint_as_float(src[1]);
+            lo4.z = __uint_as_float(src[2]); lo4.w = __uint_as_float(src[3]);
+            hi4.x = __uint_as_float(src[4]); hi4.y = __uint_as_float(src[5]);
+            hi4.z = __uint_as_float(src[6]); hi4.w = __uint_as_float(src[7]);
+            reinterpret_cast<float4*>(dst)[0] = lo4;
+            reinterpret_cast<float4*>(dst)[1] = hi4;
+          }
+        }
+        if (NORM == kRMSNorm) sp[BM * BN + row_local] = ssq;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->tempty[b]);
+        // arrival (as in the small-M kernel: the epilogue mbarrier orders the
+        // slot stores before thread et 0's acquire-release atomic)
+        if (lane == 0) mbar_arrive(&ctrl->esync);
+        if (!warp_wait(&ctrl->esync, eph, abortf, p.status, kStatusWaitDrain)) break;
+        eph ^= 1;
+        if (et == 0) {
+          const unsigned old = atom_add_acq_rel_gpu(&p.counters[t], 1u);
+          ctrl->last_flag = (old == static_cast<unsigned>(nseg - 1)) ? 1 : 0;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->esync);
+        if (!warp_wait(&ctrl->esync, eph, abortf, p.status, kStatusWaitDrain)) break;
+        eph ^= 1;
+        if (ctrl->last_flag) {
+          if (segs.done()) {   // the CTA's last segment: summed by all warps below
+            if (et == 0) {
+              ctrl->fin_t = t;
+              ctrl->fin_nseg = nseg;
+              ctrl->fin_go = 1;
+            }
+          } else {
+            k2_reduce_tile<EPI, NORM, NUM_EPI_WARPS * 32>(p, t, nseg, et, num_m, num_n);
+            if (et == 0) p.counters[t] = 0u;
+          }
+        }
+        continue;
+      }
+      float scale = 1.f;
+      if (NORM == kRMSNorm) {
+        scale = 1.f / sqrtf(ssq / static_cast<float>(K) + p.eps);
+        if (nb == 0 && row_ok && p.rstd_out != nullptr) p.rstd_out[m] = scale;
+      }
       if (EPI == kEpiSwiGLU) {
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
@@ -328,7 +534,9 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
     uint32_t s = 0, ph = 0;
     int i = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++i) {
+    Segs segs = make_segs(sk, tiles, nkb);
+    int t, kb0, nk, slot, nseg;
+    while (ok && segs.next(t, kb0, nk, slot, nseg)) {
       int mb, nb;
       tile_coords(t, num_m, num_n, mb, nb);
       float mu[RPT], rs[RPT];
@@ -346,7 +554,7 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
         }
       }
       const bool write_res = (NORM == kRMSNorm) && nb == 0;
-      for (int kb = 0; kb < nkb; ++kb) {
+      for (int kb = kb0; kb < kb0 + nk; ++kb) {
         if (!warp_wait(&ctrl->full_x[s], ph, abortf, p.status, kStatusWaitFull)) {
           ok = false;
           break;
@@ -417,23 +625,27 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
         const int b = i & 1;
         const uint32_t use = static_cast<uint32_t>(i >> 1);
         if (!warp_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty)) break;
-        if (c == 0) {
+        if (c == 0) {   // the segment's sum(h^2) per row; the epilogue turns it into 1/rms
 #pragma unroll
           for (int j = 0; j < RPT; ++j) {
             const int row = rbase + ROW_STRIDE * j;
-            if (row >= BM) continue;
-            const float r = 1.f / sqrtf(sst[j] / static_cast<float>(K) + p.eps);
-            ctrl->rs[b][row] = r;
-            const int gm = mb * BM + row;
-            if (write_res && p.rstd_out != nullptr && gm < M) p.rstd_out[gm] = r;
+            if (row < BM) ctrl->rs[b][row] = sst[j];
           }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->sfull[b]);
       }
+      ++i;
     }
   }
 
+  // Every role's loop is over (each bounded wait returns), so all warps meet
+  // here; a tile completed by this CTA's last stream-K segment is summed by all.
+  __syncthreads();
+  if (ctrl->fin_go && *abortf == 0) {
+    k2_reduce_tile<EPI, NORM, NUM_THREADS>(p, ctrl->fin_t, ctrl->fin_nseg, threadIdx.x, num_m, num_n);
+    if (threadIdx.x == 0) p.counters[ctrl->fin_t] = 0u;
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == WARP_MMA) {

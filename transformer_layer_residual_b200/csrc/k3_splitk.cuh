@@ -75,16 +75,6 @@ __host__ __device__ inline uint32_t tmem_cols(int mpad) {
   while (c < static_cast<uint32_t>(2 * mpad)) c <<= 1;
   return c;
 }
-// Index of the CTA whose unit range contains unit u (units split as g*U/G).
-__host__ __device__ inline int unit_owner(long long u, int G, long long U) {
-  return static_cast<int>(((u + 1) * G - 1) / U);
-}
-// The same in double precision (exact: every operand is an integer below 2^53
-// and a quotient that is not an integer is at least 1/U away from one).
-__device__ __forceinline__ int unit_owner_fast(long long u, int G, long long U) {
-  return static_cast<int>((static_cast<double>(u + 1) * G - 1.0) / static_cast<double>(U));
-}
-
 __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer();
   while (!mbar_try_wait(bar, parity)) {
