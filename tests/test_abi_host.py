@@ -71,3 +71,23 @@ def test_create_without_a_usable_device_fails_cleanly():
     h = ctypes.c_void_p()
     st = fnl.lib().fnl_create(ctypes.byref(h), 0, None)
     assert st in (4, 5) and not h.value
+
+
+def _header_enum_values():
+    with open(os.path.join(ROOT, "include", "fnl.h")) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    return {k: int(v) for k, v in re.findall(r"\b(FNL_[A-Z_]+)\s*=\s*(\d+)", text)}
+
+
+def test_binding_codes_match_the_header():
+    """The binding's names for paths, norms, precisions and status codes are
+    the header's enum values (a mismatch would silently pick another kernel)."""
+    e = _header_enum_values()
+    paths = {"auto": "FNL_PATH_AUTO", "tile": "FNL_PATH_TILE", "splitk": "FNL_PATH_SPLITK",
+             "wide": "FNL_PATH_TILE_WIDE", "cluster": "FNL_PATH_SPLITK_CLUSTER"}
+    assert {k: e[v] for k, v in paths.items()} == fnl.PATHS
+    assert {"layernorm": e["FNL_NORM_LAYERNORM"], "rmsnorm": e["FNL_NORM_RMSNORM"]} == fnl.NORMS
+    precisions = {"default": "FNL_PRECISION_DEFAULT", "split": "FNL_PRECISION_SPLIT",
+                  "single": "FNL_PRECISION_SINGLE"}
+    assert {k: e[v] for k, v in precisions.items()} == fnl.PRECISIONS
+    assert {e[n]: n for n in fnl.STATUS_NAMES.values()} == fnl.STATUS_NAMES
