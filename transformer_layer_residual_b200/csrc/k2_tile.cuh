@@ -12,15 +12,18 @@
 //               GELU, bf16 stores straight to the outputs;
 //   warps 6-17  converters: in place in shared memory, turn the x tile into the
 //               normalised bf16 A operand a = norm(x + r (+ bias_in)) using the
-//               residual tile, so the normalised activations never touch global
-//               memory (the "shared memory caching of normalised values /
-//               eliminating the intermediate write-back" of TensorRT-LLM
-//               深度工程实践, §2.3).
+//               residual tile, so the normalised activations stay on chip and
+//               are never written back (the LayerNorm + projection fusion of
+//               TensorRT-LLM 深度工程实践, §2.3).
 // LayerNorm: (mean, rstd) per row come from the statistics kernel (K1).
 // RMSNorm: deferred scaling. The converters write a' = bf16(gamma * h) and sum
-// h^2 per row over the K loop; 1/rms is applied per accumulator row in the
-// epilogue (y = rstd * sum_k a'_k W_nk is the same product). Tiles in the first
-// N column also write residual_out and rstd_out, so RMSNorm needs no extra pass.
+// h^2 per row over their k-blocks; the epilogue turns the sum into 1/rms and
+// applies it per accumulator row (y = rstd * sum_k a'_k W_nk is the same
+// product), writing rstd_out for the first N column. Tiles in the first N
+// column also write residual_out, so RMSNorm needs no extra pass.
+// Work: whole tiles g, g + G, ... per CTA; when the tiles are fewer than the
+// CTAs by a fifth or more, stream-K instead: even shares of the (tile, k-block)
+// units, partial tiles summed from fp32 slots by their last CTA.
 // Each stage has a weight barrier (full_w) and an activation barrier (full_x);
 // the kernel is a programmatic dependent of the previous kernel on the stream
 // (first weight tiles before griddepcontrol.wait, everything else after it).
