@@ -8,8 +8,9 @@ from the seeded generator (``synthetic.py``) as bf16 values widened to float64.
 
 What is computed, and where the pages say so:
 
-* residual add -- the graph-optimisation layer fuses "residual + LayerNorm"
-  (TensorRT-LLM 简介, "其底层架构可拆解为四个关键层次", 图优化层); the GPT-style
+* residual add -- the graph-optimisation layer fuses the residual add with the
+  LayerNorm that follows it (TensorRT-LLM 简介, the four-layer architecture,
+  图优化层); the GPT-style
   chain Input -> Add -> Bias -> LayerNorm -> GELU is the Layer Fusion figure of
   "TRT-LLM 编译优化管线 / 构建阶段详解 / 3. Layer Fusion" (trt-llm-deep-dive).
 * LayerNorm statistics in the order mean -> variance -> rsqrt(var + eps) ->
@@ -20,8 +21,8 @@ What is computed, and where the pages say so:
   pages give no formula, so the textbook one is used (reading R3 below).
 * SwiGLU: y = SiLU(x @ gate) * (x @ up), TensorRT-LLM 深度工程实践, §2.3
   ("GEMM + 激活融合（SwiGLU）").
-* LayerNorm + Linear + GELU into one kernel: trt-llm-deep-dive, 面试视角 answer on
-  "更激进的 kernel fusion".
+* LayerNorm + Linear + GELU into one kernel: trt-llm-deep-dive, the 面试视角 answer
+  on kernel fusion beyond the standard patterns.
 * QKV projection + reshape + GQA grouping: TensorRT-LLM 深度工程实践, §2.2 图构建与
   算子映射; GQA/MQA head counts come from the model config (§2.1).
 
