@@ -25,6 +25,10 @@ What is computed, and where the pages say so:
   on kernel fusion beyond the standard patterns.
 * QKV projection + reshape + GQA grouping: TensorRT-LLM 深度工程实践, §2.2 图构建与
   算子映射; GQA/MQA head counts come from the model config (§2.1).
+* Residual-stream projection: the attention output projection and the MLP's
+  down projection are the row-split GEMMs of TensorRT-LLM 深度工程实践, §4.1
+  Tensor Parallelism; the residual connection they feed is the residual add
+  that the graph-optimisation layer fuses (TensorRT-LLM 简介, 图优化层).
 
 Readings taken where the pages are silent:
   R1 variance is the population variance (divide by K), two passes about the mean.
@@ -39,6 +43,12 @@ Readings taken where the pages are silent:
      head-major Q[h, m, d] = y[m, h*D + d]. SwiGLU's W stacks gate rows [0, I)
      over up rows [I, 2I).
   R8 residual_out is h rounded once to bf16, round-to-nearest-even.
+  R9 the residual-stream projection adds the residual after the projection and
+     its bias: out = residual + a W^T + bias, with residual [M, N] (N = the
+     hidden size the projection returns to); the stored result is out rounded
+     once to bf16. The pages name the row-split output and down projections
+     but give no formula for the residual connection; this is the pre-norm
+     transformer's plain reading.
 
 Parity pins live in tests/test_oracle_pins.py; every function here is pinned.
 """
@@ -56,5 +66,6 @@ from .core import (  # noqa: F401
     add_norm_qkv,
     add_norm_swiglu,
     add_bias_norm_gelu,
+    linear_add_residual,
     run,
 )

@@ -142,9 +142,19 @@ def add_bias_norm_gelu(x, residual, bias_in, gamma, beta, norm, eps, W, bias_out
     return _stats({"residual_out": bf16_round(h), "out": gelu_tanh(z)}, mean, rstd)
 
 
+def linear_add_residual(a, W, bias, residual) -> dict:
+    """Residual-stream projection (o_proj / down_proj) with the residual add
+    fused after it: out = residual + a W^T (+ bias), in fp64 (reading R9).
+    a [M, K] is the sublayer's activation (attention output or SwiGLU output),
+    W [N, K], residual [M, N] the residual stream."""
+    return {"out": _f64(residual) + projection(a, W, bias)}
+
+
 def run(w, inputs: dict, rows=None) -> dict:
     """Evaluate workload ``w`` (a synthetic.Workload) on ``inputs`` (tensors or
-    arrays, bf16 values), optionally on a subset of rows (the op is row-wise)."""
+    arrays, bf16 values), optionally on a subset of rows (the op is row-wise).
+    For the residual-stream projection, "x" holds the activation a and
+    "residual" the [M, N] residual stream."""
     def g(name):
         t = inputs.get(name)
         if t is None:
@@ -156,6 +166,8 @@ def run(w, inputs: dict, rows=None) -> dict:
     x, r = g("x"), g("residual")
     if rows is not None:
         x, r = x[rows], r[rows]
+    if w.op == "residual":
+        return linear_add_residual(x, g("W"), g("bias_out"), r)
     if w.op == "qkv":
         return add_norm_qkv(x, r, g("gamma"), g("beta"), w.norm, w.eps, g("W"),
                             g("bias_out"), w.Hq, w.Hkv, w.D)

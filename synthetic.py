@@ -13,7 +13,9 @@ Add+Bias+LayerNorm->Linear+GELU layer):
 Every draw is fp32 from a CPU torch.Generator seeded once per workload, rounded
 to bf16 (round to nearest even). Draw order: ragged lengths (packed workload
 only), x, residual, bias_in, gamma, beta, W, bias_out; draws a workload does not
-use are skipped.
+use are skipped. The residual-stream projection draws its activation a (kept
+under the key "x") ~ N(0, 1) [M, K], the residual stream ~ N(0, 1) [M, N], W and
+bias_out, in that order.
 """
 from __future__ import annotations
 
@@ -28,6 +30,8 @@ RMSNORM = "rmsnorm"
 QKV = "qkv"
 SWIGLU = "swiglu"
 GELU = "gelu"
+RESIDUAL = "residual"   # residual-stream projection: out = residual + a W^T (+ bias)
+NONORM = "none"
 
 
 @dataclasses.dataclass(frozen=True)
@@ -48,6 +52,7 @@ class Workload:
     has_bias_in: bool = False
     has_bias_out: bool = False
     seq_lens: Optional[tuple] = None   # packed ragged batch, M = sum(seq_lens)
+    x_loc: float = 0.0    # mean of x (edge cases with |mean| >> sigma); 0 for the workloads
 
     @property
     def n_out(self) -> int:
@@ -59,8 +64,12 @@ class Workload:
 
     def algorithmic_bytes(self) -> float:
         """Bytes the fused op must move at least once: read x and residual,
-        write residual_out, read W once, write the outputs, read the vectors."""
+        write residual_out, read W once, write the outputs, read the vectors.
+        Residual-stream projection: read a [M, K], the residual [M, N] and W
+        once, write out [M, N], read the bias."""
         M, K, N = self.M, self.K, self.N
+        if self.op == RESIDUAL:
+            return float(M * K * 2 + 2 * M * N * 2 + N * K * 2 + (N * 2 if self.has_bias_out else 0))
         b = 2 * M * K * 2 + M * K * 2 + N * K * 2 + M * self.n_out * 2
         b += K * 2 * (2 if self.norm == LAYERNORM else 1)
         if self.has_bias_in:
@@ -97,7 +106,19 @@ def workloads() -> dict:
     lens = ragged_lengths()
     w["c5_70b_rms_qkv_ragged"] = qkv(
         "c5_70b_rms_qkv_ragged", sum(lens), 8192, 64, 8, 128, RMSNORM, seq_lens=lens)
+    w.update(residual_workloads())
     return w
+
+
+def residual_workloads() -> dict:
+    """The residual-stream projections that close a Llama-3-8B layer's residual
+    loop: the attention output projection at decode (M=32, K=N=4096) and the
+    MLP down projection at prefill (M=16384 tokens, K=14336, N=4096)."""
+    return {
+        "llama3_8b_o_proj_decode": Workload("llama3_8b_o_proj_decode", RESIDUAL, NONORM, 32, 4096, 4096),
+        "llama3_8b_down_proj_prefill": Workload("llama3_8b_down_proj_prefill", RESIDUAL, NONORM, 16384,
+                                                14336, 4096),
+    }
 
 
 def _bf16(t: torch.Tensor) -> torch.Tensor:
@@ -117,7 +138,14 @@ def make_inputs(w: Workload, seed: int = 0, rows: Optional[int] = None) -> dict:
     if w.seq_lens is not None:
         torch.randint(1, 2049, (len(w.seq_lens),), generator=g)   # keeps draw order
     out = {}
-    out["x"] = _bf16(torch.randn(M, K, generator=g))
+    if w.op == RESIDUAL:   # a [M, K], residual [M, N], W [N, K], bias [N]
+        out["x"] = _bf16(torch.randn(M, K, generator=g) + w.x_loc)
+        out["residual"] = _bf16(torch.randn(M, N, generator=g))
+        out["W"] = _bf16(torch.randn(N, K, generator=g) / (K ** 0.5))
+        if w.has_bias_out:
+            out["bias_out"] = _bf16(0.02 * torch.randn(N, generator=g))
+        return out
+    out["x"] = _bf16(torch.randn(M, K, generator=g) + w.x_loc)
     out["residual"] = _bf16(torch.randn(M, K, generator=g))
     if w.has_bias_in:
         out["bias_in"] = _bf16(torch.randn(K, generator=g))
@@ -131,16 +159,19 @@ def make_inputs(w: Workload, seed: int = 0, rows: Optional[int] = None) -> dict:
 
 
 def make_custom(op: str, norm: str, M: int, K: int, *, Hq=0, Hkv=0, D=0, I=0, N=0,
-                bias_in=False, bias_out=False, eps=1e-5, seed=0) -> tuple:
+                bias_in=False, bias_out=False, eps=1e-5, seed=0, x_loc=0.0) -> tuple:
     """A workload of arbitrary shape with the same distributions (tile-tail and
-    edge-case tests)."""
-    if op == QKV:
+    edge-case tests); x_loc shifts the mean of x (e.g. x ~ N(50, 1))."""
+    if op == RESIDUAL:
+        w = Workload(f"custom_residual_{M}x{K}x{N}", RESIDUAL, NONORM, M, K, N,
+                     has_bias_out=bias_out, x_loc=x_loc)
+    elif op == QKV:
         w = qkv(f"custom_qkv_{M}x{K}", M, K, Hq, Hkv, D, norm, eps=eps,
-                has_bias_in=bias_in, has_bias_out=bias_out)
+                has_bias_in=bias_in, has_bias_out=bias_out, x_loc=x_loc)
     elif op == SWIGLU:
         w = Workload(f"custom_swiglu_{M}x{K}", SWIGLU, norm, M, K, 2 * I, I=I, eps=eps,
-                     has_bias_in=bias_in, has_bias_out=bias_out)
+                     has_bias_in=bias_in, has_bias_out=bias_out, x_loc=x_loc)
     else:
         w = Workload(f"custom_gelu_{M}x{K}", GELU, norm, M, K, N, eps=eps,
-                     has_bias_in=bias_in, has_bias_out=bias_out)
+                     has_bias_in=bias_in, has_bias_out=bias_out, x_loc=x_loc)
     return w, make_inputs(w, seed=seed)

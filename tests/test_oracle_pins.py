@@ -282,9 +282,96 @@ def pin_residual_out(ora):
     assert np.array_equal(o["residual_out"][exact], s32.to(torch.bfloat16).double().numpy()[exact])
 
 
+def pin_run_maps_workload_inputs(ora):
+    """run(): the workload's tensors reach the right arguments. Every optional
+    vector present (beta, bias_in, bias_out), an unsorted non-contiguous row
+    subset, and the expected values from the per-element loops on the rows
+    picked by hand, for all three epilogues and both norms."""
+    import synthetic
+    rows = np.array([5, 0, 3, 6], dtype=np.int64)
+    cases = [synthetic.make_custom("qkv", "layernorm", 7, 16, Hq=2, Hkv=1, D=4, bias_out=True, seed=40),
+             synthetic.make_custom("qkv", "rmsnorm", 7, 16, Hq=2, Hkv=1, D=4, bias_out=True, seed=41),
+             synthetic.make_custom("swiglu", "layernorm", 7, 16, I=5, bias_out=True, seed=42),
+             synthetic.make_custom("gelu", "layernorm", 7, 16, N=6, bias_in=True, bias_out=True, seed=43),
+             synthetic.make_custom("gelu", "rmsnorm", 7, 16, N=6, bias_in=True, bias_out=True, seed=44)]
+    for w, inputs in cases:
+        f = {k: v.double().numpy() for k, v in inputs.items()}
+        beta = f.get("beta")
+        got = ora.run(w, inputs, rows=rows)
+        ref = _brute(w.op, f["x"][rows].tolist(), f["residual"][rows].tolist(), f.get("bias_in"), f["gamma"],
+                     beta, w.norm, w.eps, f["W"].tolist(), f.get("bias_out"))["rows"]
+        for i, m in enumerate(rows):
+            h = f["x"][m] + f["residual"][m] + (f["bias_in"] if "bias_in" in f else 0.0)
+            assert np.array_equal(got["residual_out"][i], ora.bf16_round(h))
+            if w.norm == "layernorm":
+                assert abs(got["mean"][i] - h.mean()) <= 1e-13
+                assert abs(got["rstd"][i] - 1.0 / math.sqrt(np.var(h) + w.eps)) <= 1e-12 * got["rstd"][i]
+            else:
+                assert abs(got["rstd"][i] - 1.0 / math.sqrt(np.mean(h * h) + w.eps)) <= 1e-12 * got["rstd"][i]
+            y = ref[i]
+            if w.op == "qkv":
+                D = w.D
+                for n in range(w.N):
+                    if n < w.Hq * D:
+                        g = got["q"][n // D, i, n % D]
+                    elif n < (w.Hq + w.Hkv) * D:
+                        g = got["k"][(n - w.Hq * D) // D, i, n % D]
+                    else:
+                        g = got["v"][(n - (w.Hq + w.Hkv) * D) // D, i, n % D]
+                    assert abs(g - y[n]) <= 1e-12
+            elif w.op == "swiglu":
+                for j in range(w.I):
+                    gate, up = y[j], y[w.I + j]
+                    assert abs(got["out"][i, j] - gate / (1.0 + math.exp(-gate)) * up) <= 1e-12
+            else:
+                c = math.sqrt(2.0 / math.pi)
+                for n in range(w.N):
+                    z = y[n]
+                    assert abs(got["out"][i, n] - 0.5 * z * (1.0 + math.tanh(c * (z + 0.044715 * z ** 3)))) <= 1e-12
+
+
+def pin_residual_projection(ora):
+    """out = residual + a W^T + bias: identity W gives residual + a + bias;
+    a one-hot row a = s e_j gives residual[n] + s W[n, j] + bias[n] (exposes
+    W's index order); per-element loops on a tiny non-square shape; run() maps
+    the workload's tensors (a under "x", the [M, N] residual) on a row subset."""
+    M, K = 4, 12
+    a, res, bias = _rand((M, K), 60), _rand((M, K), 61), _rand(K, 62, 0.02)
+    out = ora.linear_add_residual(a, np.eye(K), bias, res)["out"]
+    assert np.max(np.abs(out - (res + a + bias[None, :]))) <= 1e-15
+    N, j, sc = 7, 5, 2.5
+    W = _rand((N, K), 63)
+    oh = np.zeros((1, K))
+    oh[0, j] = sc
+    Wsq = _rand((K, K), 69)   # square: a transposed W would still have the right shape
+    out = ora.linear_add_residual(oh, Wsq, None, np.zeros((1, K)))["out"]
+    assert np.max(np.abs(out[0] - sc * Wsq[:, j])) <= 1e-14
+    r1 = _rand((1, N), 64)
+    out = ora.linear_add_residual(oh, W, None, r1)["out"]
+    assert np.max(np.abs(out[0] - (r1[0] + sc * W[:, j]))) <= 1e-14
+    a, res, b = _rand((3, K), 65), _rand((3, N), 66), _rand(N, 67, 0.02)
+    out = ora.linear_add_residual(a, W, b, res)["out"]
+    for m in range(3):
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                acc += a[m, k] * W[n, k]
+            assert abs(out[m, n] - (res[m, n] + acc + b[n])) <= 1e-12
+    import synthetic
+    w, inputs = synthetic.make_custom("residual", "none", 6, 16, N=24, bias_out=True, seed=68)
+    rows = np.array([4, 1, 2], dtype=np.int64)
+    f = {k: v.double().numpy() for k, v in inputs.items()}
+    got = ora.run(w, inputs, rows=rows)["out"]
+    for i, m in enumerate(rows):
+        for n in range(24):
+            acc = sum(f["x"][m, k] * f["W"][n, k] for k in range(16))
+            assert abs(got[i, n] - (f["residual"][m, n] + acc + f["bias_out"][n])) <= 1e-12
+
+
 PINS = [pin_layernorm_invariants, pin_rmsnorm_invariant, pin_norms_match_torch,
         pin_identity_weight, pin_one_hot, pin_brute_force, pin_epilogue_values,
-        pin_qkv_bijection, pin_bf16_round, pin_residual_out]
+        pin_qkv_bijection, pin_bf16_round, pin_residual_out,
+        pin_run_maps_workload_inputs, pin_residual_projection]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -296,7 +383,7 @@ def test_pin_holds(pin):
 # planted mistakes: every one must break at least one pin
 # --------------------------------------------------------------------------
 
-ORIG = {name: getattr(core, name) for name in ("layernorm", "rmsnorm", "split_qkv_head_major")}
+ORIG = {name: getattr(core, name) for name in ("layernorm", "rmsnorm", "split_qkv_head_major", "run")}
 
 
 def _ln_unbiased(h, gamma, beta, eps):
@@ -399,6 +486,44 @@ def _bf16_truncate(v):
     return np.ldexp(np.trunc(m * 256.0) / 256.0, e)
 
 
+def _run_subsets_x_only(w, inputs, rows=None):
+    """x is taken in the rows' order, the residual in sorted row order."""
+    if rows is None:
+        return ORIG["run"](w, inputs, rows)
+    rows = np.asarray(rows)
+    sub = {**inputs, "x": inputs["x"][rows], "residual": inputs["residual"][np.sort(rows)]}
+    return ORIG["run"](w, sub, None)
+
+
+def _run_drops(name):
+    def run(w, inputs, rows=None):
+        return ORIG["run"](w, {k: v for k, v in inputs.items() if k != name}, rows)
+    return run
+
+
+def _run_qkv_bias_dropped(w, inputs, rows=None):
+    if w.op != "qkv":
+        return ORIG["run"](w, inputs, rows)
+    return _run_drops("bias_out")(w, inputs, rows)
+
+
+def _resid_dropped(a, W, bias, residual):
+    return {"out": core.projection(a, W, bias)}
+
+
+def _resid_bias_dropped(a, W, bias, residual):
+    return {"out": np.asarray(residual, np.float64) + np.asarray(a) @ np.asarray(W).T}
+
+
+def _resid_w_untransposed(a, W, bias, residual):
+    y = np.asarray(a) @ np.asarray(W)
+    return {"out": np.asarray(residual, np.float64) + y + (0 if bias is None else np.asarray(bias)[None])}
+
+
+def _resid_subtracted(a, W, bias, residual):
+    return {"out": core.projection(a, W, bias) - np.asarray(residual, np.float64)}
+
+
 MUTANTS = {
     "variance_divides_by_K_minus_1": ("layernorm", _ln_unbiased),
     "eps_outside_sqrt": ("layernorm", _ln_eps_outside),
@@ -417,6 +542,14 @@ MUTANTS = {
     "bias_in_dropped": ("residual_add", _residual_drops_bias_in),
     "residual_ignored": ("residual_add", _residual_ignores_residual),
     "bf16_truncates": ("bf16_round", _bf16_truncate),
+    "run_residual_rows_misordered": ("run", _run_subsets_x_only),
+    "run_drops_bias_in": ("run", _run_drops("bias_in")),
+    "run_drops_beta": ("run", _run_drops("beta")),
+    "run_qkv_bias_dropped": ("run", _run_qkv_bias_dropped),
+    "residual_projection_drops_residual": ("linear_add_residual", _resid_dropped),
+    "residual_projection_drops_bias": ("linear_add_residual", _resid_bias_dropped),
+    "residual_projection_w_untransposed": ("linear_add_residual", _resid_w_untransposed),
+    "residual_projection_subtracts_residual": ("linear_add_residual", _resid_subtracted),
 }
 
 
