@@ -1,23 +1,30 @@
 """Benchmark of the fused pre-norm linear layer (one JSON line on stdout).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fnl|reference]
-                    [--workload NAME] [--sweep]
+                    [--workload NAME] [--no-sweep]
 
 A step is one fused call (residual add -> norm -> projection -> epilogue) over
-one batch of seeded synthetic inputs of the chosen workload (default: the
-Llama-3-8B-shaped decode QKV, M=32, K=4096, N=6144, RMSNorm). Inputs are
-resident in HBM before timing; the calls of the timed region are replayed from
-a CUDA graph (the host cost of a Python call is larger than a decode kernel),
-rotating over enough copies of W / x / residual to exceed 3x the L2 size so
-that every step streams its weights from HBM. `value` is the algorithmic HBM
-traffic (or FLOP) rate of the whole job; `e2e` times the same calls through the
-Python binding with the inputs copied from pinned host memory and the outputs
-copied back inside the timed region. Multi-GPU runs are independent replicas
-(the op has no exchange step): value = all ranks' work / max rank time.
+one batch of seeded synthetic inputs of the chosen workload. The default is the
+largest single-GPU workload, the Llama-2-70B-shaped packed QKV batch (64
+sequences of lengths uniform in [1, 2048], M = 62386, K = 8192, N = 10240,
+RMSNorm). Inputs are resident in HBM before timing; the calls of the timed
+region are replayed from CUDA graphs (every graph is replayed once before the
+timed region), rotating over enough copies of W / x / residual to exceed 3x the
+L2 size so that every step streams its weights from HBM. `value` is the
+algorithmic FLOP (or HBM byte) rate of the whole job; `e2e` times the same calls
+through the Python binding with the inputs copied from pinned host memory and
+the outputs copied back inside the timed region; `host_us_per_call` is the host
+cost of one bare C-ABI call (device buffers, no copies). Multi-GPU runs are
+independent replicas (the op has no exchange step): value = all ranks' work /
+max rank time.
+
+The same line carries `sweep`: one entry per workload (every shape of the
+M sweep), each timed on its own CUDA graph for at least 100 ms, with its
+fraction of the roofline, its median SM clock and, for the HBM-bound shapes, the
+time of one isolated call after an L2 flush.
 
 --impl reference times the fp64 CPU oracle (the only reference this op has) on
-the same workload; --sweep prints one line per workload to stderr after the
-main line (the main line stays the only stdout line).
+the same workload.
 """
 from __future__ import annotations
 
@@ -40,7 +47,7 @@ import torch  # noqa: E402
 import synthetic  # noqa: E402
 
 METRIC = "fused norm+GEMM TFLOP/s & GB/s (% of B200 roofline) vs M; tokens/s/layer"
-DEFAULT_WORKLOAD = "c2_decode_rms_qkv"
+DEFAULT_WORKLOAD = "c5_70b_rms_qkv_ragged"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 HBM_BOUND_AI = 250.0   # FLOP/byte below which a workload is HBM-bound on B200 (measured ridge)
 
@@ -182,110 +189,205 @@ def units(w):
 
 
 # ------------------------------------------------------------------------- fnl arm
-def bench_fnl(w, steps, warmup, world, rank, local, sweep_line=False):
-    from transformer_layer_residual_b200 import fnl
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    inputs = synthetic.make_inputs(w, seed=0)
-    per_copy = sum(t.numel() * t.element_size() for k, t in inputs.items() if k in ("x", "residual", "W"))
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    R = max(1, min(16, -(-3 * l2 // per_copy)))
-    copies = []
-    for i in range(R):
-        c = {k: v.to(dev) for k, v in inputs.items()}
-        copies.append(c)
-    M = w.M
-    h = fnl.Handle(local, max_tokens=M, max_n=w.N)
-    outs = []
-    for c in copies:   # pre-allocate outputs per copy so the graph holds fixed pointers
-        o = fnl.run_workload(h, w, c, stats=True)
-        outs.append(o)
-    h.check()
+class Bed:
+    """One workload on the device: R rotating copies of the inputs (together
+    larger than 3x L2), their pre-allocated outputs, and the call of copy i
+    through the Python binding (fixed pointers, so CUDA graphs replay the same
+    calls)."""
 
-    def call(i):
-        c, o = copies[i], outs[i]
-        if w.op == "qkv":
-            fnl.add_norm_qkv(h, c["x"], c["residual"], c["gamma"], c.get("beta"), c["W"], w.Hq, w.Hkv, w.D,
+    def __init__(self, w, local, inputs=None, tune=True, path="auto"):
+        from transformer_layer_residual_b200 import fnl
+        self.fnl = fnl
+        self.w = w
+        self.dev = torch.device("cuda", local)
+        self.inputs = synthetic.make_inputs(w, seed=0) if inputs is None else inputs
+        self.per_copy = sum(t.numel() * t.element_size() for k, t in self.inputs.items()
+                            if k in ("x", "residual", "W"))
+        self.l2 = torch.cuda.get_device_properties(self.dev).L2_cache_size
+        self.R = max(1, min(16, -(-3 * self.l2 // self.per_copy)))
+        self.copies = [{k: v.to(self.dev) for k, v in self.inputs.items()} for _ in range(self.R)]
+        # shape auto-tuning: the first call below times the candidate plans
+        self.h = fnl.Handle(local, max_tokens=w.M, max_n=w.N, tune=tune and path == "auto", path=path)
+        self.outs = [fnl.run_workload(self.h, w, c, stats=True) for c in self.copies]
+        self.h.check()
+        self.plan = self.h.last_plan()
+        self.stream = torch.cuda.Stream(self.dev)
+
+    def call(self, i):
+        fnl, w, c, o = self.fnl, self.w, self.copies[i], self.outs[i]
+        if w.op == "residual":
+            fnl.linear_add_residual(self.h, c["x"], c["W"], c["residual"], bias=c.get("bias_out"), out=o["out"])
+        elif w.op == "qkv":
+            fnl.add_norm_qkv(self.h, c["x"], c["residual"], c["gamma"], c.get("beta"), c["W"], w.Hq, w.Hkv, w.D,
                              norm=w.norm, eps=w.eps, bias=c.get("bias_out"), residual_out=o["residual_out"],
                              q=o["q"], k=o["k"], v=o["v"], mean_out=o["mean"], rstd_out=o["rstd"])
         elif w.op == "swiglu":
-            fnl.add_norm_swiglu(h, c["x"], c["residual"], c["gamma"], c.get("beta"), c["W"], w.I, norm=w.norm,
-                                eps=w.eps, bias=c.get("bias_out"), residual_out=o["residual_out"], out=o["out"],
-                                mean_out=o["mean"], rstd_out=o["rstd"])
+            fnl.add_norm_swiglu(self.h, c["x"], c["residual"], c["gamma"], c.get("beta"), c["W"], w.I,
+                                norm=w.norm, eps=w.eps, bias=c.get("bias_out"), residual_out=o["residual_out"],
+                                out=o["out"], mean_out=o["mean"], rstd_out=o["rstd"])
         else:
-            fnl.add_bias_norm_gelu(h, c["x"], c["residual"], c["gamma"], c.get("beta"), c["W"],
+            fnl.add_bias_norm_gelu(self.h, c["x"], c["residual"], c["gamma"], c.get("beta"), c["W"],
                                    bias_in=c.get("bias_in"), bias_out=c.get("bias_out"), norm=w.norm, eps=w.eps,
                                    residual_out=o["residual_out"], out=o["out"], mean_out=o["mean"],
                                    rstd_out=o["rstd"])
 
-    stream = torch.cuda.Stream(dev)
-    # graphs: one of R calls (copy 0..R-1), one of the remainder
-    def capture(n):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(stream):
-            for i in range(n):   # eager pass on the capture stream first
-                call(i % R)
-        stream.synchronize()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(n):
-                call(i % R)
-        return g
-    g_full = capture(R)
-    rem = steps % R
-    g_rem = capture(rem) if rem else None
-    n_full = steps // R
+    def raw_call(self, i):
+        """(C function, argument tuple) of the bare C-ABI call for copy i."""
+        import ctypes
+        L, w, c, o = self.fnl.lib(), self.w, self.copies[i], self.outs[i]
+        P = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())  # noqa: E731
+        st = ctypes.c_void_p(self.stream.cuda_stream)
+        if w.op == "residual":
+            return L.fnl_linear_add_residual, (self.h.ptr, st, P(c["x"]), P(c["W"]), P(c.get("bias_out")),
+                                               P(c["residual"]), P(o["out"]), w.M, w.K, w.N)
+        norm = self.fnl.NORMS[w.norm]
+        eps = ctypes.c_float(w.eps)
+        common = (P(c["x"]), P(c["residual"]))
+        if w.op == "qkv":
+            return L.fnl_add_norm_qkv, (self.h.ptr, st, *common, P(o["residual_out"]), P(c["gamma"]),
+                                        P(c.get("beta")), norm, eps, P(c["W"]), P(c.get("bias_out")), w.M, w.K,
+                                        w.Hq, w.Hkv, w.D, P(o["q"]), P(o["k"]), P(o["v"]), P(o["mean"]),
+                                        P(o["rstd"]))
+        if w.op == "swiglu":
+            return L.fnl_add_norm_swiglu, (self.h.ptr, st, *common, P(o["residual_out"]), P(c["gamma"]),
+                                           P(c.get("beta")), norm, eps, P(c["W"]), P(c.get("bias_out")), w.M,
+                                           w.K, w.I, P(o["out"]), P(o["mean"]), P(o["rstd"]))
+        return L.fnl_add_bias_norm_gelu, (self.h.ptr, st, *common, P(c.get("bias_in")), P(o["residual_out"]),
+                                          P(c["gamma"]), P(c.get("beta")), norm, eps, P(c["W"]),
+                                          P(c.get("bias_out")), w.M, w.K, w.N, P(o["out"]), P(o["mean"]),
+                                          P(o["rstd"]))
 
-    def run_steps():
-        for _ in range(n_full):
+    def graph(self, n):
+        """A CUDA graph of n calls over the copies (an eager pass first)."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(self.stream):
+            for i in range(n):
+                self.call(i % self.R)
+        self.stream.synchronize()
+        with torch.cuda.graph(g, stream=self.stream):
+            for i in range(n):
+                self.call(i % self.R)
+        return g
+
+    def timed(self, replays):
+        """Device time (ms) of the graph replays in `replays` (a list), CUDA
+        events on the launch stream."""
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(self.stream):
+            ev0.record(self.stream)
+            for g in replays:
+                g.replay()
+            ev1.record(self.stream)
+        ev1.synchronize()
+        return ev0.elapsed_time(ev1)
+
+    def host_us_per_call(self, n):
+        """Host time of one bare C-ABI call (prebuilt ctypes arguments, device
+        buffers, no copies), mean over n calls; the GPU runs them meanwhile."""
+        fn, args = self.raw_call(0)
+        self.stream.synchronize()
+        fn(*args)
+        t0 = time.perf_counter()
+        for _ in range(n):
+            st = fn(*args)
+        t1 = time.perf_counter()
+        self.stream.synchronize()
+        assert st == 0, st
+        return (t1 - t0) / n * 1e6
+
+    def isolated_us(self, reps=15):
+        """One call after an L2 flush, GPU otherwise idle: median device time of
+        the call alone (no programmatic overlap with a previous call)."""
+        g1 = self.graph(1)
+        flush = torch.empty(1 << 29, dtype=torch.uint8, device=self.dev)   # 512 MB > 3x L2
+        ts = []
+        with torch.cuda.stream(self.stream):
+            for _ in range(reps + 1):
+                flush.fill_(1)
+                ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                ev0.record(self.stream)
+                g1.replay()
+                ev1.record(self.stream)
+                ev1.synchronize()
+                ts.append(ev0.elapsed_time(ev1) * 1e3)
+        del flush
+        return float(np.median(ts[1:]))
+
+    def close(self):
+        self.h.check()
+        self.h.close()
+
+
+def _roofline(w, per_launch_ms, bound):
+    pk, pk_src = peaks()
+    if bound == "hbm":
+        achieved = w.algorithmic_bytes() / (per_launch_ms / 1e3) / 1e9
+        return achieved, pk["hbm_gbs"], "GB/s", f"{pk_src} hbm_gbs"
+    # a tensor-bound call runs back to back for the whole timed region, so its
+    # denominator is the GEMM throughput sustained under the power cap
+    achieved = w.flops() / (per_launch_ms / 1e3) / 1e12
+    return achieved, pk["bf16_tflops_sustained"], "TFLOP/s", f"{pk_src} bf16_tflops_sustained"
+
+
+def _sustain(bed, g, seconds):
+    """Keep replaying g for `seconds` (clock record of short timed regions)."""
+    t_end = time.time() + seconds
+    with torch.cuda.stream(bed.stream):
+        while time.time() < t_end:
+            g.replay()
+            bed.stream.synchronize()
+
+
+def bench_fnl(w, steps, warmup, world, rank, local, tune=True, path="auto"):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    bed = Bed(w, local, tune=tune, path=path)
+    R = bed.R
+    # graphs: one of R calls (copy 0..R-1), one of the remainder; both replayed
+    # during warm-up so that no graph's first replay lands in the timed region
+    g_full = bed.graph(R)
+    rem = steps % R
+    g_rem = bed.graph(rem) if rem else None
+    n_full = steps // R
+    with torch.cuda.stream(bed.stream):
+        for _ in range(max(1, -(-warmup // R))):
             g_full.replay()
         if g_rem is not None:
             g_rem.replay()
-
-    with torch.cuda.stream(stream):
-        for _ in range(max(1, -(-warmup // R))):
-            g_full.replay()
-    stream.synchronize()
-    h.check()
+    bed.stream.synchronize()
+    bed.h.check()
 
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
     barrier(world)
     torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_wall0 = time.time()
-    with torch.cuda.stream(stream):
-        ev0.record(stream)
-        run_steps()
-        ev1.record(stream)
-    ev1.synchronize()
+    ms = bed.timed([g_full] * n_full + ([g_rem] if g_rem is not None else []))
     t_wall1 = time.time()
     barrier(world)
     torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1)
-    # keep the same loop running ~1.5 s for the clock record if the timed region was short
-    if t_wall1 - t_wall0 < 1.0:
-        t_end = time.time() + 1.5
-        with torch.cuda.stream(stream):
-            while time.time() < t_end:
-                run_steps()
-                stream.synchronize()
+    if t_wall1 - t_wall0 < 1.0:   # keep the same loop running for the clock record
+        _sustain(bed, g_full, 1.5)
     sampler.stop()
     clocks = sampler.summary(t_wall0, t_wall1)
-    h.check()
+    bed.h.check()
     ms_max = max_over_ranks(ms, world)
 
     unit, per_step, bound = units(w)
     value = per_step * steps * world / (ms_max / 1e3)
     launches_per_step = 2 if w.norm == "layernorm" else 1
+    host_us = bed.host_us_per_call(50 if w.flops() < 1e12 else 10)
 
     # e2e: through the public binding, host buffers, copies inside the timed region
+    inputs, stream = bed.inputs, bed.stream
     x_h = inputs["x"].pin_memory()
     r_h = inputs["residual"].pin_memory()
-    c0, o0 = copies[0], outs[0]
+    c0, o0 = bed.copies[0], bed.outs[0]
     out_keys = ("q", "k", "v") if w.op == "qkv" else ("out",)
     host_out = {k: torch.empty(o0[k].shape, dtype=o0[k].dtype, pin_memory=True) for k in out_keys}
-    host_res = torch.empty(o0["residual_out"].shape, dtype=torch.bfloat16, pin_memory=True)
+    if "residual_out" in o0:
+        host_out["residual_out"] = torch.empty(o0["residual_out"].shape, dtype=torch.bfloat16, pin_memory=True)
     e2e_steps = max(3, min(steps, 200))
     with torch.cuda.stream(stream):
         for i in range(e2e_steps + 3):
@@ -296,29 +398,19 @@ def bench_fnl(w, steps, warmup, world, rank, local, sweep_line=False):
                 e0.record(stream)
             c0["x"].copy_(x_h, non_blocking=True)
             c0["residual"].copy_(r_h, non_blocking=True)
-            call(0)
-            for k in out_keys:
-                host_out[k].copy_(o0[k], non_blocking=True)
-            host_res.copy_(o0["residual_out"], non_blocking=True)
+            bed.call(0)
+            for k, t in host_out.items():
+                t.copy_(o0[k], non_blocking=True)
         e1.record(stream)
     e1.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     h2d = x_h.numel() * 2 + r_h.numel() * 2
-    d2h = sum(t.numel() * 2 for t in host_out.values()) + host_res.numel() * 2
+    d2h = sum(t.numel() * 2 for t in host_out.values())
     e2e_value = per_step * e2e_steps * world / (e2e_ms / 1e3)
+    del x_h, r_h, host_out
 
-    pk, pk_src = peaks()
     per_launch_ms = ms / steps
-    if bound == "hbm":
-        achieved = w.algorithmic_bytes() / (per_launch_ms / 1e3) / 1e9
-        peak = pk["hbm_gbs"]
-        runit = "GB/s"
-    else:
-        # a tensor-bound step runs back to back for the whole timed region, so
-        # its denominator is the GEMM throughput sustained under the power cap
-        achieved = w.flops() / (per_launch_ms / 1e3) / 1e12
-        peak = pk["bf16_tflops_sustained"]
-        runit = "TFLOP/s"
+    achieved, peak, runit, peak_src = _roofline(w, per_launch_ms, bound)
     line = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -335,25 +427,75 @@ def bench_fnl(w, steps, warmup, world, rank, local, sweep_line=False):
         "config": {"workload": w.name, "op": w.op, "norm": w.norm, "M": w.M, "K": w.K, "N": w.N,
                    **({"Hq": w.Hq, "Hkv": w.Hkv, "D": w.D} if w.op == "qkv" else {}),
                    **({"I": w.I} if w.op == "swiglu" else {}),
+                   **({"seqs": len(w.seq_lens)} if w.seq_lens else {}),
                    "l2": f"inputs larger than L2: {R} rotating copies of W/x/residual "
-                         f"({R * per_copy / 1e6:.0f} MB vs L2 {l2 / 1e6:.0f} MB)",
+                         f"({R * bed.per_copy / 1e6:.0f} MB vs L2 {bed.l2 / 1e6:.0f} MB)",
                    "timing": f"CUDA graph replays of {R} calls, CUDA events on the launch stream",
+                   "plan": bed.plan,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "tflops": round(w.flops() * steps * world / (ms_max / 1e3) / 1e12, 3),
         "gbps": round(w.algorithmic_bytes() * steps * world / (ms_max / 1e3) / 1e9, 3),
         "tokens_per_s_layer": round(w.M * steps * world / (ms_max / 1e3), 1),
         "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": runit,
-                     "frac": round(achieved / peak, 4), "peak_source": f"{pk_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops_sustained'})",
+                     "frac": round(achieved / peak, 4), "peak_source": peak_src,
                      "traffic": recorded_traffic(w.name),
                      "algorithmic_per_launch": w.algorithmic_bytes() if bound == "hbm" else w.flops(),
                      "kernel": "fused GEMM kernel" + (" + LayerNorm stats kernel (PDL)" if w.norm == "layernorm" else "")},
         "e2e": {"value": round(e2e_value, 3), "unit": unit, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "host_us_per_call": round(host_us, 2),
         "gpu_launches": launches_per_step * steps,
         "clocks": clocks,
     }
-    h.close()
+    bed.close()
+    del bed
+    torch.cuda.empty_cache()
     return line
+
+
+def sweep_entry(w, local, min_ms=100.0, tune=True):
+    """One workload of the sweep: CUDA-graph replays for at least min_ms of
+    device time, fraction of the roofline, median SM clock over the timed
+    region (sustained for 0.6 s when shorter), isolated-call time for the
+    HBM-bound shapes, host cost of one bare C-ABI call."""
+    bed = Bed(w, local, tune=tune)
+    g = bed.graph(bed.R)
+    with torch.cuda.stream(bed.stream):
+        for _ in range(3):
+            g.replay()
+    one = bed.timed([g]) / bed.R   # ms per call, to size the timed region
+    n = max(1, int(np.ceil(min_ms / max(one * bed.R, 1e-3))))
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.2)
+    t0 = time.time()
+    ms = bed.timed([g] * n)
+    t1 = time.time()
+    if t1 - t0 < 0.6:
+        _sustain(bed, g, 0.6)
+    sampler.stop()
+    clocks = sampler.summary(t0, t1)
+    calls = n * bed.R
+    per_ms = ms / calls
+    unit, _, bound = units(w)
+    achieved, peak, runit, peak_src = _roofline(w, per_ms, bound)
+    e = {"us_per_call": round(per_ms * 1e3, 2), "calls": calls, "plan": bed.plan,
+         "M": w.M, "K": w.K, "N": w.N, "op": w.op, "norm": w.norm,
+         "tflops": round(w.flops() / (per_ms / 1e3) / 1e12, 2),
+         "gbps": round(w.algorithmic_bytes() / (per_ms / 1e3) / 1e9, 1),
+         "tokens_per_s_layer": round(w.M / (per_ms / 1e3), 1),
+         "bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": runit,
+         "frac": round(achieved / peak, 4), "peak_source": peak_src,
+         "sm_mhz": clocks.get("sm_mhz"), "clock_reasons": clocks.get("reasons"),
+         "host_us_per_call": round(bed.host_us_per_call(100 if w.flops() < 1e11 else 10), 2)}
+    if bound == "hbm":
+        iso = bed.isolated_us()
+        e["isolated_us"] = round(iso, 2)
+        e["isolated_frac"] = round(w.algorithmic_bytes() / (iso / 1e6) / 1e9 / peak, 4)
+    bed.close()
+    del bed
+    torch.cuda.empty_cache()
+    return e
 
 
 # ------------------------------------------------------------------------- oracle
@@ -414,12 +556,14 @@ def bench_reference(w, steps, warmup, world, rank, budget_s=120.0):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="fnl", choices=["fnl", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--sweep", action="store_true", help="also bench every workload (lines to stderr)")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the per-workload sweep in the line")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--no-tune", action="store_true", help="untuned plans (no shape auto-tuning)")
+    ap.add_argument("--path", default="auto", help="force a kernel for the headline workload (tests/diagnosis)")
     a = ap.parse_args()
     if a.warmup < 3:
         a.warmup = 3
@@ -434,21 +578,20 @@ def main():
             torch.distributed.destroy_process_group()
         return
 
-    line = bench_fnl(w, a.steps, a.warmup, world, rank, local)
+    line = bench_fnl(w, a.steps, a.warmup, world, rank, local, tune=not a.no_tune, path=a.path)
+    if not a.no_sweep:
+        # every rank runs the same sweep (replicas); rank 0 reports its own numbers
+        sweep = {}
+        for name, ws in synthetic.workloads().items():
+            sweep[name] = sweep_entry(ws, local, tune=not a.no_tune)
+            barrier(world)
+        line["sweep"] = sweep
     if rank == 0 and world == 1:
         rate, sample, cores, _, _ = oracle_rate(w, budget_s=a.cpu_budget)
         line["cpu_baseline"] = {"value": round(rate, 6), "unit": line["unit"], "cores": cores, "kind": "oracle",
                                 "sample": sample}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if a.sweep:
-        for name, ws in synthetic.workloads().items():
-            if name == a.workload:
-                continue
-            st = max(3, min(a.steps, int(2e4 / max(1.0, ws.flops() / 2e11))))
-            l2 = bench_fnl(ws, st, 3, world, rank, local)
-            if rank == 0:
-                print(json.dumps(l2), file=sys.stderr, flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
 

@@ -43,6 +43,8 @@
  * Requirements (checked on the host before any launch):
  *   - every bf16 pointer 16-byte aligned, fp32 outputs 4-byte aligned;
  *   - K, N (and D, I) multiples of 8; 1 <= K <= 32768; M >= 0 (M = 0 is a no-op);
+ *     N <= 65535 * 128;
+ *   - eps > 0 and finite (with eps = 0 a constant row would divide by zero);
  *   - outputs overlap neither each other nor any input;
  *   - the handle is used by one host thread / one stream at a time (its
  *     workspace is shared by its calls);
@@ -78,7 +80,7 @@ typedef struct fnl_handle fnl_handle;      /* opaque: device, workspace, last er
 
 typedef enum {
   FNL_OK = 0,
-  FNL_ERR_INVALID_ARG = 1,    /* NULL where required, bad size, bad enum, eps < 0 */
+  FNL_ERR_INVALID_ARG = 1,    /* NULL where required, bad size, bad enum, eps <= 0 or not finite */
   FNL_ERR_ALIGNMENT = 2,      /* pointer or leading dimension not aligned */
   FNL_ERR_ALIAS = 3,          /* an output overlaps an input or another output */
   FNL_ERR_UNSUPPORTED = 4,    /* shape outside what the kernels handle (K > 32768, ...) */
@@ -93,8 +95,9 @@ typedef enum {
   FNL_PATH_TILE = 1,          /* force the large-M persistent kernel, 128 x 256 tiles */
   FNL_PATH_SPLITK = 2,        /* force the small-M split-K kernel, stream-K form (requires M <= 128) */
   FNL_PATH_TILE_WIDE = 3,     /* force the large-M persistent kernel, 128 x 512 tiles */
-  FNL_PATH_SPLITK_CLUSTER = 4 /* force the small-M kernel's cluster form (M <= 128; FNL_ERR_UNSUPPORTED when
-                                 the tiles cannot all run at once as clusters of 2..8 CTAs) */
+  FNL_PATH_SPLITK_CLUSTER = 4, /* force the small-M kernel's cluster form (M <= 128; FNL_ERR_UNSUPPORTED when
+                                  the tiles cannot all run at once as clusters of 2..8 CTAs) */
+  FNL_PATH_TILE_PAIR = 5       /* force the large-M kernel on CTA pairs (tcgen05 cta_group::2), 256 x 512 tiles */
 } fnl_path;
 
 /* How the normalised activation a is rounded for the bf16 tensor cores.
@@ -115,6 +118,25 @@ typedef struct {
   int path;         /* fnl_path */
   int max_ctas;     /* cap on persistent CTAs (0: one per SM) -- for tests */
   int precision;    /* fnl_precision */
+  long long wait_ns;      /* limit of the kernels' main-loop waits in ns (0: 4 s). A wait that
+                             runs out aborts its CTA and records a code for fnl_check. */
+  int debug_stall_calls;  /* fault injection for tests of the status path: the next this-many
+                             calls withhold one weight copy in their first CTA, so a wait for it
+                             runs out after wait_ns (their outputs are then incomplete and
+                             fnl_check reports FNL_ERR_DEVICE_STATUS). 0 in normal use. */
+  int tune;               /* 1: shape auto-tuning (TensorRT-LLM 深度工程实践, §2.4 内核自动调优:
+                             candidate kernels run on the target GPU, the fastest is kept). With
+                             path = FNL_PATH_AUTO, the first call of each shape (op, norm, N, K, and
+                             M up to its 16-row padding at M <= 128 or its count of 128-row
+                             blocks above) times every candidate plan on `stream` (the small-M
+                             kernel's stream-K form and each cluster size whose clusters fit, the
+                             128x256 and 128x512 tile kernels) and keeps the fastest for the
+                             handle's later calls of that shape. Each candidate is timed on
+                             launches that follow a write of twice the L2 size (weights cold in
+                             L2, as in a model's layer loop). That first call allocates the
+                             write buffer for its duration and synchronises `stream`; inside a
+                             stream capture no tuning happens (the untuned plan is used and
+                             nothing is cached). 0: the untuned plan. */
 } fnl_options;
 
 /* Create a handle on `device` (cudaSetDevice is called). opt may be NULL. */
@@ -129,8 +151,15 @@ const char* fnl_status_string(fnl_status s);
 /* Text of the handle's last error ("" if none). Valid until the next call. */
 const char* fnl_last_error(const fnl_handle* h);
 
+/* Text of the plan of the handle's last call ("" if none): the kernel, its
+ * form and grid, and whether it was tuned. Valid until the next call. */
+const char* fnl_last_plan(const fnl_handle* h);
+
 /* Synchronise `stream`, read and clear the device status word. Returns
- * FNL_ERR_DEVICE_STATUS if a kernel since the last check gave up a wait. */
+ * FNL_ERR_DEVICE_STATUS if a kernel since the last check gave up a wait; the
+ * outputs of the calls since the last check are then not to be trusted. It
+ * also resets the handle's split-K arrival counters (an aborted CTA leaves its
+ * tiles' counters part-way), so later calls on the handle compute correctly. */
 fnl_status fnl_check(fnl_handle* h, fnl_stream stream);
 
 /* Residual add -> norm -> QKV projection -> head-major GQA split.
@@ -169,27 +198,56 @@ fnl_status fnl_add_bias_norm_gelu(fnl_handle* h, fnl_stream stream,
                                   int M, int K, int N,
                                   fnl_bf16* out, float* mean_out, float* rstd_out);
 
+/* Residual-stream projection: the layer's output projection (attention o_proj
+ * or MLP down_proj) with the residual add fused into its epilogue, which closes
+ * the layer's residual loop. These are the row-split projections of
+ * TensorRT-LLM 深度工程实践, §4.1 Tensor Parallelism; the residual connection
+ * they feed is the residual add that the graph-optimisation layer fuses
+ * (TensorRT-LLM 简介, 图优化层).
+ *   out[m, n] = bf16_rne(residual[m, n] + sum_k a[m, k] W[n, k] (+ bias[n]))
+ * with the sum accumulated in fp32 on the tensor cores (a is bf16 already: no
+ * norm, no operand rounding).
+ *   a         [M, K]  the sublayer's activation (attention or SwiGLU output)
+ *   W         [N, K]  projection weight, row n = output column n
+ *   bias      [N]     nullable
+ *   residual  [M, N]  the residual stream
+ *   out       [M, N]  the updated residual stream; may be the same buffer as
+ *                     residual (in-place update: each element is read, then
+ *                     written, by one thread); any other overlap of out with
+ *                     an input is FNL_ERR_ALIAS.
+ * Requirements, asynchrony and errors as for the fused ops (K, N multiples of
+ * 8, 16-byte aligned pointers, K <= 32768). M <= 128 runs the small-M split-K
+ * kernel, larger M a tile kernel; fnl_options.path forces one as for the
+ * fused ops. */
+fnl_status fnl_linear_add_residual(fnl_handle* h, fnl_stream stream, const fnl_bf16* a, const fnl_bf16* W,
+                                   const fnl_bf16* bias, const fnl_bf16* residual, fnl_bf16* out, int M, int K,
+                                   int N);
+
 /* Allocation-free variant of fnl_add_norm_qkv for decode-sized batches.
- * The pages have no counterpart to this entry point: it exists for callers
- * that may not allocate device memory on the call path -- work recorded into
- * a CUDA graph (cudaMalloc cannot be captured), latency-critical decode loops
- * that must never hit cudaMalloc/cudaFree's implicit device synchronisation,
- * and plugins inside an inference engine that owns all device memory through
- * its own static memory plan. fnl_create allocates a workspace, so this entry
- * point takes no handle; it computes exactly what fnl_add_norm_qkv computes
- * (same arguments, same meaning, same layouts) on the calling thread's current
- * device, with the small-M split-K kernel.
+ * The pages have no counterpart to this entry point. It is for callers that
+ * cannot call cudaMalloc on the call path: plugins inside an inference engine
+ * that owns all device memory through its own static memory plan, and
+ * latency-critical decode loops that must never pay cudaMalloc/cudaFree's
+ * implicit device synchronisation. fnl_create allocates a workspace, so this
+ * entry point takes no handle. It computes the same function as
+ * fnl_add_norm_qkv (same arguments, same meaning, same layouts) on the calling
+ * thread's current device, with the same kernel as FNL_PATH_SPLITK (the
+ * small-M kernel's stream-K form over all SMs): its results are bitwise equal
+ * to those of a handle created with path = FNL_PATH_SPLITK. A handle in
+ * FNL_PATH_AUTO may pick the cluster form, whose fp32 partial sums are added
+ * in another order, so the two agree within rounding but not always bitwise.
  * Scratch: a file-scope device array of 16 MiB inside the library, held by
  * every GPU that loads it until the process exits. Calls allocate nothing and
- * share that array: it keeps the last call's contents, and the call clears the
- * parts that must start at zero (status word, arrival counters) on `stream`
- * first. Calls that overlap on one GPU (several streams or host threads at
- * once) race on the array and must be serialised by the caller.
+ * share that array: it keeps the last call's contents, and each call first
+ * clears the split-K arrival counters on `stream`. Calls that overlap on one
+ * GPU (several streams or host threads at once) race on the array and must be
+ * serialised by the caller.
  * Limits: M <= 128 (FNL_ERR_UNSUPPORTED otherwise), and the split-K partial
  * sums must fit the array (about T * segments * roundup16(M) * 516 bytes with
  * T = ceil(N/128); e.g. N = 10240, M = 128 fits, N = 65536, M = 128 does not:
  * FNL_ERR_UNSUPPORTED). Other errors as for fnl_add_norm_qkv (status code only:
- * there is no handle to hold the text or the device status word).
+ * there is no handle to hold the text). A wait that runs out inside the kernel
+ * is recorded in the array's status word, which fnl_check_static reads.
  * The first call on each device resolves the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
  * before any stream capture. */
@@ -200,6 +258,13 @@ fnl_status fnl_add_norm_qkv_static(fnl_stream stream,
                                    int M, int K, int Hq, int Hkv, int D,
                                    fnl_bf16* q, fnl_bf16* k, fnl_bf16* v,
                                    float* mean_out, float* rstd_out);
+
+/* Status check of fnl_add_norm_qkv_static on the current device: synchronise
+ * `stream` (the stream of the static calls), read the status word of the
+ * static array and clear it. Returns FNL_ERR_DEVICE_STATUS if a static call
+ * since the last check gave up a bounded wait (its outputs are then not to be
+ * trusted), FNL_OK otherwise. Allocates nothing. */
+fnl_status fnl_check_static(fnl_stream stream);
 
 #ifdef __cplusplus
 }

@@ -35,7 +35,8 @@ def run_and_check(h, w, inputs, rows=None, **hkw):
 
 
 @pytest.mark.parametrize("name", ["c1_tiny_ln_qkv", "c2_decode_rms_qkv", "c5_70b_rms_qkv_m1",
-                                  "c5_70b_rms_qkv_m8", "c5_70b_rms_qkv_m32", "c5_70b_rms_qkv_m256"])
+                                  "c5_70b_rms_qkv_m8", "c5_70b_rms_qkv_m32", "c5_70b_rms_qkv_m256",
+                                  "llama3_8b_o_proj_decode"])
 def test_full_compare(handle, name):
     w = WL[name]
     res, _ = run_and_check(handle, w, synthetic.make_inputs(w))
@@ -43,7 +44,7 @@ def test_full_compare(handle, name):
 
 
 @pytest.mark.parametrize("name", ["c3_prefill_rms_swiglu", "c4_gpt_ln_gelu", "c5_70b_rms_qkv_m2048",
-                                  "c5_70b_rms_qkv_m8192", "c5_70b_rms_qkv_ragged"])
+                                  "c5_70b_rms_qkv_m8192", "c5_70b_rms_qkv_ragged", "llama3_8b_down_proj_prefill"])
 def test_sampled_compare(handle, name):
     w = WL[name]
     inputs = synthetic.make_inputs(w)
@@ -57,10 +58,14 @@ for op in ("qkv", "swiglu", "gelu"):
     for norm in ("layernorm", "rmsnorm"):
         for M in (1, 7, 16, 129, 200):
             TAIL_CASES.append((op, norm, M))
+for M in (1, 7, 16, 129, 200):
+    TAIL_CASES.append(("residual", "none", M))
 
 
 def _tail_workload(op, norm, M, K=200, seed=3):
     # K = 200: three full 64-wide k-blocks and a ragged one; N not a tile multiple
+    if op == "residual":
+        return synthetic.make_custom(op, "none", M, K, N=328, bias_out=True, seed=seed)
     if op == "qkv":
         return synthetic.make_custom(op, norm, M, K, Hq=6, Hkv=2, D=40, bias_out=True, seed=seed)
     if op == "swiglu":
@@ -74,9 +79,12 @@ def test_tile_tails(handle, op, norm, M):
     run_and_check(handle, w, inputs)
 
 
-@pytest.mark.parametrize("path", ["tile", "wide", "splitk", "cluster"])
-@pytest.mark.parametrize("op", ["qkv", "swiglu", "gelu"])
-@pytest.mark.parametrize("norm", ["layernorm", "rmsnorm"])
+FORCED = [(op, norm) for op in ("qkv", "swiglu", "gelu") for norm in ("layernorm", "rmsnorm")]
+FORCED.append(("residual", "none"))
+
+
+@pytest.mark.parametrize("path", ["tile", "wide", "pair", "splitk", "cluster"])
+@pytest.mark.parametrize("op,norm", FORCED)
 def test_forced_paths(cuda_device, path, op, norm):
     """Both kernels on the same small-M problems (the dispatch threshold is a
     performance choice, not a correctness one)."""
@@ -178,3 +186,133 @@ def test_argument_errors(handle):
         fnl.add_norm_qkv(handle, xs, xs.clone(), torch.ones(12, **bf), None, torch.randn(32, 12, **bf), 2, 1, 8)
     assert e.value.status == 2
     handle.check()
+
+
+@pytest.mark.parametrize("path", ["splitk", "cluster", "tile", "wide", "pair"])
+def test_device_status_path(cuda_device, path):
+    """A wait that runs out: the call's first CTA withholds one weight copy
+    (fault injection), its wait gives up after 2 ms, fnl_check reports
+    FNL_ERR_DEVICE_STATUS and resets the split-K arrival counters, and the next
+    normal call on the same handle matches the oracle."""
+    h = fnl.Handle(0, path=path, wait_ns=2_000_000, debug_stall_calls=1)
+    M = 64 if path in ("splitk", "cluster") else 300
+    w, inputs = _tail_workload("qkv", "rmsnorm", M, K=1024, seed=9)
+    dev = {k: v.cuda() for k, v in inputs.items()}
+    fnl.run_workload(h, w, dev)
+    with pytest.raises(fnl.FnlError) as e:
+        h.check()
+    assert e.value.status == 6
+    for _ in range(2):
+        got = fnl.run_workload(h, w, dev)
+        h.check()
+        check(w, inputs, got)
+    h.close()
+
+
+@pytest.mark.parametrize("path", ["auto", "splitk", "tile", "wide", "pair"])
+@pytest.mark.parametrize("op", ["qkv", "gelu"])
+@pytest.mark.parametrize("M", [16, 200])
+def test_layernorm_large_mean(cuda_device, path, op, M):
+    """x ~ N(50, 1): |mean| >> sigma, where a one-pass variance would cancel;
+    the statistics kernel's two-pass fp32 reduction must still meet 1e-5."""
+    if path == "splitk" and M > 128:
+        pytest.skip("the small-M kernel takes M <= 128")
+    h = fnl.Handle(0, path=path)
+    if op == "qkv":
+        w, inputs = synthetic.make_custom(op, "layernorm", M, 4096, Hq=6, Hkv=2, D=64, bias_out=True,
+                                          seed=5, x_loc=50.0)
+    else:
+        w, inputs = synthetic.make_custom(op, "layernorm", M, 4096, N=520, bias_in=True, bias_out=True,
+                                          seed=6, x_loc=50.0)
+    res, _ = run_and_check(h, w, inputs)
+    print(path, op, M, res)
+    h.close()
+
+
+def test_eps_must_be_positive(handle):
+    K, Hq, Hkv, D, M = 64, 2, 1, 8, 4
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    x, r = torch.randn(M, K, **bf), torch.randn(M, K, **bf)
+    g = torch.ones(K, **bf)
+    W = torch.randn((Hq + 2 * Hkv) * D, K, **bf)
+    for eps in (0.0, -1e-5, float("nan"), float("inf")):
+        with pytest.raises(fnl.FnlError) as e:
+            fnl.add_norm_qkv(handle, x, r, g, None, W, Hq, Hkv, D, norm="layernorm", eps=eps)
+        assert e.value.status == 1, eps
+
+
+@pytest.mark.parametrize("M", [32, 300])
+def test_residual_projection_in_place(handle, M):
+    """out may be the residual buffer itself (the residual stream updated in
+    place); the result matches the oracle on the original residual."""
+    w, inputs = synthetic.make_custom("residual", "none", M, 4096, N=4096, bias_out=True, seed=21)
+    dev = {k: v.cuda() for k, v in inputs.items()}
+    stream_buf = dev["residual"].clone()
+    got = fnl.linear_add_residual(handle, dev["x"], dev["W"], stream_buf, bias=dev["bias_out"], out=stream_buf)
+    handle.check()
+    assert got["out"].data_ptr() == stream_buf.data_ptr()
+    print(check(w, inputs, got))
+
+
+def test_residual_projection_alias_errors(handle):
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    M, K, N = 8, 64, 64
+    a, W = torch.randn(M, K, **bf), torch.randn(N, K, **bf)
+    buf = torch.randn(2 * M * N, **bf)
+    res = buf[: M * N].view(M, N)
+    with pytest.raises(fnl.FnlError) as e:   # out partly overlaps residual
+        fnl.linear_add_residual(handle, a, W, res, out=buf[8: 8 + M * N].view(M, N))
+    assert e.value.status == 3
+    with pytest.raises(fnl.FnlError) as e:   # out overlaps a
+        fnl.linear_add_residual(handle, a, W, torch.randn(M, N, **bf), out=a)
+    assert e.value.status == 3
+    handle.check()
+
+
+@pytest.mark.parametrize("name", ["c1_tiny_ln_qkv", "c2_decode_rms_qkv", "c5_70b_rms_qkv_m256",
+                                  "llama3_8b_o_proj_decode"])
+def test_tuner(cuda_device, name):
+    """Shape auto-tuning: the first call times the candidate plans and keeps the
+    fastest (its result matches the oracle), the second call of the same shape
+    takes the cached plan without re-timing, and matches the oracle too."""
+    w = WL[name]
+    inputs = synthetic.make_inputs(w)
+    dev = {k: v.cuda() for k, v in inputs.items()}
+    h = fnl.Handle(0, tune=True)
+    got = fnl.run_workload(h, w, dev)
+    h.check()
+    first = h.last_plan()
+    assert "tuned:" in first, first
+    check(w, inputs, got)
+    got = fnl.run_workload(h, w, dev)
+    h.check()
+    second = h.last_plan()
+    assert "from the cache" in second, second
+    assert first.split(" (")[0] == second.split(" (")[0]
+    check(w, inputs, got)
+    print(name, first)
+    h.close()
+
+
+@pytest.mark.parametrize("name", ["c3_prefill_rms_swiglu", "c4_gpt_ln_gelu", "c5_70b_rms_qkv_m2048",
+                                  "llama3_8b_down_proj_prefill"])
+def test_pair_kernel_full_size(cuda_device, name):
+    """The CTA-pair kernel forced on the large workloads (sampled rows, every
+    row's residual_out and statistics)."""
+    w = WL[name]
+    h = fnl.Handle(0, path="pair")
+    inputs = synthetic.make_inputs(w)
+    res, _ = run_and_check(h, w, inputs, rows=sample_rows(w.M, w.seq_lens))
+    print(name, h.last_plan(), res)
+    h.close()
+
+
+@pytest.mark.parametrize("M", [129, 255, 256, 257, 600])
+@pytest.mark.parametrize("op,norm", [("qkv", "rmsnorm"), ("swiglu", "layernorm"), ("gelu", "layernorm"),
+                                     ("residual", "none")])
+def test_pair_kernel_row_tails(cuda_device, M, op, norm):
+    """Pair tiles cut by M: the odd CTA's rows partly or wholly past M."""
+    h = fnl.Handle(0, path="pair")
+    w, inputs = _tail_workload(op, norm, M, K=328, seed=M)
+    run_and_check(h, w, inputs)
+    h.close()

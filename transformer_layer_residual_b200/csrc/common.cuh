@@ -7,8 +7,11 @@ namespace fnl {
 
 typedef __nv_bfloat16 bf16;
 
-enum Epi : int { kEpiQKV = 0, kEpiSwiGLU = 1, kEpiGELU = 2 };
-enum Norm : int { kLayerNorm = 0, kRMSNorm = 1 };
+// kEpiResidual with kNoNorm is the residual-stream projection (o_proj /
+// down_proj): the activation operand is used as loaded (no add, no norm, no
+// converters) and the epilogue adds the residual stream: out = residual + y.
+enum Epi : int { kEpiQKV = 0, kEpiSwiGLU = 1, kEpiGELU = 2, kEpiResidual = 3 };
+enum Norm : int { kLayerNorm = 0, kRMSNorm = 1, kNoNorm = 2 };
 
 struct OpParams {
   int M, K, N;       // tokens, hidden, rows of W
@@ -28,6 +31,9 @@ struct OpParams {
   bf16* k;
   bf16* v;
   bf16* out;
+  const bf16* res_in;    // residual-stream projection: the residual [M][N] added in the epilogue
+                         // (may be the same buffer as out: each element is read, then written,
+                         // by one thread)
   // small-M split-K workspace
   float* part;           // [T][max_seg][mpad][128] fp32 partial accumulators
   float* part_ss;        // [T][max_seg][mpad] partial sums of h^2 (RMSNorm)
@@ -39,6 +45,9 @@ struct OpParams {
   int sk;                // 128x256 tile kernel: 1 = stream-K over (tile, k-block) units, 0 = whole tiles
   int split;             // 1: operand = bf16 hi + bf16 lo (two UMMAs), 0: single bf16 rounding
   int* status;           // device status word (bounded-wait failures)
+  unsigned long long wait_ns;   // limit of the main-loop waits (the drain waits keep FNL_WAIT_NS)
+  int stall;             // fault injection for the status-path tests: 1 = CTA 0's producer never
+                         // issues its first weight copy, so the wait for it runs out (0 = off)
 };
 
 __device__ __forceinline__ uint4 ldg16(const void* p) {
@@ -187,8 +196,14 @@ __device__ __forceinline__ float gelu_tanh_f(float z) {
   return __fdividef(z, 1.f + __expf(u2));
 }
 
-// Store 8 consecutive output columns [n, n+8) of row m (QKV or GELU epilogue).
-// acc is the raw fp32 accumulator, scale the deferred RMSNorm 1/rms (1 for LN).
+// 16 bytes from global memory through L2 only (no L1 allocation: read once).
+__device__ __forceinline__ uint4 ldcg16(const void* p) {
+  return __ldcg(reinterpret_cast<const uint4*>(p));
+}
+
+// Store 8 consecutive output columns [n, n+8) of row m (QKV, GELU or residual
+// epilogue). acc is the raw fp32 accumulator, scale the deferred RMSNorm 1/rms
+// (1 for LN and for the residual-stream projection).
 template <int EPI>
 __device__ __forceinline__ void store_out8(const OpParams& p, int m, int n, const float (&acc)[8], float scale) {
   float y[8];
@@ -201,7 +216,14 @@ __device__ __forceinline__ void store_out8(const OpParams& p, int m, int n, cons
     for (int e = 0; e < 8; ++e) y[e] += b[e];
   }
   bf16* dst;
-  if (EPI == kEpiGELU) {
+  if (EPI == kEpiResidual) {
+    const size_t off = static_cast<size_t>(m) * p.N + n;
+    float r[8];
+    unpack8(ldcg16(p.res_in + off), r);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] += r[e];
+    dst = p.out + off;
+  } else if (EPI == kEpiGELU) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) y[e] = gelu_tanh_f(y[e]);
     dst = p.out + static_cast<size_t>(m) * p.N + n;

@@ -23,9 +23,65 @@
 #include "k2_tile.cuh"
 #include "k2_wide.cuh"
 #include "k3_splitk.cuh"
+#include "k4_pair.cuh"
 
 using fnl::bf16;
 using fnl::OpParams;
+
+namespace fnlh {
+// A plan: which kernel runs a call, in which form, on how many CTAs.
+enum class Kern { K3, K2, K2W, K4 };
+
+struct Plan {
+  Kern kern = Kern::K3;
+  int grid = 1, threads = 0, smem = 0, mpad = 0, stages = 0, max_seg = 1, T = 0, cls = 0, sk = 0;
+};
+
+// Key of the shape auto-tuning cache (see tune()).
+struct TuneKey {
+  int op, norm, mkey, N, K, I;
+  bool operator==(const TuneKey& o) const {
+    return op == o.op && norm == o.norm && mkey == o.mkey && N == o.N && K == o.K && I == o.I;
+  }
+};
+
+struct TunedEntry {
+  TuneKey key;
+  Plan plan;
+  float us;        // median time of the plan when it was tuned
+  int candidates;  // plans timed
+};
+}  // namespace fnlh
+using fnlh::Kern;
+using fnlh::Plan;
+using fnlh::TuneKey;
+
+// Encoded TMA descriptors, keyed by what the encoding depends on. A decode
+// loop calls with the same pointers every step, so its three maps are encoded
+// once; the table is small and replaced round-robin.
+struct MapCache {
+  struct Entry {
+    const void* ptr;
+    long long rows, cols;
+    int box_rows, box_cols;
+    CUtensorMap map;
+  };
+  static constexpr int kSize = 32;
+  Entry e[kSize];
+  int used = 0, next = 0;
+  const CUtensorMap* find(const void* ptr, long long rows, long long cols, int br, int bc) const {
+    for (int i = 0; i < used; ++i)
+      if (e[i].ptr == ptr && e[i].rows == rows && e[i].cols == cols && e[i].box_rows == br && e[i].box_cols == bc)
+        return &e[i].map;
+    return nullptr;
+  }
+  void put(const void* ptr, long long rows, long long cols, int br, int bc, const CUtensorMap& m) {
+    Entry& x = e[next];
+    x.ptr = ptr; x.rows = rows; x.cols = cols; x.box_rows = br; x.box_cols = bc; x.map = m;
+    next = (next + 1) % kSize;
+    if (used < kSize) ++used;
+  }
+};
 
 struct fnl_handle {
   int device = 0;
@@ -38,6 +94,10 @@ struct fnl_handle {
     int smem, cls, clusters;
   };
   std::vector<Occ> occ;      // resident clusters of the small-M kernel per (shared memory, cluster size)
+  MapCache maps;             // encoded tensor maps of recent calls
+  std::string plan_text;     // the last call's plan (fnl_last_plan)
+  int pairs = 0;             // resident CTA pairs of the pair kernel (0: not queried yet)
+  std::vector<fnlh::TunedEntry> tuned;   // shape auto-tuning cache
 };
 
 namespace {
@@ -48,6 +108,17 @@ constexpr size_t kStatusBytes = 256;
 constexpr int kMaxTiles = 65536;
 constexpr size_t kCountersBytes = static_cast<size_t>(kMaxTiles) * 4;
 constexpr size_t kFixedBytes = kStatusBytes + kCountersBytes;
+// Largest N (rows of W) any entry point accepts: below kMaxTiles 128-row tiles
+// and far below INT_MAX, so every index derived from it fits an int.
+constexpr int kMaxN = (kMaxTiles - 1) * 128;
+
+// N = (Hq + 2 Hkv) D computed in 64 bits; 0 when a count is not positive or N
+// exceeds kMaxN.
+int qkv_columns(int Hq, int Hkv, int D) {
+  if (Hq <= 0 || Hkv <= 0 || D <= 0) return 0;
+  const long long n = (static_cast<long long>(Hq) + 2LL * Hkv) * D;
+  return n <= kMaxN ? static_cast<int>(n) : 0;
+}
 
 size_t align256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 
@@ -101,8 +172,8 @@ fnl_status get_encoder(fnl_handle* h) {
 // Row-major bf16 [rows, cols] (cols contiguous), box [box_rows, box_cols] with
 // the swizzle the UMMA descriptors expect: 128-byte swizzle for 64-wide boxes,
 // 64-byte swizzle for 32-wide boxes; out-of-range elements read 0.
-fnl_status make_map(fnl_handle* h, CUtensorMap* m, const void* ptr, long long rows, long long cols,
-                    int box_rows, int box_cols = 64) {
+fnl_status encode_map(fnl_handle* h, CUtensorMap* m, const void* ptr, long long rows, long long cols,
+                      int box_rows, int box_cols) {
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
@@ -113,6 +184,21 @@ fnl_status make_map(fnl_handle* h, CUtensorMap* m, const void* ptr, long long ro
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(h, FNL_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
   return FNL_OK;
+}
+
+// The map of a [rows, cols] operand at ptr, from the handle's cache when the
+// same operand was encoded before (h == NULL: always encoded).
+fnl_status make_map(fnl_handle* h, CUtensorMap* m, const void* ptr, long long rows, long long cols,
+                    int box_rows, int box_cols = 64) {
+  if (h) {
+    if (const CUtensorMap* c = h->maps.find(ptr, rows, cols, box_rows, box_cols)) {
+      *m = *c;
+      return FNL_OK;
+    }
+  }
+  fnl_status st = encode_map(h, m, ptr, rows, cols, box_rows, box_cols);
+  if (st == FNL_OK && h) h->maps.put(ptr, rows, cols, box_rows, box_cols, *m);
+  return st;
 }
 
 // ------------------------------------------------------------------ validation
@@ -130,7 +216,7 @@ bool overlap(const Range& a, const Range& b) {
   return a0 < b0 + b.bytes && b0 < a0 + a.bytes;
 }
 
-enum class Op { QKV, SwiGLU, GELU };
+enum class Op { QKV, SwiGLU, GELU, Residual };
 
 struct Call {
   Op op;
@@ -144,12 +230,40 @@ struct Call {
   float *mean_out, *rstd_out;
 };
 
+// Residual-stream projection: x = a [M, K], residual [M, N], out [M, N]; out
+// may be exactly the residual buffer (each element is read, then written, by
+// one thread), any other overlap is rejected.
+fnl_status validate_residual(fnl_handle* h, const Call& c) {
+  if (c.M < 0 || c.K <= 0 || c.N <= 0) return fail(h, FNL_ERR_INVALID_ARG, "need M >= 0, K > 0, N > 0");
+  if (c.K % 8 || c.N % 8) return fail(h, FNL_ERR_ALIGNMENT, "K and N must be multiples of 8 (K=%d N=%d)", c.K, c.N);
+  if (c.K > 32768) return fail(h, FNL_ERR_UNSUPPORTED, "K=%d exceeds 32768", c.K);
+  if (c.N > kMaxN) return fail(h, FNL_ERR_UNSUPPORTED, "N=%d exceeds %d", c.N, kMaxN);
+  if ((h->opt.path == FNL_PATH_SPLITK || h->opt.path == FNL_PATH_SPLITK_CLUSTER) && c.M > fnl::k3::MAX_MPAD)
+    return fail(h, FNL_ERR_UNSUPPORTED, "forced split-K path needs M <= %d", fnl::k3::MAX_MPAD);
+  if (c.M == 0) return FNL_OK;
+  if (!c.x || !c.W || !c.residual || !c.out) return fail(h, FNL_ERR_INVALID_ARG, "a, W, residual and out are required");
+  const void* p16[] = {c.x, c.W, c.bias, c.residual, c.out};
+  for (const void* p : p16)
+    if (p && !al16(p)) return fail(h, FNL_ERR_ALIGNMENT, "a bf16 pointer is not 16-byte aligned");
+  const size_t MN = static_cast<size_t>(c.M) * c.N * 2;
+  const Range out{c.out, MN, "out"};
+  const Range ins[] = {{c.x, static_cast<size_t>(c.M) * c.K * 2, "a"},
+                       {c.W, static_cast<size_t>(c.N) * c.K * 2, "W"},
+                       {c.bias, static_cast<size_t>(c.N) * 2, "bias"}};
+  for (const Range& in : ins)
+    if (overlap(out, in)) return fail(h, FNL_ERR_ALIAS, "output out overlaps input %s", in.name);
+  if (c.out != c.residual && overlap(out, Range{c.residual, MN, "residual"}))
+    return fail(h, FNL_ERR_ALIAS, "out overlaps residual without being the same buffer");
+  return FNL_OK;
+}
+
 fnl_status validate(fnl_handle* h, const Call& c) {
   if (!h) return FNL_ERR_INVALID_ARG;
+  if (c.op == Op::Residual) return validate_residual(h, c);
   if (c.norm != FNL_NORM_LAYERNORM && c.norm != FNL_NORM_RMSNORM)
     return fail(h, FNL_ERR_INVALID_ARG, "norm must be FNL_NORM_LAYERNORM or FNL_NORM_RMSNORM");
-  if (!(c.eps >= 0.f) || c.eps != c.eps || c.eps > 1e30f)
-    return fail(h, FNL_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (!(c.eps > 0.f) || c.eps > 1e30f)   // also rejects NaN
+    return fail(h, FNL_ERR_INVALID_ARG, "eps must be finite and > 0 (a constant row has zero variance)");
   if (c.M < 0 || c.K <= 0 || c.N <= 0) return fail(h, FNL_ERR_INVALID_ARG, "need M >= 0, K > 0, N > 0");
   if (c.K % 8 || c.N % 8) return fail(h, FNL_ERR_ALIGNMENT, "K and N must be multiples of 8 (K=%d N=%d)", c.K, c.N);
   if (c.K > 32768) return fail(h, FNL_ERR_UNSUPPORTED, "K=%d exceeds 32768", c.K);
@@ -160,7 +274,7 @@ fnl_status validate(fnl_handle* h, const Call& c) {
   }
   if (c.op == Op::SwiGLU && (c.I <= 0 || c.I % 8))
     return fail(h, FNL_ERR_ALIGNMENT, "I must be a positive multiple of 8 (I=%d)", c.I);
-  if (c.N / 128 + 1 > kMaxTiles) return fail(h, FNL_ERR_UNSUPPORTED, "N=%d too large", c.N);
+  if (c.N > kMaxN) return fail(h, FNL_ERR_UNSUPPORTED, "N=%d exceeds %d", c.N, kMaxN);
   if (c.norm == FNL_NORM_RMSNORM && c.beta)
     return fail(h, FNL_ERR_INVALID_ARG, "beta must be NULL for RMSNorm");
   if (c.norm == FNL_NORM_RMSNORM && c.mean_out)
@@ -182,28 +296,29 @@ fnl_status validate(fnl_handle* h, const Call& c) {
   // aliasing: outputs vs inputs and vs each other
   const size_t MK = static_cast<size_t>(c.M) * c.K * 2;
   const size_t n_out = c.op == Op::SwiGLU ? static_cast<size_t>(c.I) : static_cast<size_t>(c.N);
-  std::vector<Range> ins = {{c.x, MK, "x"},
+  const Range ins[] = {{c.x, MK, "x"},
                             {c.residual, MK, "residual"},
                             {c.bias_in, static_cast<size_t>(c.K) * 2, "bias_in"},
                             {c.gamma, static_cast<size_t>(c.K) * 2, "gamma"},
                             {c.beta, static_cast<size_t>(c.K) * 2, "beta"},
                             {c.W, static_cast<size_t>(c.N) * c.K * 2, "W"},
                             {c.bias, static_cast<size_t>(c.N) * 2, "bias"}};
-  std::vector<Range> outs = {{c.residual_out, MK, "residual_out"},
-                             {c.mean_out, static_cast<size_t>(c.M) * 4, "mean_out"},
-                             {c.rstd_out, static_cast<size_t>(c.M) * 4, "rstd_out"}};
+  Range outs[6] = {{c.residual_out, MK, "residual_out"},
+                   {c.mean_out, static_cast<size_t>(c.M) * 4, "mean_out"},
+                   {c.rstd_out, static_cast<size_t>(c.M) * 4, "rstd_out"}};
+  size_t n_outs = 3;
   if (c.op == Op::QKV) {
-    outs.push_back({c.q, static_cast<size_t>(c.Hq) * c.M * c.D * 2, "q"});
-    outs.push_back({c.k, static_cast<size_t>(c.Hkv) * c.M * c.D * 2, "k"});
-    outs.push_back({c.v, static_cast<size_t>(c.Hkv) * c.M * c.D * 2, "v"});
+    outs[n_outs++] = {c.q, static_cast<size_t>(c.Hq) * c.M * c.D * 2, "q"};
+    outs[n_outs++] = {c.k, static_cast<size_t>(c.Hkv) * c.M * c.D * 2, "k"};
+    outs[n_outs++] = {c.v, static_cast<size_t>(c.Hkv) * c.M * c.D * 2, "v"};
   } else {
-    outs.push_back({c.out, static_cast<size_t>(c.M) * n_out * 2, "out"});
+    outs[n_outs++] = {c.out, static_cast<size_t>(c.M) * n_out * 2, "out"};
   }
-  for (size_t i = 0; i < outs.size(); ++i) {
+  for (size_t i = 0; i < n_outs; ++i) {
     for (const Range& in : ins)
       if (overlap(outs[i], in))
         return fail(h, FNL_ERR_ALIAS, "output %s overlaps input %s", outs[i].name, in.name);
-    for (size_t j = i + 1; j < outs.size(); ++j)
+    for (size_t j = i + 1; j < n_outs; ++j)
       if (overlap(outs[i], outs[j]))
         return fail(h, FNL_ERR_ALIAS, "outputs %s and %s overlap", outs[i].name, outs[j].name);
   }
@@ -211,11 +326,44 @@ fnl_status validate(fnl_handle* h, const Call& c) {
 }
 
 // ------------------------------------------------------------------ launches
+// Dynamic shared-memory limit of each kernel per device, as last set by this
+// library (the attribute is per function and device, so the table is
+// process-wide). set_smem raises a limit only when it is below what the launch
+// needs, so a decode loop pays cudaFuncSetAttribute once.
+struct AttrEntry {
+  int dev;
+  const void* fn;
+  int smem;
+};
+constexpr int kMaxAttrs = 256;
+AttrEntry g_attrs[kMaxAttrs];
+int g_n_attrs = 0;
+std::mutex g_attr_mu;
+
+template <typename Kern>
+fnl_status set_smem_exact(fnl_handle* h, int dev, Kern kern, int bytes, bool exact) {
+  const void* fn = reinterpret_cast<const void*>(kern);
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  AttrEntry* a = nullptr;
+  for (int i = 0; i < g_n_attrs; ++i)
+    if (g_attrs[i].dev == dev && g_attrs[i].fn == fn) a = &g_attrs[i];
+  if (a && (exact ? a->smem == bytes : a->smem >= bytes)) return FNL_OK;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) {
+    if (a) a->smem = -1;   // unknown now
+    return cuda_fail(h, e, "cudaFuncSetAttribute");
+  }
+  if (a) a->smem = bytes;
+  else if (g_n_attrs < kMaxAttrs) g_attrs[g_n_attrs++] = {dev, fn, bytes};
+  return FNL_OK;
+}
+
 template <typename Kern>
 fnl_status set_smem(fnl_handle* h, Kern kern, int bytes) {
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e != cudaSuccess) return cuda_fail(h, e, "cudaFuncSetAttribute");
-  return FNL_OK;
+  int dev = 0;
+  if (h) dev = h->device;
+  else if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  return set_smem_exact(h, dev, kern, bytes, false);
 }
 
 template <typename Kern>
@@ -252,9 +400,14 @@ fnl_status launch_gemm(fnl_handle* h, Kern kern, int grid, int threads, int smem
 template <int EPI, bool SPLIT>
 fnl_status dispatch_gemm_p(fnl_handle* h, bool small, bool rms, int grid, int threads, int smem, bool pdl,
                            cudaStream_t stream, const CUtensorMap& mx, const CUtensorMap& mr, const CUtensorMap& mw,
-                           const OpParams& p, bool wide) {
+                           const OpParams& p, bool wide, bool pair) {
   using fnl::kLayerNorm;
   using fnl::kRMSNorm;
+  if (pair) {
+    if (rms)
+      return launch_gemm(h, fnl::k4_pair_kernel<EPI, kRMSNorm, SPLIT>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
+    return launch_gemm(h, fnl::k4_pair_kernel<EPI, kLayerNorm, SPLIT>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
+  }
   if (wide) {
     if (rms)
       return launch_gemm(h, fnl::k2w_tile_kernel<EPI, kRMSNorm, SPLIT>, grid, threads, smem, pdl, stream, mx, mr, mw, p);
@@ -277,9 +430,29 @@ fnl_status dispatch_gemm_p(fnl_handle* h, bool small, bool rms, int grid, int th
 template <int EPI>
 fnl_status dispatch_gemm(fnl_handle* h, bool small, bool rms, int grid, int threads, int smem, bool pdl,
                          cudaStream_t stream, const CUtensorMap& mx, const CUtensorMap& mr, const CUtensorMap& mw,
-                         const OpParams& p, bool wide = false) {
-  if (p.split) return dispatch_gemm_p<EPI, true>(h, small, rms, grid, threads, smem, pdl, stream, mx, mr, mw, p, wide);
-  return dispatch_gemm_p<EPI, false>(h, small, rms, grid, threads, smem, pdl, stream, mx, mr, mw, p, wide);
+                         const OpParams& p, bool wide = false, bool pair = false) {
+  if (p.split)
+    return dispatch_gemm_p<EPI, true>(h, small, rms, grid, threads, smem, pdl, stream, mx, mr, mw, p, wide, pair);
+  return dispatch_gemm_p<EPI, false>(h, small, rms, grid, threads, smem, pdl, stream, mx, mr, mw, p, wide, pair);
+}
+
+// The residual-stream projection: no norm, residual epilogue, one operand rounding.
+fnl_status dispatch_residual(fnl_handle* h, bool small, bool wide, bool pair, int grid, int threads, int smem,
+                             bool pdl, cudaStream_t stream, const CUtensorMap& mx, const CUtensorMap& mw,
+                             const OpParams& p) {
+  using fnl::kEpiResidual;
+  using fnl::kNoNorm;
+  if (pair)
+    return launch_gemm(h, fnl::k4_pair_kernel<kEpiResidual, kNoNorm, false>, grid, threads, smem, pdl, stream, mx, mx,
+                       mw, p);
+  if (wide)
+    return launch_gemm(h, fnl::k2w_tile_kernel<kEpiResidual, kNoNorm, false>, grid, threads, smem, pdl, stream, mx, mx,
+                       mw, p);
+  if (small)
+    return launch_gemm(h, fnl::k3_splitk_kernel<kEpiResidual, kNoNorm, false>, grid, threads, smem, pdl, stream, mx,
+                       mx, mw, p);
+  return launch_gemm(h, fnl::k2_tile_kernel<kEpiResidual, kNoNorm, false>, grid, threads, smem, pdl, stream, mx, mx,
+                     mw, p);
 }
 
 fnl_status launch_k1(fnl_handle* h, const Call& c, float2* stats, cudaStream_t stream) {
@@ -310,7 +483,8 @@ int resident_clusters(fnl_handle* h, int smem, int cls) {
     if (o.smem == smem && o.cls == cls) return o.clusters;
   auto kern = fnl::k3_splitk_kernel<fnl::kEpiQKV, fnl::kRMSNorm, false>;
   int n = 0;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess) {
+  // the occupancy query needs the limit at exactly `smem` (recorded in the table)
+  if (set_smem_exact(h, h->device, kern, smem, true) == FNL_OK) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(cls);
     cfg.blockDim = dim3(fnl::k3::NUM_THREADS);
@@ -329,6 +503,366 @@ int resident_clusters(fnl_handle* h, int smem, int cls) {
   return n;
 }
 
+// ------------------------------------------------------------------ plans
+
+// Largest CTA index range of one tile when U units are dealt evenly over grid
+// CTAs, tiles of nkb units each: the number of partial-sum slots per tile.
+int max_segments(int T, int nkb, int grid) {
+  const long long U = static_cast<long long>(T) * nkb;
+  int m = 1;
+  for (int t = 0; t < T; ++t) {
+    const int first = fnl::unit_owner(static_cast<long long>(t) * nkb, grid, U);
+    const int last = fnl::unit_owner(static_cast<long long>(t + 1) * nkb - 1, grid, U);
+    m = std::max(m, last - first + 1);
+  }
+  return m;
+}
+
+// Plan of kernel `kern` for call c. Small-M kernel: cls_req < 0 applies the
+// automatic rule (the cluster form when its clusters cover the GPU and are all
+// resident), 0 forces the stream-K form, >= 2 requests that cluster size
+// (FNL_ERR_UNSUPPORTED when its clusters cannot all be resident).
+// CTA pairs of the pair kernel resident at once (one CTA per SM); cached per handle.
+int resident_pairs(fnl_handle* h) {
+  if (h->pairs > 0) return h->pairs;
+  auto kern = fnl::k4_pair_kernel<fnl::kEpiQKV, fnl::kRMSNorm, false>;
+  int n = 0;
+  if (set_smem_exact(h, h->device, kern, fnl::k4::SMEM_BYTES, false) == FNL_OK) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(fnl::k4::NUM_THREADS);
+    cfg.dynamicSmemBytes = fnl::k4::SMEM_BYTES;
+    cudaLaunchAttribute a[1];
+    a[0].id = cudaLaunchAttributeClusterDimension;
+    a[0].val.clusterDim.x = 2;
+    a[0].val.clusterDim.y = 1;
+    a[0].val.clusterDim.z = 1;
+    cfg.attrs = a;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();
+  h->pairs = n > 0 ? n : 0;
+  return h->pairs;
+}
+
+fnl_status plan_kernel(fnl_handle* h, const Call& c, Kern kern, int cls_req, Plan* pl) {
+  const int max_ctas = h->opt.max_ctas > 0 ? std::min(h->opt.max_ctas, h->num_sms) : h->num_sms;
+  const int nkb = (c.K + 63) / 64;
+  Plan q;
+  q.kern = kern;
+  if (kern == Kern::K3) {
+    if (c.M > fnl::k3::MAX_MPAD) return fail(h, FNL_ERR_UNSUPPORTED, "the small-M kernel needs M <= %d", fnl::k3::MAX_MPAD);
+    q.mpad = round_up(std::max(c.M, 1), 16);
+    q.T = c.op == Op::SwiGLU ? (c.I + 63) / 64 : (c.N + 127) / 128;
+    if (q.T > kMaxTiles) return fail(h, FNL_ERR_UNSUPPORTED, "too many W tiles");
+    const long long U = static_cast<long long>(q.T) * nkb;
+    q.grid = static_cast<int>(std::min<long long>(max_ctas, U));
+    q.stages = std::min(fnl::k3::MAX_STAGES, (200 * 1024) / fnl::k3::stage_bytes(q.mpad));
+    q.smem = fnl::k3::smem_bytes(q.mpad, q.stages);
+    q.threads = fnl::k3::NUM_THREADS;
+    if (cls_req >= 2) {
+      if (cls_req > 8 || cls_req > nkb || resident_clusters(h, q.smem, cls_req) < q.T)
+        return fail(h, FNL_ERR_UNSUPPORTED, "the %d W tiles cannot run at once as clusters of %d CTAs", q.T, cls_req);
+      q.cls = cls_req;
+    } else if (cls_req < 0 && h->opt.max_ctas == 0) {
+      // Cluster form: one W tile per cluster of cls CTAs, each taking 1/cls of
+      // its k-blocks, partial sums reduced on chip. Used when the clusters cover
+      // the GPU (or every unit of work) and all of them are resident at once;
+      // the largest such cluster size (<= 8, <= the k-blocks).
+      for (int c_ = std::min({8, h->num_sms / std::max(q.T, 1), nkb}); c_ >= 2 && q.cls == 0; --c_) {
+        const bool covers = static_cast<long long>(q.T) * c_ >= std::min<long long>(U, (h->num_sms * 9) / 10);
+        if (covers && resident_clusters(h, q.smem, c_) >= q.T) q.cls = c_;
+      }
+    }
+    if (q.cls > 0) q.grid = q.T * q.cls;
+    else q.max_seg = max_segments(q.T, nkb, q.grid);
+  } else if (kern == Kern::K4) {
+    // CTA pairs, 256 tokens x 512 W rows per pair tile, one pair tile at a time per pair
+    const int pairs_max = std::min(resident_pairs(h), max_ctas / 2);
+    if (pairs_max <= 0) return fail(h, FNL_ERR_UNSUPPORTED, "the pair kernel cannot be resident");
+    const int num_m2 = (c.M + 255) / 256;
+    const long long tiles = static_cast<long long>(num_m2) *
+                            (c.op == Op::SwiGLU ? (c.I + 255) / 256 : (c.N + fnl::k4::BN - 1) / fnl::k4::BN);
+    q.grid = 2 * static_cast<int>(std::min<long long>(pairs_max, tiles));
+    q.cls = 2;
+    q.smem = fnl::k4::SMEM_BYTES;
+    q.threads = fnl::k4::NUM_THREADS;
+  } else {
+    const bool wide = kern == Kern::K2W;
+    const int num_m = (c.M + 127) / 128;
+    const long long tiles = static_cast<long long>(num_m) *
+                            (wide ? (c.op == Op::SwiGLU ? (c.I + 255) / 256 : (c.N + fnl::k2w::BN - 1) / fnl::k2w::BN)
+                                  : (c.op == Op::SwiGLU ? (c.I + 127) / 128 : (c.N + fnl::k2::BN - 1) / fnl::k2::BN));
+    q.grid = static_cast<int>(std::min<long long>(max_ctas, tiles));
+    // Fewer 128x256 tiles than CTAs by a fifth or more (e.g. 70B QKV at
+    // M = 256: 80 tiles, 148 SMs): stream-K over (tile, k-block) units, so
+    // every SM streams weights; partial tiles are summed by their last CTA.
+    if (!wide && tiles * 5 <= static_cast<long long>(max_ctas) * 4) {
+      q.sk = 1;
+      q.T = static_cast<int>(tiles);
+      if (q.T > kMaxTiles) return fail(h, FNL_ERR_UNSUPPORTED, "too many W tiles");
+      q.grid = static_cast<int>(std::min<long long>(max_ctas, tiles * nkb));
+      q.max_seg = max_segments(q.T, nkb, q.grid);
+    }
+    q.smem = wide ? fnl::k2w::SMEM_BYTES : fnl::k2::SMEM_BYTES;
+    q.threads = wide ? fnl::k2w::NUM_THREADS : fnl::k2::NUM_THREADS;
+  }
+  *pl = q;
+  return FNL_OK;
+}
+
+// The plan without tuning: the forced path, else M <= 128 -> small-M kernel,
+// else the tile shape whose waves of CTAs fit best.
+fnl_status default_plan(fnl_handle* h, const Call& c, Plan* pl) {
+  switch (h->opt.path) {
+    case FNL_PATH_TILE: return plan_kernel(h, c, Kern::K2, -1, pl);
+    case FNL_PATH_TILE_WIDE: return plan_kernel(h, c, Kern::K2W, -1, pl);
+    case FNL_PATH_TILE_PAIR: return plan_kernel(h, c, Kern::K4, -1, pl);
+    case FNL_PATH_SPLITK: return plan_kernel(h, c, Kern::K3, 0, pl);
+    case FNL_PATH_SPLITK_CLUSTER: {
+      // the largest cluster size whose clusters are all resident
+      const int T = c.op == Op::SwiGLU ? (c.I + 63) / 64 : (c.N + 127) / 128;
+      const int nkb = (c.K + 63) / 64;
+      for (int c_ = std::min({8, h->num_sms / std::max(T, 1), nkb}); c_ >= 2; --c_) {
+        Plan q;
+        if (plan_kernel(h, c, Kern::K3, c_, &q) == FNL_OK) {
+          *pl = q;
+          return FNL_OK;
+        }
+      }
+      return fail(h, FNL_ERR_UNSUPPORTED, "the %d W tiles cannot run at once as clusters of 2..8 CTAs", T);
+    }
+    default: break;
+  }
+  if (c.M <= fnl::k3::MAX_MPAD) return plan_kernel(h, c, Kern::K3, -1, pl);
+  // two tile shapes: 128 x 512 (less traffic and conversion per FLOP, the
+  // default) and 128 x 256 (finer), picked by how well the tiles fill whole
+  // waves of CTAs; a 128 x 512 tile takes about 1.6x a 128 x 256 tile
+  // (measured on B200 across the prefill shapes)
+  const int max_ctas = h->opt.max_ctas > 0 ? std::min(h->opt.max_ctas, h->num_sms) : h->num_sms;
+  const int num_m = (c.M + 127) / 128;
+  const long long tiles_n = static_cast<long long>(num_m) *
+                            (c.op == Op::SwiGLU ? (c.I + 127) / 128 : (c.N + fnl::k2::BN - 1) / fnl::k2::BN);
+  const long long tiles_w = static_cast<long long>(num_m) *
+                            (c.op == Op::SwiGLU ? (c.I + 255) / 256 : (c.N + fnl::k2w::BN - 1) / fnl::k2w::BN);
+  auto waves = [&](long long tiles) {
+    const long long g = std::min<long long>(max_ctas, tiles);
+    return static_cast<double>((tiles + g - 1) / g);
+  };
+  return plan_kernel(h, c, waves(tiles_w) * 1.6 <= waves(tiles_n) ? Kern::K2W : Kern::K2, -1, pl);
+}
+
+size_t stats_bytes_of(const Call& c) {
+  const bool ln = c.op != Op::Residual && c.norm == FNL_NORM_LAYERNORM;
+  return ln ? align256(static_cast<size_t>(c.M) * 8) : 0;
+}
+size_t ss_bytes_of(const Plan& q) {
+  return q.kern == Kern::K3 && q.cls == 0 ? align256(static_cast<size_t>(q.T) * q.max_seg * q.mpad * 4) : 0;
+}
+size_t part_bytes_of(const Plan& q) {
+  if (q.kern == Kern::K4) return 0;
+  if (q.kern == Kern::K3) return q.cls == 0 ? align256(static_cast<size_t>(q.T) * q.max_seg * q.mpad * 128 * 4) : 0;
+  if (q.sk) return align256(static_cast<size_t>(q.T) * q.max_seg * fnl::k2::SLOT_FLOATS * 4);
+  return 0;
+}
+size_t workspace_of(const Call& c, const Plan& q) {
+  return kFixedBytes + stats_bytes_of(c) + ss_bytes_of(q) + part_bytes_of(q);
+}
+
+const char* kern_name(const Plan& q) {
+  switch (q.kern) {
+    case Kern::K3: return q.cls > 0 ? "small-M split-K kernel, cluster form" : "small-M split-K kernel, stream-K form";
+    case Kern::K2: return q.sk ? "128x256 tile kernel, stream-K" : "128x256 tile kernel";
+    case Kern::K4: return "256x512 CTA-pair kernel";
+    default: return "128x512 tile kernel";
+  }
+}
+
+// Enqueue call c with plan q (the workspace must already hold workspace_of(c, q)).
+fnl_status launch_plan(fnl_handle* h, const Call& c, const Plan& q) {
+  fnl_status st;
+  const bool nonorm = c.op == Op::Residual;   // residual-stream projection: no add, no norm
+  const bool rms = !nonorm && c.norm == FNL_NORM_RMSNORM;
+  const bool small = q.kern == Kern::K3, wide = q.kern == Kern::K2W, pair = q.kern == Kern::K4;
+  const size_t sb = stats_bytes_of(c), ssb = ss_bytes_of(q);
+  uint8_t* ws = h->ws;
+  int* status = reinterpret_cast<int*>(ws);
+  unsigned* counters = reinterpret_cast<unsigned*>(ws + kStatusBytes);
+  float2* stats = reinterpret_cast<float2*>(ws + kFixedBytes);
+  float* part_ss = reinterpret_cast<float*>(ws + kFixedBytes + sb);
+  float* part = reinterpret_cast<float*>(ws + kFixedBytes + sb + ssb);
+
+  OpParams p{};
+  p.M = c.M; p.K = c.K; p.N = c.N; p.I = c.I; p.Hq = c.Hq; p.Hkv = c.Hkv; p.D = c.D; p.eps = c.eps;
+  p.x_in = c.x; p.r_in = nonorm ? nullptr : c.residual;
+  p.gamma = c.gamma; p.beta = c.beta; p.bias_in = c.bias_in; p.bias = c.bias;
+  p.residual_out = nonorm ? nullptr : c.residual_out; p.rstd_out = rms ? c.rstd_out : nullptr; p.stats = stats;
+  p.q = c.q; p.k = c.k; p.v = c.v; p.out = c.out;
+  p.res_in = nonorm ? c.residual : nullptr;
+  p.part = part; p.part_ss = part_ss; p.counters = counters; p.max_seg = q.max_seg; p.mpad = q.mpad;
+  p.stages = q.stages; p.status = status; p.cls = q.cls; p.sk = q.sk;
+  p.wait_ns = h->opt.wait_ns > 0 ? static_cast<unsigned long long>(h->opt.wait_ns) : FNL_WAIT_NS;
+  p.stall = 0;
+  if (h->opt.debug_stall_calls > 0) {   // one-shot fault injection for the status-path tests
+    p.stall = 1;
+    --h->opt.debug_stall_calls;
+  }
+  // (the residual-stream projection's operand is bf16 already: nothing to split)
+  p.split = !nonorm && (h->opt.precision == FNL_PRECISION_SPLIT ||
+                        (h->opt.precision == FNL_PRECISION_DEFAULT && c.op == Op::SwiGLU));
+
+  // tensor maps: x and residual tiles are [rows x 64] ([rows x 32] for the
+  // 128x512 kernel), W tiles [rows x 64]
+  CUtensorMap mx, mr, mw;
+  const int act_rows = small ? q.mpad : fnl::k2::BM;
+  int w_rows;
+  if (small) w_rows = c.op == Op::SwiGLU ? 64 : fnl::k3::BW;
+  else if (wide) w_rows = 256;
+  else if (pair) w_rows = 128;   // one CTA's half of an N = 256 operand
+  else w_rows = c.op == Op::SwiGLU ? 128 : fnl::k2::BN;
+  const int box_cols = wide ? fnl::k2w::BK : (pair ? fnl::k4::BK : 64);
+  if ((st = make_map(h, &mx, c.x, c.M, c.K, act_rows, box_cols)) != FNL_OK) return st;
+  if (!nonorm && (st = make_map(h, &mr, c.residual, c.M, c.K, act_rows, box_cols)) != FNL_OK) return st;
+  if ((st = make_map(h, &mw, c.W, c.N, c.K, w_rows, box_cols)) != FNL_OK) return st;
+  // Every GEMM kernel is a programmatic dependent of its predecessor: it
+  // streams its first weight tiles before griddepcontrol.wait and touches
+  // activations, statistics, workspace and outputs only after it.
+  const bool pdl = true;
+  if (nonorm) return dispatch_residual(h, small, wide, pair, q.grid, q.threads, q.smem, pdl, c.stream, mx, mw, p);
+  if (!rms) {
+    if ((st = launch_k1(h, c, stats, c.stream)) != FNL_OK) return st;
+  }
+  const int epi = c.op == Op::QKV ? fnl::kEpiQKV : (c.op == Op::SwiGLU ? fnl::kEpiSwiGLU : fnl::kEpiGELU);
+  switch (epi) {
+    case fnl::kEpiQKV:
+      return dispatch_gemm<fnl::kEpiQKV>(h, small, rms, q.grid, q.threads, q.smem, pdl, c.stream, mx, mr, mw, p, wide,
+                                         pair);
+    case fnl::kEpiSwiGLU:
+      return dispatch_gemm<fnl::kEpiSwiGLU>(h, small, rms, q.grid, q.threads, q.smem, pdl, c.stream, mx, mr, mw, p,
+                                            wide, pair);
+    default:
+      return dispatch_gemm<fnl::kEpiGELU>(h, small, rms, q.grid, q.threads, q.smem, pdl, c.stream, mx, mr, mw, p, wide,
+                                          pair);
+  }
+}
+
+// ------------------------------------------------------------------ tuner
+// Shape auto-tuning (TensorRT-LLM 深度工程实践, §2.4 内核自动调优: candidate
+// kernels with different tile shapes are run on the target GPU and the fastest
+// is kept; trt-llm-deep-dive, 构建阶段详解 "2. 算子选择": GEMMs are chosen by
+// micro-benchmark). With fnl_options.tune, the first call of each shape times
+// every candidate plan on the call's stream and caches the fastest for the
+// handle. A plan depends on M only through the small-M padding (M <= 128) or
+// the count of 128-row blocks, so those key the cache together with the op,
+// the norm, the operand precision, N and K.
+
+TuneKey tune_key(const Call& c) {
+  TuneKey k;
+  k.op = static_cast<int>(c.op);
+  k.norm = c.op == Op::Residual ? -1 : static_cast<int>(c.norm);
+  k.mkey = c.M <= fnl::k3::MAX_MPAD ? round_up(c.M, 16) : 1000 + (c.M + 127) / 128;
+  k.N = c.N; k.K = c.K; k.I = c.I;
+  return k;
+}
+
+// Time plan q on c.stream: one warm-up launch, then `reps` launches, each after
+// a write of `flush_bytes` at `flush` that evicts the operands from L2 (in a
+// model the weights of a layer are not L2-resident when its call starts);
+// median us of the launches alone.
+fnl_status time_plan(fnl_handle* h, const Call& c, const Plan& q, int reps, void* flush, size_t flush_bytes,
+                     float* us) {
+  cudaEvent_t ev[2];
+  cudaError_t e = cudaEventCreate(&ev[0]);
+  if (e == cudaSuccess) e = cudaEventCreate(&ev[1]);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventCreate");
+  fnl_status st = launch_plan(h, c, q);
+  float t[9];
+  reps = std::min(reps, 9);
+  for (int r = 0; r < reps && st == FNL_OK; ++r) {
+    if (flush) cudaMemsetAsync(flush, r & 0xff, flush_bytes, c.stream);
+    cudaEventRecord(ev[0], c.stream);
+    st = launch_plan(h, c, q);
+    cudaEventRecord(ev[1], c.stream);
+    if (st == FNL_OK) {
+      if ((e = cudaEventSynchronize(ev[1])) != cudaSuccess) st = cuda_fail(h, e, "cudaEventSynchronize");
+      else cudaEventElapsedTime(&t[r], ev[0], ev[1]);
+    }
+  }
+  cudaEventDestroy(ev[0]);
+  cudaEventDestroy(ev[1]);
+  if (st != FNL_OK) return st;
+  std::sort(t, t + reps);
+  *us = t[reps / 2] * 1e3f;
+  return FNL_OK;
+}
+
+// Same kernel, form and grid.
+bool same_plan(const Plan& a, const Plan& b) {
+  return a.kern == b.kern && a.cls == b.cls && a.sk == b.sk && a.grid == b.grid;
+}
+
+fnl_status tune(fnl_handle* h, const Call& c, Plan* best) {
+  // candidates: every kernel that takes the shape, the small-M kernel in each
+  // of its forms (stream-K and every cluster size whose clusters fit)
+  Plan cand[12];
+  int n = 0;
+  Plan q;
+  Plan dflt;
+  const bool have_dflt = default_plan(h, c, &dflt) == FNL_OK;
+  const bool small_ok = c.M <= fnl::k3::MAX_MPAD;
+  if (small_ok) {
+    if (plan_kernel(h, c, Kern::K3, 0, &q) == FNL_OK) cand[n++] = q;
+    for (int cls = 2; cls <= 8 && n < 10; ++cls)
+      if (plan_kernel(h, c, Kern::K3, cls, &q) == FNL_OK) cand[n++] = q;
+  }
+  if (plan_kernel(h, c, Kern::K2, -1, &q) == FNL_OK) cand[n++] = q;
+  if (!small_ok && plan_kernel(h, c, Kern::K2W, -1, &q) == FNL_OK) cand[n++] = q;
+  if (!small_ok && plan_kernel(h, c, Kern::K4, -1, &q) == FNL_OK) cand[n++] = q;
+  h->err.clear();   // refused candidates are not errors of the call
+  if (n == 0) return default_plan(h, c, best);
+  size_t need = 0;
+  for (int i = 0; i < n; ++i) need = std::max(need, workspace_of(c, cand[i]));
+  fnl_status st = ensure_workspace(h, c.stream, need);
+  if (st != FNL_OK) return st;
+  // an L2-sized buffer to write between timed launches (held for this call only)
+  int l2 = 0;
+  cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, h->device);
+  const size_t flush_bytes = static_cast<size_t>(std::max(l2, 1 << 20)) * 2;
+  void* flush = nullptr;
+  cudaError_t e = cudaMalloc(&flush, flush_bytes);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaMalloc(tuning L2 flush buffer)");
+  int bi = -1, di = -1;
+  float bus = 0.f, dus = 0.f;
+  for (int i = 0; i < n && st == FNL_OK; ++i) {
+    float us = 0.f;
+    if ((st = time_plan(h, c, cand[i], 5, flush, flush_bytes, &us)) != FNL_OK) break;
+    if (bi < 0 || us < bus) {
+      bi = i;
+      bus = us;
+    }
+    if (have_dflt && di < 0 && same_plan(cand[i], dflt)) {
+      di = i;
+      dus = us;
+    }
+  }
+  cudaStreamSynchronize(c.stream);
+  cudaFree(flush);
+  if (st != FNL_OK) return st;
+  // the untuned plan stays unless another is faster by more than the timing noise
+  if (di >= 0 && bus > 0.97f * dus) {
+    bi = di;
+    bus = dus;
+  }
+  *best = cand[bi];
+  h->tuned.push_back({tune_key(c), cand[bi], bus, n});
+  char buf[160];
+  snprintf(buf, sizeof(buf), "%s, grid %d (tuned: %.1f us, fastest of %d candidates)", kern_name(cand[bi]),
+           cand[bi].grid, bus, n);
+  h->plan_text = buf;
+  return FNL_OK;
+}
+
 fnl_status run(fnl_handle* h, const Call& c) {
   fnl_status st = validate(h, c);
   if (st != FNL_OK || c.M == 0) return st;
@@ -336,135 +870,36 @@ fnl_status run(fnl_handle* h, const Call& c) {
   cudaError_t e = cudaSetDevice(h->device);
   if (e != cudaSuccess) return cuda_fail(h, e, "cudaSetDevice");
 
-  const bool rms = c.norm == FNL_NORM_RMSNORM;
-  const int epi = c.op == Op::QKV ? fnl::kEpiQKV : (c.op == Op::SwiGLU ? fnl::kEpiSwiGLU : fnl::kEpiGELU);
-  bool small = c.M <= fnl::k3::MAX_MPAD;
-  if (h->opt.path == FNL_PATH_TILE || h->opt.path == FNL_PATH_TILE_WIDE) small = false;
-  if (h->opt.path == FNL_PATH_SPLITK || h->opt.path == FNL_PATH_SPLITK_CLUSTER) small = true;
-  const int max_ctas = h->opt.max_ctas > 0 ? std::min(h->opt.max_ctas, h->num_sms) : h->num_sms;
-  const int nkb = (c.K + 63) / 64;
-
-  // plan
-  int grid = 1, threads = 0, smem = 0, mpad = 0, stages = 0, max_seg = 1, T = 0, cls = 0, sk = 0;
-  bool wide = false;
-  if (small) {
-    mpad = round_up(std::max(c.M, 1), 16);
-    T = c.op == Op::SwiGLU ? (c.I + 63) / 64 : (c.N + 127) / 128;
-    const long long U = static_cast<long long>(T) * nkb;
-    grid = static_cast<int>(std::min<long long>(max_ctas, U));
-    stages = std::min(fnl::k3::MAX_STAGES, (200 * 1024) / fnl::k3::stage_bytes(mpad));
-    smem = fnl::k3::smem_bytes(mpad, stages);
-    threads = fnl::k3::NUM_THREADS;
-    // Cluster form: one W tile per cluster of cls CTAs, each taking 1/cls of
-    // its k-blocks, partial sums reduced on chip. Used when the clusters cover
-    // the GPU (or every unit of work) and all of them are resident at once.
-    if (h->opt.path == FNL_PATH_SPLITK_CLUSTER || (h->opt.path != FNL_PATH_SPLITK && h->opt.max_ctas == 0)) {
-      // the largest cluster size (<= 8, <= the k-blocks) whose T clusters are all resident
-      for (int c_ = std::min({8, h->num_sms / std::max(T, 1), nkb}); c_ >= 2 && cls == 0; --c_) {
-        const bool covers = static_cast<long long>(T) * c_ >= std::min<long long>(U, (h->num_sms * 9) / 10);
-        if ((covers || h->opt.path == FNL_PATH_SPLITK_CLUSTER) && resident_clusters(h, smem, c_) >= T) cls = c_;
+  Plan q;
+  bool planned = false;
+  if (h->opt.tune && h->opt.path == FNL_PATH_AUTO) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(c.stream, &cap);
+    const TuneKey key = tune_key(c);
+    for (const auto& t : h->tuned)
+      if (t.key == key) {
+        q = t.plan;
+        planned = true;
+        char buf[160];
+        snprintf(buf, sizeof(buf), "%s, grid %d (tuned plan from the cache: %.1f us, %d candidates)",
+                 kern_name(q), q.grid, t.us, t.candidates);
+        h->plan_text = buf;
+        break;
       }
+    // tuning synchronises the stream: never inside a stream capture
+    if (!planned && cap == cudaStreamCaptureStatusNone) {
+      if ((st = tune(h, c, &q)) != FNL_OK) return st;
+      planned = true;
     }
-    if (h->opt.path == FNL_PATH_SPLITK_CLUSTER && cls == 0)
-      return fail(h, FNL_ERR_UNSUPPORTED, "the %d W tiles cannot run at once as clusters of 2..8 CTAs", T);
-    if (cls > 0) grid = T * cls;
-    for (int t = 0; t < T && cls == 0; ++t) {
-      const int first = fnl::unit_owner(static_cast<long long>(t) * nkb, grid, U);
-      const int last = fnl::unit_owner(static_cast<long long>(t + 1) * nkb - 1, grid, U);
-      max_seg = std::max(max_seg, last - first + 1);
-    }
-    if (T > kMaxTiles) return fail(h, FNL_ERR_UNSUPPORTED, "too many W tiles");
-  } else {
-    // two tile shapes: 128 x 512 (less traffic and conversion per FLOP, the
-    // default) and 128 x 256 (finer), picked by how well the tiles fill whole
-    // waves of CTAs
-    const int num_m = (c.M + 127) / 128;
-    const long long tiles_n = static_cast<long long>(num_m) *
-                              (c.op == Op::SwiGLU ? (c.I + 127) / 128 : (c.N + fnl::k2::BN - 1) / fnl::k2::BN);
-    const long long tiles_w = static_cast<long long>(num_m) *
-                              (c.op == Op::SwiGLU ? (c.I + 255) / 256 : (c.N + fnl::k2w::BN - 1) / fnl::k2w::BN);
-    // estimated time = waves x time of one tile; a 128 x 512 tile takes about
-    // 1.6x a 128 x 256 tile (measured on B200 across the prefill shapes)
-    auto waves = [&](long long tiles) {
-      const long long g = std::min<long long>(max_ctas, tiles);
-      return static_cast<double>((tiles + g - 1) / g);
-    };
-    wide = waves(tiles_w) * 1.6 <= waves(tiles_n);
-    if (h->opt.path == FNL_PATH_TILE) wide = false;
-    if (h->opt.path == FNL_PATH_TILE_WIDE) wide = true;
-    const long long tiles = wide ? tiles_w : tiles_n;
-    grid = static_cast<int>(std::min<long long>(max_ctas, tiles));
-    // Fewer 128x256 tiles than CTAs by a fifth or more (e.g. 70B QKV at
-    // M = 256: 80 tiles, 148 SMs): stream-K over (tile, k-block) units, so
-    // every SM streams weights; partial tiles are summed by their last CTA.
-    if (!wide && tiles * 5 <= static_cast<long long>(max_ctas) * 4) {
-      sk = 1;
-      T = static_cast<int>(tiles);
-      const long long U = tiles * nkb;
-      grid = static_cast<int>(std::min<long long>(max_ctas, U));
-      for (int t = 0; t < T; ++t) {
-        const int first = fnl::unit_owner(static_cast<long long>(t) * nkb, grid, U);
-        const int last = fnl::unit_owner(static_cast<long long>(t + 1) * nkb - 1, grid, U);
-        max_seg = std::max(max_seg, last - first + 1);
-      }
-      if (T > kMaxTiles) return fail(h, FNL_ERR_UNSUPPORTED, "too many W tiles");
-    }
-    smem = wide ? fnl::k2w::SMEM_BYTES : fnl::k2::SMEM_BYTES;
-    threads = wide ? fnl::k2w::NUM_THREADS : fnl::k2::NUM_THREADS;
   }
-
-  // workspace
-  const size_t stats_bytes = rms ? 0 : align256(static_cast<size_t>(c.M) * 8);
-  const size_t ss_bytes = small && cls == 0 ? align256(static_cast<size_t>(T) * max_seg * mpad * 4) : 0;
-  size_t part_bytes = small && cls == 0 ? align256(static_cast<size_t>(T) * max_seg * mpad * 128 * 4) : 0;
-  if (sk) part_bytes = align256(static_cast<size_t>(T) * max_seg * fnl::k2::SLOT_FLOATS * 4);
-  const size_t need = kFixedBytes + stats_bytes + ss_bytes + part_bytes;
-  if ((st = ensure_workspace(h, c.stream, need)) != FNL_OK) return st;
-  uint8_t* ws = h->ws;
-  int* status = reinterpret_cast<int*>(ws);
-  unsigned* counters = reinterpret_cast<unsigned*>(ws + kStatusBytes);
-  float2* stats = reinterpret_cast<float2*>(ws + kFixedBytes);
-  float* part_ss = reinterpret_cast<float*>(ws + kFixedBytes + stats_bytes);
-  float* part = reinterpret_cast<float*>(ws + kFixedBytes + stats_bytes + ss_bytes);
-
-  OpParams p{};
-  p.M = c.M; p.K = c.K; p.N = c.N; p.I = c.I; p.Hq = c.Hq; p.Hkv = c.Hkv; p.D = c.D; p.eps = c.eps;
-  p.x_in = c.x; p.r_in = c.residual;
-  p.gamma = c.gamma; p.beta = c.beta; p.bias_in = c.bias_in; p.bias = c.bias;
-  p.residual_out = c.residual_out; p.rstd_out = rms ? c.rstd_out : nullptr; p.stats = stats;
-  p.q = c.q; p.k = c.k; p.v = c.v; p.out = c.out;
-  p.part = part; p.part_ss = part_ss; p.counters = counters; p.max_seg = max_seg; p.mpad = mpad;
-  p.stages = stages; p.status = status; p.cls = cls; p.sk = sk;
-  p.split = h->opt.precision == FNL_PRECISION_SPLIT ||
-            (h->opt.precision == FNL_PRECISION_DEFAULT && c.op == Op::SwiGLU);
-
-  // tensor maps: x and residual tiles are [rows x 64], W tiles [rows x 64]
-  CUtensorMap mx, mr, mw;
-  const int act_rows = small ? mpad : fnl::k2::BM;
-  int w_rows;
-  if (small) w_rows = c.op == Op::SwiGLU ? 64 : fnl::k3::BW;
-  else if (wide) w_rows = 256;
-  else w_rows = c.op == Op::SwiGLU ? 128 : fnl::k2::BN;
-  const int box_cols = wide ? fnl::k2w::BK : 64;
-  if ((st = make_map(h, &mx, c.x, c.M, c.K, act_rows, box_cols)) != FNL_OK) return st;
-  if ((st = make_map(h, &mr, c.residual, c.M, c.K, act_rows, box_cols)) != FNL_OK) return st;
-  if ((st = make_map(h, &mw, c.W, c.N, c.K, w_rows, box_cols)) != FNL_OK) return st;
-
-  if (!rms) {
-    if ((st = launch_k1(h, c, stats, c.stream)) != FNL_OK) return st;
+  if (!planned) {
+    if ((st = default_plan(h, c, &q)) != FNL_OK) return st;
+    char buf[160];
+    snprintf(buf, sizeof(buf), "%s, grid %d", kern_name(q), q.grid);
+    h->plan_text = buf;
   }
-  // Every GEMM kernel is a programmatic dependent of its predecessor: it
-  // streams its first weight tiles before griddepcontrol.wait and touches
-  // activations, statistics, workspace and outputs only after it.
-  const bool pdl = true;
-  switch (epi) {
-    case fnl::kEpiQKV:
-      return dispatch_gemm<fnl::kEpiQKV>(h, small, rms, grid, threads, smem, pdl, c.stream, mx, mr, mw, p, wide);
-    case fnl::kEpiSwiGLU:
-      return dispatch_gemm<fnl::kEpiSwiGLU>(h, small, rms, grid, threads, smem, pdl, c.stream, mx, mr, mw, p, wide);
-    default:
-      return dispatch_gemm<fnl::kEpiGELU>(h, small, rms, grid, threads, smem, pdl, c.stream, mx, mr, mw, p, wide);
-  }
+  if ((st = ensure_workspace(h, c.stream, workspace_of(c, q))) != FNL_OK) return st;
+  return launch_plan(h, c, q);
 }
 
 const bf16* B(const fnl_bf16* p) { return reinterpret_cast<const bf16*>(p); }
@@ -479,8 +914,9 @@ fnl_status fnl_create(fnl_handle** out, int device, const fnl_options* opt) {
   *out = nullptr;
   fnl_handle* h = new fnl_handle();
   if (opt) h->opt = *opt;
-  if (h->opt.path < FNL_PATH_AUTO || h->opt.path > FNL_PATH_SPLITK_CLUSTER || h->opt.max_tokens < 0 || h->opt.max_n < 0 ||
-      h->opt.precision < FNL_PRECISION_DEFAULT || h->opt.precision > FNL_PRECISION_SINGLE) {
+  if (h->opt.path < FNL_PATH_AUTO || h->opt.path > FNL_PATH_TILE_PAIR || h->opt.max_tokens < 0 || h->opt.max_n < 0 ||
+      h->opt.precision < FNL_PRECISION_DEFAULT || h->opt.precision > FNL_PRECISION_SINGLE || h->opt.wait_ns < 0 ||
+      h->opt.debug_stall_calls < 0 || h->opt.tune < 0 || h->opt.tune > 1) {
     delete h;
     return FNL_ERR_INVALID_ARG;
   }
@@ -539,6 +975,8 @@ const char* fnl_status_string(fnl_status s) {
 
 const char* fnl_last_error(const fnl_handle* h) { return h ? h->err.c_str() : ""; }
 
+const char* fnl_last_plan(const fnl_handle* h) { return h ? h->plan_text.c_str() : ""; }
+
 fnl_status fnl_check(fnl_handle* h, fnl_stream stream) {
   if (!h) return FNL_ERR_INVALID_ARG;
   cudaSetDevice(h->device);
@@ -548,7 +986,12 @@ fnl_status fnl_check(fnl_handle* h, fnl_stream stream) {
   e = cudaMemcpy(&status, h->ws, sizeof(int), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemcpy(status)");
   if (status != 0) {
-    cudaMemset(h->ws, 0, sizeof(int));
+    // A CTA that gave up never made its split-K arrival, so its tiles' arrival
+    // counters are left part-way; clear them with the status word, or every later
+    // call would elect the wrong last CTA.
+    e = cudaMemset(h->ws, 0, kFixedBytes);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemset(status, counters)");
     return fail(h, FNL_ERR_DEVICE_STATUS, "a kernel gave up a bounded wait (code %d)", status);
   }
   return FNL_OK;
@@ -564,10 +1007,10 @@ fnl_status fnl_add_norm_qkv(fnl_handle* h, fnl_stream stream, const fnl_bf16* x,
   c.x = B(x); c.residual = B(residual); c.bias_in = nullptr; c.gamma = B(gamma); c.beta = B(beta);
   c.W = B(W); c.bias = B(bias); c.residual_out = Bm(residual_out);
   c.norm = norm; c.eps = eps; c.M = M; c.K = K; c.Hq = Hq; c.Hkv = Hkv; c.D = D;
-  c.N = (Hq > 0 && Hkv > 0 && D > 0) ? (Hq + 2 * Hkv) * D : 0;
+  c.N = qkv_columns(Hq, Hkv, D);
   c.q = Bm(q); c.k = Bm(k); c.v = Bm(v); c.out = nullptr;
   c.mean_out = mean_out; c.rstd_out = rstd_out;
-  if (c.N <= 0 && h) return fail(h, FNL_ERR_INVALID_ARG, "Hq, Hkv, D must be > 0");
+  if (c.N <= 0 && h) return fail(h, FNL_ERR_INVALID_ARG, "Hq, Hkv, D must be > 0 and (Hq + 2 Hkv) D <= %d", kMaxN);
   return run(h, c);
 }
 
@@ -580,10 +1023,10 @@ fnl_status fnl_add_norm_swiglu(fnl_handle* h, fnl_stream stream, const fnl_bf16*
   c.stream = reinterpret_cast<cudaStream_t>(stream);
   c.x = B(x); c.residual = B(residual); c.bias_in = nullptr; c.gamma = B(gamma); c.beta = B(beta);
   c.W = B(W); c.bias = B(bias); c.residual_out = Bm(residual_out);
-  c.norm = norm; c.eps = eps; c.M = M; c.K = K; c.I = I; c.N = I > 0 ? 2 * I : 0;
+  c.norm = norm; c.eps = eps; c.M = M; c.K = K; c.I = I; c.N = (I > 0 && I <= kMaxN / 2) ? 2 * I : 0;
   c.out = Bm(out);
   c.mean_out = mean_out; c.rstd_out = rstd_out;
-  if (c.N <= 0 && h) return fail(h, FNL_ERR_INVALID_ARG, "I must be > 0");
+  if (c.N <= 0 && h) return fail(h, FNL_ERR_INVALID_ARG, "I must be > 0 and 2 I <= %d", kMaxN);
   return run(h, c);
 }
 
@@ -600,6 +1043,18 @@ fnl_status fnl_add_bias_norm_gelu(fnl_handle* h, fnl_stream stream, const fnl_bf
   c.norm = norm; c.eps = eps; c.M = M; c.K = K; c.N = N;
   c.out = Bm(out);
   c.mean_out = mean_out; c.rstd_out = rstd_out;
+  return run(h, c);
+}
+
+fnl_status fnl_linear_add_residual(fnl_handle* h, fnl_stream stream, const fnl_bf16* a, const fnl_bf16* W,
+                                   const fnl_bf16* bias, const fnl_bf16* residual, fnl_bf16* out, int M, int K,
+                                   int N) {
+  Call c{};
+  c.op = Op::Residual;
+  c.stream = reinterpret_cast<cudaStream_t>(stream);
+  c.x = B(a); c.W = B(W); c.bias = B(bias); c.residual = B(residual); c.out = Bm(out);
+  c.norm = FNL_NORM_RMSNORM; c.eps = 1.f;   // unused (no norm)
+  c.M = M; c.K = K; c.N = N;
   return run(h, c);
 }
 
@@ -654,8 +1109,8 @@ fnl_status static_setup(int dev, void** ptr, int* sms) {
 // Argument checks of fnl_add_norm_qkv, without a handle (and without heap use).
 fnl_status validate_static(const Call& c) {
   if (c.norm != FNL_NORM_LAYERNORM && c.norm != FNL_NORM_RMSNORM) return FNL_ERR_INVALID_ARG;
-  if (!(c.eps >= 0.f) || c.eps > 1e30f) return FNL_ERR_INVALID_ARG;
-  if (c.M < 0 || c.K <= 0 || c.Hq <= 0 || c.Hkv <= 0 || c.D <= 0) return FNL_ERR_INVALID_ARG;
+  if (!(c.eps > 0.f) || c.eps > 1e30f) return FNL_ERR_INVALID_ARG;
+  if (c.M < 0 || c.K <= 0 || c.Hq <= 0 || c.Hkv <= 0 || c.D <= 0 || c.N <= 0) return FNL_ERR_INVALID_ARG;
   if (c.Hq % c.Hkv) return FNL_ERR_INVALID_ARG;
   if (c.K % 8 || c.D % 8) return FNL_ERR_ALIGNMENT;
   if (c.K > 32768 || c.M > fnl::k3::MAX_MPAD) return FNL_ERR_UNSUPPORTED;
@@ -702,7 +1157,7 @@ extern "C" fnl_status fnl_add_norm_qkv_static(fnl_stream stream, const fnl_bf16*
   c.x = B(x); c.residual = B(residual); c.bias_in = nullptr; c.gamma = B(gamma); c.beta = B(beta);
   c.W = B(W); c.bias = B(bias); c.residual_out = Bm(residual_out);
   c.norm = norm; c.eps = eps; c.M = M; c.K = K; c.Hq = Hq; c.Hkv = Hkv; c.D = D;
-  c.N = (Hq > 0 && Hkv > 0 && D > 0) ? (Hq + 2 * Hkv) * D : 0;
+  c.N = qkv_columns(Hq, Hkv, D);
   c.q = Bm(q); c.k = Bm(k); c.v = Bm(v); c.out = nullptr;
   c.mean_out = mean_out; c.rstd_out = rstd_out;
   fnl_status st = validate_static(c);
@@ -731,14 +1186,17 @@ extern "C" fnl_status fnl_add_norm_qkv_static(fnl_stream stream, const fnl_bf16*
   }
   // scratch layout: [status][counters][stats][partial h^2 sums][partial accumulators]
   const size_t zero_bytes = align256(kStatusBytes + static_cast<size_t>(T) * 4);
+  const size_t counter_bytes = zero_bytes - kStatusBytes;
   const size_t stats_bytes = rms ? 0 : align256(static_cast<size_t>(c.M) * 8);
   const size_t ss_bytes = align256(static_cast<size_t>(T) * max_seg * mpad * 4);
   const size_t part_bytes = align256(static_cast<size_t>(T) * max_seg * mpad * 128 * 4);
   if (zero_bytes + stats_bytes + ss_bytes + part_bytes > kStaticScratchBytes) return FNL_ERR_UNSUPPORTED;
   uint8_t* base = static_cast<uint8_t*>(scratch);
-  // the array keeps the previous call's contents: the status word and the
-  // arrival counters must start at zero (the rest is written before it is read)
-  cudaError_t e = cudaMemsetAsync(base, 0, zero_bytes, c.stream);
+  // The array keeps the previous call's contents: the arrival counters must
+  // start at zero (the rest is written before it is read). The status word is
+  // left alone: it keeps the first failure code until fnl_check_static reads
+  // and clears it.
+  cudaError_t e = cudaMemsetAsync(base + kStatusBytes, 0, counter_bytes, c.stream);
   if (e != cudaSuccess) return FNL_ERR_CUDA;
 
   OpParams p{};
@@ -753,6 +1211,8 @@ extern "C" fnl_status fnl_add_norm_qkv_static(fnl_stream stream, const fnl_bf16*
   p.part = reinterpret_cast<float*>(base + zero_bytes + stats_bytes + ss_bytes);
   p.max_seg = max_seg; p.mpad = mpad; p.stages = stages; p.split = 0;
   p.status = reinterpret_cast<int*>(base);
+  p.wait_ns = FNL_WAIT_NS;
+  p.stall = 0;
 
   CUtensorMap mx, mr, mw;
   if ((st = make_map(nullptr, &mx, c.x, c.M, c.K, mpad)) != FNL_OK) return st;
@@ -762,4 +1222,21 @@ extern "C" fnl_status fnl_add_norm_qkv_static(fnl_stream stream, const fnl_bf16*
     return st;
   return dispatch_gemm<fnl::kEpiQKV>(nullptr, true, rms, grid, fnl::k3::NUM_THREADS,
                                      fnl::k3::smem_bytes(mpad, stages), !rms, c.stream, mx, mr, mw, p);
+}
+
+extern "C" fnl_status fnl_check_static(fnl_stream stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FNL_ERR_CUDA;
+  void* scratch = nullptr;
+  int sms = 0;
+  fnl_status st = static_setup(dev, &scratch, &sms);
+  if (st != FNL_OK) return st;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return FNL_ERR_CUDA;
+  int status = 0;
+  if (cudaMemcpy(&status, scratch, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FNL_ERR_CUDA;
+  if (status == 0) return FNL_OK;
+  // clear the status word (the next call clears the arrival counters itself)
+  if (cudaMemset(scratch, 0, sizeof(int)) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+    return FNL_ERR_CUDA;
+  return FNL_ERR_DEVICE_STATUS;
 }

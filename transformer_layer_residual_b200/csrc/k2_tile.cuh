@@ -273,6 +273,8 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
       const int npre = P < STAGES ? P : STAGES;
       uint32_t armed_w = 0, armed_x = 0, par_w = 0, par_x = 0;
       bool ok = true;
+      // fault injection (status-path tests only): CTA 0 withholds its first weight copy
+      bool withhold = p.stall != 0 && blockIdx.x == 0;
       struct Cur {
         int t, mb, nb, kb, s;
         uint32_t ph;
@@ -296,6 +298,10 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
         }
       };
       auto issue_w = [&](const Cur& c) {
+        if (withhold) {
+          withhold = false;
+          return;
+        }
         uint8_t* st = smem + c.s * STAGE_BYTES;
         mbar_arrive_expect_tx(&ctrl->full_w[c.s], W_BYTES);
         if (EPI == kEpiSwiGLU) {
@@ -309,6 +315,13 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
       };
       auto issue_x = [&](const Cur& c) {
         uint8_t* st = smem + c.s * STAGE_BYTES;
+        if (NORM == kNoNorm) {   // the activation tile is the operand as loaded
+          mbar_arrive_expect_tx(&ctrl->full_x[c.s], X_BYTES);
+          tma_load_2d(st, &tm_x, &ctrl->full_x[c.s], c.kb * BK, c.mb * BM);
+          armed_x |= 1u << c.s;
+          par_x = (par_x & ~(1u << c.s)) | (c.ph << c.s);
+          return;
+        }
         mbar_arrive_expect_tx(&ctrl->full_x[c.s], 2 * X_BYTES + vec_bytes(p, has_beta, has_bias_in, c.kb));
         issue_vec_loads(p, has_beta, has_bias_in, c.kb, vecs + c.s * 3 * kVecElems, &ctrl->full_x[c.s]);
         tma_load_2d(st, &tm_x, &ctrl->full_x[c.s], c.kb * BK, c.mb * BM);
@@ -325,7 +338,7 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
       pdl_wait();
       for (int q = 0; q < P; ++q) {
         if (q >= npre) {
-          if (!mbar_wait(&ctrl->empty[cw.s], cw.ph ^ 1, abortf, p.status, kStatusWaitEmpty)) {
+          if (!mbar_wait(&ctrl->empty[cw.s], cw.ph ^ 1, abortf, p.status, kStatusWaitEmpty, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -355,12 +368,14 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
         const int b = i & 1;
         const uint32_t use = static_cast<uint32_t>(i >> 1);
         ++i;
-        if (!mbar_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty)) break;
+        if (!mbar_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty, p.wait_ns)) break;
         tc_fence_after();
         const uint32_t d = tmem + b * BN;
         for (int kb = 0; kb < nk; ++kb) {   // kb counts the segment's k-blocks
-          if (!mbar_wait(&ctrl->conv[s], ph, abortf, p.status, kStatusWaitConv) ||
-              !mbar_wait(&ctrl->full_w[s], ph, abortf, p.status, kStatusWaitFull)) {
+          // the converted operand (or, without a norm, the activation tile as loaded)
+          uint64_t* ready = NORM == kNoNorm ? &ctrl->full_x[s] : &ctrl->conv[s];
+          if (!mbar_wait(ready, ph, abortf, p.status, kStatusWaitConv, p.wait_ns) ||
+              !mbar_wait(&ctrl->full_w[s], ph, abortf, p.status, kStatusWaitFull, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -402,10 +417,10 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
       const int b = i & 1;
       const uint32_t use = static_cast<uint32_t>(i >> 1);
       ++i;
-      if (!warp_wait(&ctrl->tfull[b], use & 1, abortf, p.status, kStatusWaitTmemFull)) break;
+      if (!warp_wait(&ctrl->tfull[b], use & 1, abortf, p.status, kStatusWaitTmemFull, p.wait_ns)) break;
       float ssq = 0.f;
       if (NORM == kRMSNorm) {
-        if (!warp_wait(&ctrl->sfull[b], use & 1, abortf, p.status, kStatusWaitStats)) break;
+        if (!warp_wait(&ctrl->sfull[b], use & 1, abortf, p.status, kStatusWaitStats, p.wait_ns)) break;
         ssq = ctrl->rs[b][row_local];
       }
       tc_fence_after();
@@ -444,7 +459,7 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
         // arrival (as in the small-M kernel: the epilogue mbarrier orders the
         // slot stores before thread et 0's acquire-release atomic)
         if (lane == 0) mbar_arrive(&ctrl->esync);
-        if (!warp_wait(&ctrl->esync, eph, abortf, p.status, kStatusWaitDrain)) break;
+        if (!warp_wait(&ctrl->esync, eph, abortf, p.status, kStatusWaitDrain, p.wait_ns)) break;
         eph ^= 1;
         if (et == 0) {
           const unsigned old = atom_add_acq_rel_gpu(&p.counters[t], 1u);
@@ -452,7 +467,7 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->esync);
-        if (!warp_wait(&ctrl->esync, eph, abortf, p.status, kStatusWaitDrain)) break;
+        if (!warp_wait(&ctrl->esync, eph, abortf, p.status, kStatusWaitDrain, p.wait_ns)) break;
         eph ^= 1;
         if (ctrl->last_flag) {
           if (segs.done()) {   // the CTA's last segment: summed by all warps below
@@ -527,7 +542,7 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctrl->tempty[b]);
     }
-  } else {
+  } else if (NORM != kNoNorm) {
     // ------------------------------------------------------------ converters
     const int ct = threadIdx.x - WARP_CONV0 * 32;   // 0 .. NUM_CONV_WARPS*32-1
     const int c = ct & 7;                            // 16-byte chunk of the 128-byte row
@@ -558,7 +573,7 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
       }
       const bool write_res = (NORM == kRMSNorm) && nb == 0;
       for (int kb = kb0; kb < kb0 + nk; ++kb) {
-        if (!warp_wait(&ctrl->full_x[s], ph, abortf, p.status, kStatusWaitFull)) {
+        if (!warp_wait(&ctrl->full_x[s], ph, abortf, p.status, kStatusWaitFull, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -627,7 +642,7 @@ __global__ void __launch_bounds__(k2::NUM_THREADS, 1)
         }
         const int b = i & 1;
         const uint32_t use = static_cast<uint32_t>(i >> 1);
-        if (!warp_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty)) break;
+        if (!warp_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty, p.wait_ns)) break;
         if (c == 0) {   // the segment's sum(h^2) per row; the epilogue turns it into 1/rms
 #pragma unroll
           for (int j = 0; j < RPT; ++j) {

@@ -136,6 +136,8 @@ __global__ void __launch_bounds__(k2w::NUM_THREADS, 1)
       const int npre = P < STAGES ? P : STAGES;
       uint32_t armed_w = 0, armed_x = 0, par_w = 0, par_x = 0;
       bool ok = true;
+      // fault injection (status-path tests only): CTA 0 withholds its first weight copy
+      bool withhold = p.stall != 0 && blockIdx.x == 0;
       struct Cur {
         int t, mb, nb, kb, s;
         uint32_t ph;
@@ -155,6 +157,10 @@ __global__ void __launch_bounds__(k2w::NUM_THREADS, 1)
         }
       };
       auto issue_w = [&](const Cur& c) {
+        if (withhold) {
+          withhold = false;
+          return;
+        }
         uint8_t* st = smem + c.s * STAGE_BYTES + 2 * X_BYTES;
         mbar_arrive_expect_tx(&ctrl->full_w[c.s], W_BYTES);
         if (EPI == kEpiSwiGLU) {
@@ -169,6 +175,13 @@ __global__ void __launch_bounds__(k2w::NUM_THREADS, 1)
       };
       auto issue_x = [&](const Cur& c) {
         uint8_t* st = smem + c.s * STAGE_BYTES;
+        if (NORM == kNoNorm) {   // the activation tile is the operand as loaded
+          mbar_arrive_expect_tx(&ctrl->full_x[c.s], X_BYTES);
+          tma_load_2d(st, &tm_x, &ctrl->full_x[c.s], c.kb * BK, c.mb * BM);
+          armed_x |= 1u << c.s;
+          par_x = (par_x & ~(1u << c.s)) | (c.ph << c.s);
+          return;
+        }
         bf16* vec = vecs + c.s * 3 * VEC;
         const int k0 = c.kb * BK;
         const uint32_t vb = static_cast<uint32_t>(min(VEC, K - k0)) * 2;
@@ -189,7 +202,7 @@ __global__ void __launch_bounds__(k2w::NUM_THREADS, 1)
       pdl_wait();
       for (int q = 0; q < P; ++q) {
         if (q >= npre) {
-          if (!mbar_wait(&ctrl->empty[cw.s], cw.ph ^ 1, abortf, p.status, kStatusWaitEmpty)) {
+          if (!mbar_wait(&ctrl->empty[cw.s], cw.ph ^ 1, abortf, p.status, kStatusWaitEmpty, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -214,12 +227,14 @@ __global__ void __launch_bounds__(k2w::NUM_THREADS, 1)
       const uint32_t idesc = idesc_bf16(BM, 256);
       int i = 0;
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++i) {
-        if (!mbar_wait(&ctrl->tempty, (static_cast<uint32_t>(i) & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty))
+        if (!mbar_wait(&ctrl->tempty, (static_cast<uint32_t>(i) & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty, p.wait_ns))
           break;
         tc_fence_after();
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&ctrl->full_w[s], ph, abortf, p.status, kStatusWaitFull) ||
-              !mbar_wait(&ctrl->conv[s], ph, abortf, p.status, kStatusWaitConv)) {
+          // the converted operand (or, without a norm, the activation tile as loaded)
+          uint64_t* ready = NORM == kNoNorm ? &ctrl->full_x[s] : &ctrl->conv[s];
+          if (!mbar_wait(&ctrl->full_w[s], ph, abortf, p.status, kStatusWaitFull, p.wait_ns) ||
+              !mbar_wait(ready, ph, abortf, p.status, kStatusWaitConv, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -259,10 +274,10 @@ __global__ void __launch_bounds__(k2w::NUM_THREADS, 1)
     int i = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
       const uint32_t par = static_cast<uint32_t>(i) & 1;
-      if (!warp_wait(&ctrl->tfull, par, abortf, p.status, kStatusWaitTmemFull)) break;
+      if (!warp_wait(&ctrl->tfull, par, abortf, p.status, kStatusWaitTmemFull, p.wait_ns)) break;
       float scale = 1.f;
       if (NORM == kRMSNorm) {
-        if (!warp_wait(&ctrl->sfull, par, abortf, p.status, kStatusWaitStats)) break;
+        if (!warp_wait(&ctrl->sfull, par, abortf, p.status, kStatusWaitStats, p.wait_ns)) break;
         scale = ctrl->rs[row_local];
       }
       tc_fence_after();
@@ -325,7 +340,7 @@ __global__ void __launch_bounds__(k2w::NUM_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctrl->tempty);
     }
-  } else {
+  } else if (NORM != kNoNorm) {
     // ------------------------------------------------------------ converters
     // Thread ct: 16-byte chunk c (0..3) of the 64-byte row, rows rbase and
     // rbase + 64. 64-byte swizzle: chunk c of row r sits at c ^ ((r >> 1) & 3).
@@ -355,7 +370,7 @@ __global__ void __launch_bounds__(k2w::NUM_THREADS, 1)
       }
       const bool write_res = (NORM == kRMSNorm) && nb == 0;
       for (int kb = 0; kb < nkb; ++kb) {
-        if (!warp_wait(&ctrl->full_x[s], ph, abortf, p.status, kStatusWaitFull)) {
+        if (!warp_wait(&ctrl->full_x[s], ph, abortf, p.status, kStatusWaitFull, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -418,7 +433,7 @@ __global__ void __launch_bounds__(k2w::NUM_THREADS, 1)
         }
         // the epilogue of the previous tile has read rs once tempty completes
         if (!warp_wait(&ctrl->tempty, (static_cast<uint32_t>(i) & 1) ^ 1, abortf, p.status,
-                       kStatusWaitTmemEmpty))
+                       kStatusWaitTmemEmpty, p.wait_ns))
           break;
         if (c == 0) {
 #pragma unroll

@@ -365,6 +365,8 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
       const int npre = P < S ? P : S;
       uint32_t armed_w = 0, armed_x = 0, par_w = 0, par_x = 0;
       bool ok = true;
+      // fault injection (status-path tests only): CTA 0 withholds its first weight copy
+      bool withhold = p.stall != 0 && blockIdx.x == 0;
       const uint64_t pol_w = policy_evict_first();   // W is streamed exactly once
       // two cursors over the unit sequence (tile t, k-block kb, stage s, parity)
       struct Cur {
@@ -385,6 +387,10 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
         }
       };
       auto issue_w = [&](const Cur& c) {
+        if (withhold) {
+          withhold = false;
+          return;
+        }
         uint8_t* st = smem + c.s * SB;
         mbar_arrive_expect_tx(&ctrl->full_w[c.s], W_BYTES);
         if (EPI == kEpiSwiGLU) {
@@ -398,6 +404,13 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
       };
       auto issue_x = [&](const Cur& c) {
         uint8_t* st = smem + c.s * SB;
+        if (NORM == kNoNorm) {   // the activation tile is the operand as loaded
+          mbar_arrive_expect_tx(&ctrl->full_x[c.s], XB);
+          tma_load_2d(st + W_BYTES, &tm_x, &ctrl->full_x[c.s], c.kb * BK, 0);
+          armed_x |= 1u << c.s;
+          par_x = (par_x & ~(1u << c.s)) | (c.ph << c.s);
+          return;
+        }
         mbar_arrive_expect_tx(&ctrl->full_x[c.s], 2 * XB + vec_bytes(p, has_beta, has_bias_in, c.kb));
         issue_vec_loads(p, has_beta, has_bias_in, c.kb, vecs + c.s * 3 * kVecElems, &ctrl->full_x[c.s]);
         tma_load_2d(st + W_BYTES, &tm_x, &ctrl->full_x[c.s], c.kb * BK, 0);
@@ -418,7 +431,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
           issue_w(cw);
           step(cw);
         } else if (q >= npre) {
-          if (!mbar_wait(&ctrl->empty[cw.s], cw.ph ^ 1, abortf, p.status, kStatusWaitEmpty)) {
+          if (!mbar_wait(&ctrl->empty[cw.s], cw.ph ^ 1, abortf, p.status, kStatusWaitEmpty, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -447,12 +460,14 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
       while (ok && it.next(t, kb0, nk, slot, nseg)) {
         const int b = i & 1;
         const uint32_t use = static_cast<uint32_t>(i >> 1);
-        if (!mbar_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty)) break;
+        if (!mbar_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty, p.wait_ns)) break;
         tc_fence_after();
         const uint32_t d = tmem + b * mpad;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(&ctrl->conv[s], ph, abortf, p.status, kStatusWaitConv) ||
-              !mbar_wait(&ctrl->full_w[s], ph, abortf, p.status, kStatusWaitFull)) {
+          // the converted operand (or, without a norm, the activation tile as loaded)
+          uint64_t* ready = NORM == kNoNorm ? &ctrl->full_x[s] : &ctrl->conv[s];
+          if (!mbar_wait(ready, ph, abortf, p.status, kStatusWaitConv, p.wait_ns) ||
+              !mbar_wait(&ctrl->full_w[s], ph, abortf, p.status, kStatusWaitFull, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -519,9 +534,9 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     while (it.next(t, kb0, nk, slot, nseg)) {
       const int b = i & 1;
       const uint32_t use = static_cast<uint32_t>(i >> 1);
-      if (!warp_wait(&ctrl->tfull[b], use & 1, abortf, p.status, kStatusWaitTmemFull)) break;
+      if (!warp_wait(&ctrl->tfull[b], use & 1, abortf, p.status, kStatusWaitTmemFull, p.wait_ns)) break;
       if (NORM == kRMSNorm) {
-        if (!warp_wait(&ctrl->sfull[b], use & 1, abortf, p.status, kStatusWaitStats)) break;
+        if (!warp_wait(&ctrl->sfull[b], use & 1, abortf, p.status, kStatusWaitStats, p.wait_ns)) break;
       }
       tc_fence_after();
       // stream-K form: the partial goes to the tile's workspace slot; cluster
@@ -562,7 +577,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
       // threads that read the slots (L2 loads).
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctrl->esync);
-      if (!warp_wait(&ctrl->esync, eph, abortf, p.status, kStatusWaitDrain)) break;
+      if (!warp_wait(&ctrl->esync, eph, abortf, p.status, kStatusWaitDrain, p.wait_ns)) break;
       eph ^= 1;
       if (et == 0) {
         const unsigned old = atom_add_acq_rel_gpu(&p.counters[t], 1u);
@@ -570,7 +585,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctrl->esync);
-      if (!warp_wait(&ctrl->esync, eph, abortf, p.status, kStatusWaitDrain)) break;
+      if (!warp_wait(&ctrl->esync, eph, abortf, p.status, kStatusWaitDrain, p.wait_ns)) break;
       eph ^= 1;
       if (ctrl->last_flag) {
         if (it.u >= it.u1) {   // the CTA's last segment: handed to all warps below
@@ -585,7 +600,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
         }
       }
     }
-  } else {
+  } else if (NORM != kNoNorm) {
     // ------------------------------------------------------------ converters
     // Converter warp cw owns pipeline positions cw, cw + 4, cw + 8, ... of this
     // CTA's unit sequence, so up to four stages are converted at once. Lanes
@@ -635,7 +650,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
           cph ^= 1u;
         }
         const int kb = kb0 + (q - pos);
-        if (!warp_wait(&ctrl->full_x[s], ph, abortf, p.status, kStatusWaitFull)) {
+        if (!warp_wait(&ctrl->full_x[s], ph, abortf, p.status, kStatusWaitFull, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -689,7 +704,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
         // publish this warp's share once the epilogue has read the segment
         // that used this buffer two segments ago
         const uint32_t use = static_cast<uint32_t>(i >> 1);
-        if (!warp_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty)) break;
+        if (!warp_wait(&ctrl->tempty[b], (use & 1) ^ 1, abortf, p.status, kStatusWaitTmemEmpty, p.wait_ns)) break;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           float lo_, hi_;
@@ -740,7 +755,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
                       &ctrl->rbar);
         }
       }
-      if (warp_wait(&ctrl->rbar, 0, abortf, p.status, kStatusWaitFull)) {
+      if (warp_wait(&ctrl->rbar, 0, abortf, p.status, kStatusWaitFull, p.wait_ns)) {
         k3_reduce_tile_smem<EPI, NORM>(p, t, nseg, reinterpret_cast<const float*>(smem),
                                        reinterpret_cast<const float*>(smem + nseg * slot_bytes));
       } else if (threadIdx.x == 0) {

@@ -1,0 +1,522 @@
+// K4: large-M fused norm + GEMM + epilogue on CTA pairs (tcgen05 cta_group::2).
+//
+// Same dataflow as the 128 x 512 kernel (TMA x / residual / W tiles ->
+// converter warps build the normalised bf16 operand in place in shared memory
+// -> tcgen05.mma into TMEM -> fused epilogue), with the pair tile spread over
+// two CTAs of a cluster: 256 tokens x 512 W rows (SwiGLU: 256 gate rows + the
+// matching 256 up rows). Each CTA holds its 128 tokens' x, residual and
+// normalised operand, and half of each weight operand; the pair's even CTA
+// issues tcgen05.mma.cta_group::2 M=256 N=256 K=16, which reads A from both
+// CTAs' shared memory (128 rows each) and B from both (128 of the 256 W rows
+// each) and writes each CTA's 128 accumulator rows into its own TMEM. Per CTA
+// and 32-wide k-block that is x 8 KB + residual 8 KB + W 16 KB of tensor copies
+// and 32 KB of UMMA operand reads for 512 tensor cycles, against 48 KB and
+// 48 KB in the single-CTA 128 x 512 kernel: shared-memory bytes per FLOP, the
+// bound of the fused operand's pipeline, drop by about a quarter.
+//
+// Warp roles (14 warps per CTA): 0 TMA producer (own tiles only), 1 TMEM
+// (allocated for the pair) and, in the even CTA, UMMA issuer; 2-5 epilogue
+// (own 128 rows); 6-13 converters. A stage is ready for the UMMA when both
+// CTAs' converters have built their operand and seen their own weight half
+// land: every converter warp of both CTAs arrives on the even CTA's conv[s]
+// after waiting for its CTA's full_x[s] and full_w[s], so no tensor copy ever
+// signals the other CTA and each CTA drains only its own copies. The UMMA
+// commits arrive on both CTAs' empty[s] / tfull (multicast commit); the
+// epilogue warps of both CTAs arrive on the even CTA's tempty. RMSNorm uses the
+// deferred scale of the other kernels (each CTA's converters sum h^2 of its
+// rows for its own epilogue); LayerNorm statistics come from the statistics
+// kernel. A wait that gives up raises the abort flag of both CTAs; both CTAs
+// meet at a cluster barrier after their role loops (and after the last UMMA
+// completed), so neither leaves while the other may still touch its shared
+// memory.
+#pragma once
+
+#include "common.cuh"
+
+namespace fnl {
+namespace k4 {
+
+constexpr int BM = 128;            // tokens per CTA (256 per pair)
+constexpr int BN = 512;            // W rows per pair tile (all in each CTA's TMEM)
+constexpr int BK = 32;             // k-block: 64-byte rows, 64-byte swizzle
+constexpr int STAGES = 6;
+constexpr int X_BYTES = BM * BK * 2;              // 8 KB
+constexpr int WH_BYTES = 128 * BK * 2;            // 8 KB: one 128-row half of an N=256 operand
+constexpr int STAGE_BYTES = 2 * X_BYTES + 2 * WH_BYTES;   // 32 KB: x, residual, W half 0, W half 1
+constexpr int VEC = BK;
+constexpr int VEC_STAGE_BYTES = 3 * VEC * 2;
+constexpr int VEC_BYTES = STAGES * VEC_STAGE_BYTES;
+constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_EPI0 = 2, NUM_EPI_WARPS = 4;
+constexpr int WARP_CONV0 = 6, NUM_CONV_WARPS = 8;
+constexpr int NUM_THREADS = (WARP_CONV0 + NUM_CONV_WARPS) * 32;   // 448
+constexpr int TMEM_COLS = 512;
+constexpr int GROUP_M = 8;         // pair rows (of 256 tokens) sharing a W tile while it is hot in L2
+
+struct Ctrl {
+  uint64_t full_w[STAGES], full_x[STAGES], conv[STAGES], empty[STAGES];
+  uint64_t tfull, tempty, sfull[2], efree[2], drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  float rs[2][BM];
+};
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + VEC_BYTES + static_cast<int>(sizeof(Ctrl)) + 1024;
+
+__device__ __forceinline__ void tile_coords(int t, int num_m2, int num_n, int& mb2, int& nb) {
+  const int per_group = GROUP_M * num_n;
+  const int group = t / per_group;
+  const int first_m = group * GROUP_M;
+  const int gm = min(GROUP_M, num_m2 - first_m);
+  const int r = t - group * per_group;
+  mb2 = first_m + r % gm;
+  nb = r / gm;
+}
+
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > FNL_WAIT_NS) return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(1) << 16;
+  d |= static_cast<uint64_t>(512 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(4) << 61;   // SWIZZLE_64B
+  return d;
+}
+
+}  // namespace k4
+
+template <int EPI, int NORM, bool SPLIT>
+__global__ void __launch_bounds__(k4::NUM_THREADS, 1)
+    k4_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_r,
+                   const __grid_constant__ CUtensorMap tm_w, const OpParams p) {
+  using namespace k4;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  bf16* vecs = reinterpret_cast<bf16*>(smem + STAGES * STAGE_BYTES);   // [STAGES][3][32]
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + STAGES * STAGE_BYTES + VEC_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();       // 0: the pair's UMMA issuer
+  const uint32_t peer = rank ^ 1u;
+  const bool leader = rank == 0;
+  const bool has_beta = NORM == kLayerNorm && p.beta != nullptr;
+  const bool has_bias_in = EPI == kEpiGELU && p.bias_in != nullptr;
+  constexpr bool BIAS_IN = EPI == kEpiGELU;
+
+  const int M = p.M, K = p.K;
+  const int num_m2 = (M + 2 * BM - 1) / (2 * BM);
+  const int num_n = (EPI == kEpiSwiGLU) ? (p.I + 255) / 256 : (p.N + BN - 1) / BN;
+  const int tiles = num_m2 * num_n;
+  const int nkb = (K + BK - 1) / BK;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    pdl_launch_dependents();
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&ctrl->full_w[s], 1);
+      mbar_init(&ctrl->full_x[s], 1);
+      mbar_init(&ctrl->conv[s], 2 * NUM_CONV_WARPS);   // (even CTA) converter warps of both CTAs
+      mbar_init(&ctrl->empty[s], 1);                   // multicast UMMA commit
+    }
+    mbar_init(&ctrl->tfull, 1);
+    mbar_init(&ctrl->tempty, 2 * NUM_EPI_WARPS);       // (even CTA) epilogue warps of both CTAs
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctrl->sfull[b], NUM_CONV_WARPS);
+      mbar_init(&ctrl->efree[b], NUM_EPI_WARPS);
+    }
+    mbar_init(&ctrl->drain, 1);
+    ctrl->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == WARP_TMA && lane == 0) {
+    prefetch_tmap(&tm_x);
+    prefetch_tmap(&tm_r);
+    prefetch_tmap(&tm_w);
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc_pair(&ctrl->tmem_base, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  zero_vec_slices(vecs, STAGES * 3 * VEC);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();   // both CTAs' barriers are initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+  volatile int* abortf = &ctrl->abort_flag;
+  // a wait that gave up (or saw the flag) also stops the other CTA of the pair
+  auto abort_pair = [&]() { st_remote_u32(&ctrl->abort_flag, peer, 1u); };
+
+  if (warp == WARP_TMA) {
+    // ------------------------------------------------------------ producer (own tiles)
+    if (lane == 0) {
+      const int my_tiles = pair < tiles ? (tiles - 1 - pair) / npairs + 1 : 0;
+      const int P = my_tiles * nkb;
+      const int npre = P < STAGES ? P : STAGES;
+      uint32_t armed_w = 0, armed_x = 0, par_w = 0, par_x = 0;
+      bool ok = true;
+      bool withhold = p.stall != 0 && blockIdx.x == 0;   // fault injection (status-path tests only)
+      struct Cur {
+        int t, mb2, nb, kb, s;
+        uint32_t ph;
+      };
+      Cur cw{pair, 0, 0, 0, 0, 0u};
+      if (P > 0) tile_coords(cw.t, num_m2, num_n, cw.mb2, cw.nb);
+      Cur cx = cw;
+      auto step = [&](Cur& c) {
+        if (++c.kb == nkb) {
+          c.kb = 0;
+          c.t += npairs;
+          if (c.t < tiles) tile_coords(c.t, num_m2, num_n, c.mb2, c.nb);
+        }
+        if (++c.s == STAGES) {
+          c.s = 0;
+          c.ph ^= 1u;
+        }
+      };
+      auto issue_w = [&](const Cur& c) {
+        if (withhold) {
+          withhold = false;
+          return;
+        }
+        uint8_t* st = smem + c.s * STAGE_BYTES + 2 * X_BYTES;
+        mbar_arrive_expect_tx(&ctrl->full_w[c.s], 2 * WH_BYTES);
+        // this CTA's 128-row halves of the two N=256 operands
+        int r0, r1;
+        if (EPI == kEpiSwiGLU) {
+          r0 = c.nb * 256 + static_cast<int>(rank) * 128;          // gate rows
+          r1 = p.I + c.nb * 256 + static_cast<int>(rank) * 128;    // the matching up rows
+        } else {
+          r0 = c.nb * BN + static_cast<int>(rank) * 128;
+          r1 = c.nb * BN + 256 + static_cast<int>(rank) * 128;
+        }
+        tma_load_2d(st, &tm_w, &ctrl->full_w[c.s], c.kb * BK, r0);
+        tma_load_2d(st + WH_BYTES, &tm_w, &ctrl->full_w[c.s], c.kb * BK, r1);
+        armed_w |= 1u << c.s;
+        par_w = (par_w & ~(1u << c.s)) | (c.ph << c.s);
+      };
+      auto issue_x = [&](const Cur& c) {
+        uint8_t* st = smem + c.s * STAGE_BYTES;
+        const int k0 = c.kb * BK;
+        const int row0 = c.mb2 * 2 * BM + static_cast<int>(rank) * BM;
+        if (NORM == kNoNorm) {
+          mbar_arrive_expect_tx(&ctrl->full_x[c.s], X_BYTES);
+          tma_load_2d(st, &tm_x, &ctrl->full_x[c.s], k0, row0);
+        } else {
+          bf16* vec = vecs + c.s * 3 * VEC;
+          const uint32_t vb = static_cast<uint32_t>(min(VEC, K - k0)) * 2;
+          const uint32_t nvec = 1 + (has_beta ? 1 : 0) + (has_bias_in ? 1 : 0);
+          mbar_arrive_expect_tx(&ctrl->full_x[c.s], 2 * X_BYTES + vb * nvec);
+          bulk_load(vec, p.gamma + k0, vb, &ctrl->full_x[c.s]);
+          if (has_beta) bulk_load(vec + VEC, p.beta + k0, vb, &ctrl->full_x[c.s]);
+          if (has_bias_in) bulk_load(vec + 2 * VEC, p.bias_in + k0, vb, &ctrl->full_x[c.s]);
+          tma_load_2d(st, &tm_x, &ctrl->full_x[c.s], k0, row0);
+          tma_load_2d(st + X_BYTES, &tm_r, &ctrl->full_x[c.s], k0, row0);
+        }
+        armed_x |= 1u << c.s;
+        par_x = (par_x & ~(1u << c.s)) | (c.ph << c.s);
+      };
+      for (int q = 0; q < npre; ++q) {   // weights stream before the dependency wait
+        issue_w(cw);
+        step(cw);
+      }
+      pdl_wait();
+      for (int q = 0; q < P; ++q) {
+        if (q >= npre) {
+          if (!mbar_wait(&ctrl->empty[cw.s], cw.ph ^ 1, abortf, p.status, kStatusWaitEmpty, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          issue_w(cw);
+          step(cw);
+        }
+        issue_x(cx);
+        step(cx);
+      }
+      if (!ok) {
+        abort_pair();
+        for (int i = 0; i < STAGES; ++i) {   // let every issued copy land before the CTA can exit
+          if (armed_w & (1u << i)) drain_wait(&ctrl->full_w[i], (par_w >> i) & 1);
+          if (armed_x & (1u << i)) drain_wait(&ctrl->full_x[i], (par_x >> i) & 1);
+        }
+      }
+    }
+  } else if (warp == WARP_MMA) {
+    // ------------------------------------------------------------ UMMA issuer (even CTA)
+    if (leader && lane == 0) {
+      uint32_t s = 0, ph = 0;
+      bool ok = true;
+      const uint32_t idesc = idesc_bf16(2 * BM, 256);
+      int i = 0;
+      for (int t = pair; t < tiles && ok; t += npairs, ++i) {
+        if (!mbar_wait_cluster(&ctrl->tempty, (static_cast<uint32_t>(i) & 1) ^ 1, abortf, p.status,
+                               kStatusWaitTmemEmpty, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_cluster(&ctrl->conv[s], ph, abortf, p.status, kStatusWaitConv, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t xa = smem_u32(smem + s * STAGE_BYTES);
+          const uint64_t ad = k4::sw64_desc(xa);
+          const uint64_t ld = k4::sw64_desc(xa + X_BYTES);
+          const uint64_t bd0 = k4::sw64_desc(xa + 2 * X_BYTES);
+          const uint64_t bd1 = k4::sw64_desc(xa + 2 * X_BYTES + WH_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            umma_bf16_pair(tmem, ad + 2 * kk, bd0 + 2 * kk, idesc, acc);
+            umma_bf16_pair(tmem + 256, ad + 2 * kk, bd1 + 2 * kk, idesc, acc);
+            if (SPLIT) {   // + lo(a) W^T into the same accumulators
+              umma_bf16_pair(tmem, ld + 2 * kk, bd0 + 2 * kk, idesc, 1u);
+              umma_bf16_pair(tmem + 256, ld + 2 * kk, bd1 + 2 * kk, idesc, 1u);
+            }
+          }
+          umma_commit_pair(&ctrl->empty[s], 0x3);   // the stage is free in both CTAs
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(&ctrl->tfull, 0x3);
+      }
+      if (!ok) abort_pair();
+      umma_commit_pair(&ctrl->drain, 0x1);   // every issued UMMA done before the pair's exit
+      drain_wait(&ctrl->drain, 0);
+    }
+  } else if (warp < WARP_CONV0) {
+    // ------------------------------------------------------------ epilogue (own 128 rows)
+    const int q = warp & 3;
+    const int row_local = q * 32 + lane;
+    pdl_wait();
+    int i = 0;
+    for (int t = pair; t < tiles; t += npairs, ++i) {
+      const uint32_t par = static_cast<uint32_t>(i) & 1;
+      if (!warp_wait(&ctrl->tfull, par, abortf, p.status, kStatusWaitTmemFull, p.wait_ns)) {
+        if (lane == 0) abort_pair();
+        break;
+      }
+      float scale = 1.f;
+      if (NORM == kRMSNorm) {
+        const int b = i & 1;
+        if (!warp_wait(&ctrl->sfull[b], static_cast<uint32_t>(i >> 1) & 1, abortf, p.status, kStatusWaitStats,
+                       p.wait_ns)) {
+          if (lane == 0) abort_pair();
+          break;
+        }
+        scale = ctrl->rs[b][row_local];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->efree[b]);   // the converters may refill rs[b]
+      }
+      tc_fence_after();
+      int mb2, nb;
+      tile_coords(t, num_m2, num_n, mb2, nb);
+      const int m = mb2 * 2 * BM + static_cast<int>(rank) * BM + row_local;
+      const bool row_ok = m < M;
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      if (EPI == kEpiSwiGLU) {
+#pragma unroll 1
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t g0[16], g1[16], u0[16], u1[16];
+          tmem_ld16(tbase + cc * 32, g0);
+          tmem_ld16(tbase + cc * 32 + 16, g1);
+          tmem_ld16(tbase + 256 + cc * 32, u0);
+          tmem_ld16(tbase + 256 + cc * 32 + 16, u1);
+          tmem_ld_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) {
+              const int j = nb * 256 + cc * 32 + g8 * 8;
+              if (j < p.I) {
+                float gv[8], uv[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const int c = g8 * 8 + e;
+                  gv[e] = __uint_as_float(c < 16 ? g0[c] : g1[c - 16]);
+                  uv[e] = __uint_as_float(c < 16 ? u0[c] : u1[c - 16]);
+                }
+                store_swiglu8(p, m, j, gv, uv, scale);
+              }
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 32; ++cc) {
+          uint32_t a0[16], a1[16];
+          tmem_ld16(tbase + cc * 32, a0);
+          tmem_ld16(tbase + cc * 32 + 16, a1);
+          tmem_ld_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int g8 = 0; g8 < 4; ++g8) {
+              const int n = nb * BN + cc * 32 + g8 * 8;
+              if (n < p.N) {
+                float av[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  const int c = g8 * 8 + e;
+                  av[e] = __uint_as_float(c < 16 ? a0[c] : a1[c - 16]);
+                }
+                store_out8<EPI>(p, m, n, av, scale);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {   // the pair's accumulator may be overwritten once both CTAs read it
+        if (leader) mbar_arrive(&ctrl->tempty);
+        else mbar_arrive_remote(&ctrl->tempty, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ converters (own 128 rows)
+    // Thread ct: 16-byte chunk c (0..3) of the 64-byte row, rows rbase and
+    // rbase + 64. 64-byte swizzle: chunk c of row r sits at c ^ ((r >> 1) & 3).
+    // Without a norm (residual-stream projection) the warps only relay the
+    // stage's readiness to the even CTA.
+    const int ct = threadIdx.x - WARP_CONV0 * 32;   // 0..255
+    const int c = ct & 3;
+    const int rbase = ct >> 2;                       // 0..63
+    if (NORM == kLayerNorm) pdl_wait();
+    uint32_t s = 0, ph = 0;
+    int i = 0;
+    bool ok = true;
+    for (int t = pair; t < tiles && ok; t += npairs, ++i) {
+      int mb2, nb;
+      tile_coords(t, num_m2, num_n, mb2, nb);
+      const int mrow0 = mb2 * 2 * BM + static_cast<int>(rank) * BM;
+      float mu[2], rs[2];
+      f32x2 ss[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int gm = mrow0 + rbase + 64 * j;
+        ss[j] = 0ull;
+        mu[j] = 0.f;
+        rs[j] = 0.f;
+        if (NORM == kLayerNorm && gm < M) {
+          const float2 st = p.stats[gm];
+          mu[j] = st.x;
+          rs[j] = st.y;
+        }
+      }
+      const bool write_res = (NORM == kRMSNorm) && nb == 0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!warp_wait(&ctrl->full_x[s], ph, abortf, p.status, kStatusWaitFull, p.wait_ns) ||
+            !warp_wait(&ctrl->full_w[s], ph, abortf, p.status, kStatusWaitFull, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        if (NORM != kNoNorm) {
+          bf16* vec = vecs + s * 3 * VEC;
+          if (K - kb * BK < BK) zero_vec_tails(vec, VEC, K - kb * BK);
+          const uint32_t vaddr = smem_u32(vec) + c * 16;
+          f32x2 g2[4], be2[4] = {}, bi2[4] = {};
+          vec_pairs(vaddr, g2);
+          if (NORM == kLayerNorm) vec_pairs(vaddr + 2 * VEC, be2);
+          if (BIAS_IN) vec_pairs(vaddr + 4 * VEC, bi2);
+          const uint32_t xs = smem_u32(smem + s * STAGE_BYTES);
+          const uint32_t rsm = xs + X_BYTES;
+          uint4 xv[2], rv[2];
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int row = rbase + 64 * j;
+            const uint32_t off = row * 64 + ((c ^ ((row >> 1) & 3)) << 4);
+            xv[j] = ld_shared_v4(xs + off);
+            rv[j] = ld_shared_v4(rsm + off);
+          }
+          // instantiated with and without the residual_out store (first N column)
+          auto convert_stage = [&](auto wres_tag) {
+            constexpr bool WRES = decltype(wres_tag)::value;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int row = rbase + 64 * j;
+              const uint32_t off = row * 64 + ((c ^ ((row >> 1) & 3)) << 4);
+              uint4 hi, lo, hres;
+              convert8<(NORM == kNoNorm ? kRMSNorm : NORM), BIAS_IN, SPLIT, WRES>(
+                  xv[j], rv[j], g2, be2, bi2, mu[j], rs[j], ss[j], hi, lo, hres);
+              st_shared_v4(xs + off, hi);
+              if (SPLIT) st_shared_v4(rsm + off, lo);
+              if (WRES) {
+                const int gm = mrow0 + row;
+                const int k0 = kb * BK + c * 8;
+                if (gm < M && k0 < K)
+                  *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(gm) * K + k0) = hres;
+              }
+            }
+          };
+          if (write_res) convert_stage(BoolC<true>{});
+          else convert_stage(BoolC<false>{});
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) {   // this CTA's half of stage s is ready for the pair's UMMA
+          if (leader) mbar_arrive(&ctrl->conv[s]);
+          else mbar_arrive_remote(&ctrl->conv[s], 0);
+        }
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1;
+        }
+      }
+      if (!ok) {
+        if (lane == 0) abort_pair();
+        break;
+      }
+      if (NORM == kRMSNorm) {
+        float sst[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          float lo_, hi_;
+          unpk2(ss[j], lo_, hi_);
+          sst[j] = lo_ + hi_;
+          sst[j] += __shfl_xor_sync(0xffffffffu, sst[j], 1);
+          sst[j] += __shfl_xor_sync(0xffffffffu, sst[j], 2);
+        }
+        const int b = i & 1;
+        // the epilogue of the tile two back has read rs[b]
+        if (!warp_wait(&ctrl->efree[b], (static_cast<uint32_t>(i >> 1) & 1) ^ 1, abortf, p.status,
+                       kStatusWaitTmemEmpty, p.wait_ns)) {
+          if (lane == 0) abort_pair();
+          break;
+        }
+        if (c == 0) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int row = rbase + 64 * j;
+            const float r = 1.f / sqrtf(sst[j] / static_cast<float>(K) + p.eps);
+            ctrl->rs[b][row] = r;
+            const int gm = mrow0 + row;
+            if (write_res && p.rstd_out != nullptr && gm < M) p.rstd_out[gm] = r;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->sfull[b]);
+      }
+    }
+  }
+
+  // Every role's loop is over and the even CTA's last UMMA has completed (its
+  // issuer waited for it): meet the other CTA, then free the pair's TMEM.
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace fnl

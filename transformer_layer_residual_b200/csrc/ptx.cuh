@@ -1,9 +1,11 @@
 // Thin inline-PTX wrappers for sm_100a: mbarriers, TMA tile loads, tcgen05
 // (TMEM allocation, UMMA issue/commit, TMEM loads), proxy fences, programmatic
-// dependent launch. Every spin on an mbarrier is bounded: after FNL_WAIT_NS of
-// wall time the waiter records an error code in a device status word, raises a
-// CTA-wide abort flag and returns false, so no kernel in this library can hang
-// a GPU on a wait.
+// dependent launch. Every spin on an mbarrier is bounded: after a limit of
+// wall time (FNL_WAIT_NS by default, a per-call value for the main-loop waits)
+// the waiter records an error code in a device status word, raises a CTA-wide
+// abort flag and returns false, so no kernel in this library can hang a GPU on
+// a wait. Waits for a CTA's own copies to land before it exits keep the long
+// default limit.
 #pragma once
 
 #include <cuda.h>
@@ -69,10 +71,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity. Returns false (and raises
-// the CTA abort flag, recording `code` in *status) when the wait gives up or
-// another role of the CTA already aborted.
+// the CTA abort flag, recording `code` in *status) when the wait gives up after
+// limit_ns nanoseconds or another role of the CTA already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status, int code) {
+                                          int* status, int code, uint64_t limit_ns = FNL_WAIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
@@ -80,7 +82,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer() - t0 > FNL_WAIT_NS) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort_flag = 1;
       if (status) atomicCAS(status, 0, code);
       return false;
@@ -94,7 +96,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // could stay split into two groups that the scheduler runs one after the other,
 // which doubles the cost of all the warp-wide work that follows the wait.)
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status, int code) {
+                                          int* status, int code, uint64_t limit_ns = FNL_WAIT_NS) {
   constexpr unsigned kAll = 0xffffffffu;
   if (__any_sync(kAll, mbar_try_wait(bar, parity))) return true;
   const uint64_t t0 = globaltimer();
@@ -103,7 +105,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
     for (int i = 0; i < 32; ++i)
       if (__any_sync(kAll, mbar_try_wait(bar, parity))) return true;
     if (__any_sync(kAll, *abort_flag != 0)) return false;
-    if (__any_sync(kAll, globaltimer() - t0 > FNL_WAIT_NS)) {
+    if (__any_sync(kAll, globaltimer() - t0 > limit_ns)) {
       if ((threadIdx.x & 31) == 0) {
         *abort_flag = 1;
         if (status) atomicCAS(status, 0, code);
@@ -273,6 +275,96 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
          | (1u << 10)                               // B format: bf16
          | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
+}
+
+// ---------------------------------------------------------------- CTA pairs (cta_group::2)
+// Rank of this CTA in its cluster.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Test of a phase whose arrivals may come from the other CTA of the pair
+// (acquire at cluster scope, so the arriving CTA's prior writes are visible).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(1000u)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  int* status, int code, uint64_t limit_ns) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > limit_ns) {
+      *abort_flag = 1;
+      if (status) atomicCAS(status, 0, code);
+      return false;
+    }
+  }
+}
+// Arrive on the mbarrier at the same shared-memory offset in CTA `rank` of the
+// cluster, releasing this thread's prior writes at cluster scope.
+__device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t rank) {
+  asm volatile(
+      "{\n\t.reg .b32 ra;\n\t"
+      "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_u32(bar)),
+      "r"(rank)
+      : "memory");
+}
+// Store a 32-bit value at the same shared-memory offset in CTA `rank`.
+__device__ __forceinline__ void st_remote_u32(void* p, uint32_t rank, uint32_t v) {
+  asm volatile(
+      "{\n\t.reg .b32 ra;\n\t"
+      "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+      "st.shared::cluster.u32 [ra], %2;\n\t}" ::"r"(smem_u32(p)),
+      "r"(rank), "r"(v)
+      : "memory");
+}
+// TMEM allocation shared by the two CTAs of a pair: one warp of each CTA (the
+// same warp index) executes these together.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D[tmem of both CTAs] (+)= A[256 rows: 128 from each CTA's smem] *
+// B[N cols: N/2 from each CTA's smem]^T, bf16 in, fp32 accumulate; issued by
+// one thread of the pair's even CTA.
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the mbarrier at this offset in every CTA of `mask` when every
+// UMMA issued so far by this thread is done.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
 }
 
 // ---------------------------------------------------------------- misc

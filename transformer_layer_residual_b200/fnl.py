@@ -21,11 +21,12 @@ FNL_OK = 0
 STATUS_NAMES = {0: "FNL_OK", 1: "FNL_ERR_INVALID_ARG", 2: "FNL_ERR_ALIGNMENT", 3: "FNL_ERR_ALIAS",
                 4: "FNL_ERR_UNSUPPORTED", 5: "FNL_ERR_CUDA", 6: "FNL_ERR_DEVICE_STATUS"}
 NORMS = {"layernorm": 0, "rmsnorm": 1}
-PATHS = {"auto": 0, "tile": 1, "splitk": 2, "wide": 3, "cluster": 4}
+PATHS = {"auto": 0, "tile": 1, "splitk": 2, "wide": 3, "cluster": 4, "pair": 5}
 PRECISIONS = {"default": 0, "split": 1, "single": 2}
 
-EXPORTED = ("fnl_create", "fnl_destroy", "fnl_status_string", "fnl_last_error", "fnl_check",
-            "fnl_add_norm_qkv", "fnl_add_norm_swiglu", "fnl_add_bias_norm_gelu", "fnl_add_norm_qkv_static")
+EXPORTED = ("fnl_create", "fnl_destroy", "fnl_status_string", "fnl_last_error", "fnl_last_plan", "fnl_check",
+            "fnl_add_norm_qkv", "fnl_add_norm_swiglu", "fnl_add_bias_norm_gelu", "fnl_linear_add_residual",
+            "fnl_add_norm_qkv_static", "fnl_check_static")
 
 
 class FnlError(RuntimeError):
@@ -36,7 +37,8 @@ class FnlError(RuntimeError):
 
 class _Options(ctypes.Structure):
     _fields_ = [("max_tokens", ctypes.c_int), ("max_n", ctypes.c_int), ("path", ctypes.c_int),
-                ("max_ctas", ctypes.c_int), ("precision", ctypes.c_int)]
+                ("max_ctas", ctypes.c_int), ("precision", ctypes.c_int), ("wait_ns", ctypes.c_longlong),
+                ("debug_stall_calls", ctypes.c_int), ("tune", ctypes.c_int)]
 
 
 def lib_path() -> str:
@@ -59,13 +61,17 @@ def lib() -> ctypes.CDLL:
     L.fnl_status_string.restype = ctypes.c_char_p
     L.fnl_last_error.argtypes = [P]
     L.fnl_last_error.restype = ctypes.c_char_p
+    L.fnl_last_plan.argtypes = [P]
+    L.fnl_last_plan.restype = ctypes.c_char_p
     L.fnl_check.argtypes = [P, P]
     L.fnl_add_norm_qkv.argtypes = [P, P, P, P, P, P, P, I, F, P, P, I, I, I, I, I, P, P, P, P, P]
     L.fnl_add_norm_swiglu.argtypes = [P, P, P, P, P, P, P, I, F, P, P, I, I, I, P, P, P]
     L.fnl_add_bias_norm_gelu.argtypes = [P, P, P, P, P, P, P, P, I, F, P, P, I, I, I, P, P, P]
+    L.fnl_linear_add_residual.argtypes = [P, P, P, P, P, P, P, I, I, I]
     L.fnl_add_norm_qkv_static.argtypes = [P, P, P, P, P, P, I, F, P, P, I, I, I, I, I, P, P, P, P, P]
+    L.fnl_check_static.argtypes = [P]
     for name in EXPORTED:
-        if getattr(L, name).restype is None and name not in ("fnl_status_string", "fnl_last_error"):
+        if getattr(L, name).restype is None and name not in ("fnl_status_string", "fnl_last_error", "fnl_last_plan"):
             getattr(L, name).restype = I
     _lib = L
     return L
@@ -78,14 +84,20 @@ class Handle:
     no stream synchronisation, on later calls up to that size). path forces a
     kernel: "auto" (by M), "splitk" (small-M kernel, stream-K form), "cluster"
     (small-M kernel, cluster form), "tile" (128x256 tiles), "wide" (128x512
-    tiles). max_ctas caps the grid (0 = all SMs). precision: "default" (split
-    hi + lo operand for SwiGLU only), "split", "single"."""
+    tiles), "pair" (256x512 tiles on CTA pairs). max_ctas caps the grid (0 = all SMs). precision: "default" (split
+    hi + lo operand for SwiGLU only), "split", "single". wait_ns: limit of the
+    kernels' main-loop waits (0 = 4 s). debug_stall_calls: fault injection for
+    tests of the status path (the next that-many calls withhold one weight copy,
+    so a wait runs out and check() raises). tune: shape auto-tuning (the first
+    call of each shape times the candidate plans and keeps the fastest)."""
 
     def __init__(self, device: int = 0, max_tokens: int = 0, max_n: int = 0, path: str = "auto",
-                 max_ctas: int = 0, precision: str = "default"):
+                 max_ctas: int = 0, precision: str = "default", wait_ns: int = 0, debug_stall_calls: int = 0,
+                 tune: bool = False):
         L = lib()
         self._h = ctypes.c_void_p()
-        opt = _Options(max_tokens, max_n, PATHS[path], max_ctas, PRECISIONS[precision])
+        opt = _Options(max_tokens, max_n, PATHS[path], max_ctas, PRECISIONS[precision], wait_ns,
+                       debug_stall_calls, int(bool(tune)))
         st = L.fnl_create(ctypes.byref(self._h), device, ctypes.byref(opt))
         if st != FNL_OK:
             raise FnlError(st, f"fnl_create(device={device}) failed")
@@ -109,6 +121,11 @@ class Handle:
     def _raise(self, st: int, what: str):
         msg = lib().fnl_last_error(self._h)
         raise FnlError(st, f"{what}: {msg.decode() if msg else ''}")
+
+    def last_plan(self) -> str:
+        """fnl_last_plan: the kernel, form and grid of the last call."""
+        t = lib().fnl_last_plan(self._h)
+        return t.decode() if t else ""
 
     def check(self, stream: Optional[torch.cuda.Stream] = None):
         """Synchronise the stream and raise if a kernel gave up a bounded wait."""
@@ -211,9 +228,32 @@ def add_bias_norm_gelu(h: Handle, x, residual, gamma, beta, W, bias_in=None, bia
     return {"residual_out": residual_out, "out": out, "mean": mean_out, "rstd": rstd_out}
 
 
+def linear_add_residual(h: Handle, a, W, residual, bias=None, out=None, stream=None):
+    """fnl_linear_add_residual: out = residual + a W^T (+ bias), bf16. a [M, K],
+    W [N, K], residual [M, N]; out may be `residual` itself (in-place update of
+    the residual stream). Returns dict(out)."""
+    M, K = a.shape
+    _need(a, "a", (M, K))
+    _need(W, "W")
+    if W.dim() != 2 or W.shape[1] != K:
+        raise ValueError("W must be [N, K]")
+    N = W.shape[0]
+    _need(bias, "bias", (N,))
+    _need(residual, "residual", (M, N))
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=a.device) if out is None else out
+    _need(out, "out", (M, N))
+    st = lib().fnl_linear_add_residual(h.ptr, _stream_ptr(stream), _p(a), _p(W), _p(bias), _p(residual), _p(out),
+                                       M, K, N)
+    if st != FNL_OK:
+        h._raise(st, "fnl_linear_add_residual")
+    return {"out": out}
+
+
 def run_workload(h: Handle, w, dev: dict, stats: bool = True, stream=None) -> dict:
     """Run a synthetic.Workload on device tensors `dev` (same keys as
     synthetic.make_inputs). Allocates the outputs and statistics buffers."""
+    if w.op == "residual":
+        return linear_add_residual(h, dev["x"], dev["W"], dev["residual"], bias=dev.get("bias_out"), stream=stream)
     M = dev["x"].shape[0]
     rstd = torch.empty(M, dtype=torch.float32, device=dev["x"].device) if stats else None
     mean = (torch.empty(M, dtype=torch.float32, device=dev["x"].device)
@@ -248,3 +288,11 @@ def add_norm_qkv_static(x, residual, gamma, beta, W, Hq, Hkv, D, norm="rmsnorm",
     if st != FNL_OK:
         raise FnlError(st, "fnl_add_norm_qkv_static")
     return {"residual_out": residual_out, "q": q, "k": k, "v": v, "mean": mean_out, "rstd": rstd_out}
+
+
+def check_static(stream=None):
+    """fnl_check_static: synchronise the stream and raise if a call of the
+    allocation-free entry point gave up a bounded wait since the last check."""
+    st = lib().fnl_check_static(_stream_ptr(stream))
+    if st != FNL_OK:
+        raise FnlError(st, "fnl_check_static")
