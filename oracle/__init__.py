@@ -25,6 +25,8 @@ What is computed, and where the pages say so:
   on kernel fusion beyond the standard patterns.
 * QKV projection + reshape + GQA grouping: TensorRT-LLM 深度工程实践, §2.2 图构建与
   算子映射; GQA/MQA head counts come from the model config (§2.1).
+* FP8 W8A8 quantisation of the fused op: TensorRT-LLM 深度工程实践, §3.3 FP4/FP8
+  动态量化加速 (W8A8_FP8, dynamic activation ranges, no calibration for FP8).
 * Residual-stream projection: the attention output projection and the MLP's
   down projection are the row-split GEMMs of TensorRT-LLM 深度工程实践, §4.1
   Tensor Parallelism; the residual connection they feed is the residual add
@@ -43,6 +45,14 @@ Readings taken where the pages are silent:
      head-major Q[h, m, d] = y[m, h*D + d]. SwiGLU's W stacks gate rows [0, I)
      over up rows [I, 2I).
   R8 residual_out is h rounded once to bf16, round-to-nearest-even.
+  R11 FP8 W8A8 (the pages name the W8A8_FP8 scheme and say its activation
+     ranges adapt online from runtime statistics, no calibration; they give
+     no granularity): e4m3 codes (round to nearest, ties to even, saturating at
+     +-448); weights get one static scale per output channel, s_w[n] =
+     max_k |W[n, k]| / 448; activations one dynamic scale per token, taken on
+     the normalised row, s_a[m] = max_k |a[m, k]| / 448; y = s_a s_w sum of
+     code products. Every decision that picks a code is taken in fp32, the
+     kernel's precision; the rest is fp64.
   R9 the residual-stream projection adds the residual after the projection and
      its bias: out = residual + a W^T + bias, with residual [M, N] (N = the
      hidden size the projection returns to); the stored result is out rounded
@@ -67,5 +77,11 @@ from .core import (  # noqa: F401
     add_norm_swiglu,
     add_bias_norm_gelu,
     linear_add_residual,
+    E4M3_MAX,
+    e4m3_round,
+    fp8_row_scale_and_codes,
+    quantize_weight_fp8,
+    fp8_linear,
+    add_norm_qkv_fp8,
     run,
 )

@@ -150,6 +150,67 @@ def linear_add_residual(a, W, bias, residual) -> dict:
     return {"out": _f64(residual) + projection(a, W, bias)}
 
 
+# ---------------------------------------------------------------- FP8 (W8A8)
+E4M3_MAX = 448.0   # largest finite value of the e4m3 format (1 sign, 4 exponent bits with bias 7, 3 mantissa bits)
+
+
+def e4m3_round(v) -> np.ndarray:
+    """Round to the nearest e4m3 value, ties to even, saturating at +-448
+    (reading R11). Normal binades [2^e, 2^(e+1)) for e >= -6 have 8 steps of
+    2^(e-3); below 2^-6 the subnormal step is 2^-9."""
+    v = _f64(v)
+    a = np.abs(v)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -6.0)                       # subnormals share the 2^-9 step of e = -6
+    quantum = np.ldexp(1.0, (e - 3).astype(np.int64))
+    q = np.rint(a / quantum) * quantum            # np.rint: halves to even
+    q = np.minimum(q, E4M3_MAX)
+    return np.where(a > 0, np.sign(v) * q, 0.0)
+
+
+def _f32(a) -> np.ndarray:
+    return np.asarray(a, dtype=np.float32)
+
+
+def fp8_row_scale_and_codes(v32):
+    """Per-row symmetric e4m3 quantisation, every decision in fp32 (reading
+    R11): amax = max |v| of the row, s = amax / 448 (1 for an all-zero row),
+    code = e4m3(v / s). Returns (codes as fp64 values, s as fp32)."""
+    v32 = _f32(v32)
+    amax = np.max(np.abs(v32), axis=1)
+    s = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    q = e4m3_round((v32 / s[:, None]).astype(np.float32))
+    return q, s
+
+
+def quantize_weight_fp8(W):
+    """Static per-output-channel FP8 weights: row n of W [N, K] (bf16 values)
+    gets scale s_w[n] = max_k |W[n, k]| / 448 and codes e4m3(W / s_w[n])."""
+    return fp8_row_scale_and_codes(_f64(W).astype(np.float32))
+
+
+def fp8_linear(a, Wq, w_scale, bias=None):
+    """Dynamic per-token FP8 activations against per-channel FP8 weights
+    (W8A8): a [M, K] is quantised row by row in fp32 (R11), then
+    y = s_a[m] s_w[n] sum_k code_a[m, k] code_w[n, k] (+ bias[n]) in fp64."""
+    qa, sa = fp8_row_scale_and_codes(_f64(a).astype(np.float32))
+    y = (qa @ _f64(Wq).T) * _f64(sa)[:, None] * _f64(w_scale)[None, :]
+    if bias is not None:
+        y = y + _f64(bias)[None, :]
+    return y
+
+
+def add_norm_qkv_fp8(x, residual, gamma, beta, norm, eps, Wq, w_scale, bias, Hq, Hkv, D) -> dict:
+    """The fused QKV op on FP8 tensor cores: residual add -> norm -> per-token
+    FP8 quantisation of the normalised activation -> projection with the FP8
+    weights and their scales -> head-major Q/K/V split."""
+    h = residual_add(x, residual)
+    a, mean, rstd = normalize(h, gamma, beta, norm, eps)
+    y = fp8_linear(a, Wq, w_scale, bias)
+    q, k, v = split_qkv_head_major(y, Hq, Hkv, D)
+    return _stats({"residual_out": bf16_round(h), "q": q, "k": k, "v": v}, mean, rstd)
+
+
 def run(w, inputs: dict, rows=None) -> dict:
     """Evaluate workload ``w`` (a synthetic.Workload) on ``inputs`` (tensors or
     arrays, bf16 values), optionally on a subset of rows (the op is row-wise).
@@ -168,6 +229,9 @@ def run(w, inputs: dict, rows=None) -> dict:
         x, r = x[rows], r[rows]
     if w.op == "residual":
         return linear_add_residual(x, g("W"), g("bias_out"), r)
+    if w.op == "qkv_fp8":   # "W_fp8" / "w_scale": the FP8 weights (codes as values) and their scales
+        return add_norm_qkv_fp8(x, r, g("gamma"), g("beta"), w.norm, w.eps, g("W_fp8"), g("w_scale"),
+                                g("bias_out"), w.Hq, w.Hkv, w.D)
     if w.op == "qkv":
         return add_norm_qkv(x, r, g("gamma"), g("beta"), w.norm, w.eps, g("W"),
                             g("bias_out"), w.Hq, w.Hkv, w.D)

@@ -368,10 +368,127 @@ def pin_residual_projection(ora):
             assert abs(got[i, n] - (f["residual"][m, n] + acc + f["bias_out"][n])) <= 1e-12
 
 
+def _e4m3_values():
+    """All finite e4m3 values, from the format's definition: sign, 4 exponent
+    bits (bias 7), 3 mantissa bits; exponent 0 is subnormal (m/8 * 2^-6);
+    exponent 15 with mantissa 7 is NaN."""
+    vals = set()
+    for sign in (1.0, -1.0):
+        for e in range(16):
+            for m in range(8):
+                if e == 15 and m == 7:
+                    continue
+                v = (m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7)
+                vals.add(sign * v)
+    return np.array(sorted(vals))
+
+
+def pin_e4m3_format(ora):
+    """e4m3 rounding: every finite value of the format rounds to itself, the
+    largest is 448, midpoints go to the even mantissa, values past 448
+    saturate, and torch's float8_e4m3fn conversion agrees on +-448."""
+    vals = _e4m3_values()
+    assert len(vals) == 253 and vals.max() == 448.0   # +0 and -0 are one value
+    assert np.array_equal(ora.e4m3_round(vals), vals)
+    pos = vals[vals > 0]
+    mids = (pos[:-1] + pos[1:]) / 2
+    got = ora.e4m3_round(mids)
+    # the even neighbour: mantissa field even (bit pattern of the value's code)
+    def mant(v):
+        if v < 2.0 ** -6:
+            return int(round(v / 2.0 ** -9))
+        e = math.floor(math.log2(v))
+        return int(round((v / 2.0 ** e - 1.0) * 8))
+    for g, lo, hi in zip(got, pos[:-1], pos[1:]):
+        assert g in (lo, hi)
+        assert mant(g) % 2 == 0, (lo, hi, g)
+    assert np.array_equal(ora.e4m3_round(np.array([460.0, 1e6, -1e9])), np.array([448.0, 448.0, -448.0]))
+    rng = np.random.default_rng(70)
+    v = np.concatenate([rng.uniform(-448, 448, 20000), rng.normal(0, 0.02, 20000), mids, -mids])
+    ref = torch.tensor(v).to(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(ora.e4m3_round(v), ref)
+
+
+def pin_fp8_quantisers(ora):
+    """Per-row FP8 quantisation: the row's largest magnitude maps to exactly
+    +-448, scale = amax / 448 in fp32, the error is within half a step
+    (2^-4 relative for normals, 2^-10 s below 2^-6 s), signs are symmetric,
+    a power-of-two row scaling moves only the scale, a zero row has scale 1."""
+    rng = np.random.default_rng(71)
+    W = rng.normal(0, 0.02, (6, 64))
+    W[3] = 0.0
+    q, s_ = ora.quantize_weight_fp8(W)
+    assert s_.dtype == np.float32 and s_[3] == 1.0 and np.all(q[3] == 0)
+    for n in (0, 1, 2, 4, 5):
+        j = int(np.argmax(np.abs(W[n])))
+        assert abs(q[n, j]) == 448.0 and np.sign(q[n, j]) == np.sign(W[n, j])
+        assert s_[n] == np.float32(np.float32(abs(W[n, j])) / np.float32(448.0))
+        err = np.abs(W[n] - q[n] * np.float64(s_[n]))
+        assert np.all(err <= 2.0 ** -4 * np.abs(W[n]) + 2.0 ** -10 * np.float64(s_[n]) + 1e-12)
+    q2, s2 = ora.quantize_weight_fp8(-W)
+    assert np.array_equal(q2, -q) and np.array_equal(s2, s_)
+    q3, s3 = ora.quantize_weight_fp8(W * 8.0)
+    assert np.array_equal(q3, q) and np.array_equal(s3[[0, 1, 2, 4, 5]], 8 * s_[[0, 1, 2, 4, 5]])
+
+
+def pin_fp8_linear(ora):
+    """W8A8 projection: a one-hot activation row gives y_n = c W~[n, j]
+    (W~ = codes * s_w), per-element loops over the codes on a tiny case, and
+    the result stays within the quantisation error bound of the exact
+    product."""
+    rng = np.random.default_rng(72)
+    K, N = 32, 12
+    W = rng.normal(0, 0.2, (N, K))
+    Wq, sw = ora.quantize_weight_fp8(W)
+    Wd = Wq * sw.astype(np.float64)[:, None]
+    a = np.zeros((1, K))
+    a[0, 5] = -2.5
+    y = ora.fp8_linear(a, Wq, sw)
+    # exact but for the fp32 rounding of s_a = 2.5 / 448 (relative 2^-24)
+    assert np.max(np.abs(y[0] - (-2.5) * Wd[:, 5])) <= 2.0 ** -23 * np.max(np.abs(2.5 * Wd[:, 5]))
+    a = rng.normal(0, 1, (3, K))
+    b = rng.normal(0, 0.02, N)
+    y = ora.fp8_linear(a, Wq, sw, b)
+    qa, sa = ora.fp8_row_scale_and_codes(a.astype(np.float32))
+    for m in range(3):
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                acc += qa[m, k] * Wq[n, k]
+            assert abs(y[m, n] - (acc * float(sa[m]) * float(sw[n]) + b[n])) <= 1e-12 * (1 + abs(y[m, n]))
+    exact = a @ Wd.T + b
+    bound = (2.0 ** -4 * np.abs(a) + 2.0 ** -10 * sa.astype(np.float64)[:, None]) @ np.abs(Wd).T + 1e-6
+    assert np.all(np.abs(y - exact) <= bound)
+
+
+def pin_fp8_fused_qkv(ora):
+    """The FP8 fused QKV op: one-hot x (RMSNorm) gives y_n = W~[n, j] gamma_j s /
+    sqrt(s^2/K + eps); residual_out and the statistics are those of the bf16 op."""
+    Hq, Hkv, D = 2, 1, 4
+    N, K = (Hq + 2 * Hkv) * D, 24
+    j, sc, eps = 9, 3.0, 1e-3
+    rng = np.random.default_rng(73)
+    g = 1.0 + 0.1 * rng.normal(size=K)
+    Wq, sw = ora.quantize_weight_fp8(rng.normal(0, 0.2, (N, K)))
+    Wd = Wq * sw.astype(np.float64)[:, None]
+    x = np.zeros((1, K))
+    x[0, j] = sc
+    out = ora.add_norm_qkv_fp8(x, np.zeros((1, K)), g, None, "rmsnorm", eps, Wq, sw, None, Hq, Hkv, D)
+    y = np.concatenate([out["q"][:, 0, :].reshape(-1), out["k"][:, 0, :].reshape(-1), out["v"][:, 0, :].reshape(-1)])
+    ref = Wd[:, j] * g[j] * sc / math.sqrt(sc * sc / K + eps)
+    assert np.max(np.abs(y - ref)) <= 1e-6 * np.max(np.abs(ref))
+    xr, rr = rng.normal(size=(3, K)), rng.normal(size=(3, K))
+    o8 = ora.add_norm_qkv_fp8(xr, rr, g, None, "layernorm", 1e-5, Wq, sw, None, Hq, Hkv, D)
+    o16 = ora.add_norm_qkv(xr, rr, g, None, "layernorm", 1e-5, Wd, None, Hq, Hkv, D)
+    for key in ("residual_out", "mean", "rstd"):
+        assert np.array_equal(o8[key], o16[key])
+
+
 PINS = [pin_layernorm_invariants, pin_rmsnorm_invariant, pin_norms_match_torch,
         pin_identity_weight, pin_one_hot, pin_brute_force, pin_epilogue_values,
         pin_qkv_bijection, pin_bf16_round, pin_residual_out,
-        pin_run_maps_workload_inputs, pin_residual_projection]
+        pin_run_maps_workload_inputs, pin_residual_projection, pin_e4m3_format, pin_fp8_quantisers,
+        pin_fp8_linear, pin_fp8_fused_qkv]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -383,7 +500,8 @@ def test_pin_holds(pin):
 # planted mistakes: every one must break at least one pin
 # --------------------------------------------------------------------------
 
-ORIG = {name: getattr(core, name) for name in ("layernorm", "rmsnorm", "split_qkv_head_major", "run")}
+ORIG = {name: getattr(core, name) for name in ("layernorm", "rmsnorm", "split_qkv_head_major", "run",
+                                               "e4m3_round", "fp8_row_scale_and_codes", "fp8_linear")}
 
 
 def _ln_unbiased(h, gamma, beta, eps):
@@ -524,6 +642,45 @@ def _resid_subtracted(a, W, bias, residual):
     return {"out": core.projection(a, W, bias) - np.asarray(residual, np.float64)}
 
 
+def _e4m3_truncates(v):
+    v = np.asarray(v, np.float64)
+    a = np.abs(v)
+    e = np.maximum(np.floor(np.log2(np.where(a > 0, a, 1.0))), -6.0)
+    quantum = np.ldexp(1.0, (e - 3).astype(np.int64))
+    q = np.minimum(np.floor(a / quantum) * quantum, 448.0)
+    return np.where(a > 0, np.sign(v) * q, 0.0)
+
+
+def _e4m3_no_subnormals(v):
+    q = ORIG["e4m3_round"](v)
+    return np.where(np.abs(q) < 2.0 ** -6, 0.0, q)
+
+
+def _e4m3_e5m2_max(v):
+    v = np.asarray(v, np.float64)
+    a = np.abs(v)
+    e = np.maximum(np.floor(np.log2(np.where(a > 0, a, 1.0))), -6.0)
+    quantum = np.ldexp(1.0, (e - 3).astype(np.int64))
+    q = np.minimum(np.rint(a / quantum) * quantum, 480.0)
+    return np.where(a > 0, np.sign(v) * q, 0.0)
+
+
+def _fp8_per_tensor(v32):
+    v32 = np.asarray(v32, np.float32)
+    amax = np.float32(np.max(np.abs(v32)))
+    s_ = np.full(v32.shape[0], amax / np.float32(448.0) if amax > 0 else np.float32(1.0), np.float32)
+    return core.e4m3_round((v32 / s_[:, None]).astype(np.float32)), s_
+
+
+def _fp8_scale_inverted(v32):
+    q, s_ = ORIG["fp8_row_scale_and_codes"](v32)
+    return q, (np.float32(1.0) / s_).astype(np.float32)
+
+
+def _fp8_linear_no_weight_scale(a, Wq, w_scale, bias=None):
+    return ORIG["fp8_linear"](a, Wq, np.ones_like(np.asarray(w_scale)), bias)
+
+
 MUTANTS = {
     "variance_divides_by_K_minus_1": ("layernorm", _ln_unbiased),
     "eps_outside_sqrt": ("layernorm", _ln_eps_outside),
@@ -550,6 +707,12 @@ MUTANTS = {
     "residual_projection_drops_bias": ("linear_add_residual", _resid_bias_dropped),
     "residual_projection_w_untransposed": ("linear_add_residual", _resid_w_untransposed),
     "residual_projection_subtracts_residual": ("linear_add_residual", _resid_subtracted),
+    "e4m3_truncates": ("e4m3_round", _e4m3_truncates),
+    "e4m3_flushes_subnormals": ("e4m3_round", _e4m3_no_subnormals),
+    "e4m3_saturates_at_480": ("e4m3_round", _e4m3_e5m2_max),
+    "fp8_scale_per_tensor": ("fp8_row_scale_and_codes", _fp8_per_tensor),
+    "fp8_scale_inverted": ("fp8_row_scale_and_codes", _fp8_scale_inverted),
+    "fp8_weight_scale_dropped": ("fp8_linear", _fp8_linear_no_weight_scale),
 }
 
 
