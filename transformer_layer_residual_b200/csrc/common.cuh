@@ -31,6 +31,8 @@ struct OpParams {
   bf16* k;
   bf16* v;
   bf16* out;
+  const float4* stats8;  // FP8 ops: per token (mean, rstd, activation scale s_a, 448 / amax), from the pre-pass
+  const float* w_scale;  // FP8 ops: per W row dequantisation scale s_w [N] (null for the bf16 ops)
   const bf16* res_in;    // residual-stream projection: the residual [M][N] added in the epilogue
                          // (may be the same buffer as out: each element is read, then written,
                          // by one thread)
@@ -204,11 +206,22 @@ __device__ __forceinline__ uint4 ldcg16(const void* p) {
 // Store 8 consecutive output columns [n, n+8) of row m (QKV, GELU or residual
 // epilogue). acc is the raw fp32 accumulator, scale the deferred RMSNorm 1/rms
 // (1 for LN and for the residual-stream projection).
+// FP8 ops: the accumulator holds sum of code products; y = acc s_a[m] s_w[n].
+__device__ __forceinline__ void fp8_dequant8(const OpParams& p, int m, int n, float (&y)[8]) {
+  const float sa = p.stats8[m].z;
+  const float4 w0 = __ldg(reinterpret_cast<const float4*>(p.w_scale + n));
+  const float4 w1 = __ldg(reinterpret_cast<const float4*>(p.w_scale + n + 4));
+  const float ws[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+  for (int e = 0; e < 8; ++e) y[e] *= sa * ws[e];
+}
+
 template <int EPI>
 __device__ __forceinline__ void store_out8(const OpParams& p, int m, int n, const float (&acc)[8], float scale) {
   float y[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) y[e] = acc[e] * scale;
+  if (p.w_scale != nullptr) fp8_dequant8(p, m, n, y);
   if (p.bias != nullptr) {
     float b[8];
     unpack8(ldg16(p.bias + n), b);
@@ -253,6 +266,10 @@ __device__ __forceinline__ void store_swiglu8(const OpParams& p, int m, int j, c
   for (int e = 0; e < 8; ++e) {
     g[e] = gate[e] * scale;
     u[e] = up[e] * scale;
+  }
+  if (p.w_scale != nullptr) {
+    fp8_dequant8(p, m, j, g);
+    fp8_dequant8(p, m, p.I + j, u);
   }
   if (p.bias != nullptr) {
     float bg[8], bu[8];

@@ -636,21 +636,28 @@ fnl_status default_plan(fnl_handle* h, const Call& c, Plan* pl) {
     default: break;
   }
   if (c.M <= fnl::k3::MAX_MPAD) return plan_kernel(h, c, Kern::K3, -1, pl);
-  // two tile shapes: 128 x 512 (less traffic and conversion per FLOP, the
-  // default) and 128 x 256 (finer), picked by how well the tiles fill whole
-  // waves of CTAs; a 128 x 512 tile takes about 1.6x a 128 x 256 tile
+  // three tile shapes: 256 x 512 on CTA pairs (least shared-memory traffic per
+  // FLOP), 128 x 512 and 128 x 256 (finer), picked by how well their tiles
+  // fill whole waves of CTAs (pairs): per SM, a 128 x 512 tile takes about
+  // 1.6x a 128 x 256 tile and a pair tile about 0.9x a 128 x 512 tile
   // (measured on B200 across the prefill shapes)
   const int max_ctas = h->opt.max_ctas > 0 ? std::min(h->opt.max_ctas, h->num_sms) : h->num_sms;
-  const int num_m = (c.M + 127) / 128;
+  const int num_m = (c.M + 127) / 128, num_m2 = (c.M + 255) / 256;
   const long long tiles_n = static_cast<long long>(num_m) *
                             (c.op == Op::SwiGLU ? (c.I + 127) / 128 : (c.N + fnl::k2::BN - 1) / fnl::k2::BN);
   const long long tiles_w = static_cast<long long>(num_m) *
                             (c.op == Op::SwiGLU ? (c.I + 255) / 256 : (c.N + fnl::k2w::BN - 1) / fnl::k2w::BN);
-  auto waves = [&](long long tiles) {
-    const long long g = std::min<long long>(max_ctas, tiles);
+  const long long tiles_p = static_cast<long long>(num_m2) *
+                            (c.op == Op::SwiGLU ? (c.I + 255) / 256 : (c.N + fnl::k4::BN - 1) / fnl::k4::BN);
+  auto waves = [](long long tiles, long long slots) {
+    const long long g = std::min<long long>(slots, tiles);
     return static_cast<double>((tiles + g - 1) / g);
   };
-  return plan_kernel(h, c, waves(tiles_w) * 1.6 <= waves(tiles_n) ? Kern::K2W : Kern::K2, -1, pl);
+  const double t_n = waves(tiles_n, max_ctas), t_w = 1.6 * waves(tiles_w, max_ctas);
+  const int pairs = h->opt.max_ctas == 0 ? resident_pairs(h) : 0;
+  const double t_p = pairs > 0 ? 1.45 * waves(tiles_p, pairs) : 1e30;
+  if (t_p <= t_w && t_p <= t_n) return plan_kernel(h, c, Kern::K4, -1, pl);
+  return plan_kernel(h, c, t_w <= t_n ? Kern::K2W : Kern::K2, -1, pl);
 }
 
 size_t stats_bytes_of(const Call& c) {

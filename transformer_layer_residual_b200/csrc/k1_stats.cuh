@@ -90,4 +90,149 @@ __global__ void __launch_bounds__(kK1Threads) k1_layernorm_stats(const bf16* __r
   }
 }
 
+__device__ __forceinline__ float block_max_256(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float m = 0.f;
+#pragma unroll
+  for (int w = 0; w < kK1Threads / 32; ++w) m = fmaxf(m, red[w]);
+  return m;
+}
+
+// FP8 pre-pass of the fused ops (per-token dynamic quantisation, TensorRT-LLM
+// 深度工程实践, §3.3 FP4/FP8 动态量化加速: activation ranges from runtime
+// statistics). One CTA per row: h = x + r (+ bias_in) in fp32, residual_out =
+// bf16(h), the row's statistics (LayerNorm: two-pass mean and variance;
+// RMSNorm: mean 0, mean of h^2), then a = (h - mean) rstd gamma + beta computed
+// exactly as the FP8 converters compute it, and its amax. Writes
+// stats8[row] = (mean, rstd, s_a = amax / 448, 448 / amax) (1, 1 for a zero row).
+template <int MAXV, bool RMS>
+__global__ void __launch_bounds__(kK1Threads) k1_fp8_prepass(const bf16* __restrict__ x,
+                                                             const bf16* __restrict__ residual,
+                                                             const bf16* __restrict__ bias_in,
+                                                             const bf16* __restrict__ gamma,
+                                                             const bf16* __restrict__ beta,
+                                                             bf16* __restrict__ residual_out,
+                                                             float4* __restrict__ stats8,
+                                                             float* __restrict__ mean_out,
+                                                             float* __restrict__ rstd_out, int M, int K,
+                                                             float eps) {
+  pdl_launch_dependents();
+  __shared__ float red[kK1Threads / 32];
+  const int row = blockIdx.x;
+  if (row >= M) return;
+  const int nvec = K >> 3;
+  const size_t rbase = static_cast<size_t>(row) * K;
+  f32x2 h[MAXV][4];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int v = threadIdx.x + i * kK1Threads;
+    if (v < nvec) {
+      const uint4 xv = ldg16(x + rbase + v * 8), rv = ldg16(residual + rbase + v * 8);
+      const uint4 bv = bias_in != nullptr ? ldg16(bias_in + v * 8) : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, rw[4] = {rv.x, rv.y, rv.z, rv.w};
+      const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+      uint32_t ho[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        h[i][e] = add2(bf2_to_f2(xw[e]), bf2_to_f2(rw[e]));
+        if (bias_in != nullptr) h[i][e] = add2(h[i][e], bf2_to_f2(bw[e]));
+        float lo, hi;
+        unpk2(h[i][e], lo, hi);
+        s += RMS ? fmaf(lo, lo, hi * hi) : lo + hi;
+        ho[e] = f2_to_bf2(h[i][e]);
+      }
+      *reinterpret_cast<uint4*>(residual_out + rbase + v * 8) = make_uint4(ho[0], ho[1], ho[2], ho[3]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) h[i][e] = 0ull;
+    }
+  }
+  float mean = 0.f, rstd;
+  if (RMS) {
+    rstd = 1.f / sqrtf(block_sum_256(s, red) / static_cast<float>(K) + eps);
+  } else {
+    mean = block_sum_256(s, red) / static_cast<float>(K);
+    float s2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < MAXV; ++i) {
+      const int v = threadIdx.x + i * kK1Threads;
+      if (v < nvec) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float lo, hi;
+          unpk2(h[i][e], lo, hi);
+          const float d0 = lo - mean, d1 = hi - mean;
+          s2 = fmaf(d0, d0, s2);
+          s2 = fmaf(d1, d1, s2);
+        }
+      }
+    }
+    rstd = 1.f / sqrtf(block_sum_256(s2, red) / static_cast<float>(K) + eps);
+  }
+  const f32x2 mu2 = pk2(mean, mean), rs2 = pk2(rstd, rstd);
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int v = threadIdx.x + i * kK1Threads;
+    if (v < nvec) {
+      const uint4 gv = ldg16(gamma + v * 8);
+      const uint4 bv = beta != nullptr ? ldg16(beta + v * 8) : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const f32x2 a = fma2(mul2(sub2(h[i][e], mu2), rs2), bf2_to_f2(gw[e]), bf2_to_f2(bw[e]));
+        float lo, hi;
+        unpk2(a, lo, hi);
+        amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+      }
+    }
+  }
+  amax = block_max_256(amax, red);
+  if (threadIdx.x == 0) {
+    const float sa = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+    const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
+    stats8[row] = make_float4(mean, rstd, sa, inv);
+    if (mean_out) mean_out[row] = mean;
+    if (rstd_out) rstd_out[row] = rstd;
+  }
+}
+
+// Static per-output-channel FP8 weights: one CTA per W row, s_w = amax / 448
+// (1 for a zero row) and codes e4m3(w / s_w), both divisions IEEE in fp32.
+__global__ void __launch_bounds__(kK1Threads) k0_quantize_weight_fp8(const bf16* __restrict__ W,
+                                                                    uint8_t* __restrict__ Wq,
+                                                                    float* __restrict__ w_scale, int N, int K) {
+  __shared__ float red[kK1Threads / 32];
+  const int row = blockIdx.x;
+  if (row >= N) return;
+  const size_t base = static_cast<size_t>(row) * K;
+  const int nvec = K >> 3;
+  float amax = 0.f;
+  for (int v = threadIdx.x; v < nvec; v += kK1Threads) {
+    float f[8];
+    unpack8(ldg16(W + base + v * 8), f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+  }
+  amax = block_max_256(amax, red);
+  const float sw = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+  for (int v = threadIdx.x; v < nvec; v += kK1Threads) {
+    float f[8];
+    unpack8(ldg16(W + base + v * 8), f);
+    uint32_t c[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+      c[e] = e4m3x4(pk2(__fdiv_rn(f[4 * e], sw), __fdiv_rn(f[4 * e + 1], sw)),
+                    pk2(__fdiv_rn(f[4 * e + 2], sw), __fdiv_rn(f[4 * e + 3], sw)));
+    *reinterpret_cast<uint2*>(Wq + base + v * 8) = make_uint2(c[0], c[1]);
+  }
+  if (threadIdx.x == 0) w_scale[row] = sw;
+}
+
 }  // namespace fnl

@@ -63,18 +63,6 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-// UMMA descriptor, K-major operand in the 64-byte swizzle layout: 64-byte rows,
-// 8-row groups 512 bytes apart.
-__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
-  d |= static_cast<uint64_t>(1) << 16;
-  d |= static_cast<uint64_t>(512 >> 4) << 32;
-  d |= static_cast<uint64_t>(1) << 46;
-  d |= static_cast<uint64_t>(4) << 61;   // SWIZZLE_64B
-  return d;
-}
-
 }  // namespace k2w
 
 template <int EPI, int NORM, bool SPLIT>

@@ -66,9 +66,14 @@ struct Ctrl {
 };
 
 __host__ __device__ inline int stage_bytes(int mpad) { return W_BYTES + 2 * mpad * BK * 2; }
+// FP8 form: the W tile is 128 rows x 64 e4m3 (8 KB, 64-byte swizzle), the x and
+// residual tiles stay bf16, and the converters write the e4m3 activation
+// operand [mpad][64] (64-byte swizzle) after them.
+constexpr int W8_BYTES = BW * BK;   // 8 KB
+__host__ __device__ inline int stage_bytes8(int mpad) { return W8_BYTES + 2 * mpad * BK * 2 + mpad * BK; }
 constexpr int VEC_BYTES = MAX_STAGES * kVecStageBytes;   // 3 KB
-__host__ __device__ inline int smem_bytes(int mpad, int stages) {
-  return stages * stage_bytes(mpad) + VEC_BYTES + static_cast<int>(sizeof(Ctrl)) + 1024;
+__host__ __device__ inline int smem_bytes(int mpad, int stages, bool fp8 = false) {
+  return stages * (fp8 ? stage_bytes8(mpad) : stage_bytes(mpad)) + VEC_BYTES + static_cast<int>(sizeof(Ctrl)) + 1024;
 }
 __host__ __device__ inline uint32_t tmem_cols(int mpad) {
   uint32_t c = 32;
@@ -288,7 +293,11 @@ __device__ __forceinline__ void k3_cluster_reduce(const OpParams& p, uint32_t pa
   }
 }
 
-template <int EPI, int NORM, bool SPLIT>
+// FP8 (e4m3 weights and activations, kind::f8f6f4 UMMA): the normalisation uses
+// the pre-pass statistics (p.stats8: mean, rstd and the token's quantisation
+// scale) for both norms, so it is instantiated with NORM = kLayerNorm (beta
+// absent and mean 0 for RMSNorm); the epilogue multiplies by s_a[m] s_w[n].
+template <int EPI, int NORM, bool SPLIT, bool FP8 = false>
 __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     k3_splitk_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_r,
                      const __grid_constant__ CUtensorMap tm_w, const OpParams p) {
@@ -296,7 +305,8 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int mpad = p.mpad, S = p.stages;
-  const int SB = stage_bytes(mpad);
+  const int SB = FP8 ? stage_bytes8(mpad) : stage_bytes(mpad);
+  const int WB = FP8 ? W8_BYTES : W_BYTES;   // x tile offset within a stage
   const int XB = mpad * BK * 2;
   bf16* vecs = reinterpret_cast<bf16*>(smem + S * SB);   // [S][3][64]
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + S * SB + VEC_BYTES);
@@ -392,10 +402,10 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
           return;
         }
         uint8_t* st = smem + c.s * SB;
-        mbar_arrive_expect_tx(&ctrl->full_w[c.s], W_BYTES);
+        mbar_arrive_expect_tx(&ctrl->full_w[c.s], WB);
         if (EPI == kEpiSwiGLU) {
           tma_load_2d_hint(st, &tm_w, &ctrl->full_w[c.s], c.kb * BK, c.t * 64, pol_w);
-          tma_load_2d_hint(st + W_BYTES / 2, &tm_w, &ctrl->full_w[c.s], c.kb * BK, p.I + c.t * 64, pol_w);
+          tma_load_2d_hint(st + WB / 2, &tm_w, &ctrl->full_w[c.s], c.kb * BK, p.I + c.t * 64, pol_w);
         } else {
           tma_load_2d_hint(st, &tm_w, &ctrl->full_w[c.s], c.kb * BK, c.t * BW, pol_w);
         }
@@ -406,15 +416,15 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
         uint8_t* st = smem + c.s * SB;
         if (NORM == kNoNorm) {   // the activation tile is the operand as loaded
           mbar_arrive_expect_tx(&ctrl->full_x[c.s], XB);
-          tma_load_2d(st + W_BYTES, &tm_x, &ctrl->full_x[c.s], c.kb * BK, 0);
+          tma_load_2d(st + WB, &tm_x, &ctrl->full_x[c.s], c.kb * BK, 0);
           armed_x |= 1u << c.s;
           par_x = (par_x & ~(1u << c.s)) | (c.ph << c.s);
           return;
         }
         mbar_arrive_expect_tx(&ctrl->full_x[c.s], 2 * XB + vec_bytes(p, has_beta, has_bias_in, c.kb));
         issue_vec_loads(p, has_beta, has_bias_in, c.kb, vecs + c.s * 3 * kVecElems, &ctrl->full_x[c.s]);
-        tma_load_2d(st + W_BYTES, &tm_x, &ctrl->full_x[c.s], c.kb * BK, 0);
-        tma_load_2d(st + W_BYTES + XB, &tm_r, &ctrl->full_x[c.s], c.kb * BK, 0);
+        tma_load_2d(st + WB, &tm_x, &ctrl->full_x[c.s], c.kb * BK, 0);
+        tma_load_2d(st + WB + XB, &tm_r, &ctrl->full_x[c.s], c.kb * BK, 0);
         armed_x |= 1u << c.s;
         par_x = (par_x & ~(1u << c.s)) | (c.ph << c.s);
       };
@@ -455,7 +465,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
       int t, kb0, nk, slot, nseg;
       uint32_t s = 0, ph = 0;
       bool ok = true;
-      const uint32_t idesc = idesc_bf16(BW, mpad);
+      const uint32_t idesc = FP8 ? idesc_e4m3(BW, mpad) : idesc_bf16(BW, mpad);
       int i = 0;
       while (ok && it.next(t, kb0, nk, slot, nseg)) {
         const int b = i & 1;
@@ -473,15 +483,23 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
           }
           tc_fence_after();
           const uint32_t wa = smem_u32(smem + s * SB);
-          const uint64_t ad = sw128_desc(wa);
-          const uint64_t bd = sw128_desc(wa + W_BYTES);
+          if (FP8) {   // 64 e4m3 per row: two K = 32 steps of 32 bytes
+            const uint64_t ad = sw64_desc(wa);
+            const uint64_t bd = sw64_desc(wa + WB + 2 * XB);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
-          if (SPLIT) {
-            const uint64_t ld = sw128_desc(wa + W_BYTES + XB);
+            for (int kk = 0; kk < BK / 32; ++kk)
+              umma_f8(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+          } else {
+            const uint64_t ad = sw128_desc(wa);
+            const uint64_t bd = sw128_desc(wa + WB);
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) umma_bf16(d, ad + 2 * kk, ld + 2 * kk, idesc, 1u);
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma_bf16(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+            if (SPLIT) {
+              const uint64_t ld = sw128_desc(wa + WB + XB);
+#pragma unroll
+              for (int kk = 0; kk < BK / 16; ++kk) umma_bf16(d, ad + 2 * kk, ld + 2 * kk, idesc, 1u);
+            }
           }
           umma_commit(&ctrl->empty[s]);
           if (++s == static_cast<uint32_t>(S)) {
@@ -598,6 +616,68 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
           k3_reduce_tile<EPI, NORM, NUM_EPI_WARPS * 32>(p, t, nseg, et);
           if (et == 0) p.counters[t] = 0u;
         }
+      }
+    }
+  } else if (FP8) {
+    // ------------------------------------------------------------ converters (FP8)
+    // Converter warp cw owns positions cw, cw + 4, ... as below. A lane task is
+    // (token row, 16-byte e4m3 chunk j of the row's 64): it reads the bf16
+    // chunks 2j and 2j + 1 of x and the residual, forms h (+ bias_in), normalises
+    // with the pre-pass statistics, a = (h - mean) rstd gamma + beta (the
+    // pre-pass computes the same expression for the token's amax), and stores
+    // e4m3(a * 448 / amax) (round to nearest even, saturating).
+    const int cw = warp - WARP_CONV0;
+    pdl_wait();   // statistics come from the pre-pass
+    const int P = static_cast<int>(u1 - u0);
+    int s = cw;
+    uint32_t ph = 0;
+    for (int q = cw; q < P; q += NUM_CONV_WARPS) {
+      const long long u = u0 + q;
+      const int kb = static_cast<int>(u % nkb);
+      if (!warp_wait(&ctrl->full_x[s], ph, abortf, p.status, kStatusWaitFull, p.wait_ns)) break;
+      const uint32_t xs = smem_u32(smem + s * SB) + WB;
+      const uint32_t rsm = xs + XB;
+      const uint32_t qs = rsm + XB;
+      bf16* vec = vecs + s * 3 * kVecElems;
+      if (K - kb * BK < BK) zero_vec_tails(vec, kVecElems, K - kb * BK);
+      const uint32_t vaddr = smem_u32(vec);
+      for (int task = lane; task < M * 4; task += 32) {
+        const int row = task >> 2, j = task & 3;
+        const float4 st = __ldg(p.stats8 + row);
+        const f32x2 mu2 = pk2(st.x, st.x), rs2 = pk2(st.y, st.y), inv2 = pk2(st.w, st.w);
+        uint32_t codes[4];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int c = 2 * j + hh;
+          const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
+          const uint4 xv = ld_shared_v4(xs + off), rv = ld_shared_v4(rsm + off);
+          f32x2 g2[4], be2[4] = {}, bi2[4] = {};
+          vec_pairs(vaddr + c * 16, g2);
+          if (p.beta != nullptr) vec_pairs(vaddr + 2 * kVecElems + c * 16, be2);
+          if (BIAS_IN) vec_pairs(vaddr + 4 * kVecElems + c * 16, bi2);
+          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, rw[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+          for (int i = 0; i < 4; i += 2) {
+            f32x2 h0 = add2(bf2_to_f2(xw[i]), bf2_to_f2(rw[i]));
+            f32x2 h1 = add2(bf2_to_f2(xw[i + 1]), bf2_to_f2(rw[i + 1]));
+            if (BIAS_IN) {
+              h0 = add2(h0, bi2[i]);
+              h1 = add2(h1, bi2[i + 1]);
+            }
+            const f32x2 a0 = mul2(fma2(mul2(sub2(h0, mu2), rs2), g2[i], be2[i]), inv2);
+            const f32x2 a1 = mul2(fma2(mul2(sub2(h1, mu2), rs2), g2[i + 1], be2[i + 1]), inv2);
+            codes[hh * 2 + i / 2] = e4m3x4(a0, a1);
+          }
+        }
+        st_shared_v4(qs + row * 64 + ((j ^ ((row >> 1) & 3)) << 4), make_uint4(codes[0], codes[1], codes[2], codes[3]));
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctrl->conv[s]);
+      s += NUM_CONV_WARPS;
+      if (s >= S) {
+        s -= S;
+        ph ^= 1u;
       }
     }
   } else if (NORM != kNoNorm) {

@@ -79,16 +79,6 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
-  d |= static_cast<uint64_t>(1) << 16;
-  d |= static_cast<uint64_t>(512 >> 4) << 32;
-  d |= static_cast<uint64_t>(1) << 46;
-  d |= static_cast<uint64_t>(4) << 61;   // SWIZZLE_64B
-  return d;
-}
-
 }  // namespace k4
 
 template <int EPI, int NORM, bool SPLIT>
@@ -267,10 +257,10 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
           }
           tc_fence_after();
           const uint32_t xa = smem_u32(smem + s * STAGE_BYTES);
-          const uint64_t ad = k4::sw64_desc(xa);
-          const uint64_t ld = k4::sw64_desc(xa + X_BYTES);
-          const uint64_t bd0 = k4::sw64_desc(xa + 2 * X_BYTES);
-          const uint64_t bd1 = k4::sw64_desc(xa + 2 * X_BYTES + WH_BYTES);
+          const uint64_t ad = sw64_desc(xa);
+          const uint64_t ld = sw64_desc(xa + X_BYTES);
+          const uint64_t bd0 = sw64_desc(xa + 2 * X_BYTES);
+          const uint64_t bd1 = sw64_desc(xa + 2 * X_BYTES + WH_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;

@@ -235,6 +235,18 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
       : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, e4m3 inputs (K = 32 per
+// instruction), fp32 accumulate.
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on `bar` when every previously issued UMMA of this thread is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -284,13 +296,17 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
-// Test of a phase whose arrivals may come from the other CTA of the pair
-// (acquire at cluster scope, so the arriving CTA's prior writes are visible).
+// Test of a phase whose arrivals may come from the other CTA of the pair.
+// What the arriving CTA hands over is its shared-memory operand, read by the
+// pair's UMMA through the async proxy: its proxy fence before the arrive orders
+// it, so the wait is the ordinary CTA-scope one (cluster-scope acquire/release
+// on every stage doubled the pair kernel's time: 446 -> 960 us at 70B QKV,
+// M = 2048).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity), "r"(1000u)
@@ -314,12 +330,12 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   }
 }
 // Arrive on the mbarrier at the same shared-memory offset in CTA `rank` of the
-// cluster, releasing this thread's prior writes at cluster scope.
+// cluster (default semantics: release at CTA scope; see mbar_try_wait_cluster).
 __device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t rank) {
   asm volatile(
       "{\n\t.reg .b32 ra;\n\t"
       "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
-      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_u32(bar)),
+      "mbarrier.arrive.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_u32(bar)),
       "r"(rank)
       : "memory");
 }
@@ -365,6 +381,28 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t mask) {
           smem_u32(bar)),
       "h"(mask)
       : "memory");
+}
+
+// Instruction descriptor, kind::f8f6f4: e4m3 A and B (K-major), fp32 D, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
+  return (1u << 4)                                  // D format: f32
+         | (0u << 7)                                // A format: e4m3
+         | (0u << 10)                               // B format: e4m3
+         | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
+}
+
+// UMMA shared-memory descriptor, K-major operand in the 64-byte swizzle layout
+// that TMA writes with CU_TENSOR_MAP_SWIZZLE_64B: 64-byte rows, 8-row groups
+// 512 bytes apart.
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(1) << 16;
+  d |= static_cast<uint64_t>(512 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(4) << 61;   // SWIZZLE_64B
+  return d;
 }
 
 // ---------------------------------------------------------------- misc
@@ -417,6 +455,20 @@ __device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
   f32x2 r;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
   return r;
+}
+
+// Four fp32 values (two pairs, first element lowest) -> four e4m3 codes in one
+// 32-bit word (first element in the lowest byte), round to nearest even,
+// saturating at +-448.
+__device__ __forceinline__ uint32_t e4m3x4(f32x2 a, f32x2 b) {
+  float a0, a1, b0, b1;
+  unpk2(a, a0, a1);
+  unpk2(b, b0, b1);
+  uint16_t lo, hi;
+  // cvt packs its first source into the upper byte
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(a1), "f"(a0));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(b1), "f"(b0));
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
 // bf16 pair <-> two floats (low half = lower address = first element)
