@@ -52,7 +52,12 @@ Readings taken where the pages are silent:
      max_k |W[n, k]| / 448; activations one dynamic scale per token, taken on
      the normalised row, s_a[m] = max_k |a[m, k]| / 448; y = s_a s_w sum of
      code products. Every decision that picks a code is taken in fp32, the
-     kernel's precision; the rest is fp64.
+     kernel's precision, with the kernel's formula: weights e4m3(w / s_w);
+     activations formed in fp32 from the statistics, t = (h - mean) rstd,
+     a = t gamma + beta, then e4m3(a * (448 / amax)). RMSNorm's 1/rms is a
+     positive per-token factor: its codes are decided on h * gamma and rstd
+     joins the token's scale. The statistics, the sums of code products and
+     the dequantisation are fp64.
   R9 the residual-stream projection adds the residual after the projection and
      its bias: out = residual + a W^T + bias, with residual [M, N] (N = the
      hidden size the projection returns to); the stored result is out rounded
@@ -80,6 +85,8 @@ from .core import (  # noqa: F401
     E4M3_MAX,
     e4m3_round,
     fp8_row_scale_and_codes,
+    fp8_activation_codes,
+    fp8_normalised32,
     quantize_weight_fp8,
     fp8_linear,
     add_norm_qkv_fp8,

@@ -173,13 +173,28 @@ def _f32(a) -> np.ndarray:
 
 
 def fp8_row_scale_and_codes(v32):
-    """Per-row symmetric e4m3 quantisation, every decision in fp32 (reading
-    R11): amax = max |v| of the row, s = amax / 448 (1 for an all-zero row),
-    code = e4m3(v / s). Returns (codes as fp64 values, s as fp32)."""
+    """Per-row symmetric e4m3 quantisation of a weight row (R11), every step
+    in fp32: amax = max |v| of the row, s = amax / 448 (1 for an all-zero
+    row), code = e4m3(v / s). Returns (codes as fp64 values, s as fp32)."""
     v32 = _f32(v32)
     amax = np.max(np.abs(v32), axis=1)
     s = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
     q = e4m3_round((v32 / s[:, None]).astype(np.float32))
+    return q, s
+
+
+def fp8_activation_codes(a32):
+    """Per-token dynamic quantisation of the normalised activation (R11), the
+    decision in fp32 as the kernel takes it: amax = max_k |a|, code =
+    e4m3(a * (448 / amax)), dequantisation scale s_a = amax / 448 (448 / amax
+    and s_a are 1 for an all-zero row). Returns (codes as fp64 values, s_a)."""
+    a32 = _f32(a32)
+    amax = np.max(np.abs(a32), axis=1)
+    nz = amax > 0
+    safe = np.where(nz, amax, np.float32(1.0)).astype(np.float32)
+    inv = np.where(nz, np.float32(E4M3_MAX) / safe, np.float32(1.0)).astype(np.float32)
+    s = np.where(nz, safe / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    q = e4m3_round((a32 * inv[:, None]).astype(np.float32))
     return q, s
 
 
@@ -189,24 +204,47 @@ def quantize_weight_fp8(W):
     return fp8_row_scale_and_codes(_f64(W).astype(np.float32))
 
 
-def fp8_linear(a, Wq, w_scale, bias=None):
+def fp8_linear(a32, Wq, w_scale, bias=None):
     """Dynamic per-token FP8 activations against per-channel FP8 weights
-    (W8A8): a [M, K] is quantised row by row in fp32 (R11), then
-    y = s_a[m] s_w[n] sum_k code_a[m, k] code_w[n, k] (+ bias[n]) in fp64."""
-    qa, sa = fp8_row_scale_and_codes(_f64(a).astype(np.float32))
+    (W8A8): a [M, K] (fp32) is quantised row by row (fp8_activation_codes),
+    then y = s_a[m] s_w[n] sum_k code_a[m, k] code_w[n, k] (+ bias[n]) in fp64."""
+    qa, sa = fp8_activation_codes(a32)
     y = (qa @ _f64(Wq).T) * _f64(sa)[:, None] * _f64(w_scale)[None, :]
     if bias is not None:
         y = y + _f64(bias)[None, :]
     return y
 
 
+def fp8_normalised32(h, mean, rstd, gamma, beta):
+    """The normalised activation in fp32, as the FP8 path forms it before the
+    code decision (R11): h in fp32, the statistics rounded to fp32,
+    t = fp32(fp32(h - mean) * rstd), a = fp32(t * gamma + beta) with one
+    rounding (mean 0 and beta 0 for RMSNorm)."""
+    h32 = _f32(h)
+    m32 = _f32(np.zeros(h32.shape[0]) if mean is None else mean)
+    r32 = _f32(rstd)
+    t = ((h32 - m32[:, None]).astype(np.float32) * r32[:, None]).astype(np.float32)
+    b = np.zeros(h32.shape[1]) if beta is None else _f64(beta)
+    return (_f64(t) * _f64(gamma)[None, :] + b[None, :]).astype(np.float32)
+
+
 def add_norm_qkv_fp8(x, residual, gamma, beta, norm, eps, Wq, w_scale, bias, Hq, Hkv, D) -> dict:
-    """The fused QKV op on FP8 tensor cores: residual add -> norm -> per-token
-    FP8 quantisation of the normalised activation -> projection with the FP8
-    weights and their scales -> head-major Q/K/V split."""
+    """The fused QKV op on FP8 tensor cores: residual add -> norm statistics ->
+    the activation in fp32 -> per-token FP8 quantisation -> projection with the
+    FP8 weights and their scales -> head-major Q/K/V split. RMSNorm's 1/rms is
+    a positive per-token factor, so its codes are decided on h * gamma (the same
+    codes as on the normalised row, but for fp32 rounding) and rstd multiplies
+    the token's scale (reading R11)."""
     h = residual_add(x, residual)
-    a, mean, rstd = normalize(h, gamma, beta, norm, eps)
-    y = fp8_linear(a, Wq, w_scale, bias)
+    _, mean, rstd = normalize(h, gamma, beta, norm, eps)
+    if norm == "rmsnorm":
+        a32 = (_f32(h) * _f32(gamma)[None, :]).astype(np.float32)
+        qa, sa = fp8_activation_codes(a32)
+        y = (qa @ _f64(Wq).T) * (_f64(sa) * rstd)[:, None] * _f64(w_scale)[None, :]
+        if bias is not None:
+            y = y + _f64(bias)[None, :]
+    else:
+        y = fp8_linear(fp8_normalised32(h, mean, rstd, gamma, beta), Wq, w_scale, bias)
     q, k, v = split_qkv_head_major(y, Hq, Hkv, D)
     return _stats({"residual_out": bf16_round(h), "q": q, "k": k, "v": v}, mean, rstd)
 

@@ -446,19 +446,48 @@ def pin_fp8_linear(ora):
     y = ora.fp8_linear(a, Wq, sw)
     # exact but for the fp32 rounding of s_a = 2.5 / 448 (relative 2^-24)
     assert np.max(np.abs(y[0] - (-2.5) * Wd[:, 5])) <= 2.0 ** -23 * np.max(np.abs(2.5 * Wd[:, 5]))
-    a = rng.normal(0, 1, (3, K))
+    a = rng.normal(0, 1, (3, K)).astype(np.float32)
     b = rng.normal(0, 0.02, N)
     y = ora.fp8_linear(a, Wq, sw, b)
-    qa, sa = ora.fp8_row_scale_and_codes(a.astype(np.float32))
+    qa, sa = ora.fp8_activation_codes(a)
     for m in range(3):
         for n in range(N):
             acc = 0.0
             for k in range(K):
                 acc += qa[m, k] * Wq[n, k]
             assert abs(y[m, n] - (acc * float(sa[m]) * float(sw[n]) + b[n])) <= 1e-12 * (1 + abs(y[m, n]))
-    exact = a @ Wd.T + b
+    exact = a.astype(np.float64) @ Wd.T + b
     bound = (2.0 ** -4 * np.abs(a) + 2.0 ** -10 * sa.astype(np.float64)[:, None]) @ np.abs(Wd).T + 1e-6
     assert np.all(np.abs(y - exact) <= bound)
+
+
+def pin_fp8_activation_codes(ora):
+    """Per-token activation codes: the row's amax element maps to +-448, every
+    code is within half a step of a * 448 / amax, s_a * 448 recovers amax,
+    a zero row gives zero codes and scale 1; the fp32 normalisation used for the
+    decision is the fp64 normalisation within two fp32 rounding steps."""
+    rng = np.random.default_rng(74)
+    a = rng.normal(0, 1.5, (5, 96)).astype(np.float32)
+    a[2] = 0.0
+    q, s_ = ora.fp8_activation_codes(a)
+    assert s_[2] == 1.0 and np.all(q[2] == 0)
+    for m in (0, 1, 3, 4):
+        j = int(np.argmax(np.abs(a[m])))
+        assert abs(q[m, j]) == 448.0
+        amax = float(np.abs(a[m]).max())
+        assert abs(float(s_[m]) * 448.0 - amax) <= 2.0 ** -23 * amax
+        v = a[m].astype(np.float64) * 448.0 / amax
+        step = np.where(np.abs(v) < 2.0 ** -6, 2.0 ** -9, 2.0 ** (np.floor(np.log2(np.maximum(np.abs(v), 1e-30))) - 3))
+        assert np.all(np.abs(q[m] - v) <= 0.5 * step * (1 + 1e-6))
+    h = rng.normal(0, 1, (4, 64))
+    g, be = 1 + 0.1 * rng.normal(size=64), 0.1 * rng.normal(size=64)
+    a64, mean, rstd = ora.layernorm(h, g, be, 1e-5)
+    a32 = ora.fp8_normalised32(h, mean, rstd, g, be)
+    assert a32.dtype == np.float32
+    assert np.all(np.abs(a32 - a64) <= 4 * 2.0 ** -24 * (np.abs(a64) + np.abs(be)[None, :] + 1))
+    r64, rs = ora.rmsnorm(h, g, 1e-5)
+    r32 = ora.fp8_normalised32(h, None, rs, g, None)
+    assert np.all(np.abs(r32 - r64) <= 4 * 2.0 ** -24 * (np.abs(r64) + 1))
 
 
 def pin_fp8_fused_qkv(ora):
@@ -488,7 +517,7 @@ PINS = [pin_layernorm_invariants, pin_rmsnorm_invariant, pin_norms_match_torch,
         pin_identity_weight, pin_one_hot, pin_brute_force, pin_epilogue_values,
         pin_qkv_bijection, pin_bf16_round, pin_residual_out,
         pin_run_maps_workload_inputs, pin_residual_projection, pin_e4m3_format, pin_fp8_quantisers,
-        pin_fp8_linear, pin_fp8_fused_qkv]
+        pin_fp8_linear, pin_fp8_activation_codes, pin_fp8_fused_qkv]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -501,7 +530,8 @@ def test_pin_holds(pin):
 # --------------------------------------------------------------------------
 
 ORIG = {name: getattr(core, name) for name in ("layernorm", "rmsnorm", "split_qkv_head_major", "run",
-                                               "e4m3_round", "fp8_row_scale_and_codes", "fp8_linear")}
+                                               "e4m3_round", "fp8_row_scale_and_codes", "fp8_activation_codes",
+                                               "fp8_linear", "fp8_normalised32")}
 
 
 def _ln_unbiased(h, gamma, beta, eps):
@@ -681,6 +711,21 @@ def _fp8_linear_no_weight_scale(a, Wq, w_scale, bias=None):
     return ORIG["fp8_linear"](a, Wq, np.ones_like(np.asarray(w_scale)), bias)
 
 
+def _fp8_act_per_tensor(a32):
+    a32 = np.asarray(a32, np.float32)
+    q, s_ = ORIG["fp8_activation_codes"](a32.reshape(1, -1))
+    return q.reshape(a32.shape), np.full(a32.shape[0], s_[0], np.float32)
+
+
+def _fp8_act_no_dequant(a32):
+    q, s_ = ORIG["fp8_activation_codes"](a32)
+    return q, np.ones_like(s_)
+
+
+def _fp8_norm32_drops_beta(h, mean, rstd, gamma, beta):
+    return ORIG["fp8_normalised32"](h, mean, rstd, gamma, None)
+
+
 MUTANTS = {
     "variance_divides_by_K_minus_1": ("layernorm", _ln_unbiased),
     "eps_outside_sqrt": ("layernorm", _ln_eps_outside),
@@ -713,6 +758,9 @@ MUTANTS = {
     "fp8_scale_per_tensor": ("fp8_row_scale_and_codes", _fp8_per_tensor),
     "fp8_scale_inverted": ("fp8_row_scale_and_codes", _fp8_scale_inverted),
     "fp8_weight_scale_dropped": ("fp8_linear", _fp8_linear_no_weight_scale),
+    "fp8_activation_scale_per_tensor": ("fp8_activation_codes", _fp8_act_per_tensor),
+    "fp8_activation_scale_dropped": ("fp8_activation_codes", _fp8_act_no_dequant),
+    "fp8_normalisation_drops_beta": ("fp8_normalised32", _fp8_norm32_drops_beta),
 }
 
 
