@@ -201,13 +201,17 @@ class Bed:
         self.w = w
         self.dev = torch.device("cuda", local)
         self.inputs = synthetic.make_inputs(w, seed=0) if inputs is None else inputs
-        self.per_copy = sum(t.numel() * t.element_size() for k, t in self.inputs.items()
-                            if k in ("x", "residual", "W"))
+        wbytes = 1 if w.op == "qkv_fp8" else 2   # the FP8 form streams one byte per weight
+        self.per_copy = sum(t.numel() * (wbytes if k == "W" else t.element_size())
+                            for k, t in self.inputs.items() if k in ("x", "residual", "W"))
         self.l2 = torch.cuda.get_device_properties(self.dev).L2_cache_size
         self.R = max(1, min(16, -(-3 * self.l2 // self.per_copy)))
         self.copies = [{k: v.to(self.dev) for k, v in self.inputs.items()} for _ in range(self.R)]
         # shape auto-tuning: the first call below times the candidate plans
         self.h = fnl.Handle(local, max_tokens=w.M, max_n=w.N, tune=tune and path == "auto", path=path)
+        if w.op == "qkv_fp8":   # FP8 weights from the library's own quantiser
+            for c in self.copies:
+                c["W_fp8"], c["w_scale"] = fnl.quantize_weight_fp8(self.h, c.pop("W"))
         self.outs = [fnl.run_workload(self.h, w, c, stats=True) for c in self.copies]
         self.h.check()
         self.plan = self.h.last_plan()
@@ -217,6 +221,11 @@ class Bed:
         fnl, w, c, o = self.fnl, self.w, self.copies[i], self.outs[i]
         if w.op == "residual":
             fnl.linear_add_residual(self.h, c["x"], c["W"], c["residual"], bias=c.get("bias_out"), out=o["out"])
+        elif w.op == "qkv_fp8":
+            fnl.add_norm_qkv_fp8(self.h, c["x"], c["residual"], c["gamma"], c.get("beta"), c["W_fp8"], c["w_scale"],
+                                 w.Hq, w.Hkv, w.D, norm=w.norm, eps=w.eps, bias=c.get("bias_out"),
+                                 residual_out=o["residual_out"], q=o["q"], k=o["k"], v=o["v"], mean_out=o["mean"],
+                                 rstd_out=o["rstd"])
         elif w.op == "qkv":
             fnl.add_norm_qkv(self.h, c["x"], c["residual"], c["gamma"], c.get("beta"), c["W"], w.Hq, w.Hkv, w.D,
                              norm=w.norm, eps=w.eps, bias=c.get("bias_out"), residual_out=o["residual_out"],
@@ -243,6 +252,11 @@ class Bed:
         norm = self.fnl.NORMS[w.norm]
         eps = ctypes.c_float(w.eps)
         common = (P(c["x"]), P(c["residual"]))
+        if w.op == "qkv_fp8":
+            return L.fnl_add_norm_qkv_fp8, (self.h.ptr, st, *common, P(o["residual_out"]), P(c["gamma"]),
+                                            P(c.get("beta")), norm, eps, P(c["W_fp8"]), P(c["w_scale"]),
+                                            P(c.get("bias_out")), w.M, w.K, w.Hq, w.Hkv, w.D, P(o["q"]), P(o["k"]),
+                                            P(o["v"]), P(o["mean"]), P(o["rstd"]))
         if w.op == "qkv":
             return L.fnl_add_norm_qkv, (self.h.ptr, st, *common, P(o["residual_out"]), P(c["gamma"]),
                                         P(c.get("beta")), norm, eps, P(c["W"]), P(c.get("bias_out")), w.M, w.K,
@@ -376,7 +390,7 @@ def bench_fnl(w, steps, warmup, world, rank, local, tune=True, path="auto"):
 
     unit, per_step, bound = units(w)
     value = per_step * steps * world / (ms_max / 1e3)
-    launches_per_step = 2 if w.norm == "layernorm" else 1
+    launches_per_step = 2 if (w.norm == "layernorm" or w.op == "qkv_fp8") else 1   # + the stats pre-pass
     host_us = bed.host_us_per_call(50 if w.flops() < 1e12 else 10)
 
     # e2e: through the public binding, host buffers, copies inside the timed region
@@ -384,7 +398,7 @@ def bench_fnl(w, steps, warmup, world, rank, local, tune=True, path="auto"):
     x_h = inputs["x"].pin_memory()
     r_h = inputs["residual"].pin_memory()
     c0, o0 = bed.copies[0], bed.outs[0]
-    out_keys = ("q", "k", "v") if w.op == "qkv" else ("out",)
+    out_keys = ("q", "k", "v") if w.op in ("qkv", "qkv_fp8") else ("out",)
     host_out = {k: torch.empty(o0[k].shape, dtype=o0[k].dtype, pin_memory=True) for k in out_keys}
     if "residual_out" in o0:
         host_out["residual_out"] = torch.empty(o0["residual_out"].shape, dtype=torch.bfloat16, pin_memory=True)
@@ -422,10 +436,10 @@ def bench_fnl(w, steps, warmup, world, rank, local, tune=True, path="auto"):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "e4m3" if w.op == "qkv_fp8" else "bf16",
         "data": "synthetic (seeded normal draws rounded to bf16; random-init weights)",
         "config": {"workload": w.name, "op": w.op, "norm": w.norm, "M": w.M, "K": w.K, "N": w.N,
-                   **({"Hq": w.Hq, "Hkv": w.Hkv, "D": w.D} if w.op == "qkv" else {}),
+                   **({"Hq": w.Hq, "Hkv": w.Hkv, "D": w.D} if w.op in ("qkv", "qkv_fp8") else {}),
                    **({"I": w.I} if w.op == "swiglu" else {}),
                    **({"seqs": len(w.seq_lens)} if w.seq_lens else {}),
                    "l2": f"inputs larger than L2: {R} rotating copies of W/x/residual "
@@ -513,6 +527,9 @@ def oracle_rate(w, budget_s=10.0, max_steps=None, rows=None):
     cores = len(os.sched_getaffinity(0))
     rows = min(w.M, 256) if rows is None else rows
     inputs = synthetic.make_inputs(w, rows=rows)
+    if w.op == "qkv_fp8":   # the FP8 weights: an offline step, outside the timed passes
+        codes, scale = oracle.quantize_weight_fp8(inputs["W"].double().numpy())
+        inputs["W_fp8"], inputs["w_scale"] = codes, scale
     ws = synthetic.Workload(**{**w.__dict__, "M": rows, "seq_lens": None})
     unit, per_step, _ = units(w)
     n, t0 = 0, time.perf_counter()

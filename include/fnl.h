@@ -198,6 +198,37 @@ fnl_status fnl_add_bias_norm_gelu(fnl_handle* h, fnl_stream stream,
                                   int M, int K, int N,
                                   fnl_bf16* out, float* mean_out, float* rstd_out);
 
+/* FP8 (W8A8) form of fnl_add_norm_qkv for decode-sized batches (M <= 128),
+ * on the e4m3 tensor cores (tcgen05.mma kind::f8f6f4). TensorRT-LLM
+ * 深度工程实践, §3.3 FP4/FP8 动态量化加速: W8A8_FP8 with activation ranges taken
+ * from runtime statistics (no calibration). Per token m, the normalised row a
+ * (as in fnl_add_norm_qkv, in fp32) is quantised with its own scale,
+ * s_a[m] = max_k |a[m, k]| / 448, codes e4m3(a * 448 / max|a|) (round to
+ * nearest even, saturating at +-448); W is given as e4m3 codes Wq [N, K] (one
+ * byte each, K-contiguous) with one scale per row, w_scale [N] (fp32, see
+ * fnl_quantize_weight_fp8), and
+ *   y[m, n] = s_a[m] w_scale[n] sum_k code_a[m, k] Wq[n, k] (+ bias[n]),
+ * accumulated in fp32, then the QKV split as in fnl_add_norm_qkv. Two kernels
+ * per call: a pre-pass (one CTA per token: residual_out, the statistics and
+ * the token's amax) and the small-M split-K kernel's FP8 form. Requirements as
+ * for fnl_add_norm_qkv plus: K a multiple of 16, Wq 16-byte aligned, w_scale
+ * 16-byte aligned; M > 128 or a forced tile path -> FNL_ERR_UNSUPPORTED. */
+fnl_status fnl_add_norm_qkv_fp8(fnl_handle* h, fnl_stream stream,
+                                const fnl_bf16* x, const fnl_bf16* residual, fnl_bf16* residual_out,
+                                const fnl_bf16* gamma, const fnl_bf16* beta, fnl_norm norm, float eps,
+                                const uint8_t* Wq, const float* w_scale, const fnl_bf16* bias,
+                                int M, int K, int Hq, int Hkv, int D,
+                                fnl_bf16* q, fnl_bf16* k, fnl_bf16* v,
+                                float* mean_out, float* rstd_out);
+
+/* Static per-output-channel FP8 quantisation of a bf16 weight W [N, K] for
+ * the FP8 form: w_scale[n] = max_k |W[n, k]| / 448 (1 for an all-zero row) and
+ * Wq[n, k] = e4m3(W[n, k] / w_scale[n]), both divisions IEEE fp32, round to
+ * nearest even, saturating. One CTA per row on `stream`. K a multiple of 8;
+ * W 16-byte, Wq 8-byte, w_scale 4-byte aligned; outputs must not overlap W. */
+fnl_status fnl_quantize_weight_fp8(fnl_handle* h, fnl_stream stream, const fnl_bf16* W, int N, int K,
+                                   uint8_t* Wq, float* w_scale);
+
 /* Residual-stream projection: the layer's output projection (attention o_proj
  * or MLP down_proj) with the residual add fused into its epilogue, which closes
  * the layer's residual loop. These are the row-split projections of

@@ -31,6 +31,7 @@ QKV = "qkv"
 SWIGLU = "swiglu"
 GELU = "gelu"
 RESIDUAL = "residual"   # residual-stream projection: out = residual + a W^T (+ bias)
+QKV_FP8 = "qkv_fp8"     # the QKV op with FP8 (e4m3) weights and activations; W is drawn in bf16
 NONORM = "none"
 
 
@@ -70,6 +71,9 @@ class Workload:
         M, K, N = self.M, self.K, self.N
         if self.op == RESIDUAL:
             return float(M * K * 2 + 2 * M * N * 2 + N * K * 2 + (N * 2 if self.has_bias_out else 0))
+        if self.op == QKV_FP8:   # one byte per weight plus a 4-byte scale per row
+            b = 2 * M * K * 2 + M * K * 2 + N * K + N * 4 + M * N * 2
+            return float(b + K * 2 * (2 if self.norm == LAYERNORM else 1) + (N * 2 if self.has_bias_out else 0))
         b = 2 * M * K * 2 + M * K * 2 + N * K * 2 + M * self.n_out * 2
         b += K * 2 * (2 if self.norm == LAYERNORM else 1)
         if self.has_bias_in:
@@ -107,7 +111,21 @@ def workloads() -> dict:
     w["c5_70b_rms_qkv_ragged"] = qkv(
         "c5_70b_rms_qkv_ragged", sum(lens), 8192, 64, 8, 128, RMSNORM, seq_lens=lens)
     w.update(residual_workloads())
+    w.update(fp8_workloads())
     return w
+
+
+def fp8_workloads() -> dict:
+    """The decode QKV shapes with FP8 (e4m3) weights and activations: Llama-3-8B
+    (M=32, K=4096, N=6144) and Llama-2-70B (M=32, K=8192, N=10240), RMSNorm.
+    The bf16 W is drawn as for the bf16 op; its FP8 codes and scales are
+    derived from it by the quantiser under test (or the oracle's)."""
+    return {
+        "c2_decode_rms_qkv_fp8": Workload("c2_decode_rms_qkv_fp8", QKV_FP8, RMSNORM, 32, 4096, 6144,
+                                          Hq=32, Hkv=8, D=128),
+        "c5_70b_rms_qkv_m32_fp8": Workload("c5_70b_rms_qkv_m32_fp8", QKV_FP8, RMSNORM, 32, 8192, 10240,
+                                           Hq=64, Hkv=8, D=128),
+    }
 
 
 def residual_workloads() -> dict:
@@ -168,6 +186,9 @@ def make_custom(op: str, norm: str, M: int, K: int, *, Hq=0, Hkv=0, D=0, I=0, N=
     elif op == QKV:
         w = qkv(f"custom_qkv_{M}x{K}", M, K, Hq, Hkv, D, norm, eps=eps,
                 has_bias_in=bias_in, has_bias_out=bias_out, x_loc=x_loc)
+    elif op == QKV_FP8:
+        w = Workload(f"custom_qkv_fp8_{M}x{K}", QKV_FP8, norm, M, K, (Hq + 2 * Hkv) * D, Hq=Hq, Hkv=Hkv, D=D,
+                     eps=eps, has_bias_in=bias_in, has_bias_out=bias_out, x_loc=x_loc)
     elif op == SWIGLU:
         w = Workload(f"custom_swiglu_{M}x{K}", SWIGLU, norm, M, K, 2 * I, I=I, eps=eps,
                      has_bias_in=bias_in, has_bias_out=bias_out, x_loc=x_loc)

@@ -16,7 +16,7 @@ def declared_symbols():
     with open(os.path.join(ROOT, "include", "fnl.h")) as f:
         text = f.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(fnl_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(fnl_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_boundary():

@@ -31,7 +31,8 @@ struct OpParams {
   bf16* k;
   bf16* v;
   bf16* out;
-  const float4* stats8;  // FP8 ops: per token (mean, rstd, activation scale s_a, 448 / amax), from the pre-pass
+  const float4* stats8;  // FP8 ops: per token (mean, rstd, dequantisation scale, 448 / amax), from the pre-pass
+  int fp8_rms;           // FP8 ops: 1 = RMSNorm (codes of h * gamma, rstd in the scale), 0 = LayerNorm
   const float* w_scale;  // FP8 ops: per W row dequantisation scale s_w [N] (null for the bf16 ops)
   const bf16* res_in;    // residual-stream projection: the residual [M][N] added in the epilogue
                          // (may be the same buffer as out: each element is read, then written,
@@ -206,7 +207,8 @@ __device__ __forceinline__ uint4 ldcg16(const void* p) {
 // Store 8 consecutive output columns [n, n+8) of row m (QKV, GELU or residual
 // epilogue). acc is the raw fp32 accumulator, scale the deferred RMSNorm 1/rms
 // (1 for LN and for the residual-stream projection).
-// FP8 ops: the accumulator holds sum of code products; y = acc s_a[m] s_w[n].
+// FP8 ops: the accumulator holds sum of code products; y = acc s_a[m] s_w[n]
+// (s_a includes rstd for RMSNorm).
 __device__ __forceinline__ void fp8_dequant8(const OpParams& p, int m, int n, float (&y)[8]) {
   const float sa = p.stats8[m].z;
   const float4 w0 = __ldg(reinterpret_cast<const float4*>(p.w_scale + n));

@@ -107,9 +107,12 @@ __device__ __forceinline__ float block_max_256(float v, float* red) {
 // 深度工程实践, §3.3 FP4/FP8 动态量化加速: activation ranges from runtime
 // statistics). One CTA per row: h = x + r (+ bias_in) in fp32, residual_out =
 // bf16(h), the row's statistics (LayerNorm: two-pass mean and variance;
-// RMSNorm: mean 0, mean of h^2), then a = (h - mean) rstd gamma + beta computed
-// exactly as the FP8 converters compute it, and its amax. Writes
-// stats8[row] = (mean, rstd, s_a = amax / 448, 448 / amax) (1, 1 for a zero row).
+// RMSNorm: mean of h^2), then the value the FP8 converters quantise, computed
+// exactly as they compute it, and its amax: LayerNorm a = (h - mean) rstd
+// gamma + beta; RMSNorm a = h gamma (1/rms is a positive per-token factor, so
+// it joins the token's dequantisation scale instead). Writes stats8[row] =
+// (mean, rstd, dequantisation scale, 448 / amax) with the scale amax / 448
+// (times rstd for RMSNorm); 1 and 1 for a zero row.
 template <int MAXV, bool RMS>
 __global__ void __launch_bounds__(kK1Threads) k1_fp8_prepass(const bf16* __restrict__ x,
                                                              const bf16* __restrict__ residual,
@@ -186,7 +189,8 @@ __global__ void __launch_bounds__(kK1Threads) k1_fp8_prepass(const bf16* __restr
       const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const f32x2 a = fma2(mul2(sub2(h[i][e], mu2), rs2), bf2_to_f2(gw[e]), bf2_to_f2(bw[e]));
+        const f32x2 a = RMS ? mul2(h[i][e], bf2_to_f2(gw[e]))
+                            : fma2(mul2(sub2(h[i][e], mu2), rs2), bf2_to_f2(gw[e]), bf2_to_f2(bw[e]));
         float lo, hi;
         unpk2(a, lo, hi);
         amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
@@ -197,7 +201,7 @@ __global__ void __launch_bounds__(kK1Threads) k1_fp8_prepass(const bf16* __restr
   if (threadIdx.x == 0) {
     const float sa = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
     const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
-    stats8[row] = make_float4(mean, rstd, sa, inv);
+    stats8[row] = make_float4(mean, rstd, RMS ? rstd * sa : sa, inv);
     if (mean_out) mean_out[row] = mean;
     if (rstd_out) rstd_out[row] = rstd;
   }

@@ -623,9 +623,10 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     // Converter warp cw owns positions cw, cw + 4, ... as below. A lane task is
     // (token row, 16-byte e4m3 chunk j of the row's 64): it reads the bf16
     // chunks 2j and 2j + 1 of x and the residual, forms h (+ bias_in), normalises
-    // with the pre-pass statistics, a = (h - mean) rstd gamma + beta (the
-    // pre-pass computes the same expression for the token's amax), and stores
-    // e4m3(a * 448 / amax) (round to nearest even, saturating).
+    // with the pre-pass statistics, a = (h - mean) rstd gamma + beta for
+    // LayerNorm, a = h gamma for RMSNorm (the pre-pass computes the same
+    // expression for the token's amax), and stores e4m3(a * 448 / amax) (round
+    // to nearest even, saturating).
     const int cw = warp - WARP_CONV0;
     pdl_wait();   // statistics come from the pre-pass
     const int P = static_cast<int>(u1 - u0);
@@ -664,8 +665,11 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
               h0 = add2(h0, bi2[i]);
               h1 = add2(h1, bi2[i + 1]);
             }
-            const f32x2 a0 = mul2(fma2(mul2(sub2(h0, mu2), rs2), g2[i], be2[i]), inv2);
-            const f32x2 a1 = mul2(fma2(mul2(sub2(h1, mu2), rs2), g2[i + 1], be2[i + 1]), inv2);
+            // RMSNorm: codes of h * gamma (rstd joins the token's scale); LayerNorm:
+            // of the normalised value
+            const f32x2 a0 = mul2(p.fp8_rms ? mul2(h0, g2[i]) : fma2(mul2(sub2(h0, mu2), rs2), g2[i], be2[i]), inv2);
+            const f32x2 a1 =
+                mul2(p.fp8_rms ? mul2(h1, g2[i + 1]) : fma2(mul2(sub2(h1, mu2), rs2), g2[i + 1], be2[i + 1]), inv2);
             codes[hh * 2 + i / 2] = e4m3x4(a0, a1);
           }
         }

@@ -26,6 +26,7 @@ PRECISIONS = {"default": 0, "split": 1, "single": 2}
 
 EXPORTED = ("fnl_create", "fnl_destroy", "fnl_status_string", "fnl_last_error", "fnl_last_plan", "fnl_check",
             "fnl_add_norm_qkv", "fnl_add_norm_swiglu", "fnl_add_bias_norm_gelu", "fnl_linear_add_residual",
+            "fnl_add_norm_qkv_fp8", "fnl_quantize_weight_fp8",
             "fnl_add_norm_qkv_static", "fnl_check_static")
 
 
@@ -68,6 +69,8 @@ def lib() -> ctypes.CDLL:
     L.fnl_add_norm_swiglu.argtypes = [P, P, P, P, P, P, P, I, F, P, P, I, I, I, P, P, P]
     L.fnl_add_bias_norm_gelu.argtypes = [P, P, P, P, P, P, P, P, I, F, P, P, I, I, I, P, P, P]
     L.fnl_linear_add_residual.argtypes = [P, P, P, P, P, P, P, I, I, I]
+    L.fnl_add_norm_qkv_fp8.argtypes = [P, P, P, P, P, P, P, I, F, P, P, P, I, I, I, I, I, P, P, P, P, P]
+    L.fnl_quantize_weight_fp8.argtypes = [P, P, P, I, I, P, P]
     L.fnl_add_norm_qkv_static.argtypes = [P, P, P, P, P, P, I, F, P, P, I, I, I, I, I, P, P, P, P, P]
     L.fnl_check_static.argtypes = [P]
     for name in EXPORTED:
@@ -249,12 +252,69 @@ def linear_add_residual(h: Handle, a, W, residual, bias=None, out=None, stream=N
     return {"out": out}
 
 
+def quantize_weight_fp8(h: Handle, W, stream=None):
+    """fnl_quantize_weight_fp8: (Wq uint8 [N, K] e4m3 codes, w_scale fp32 [N])."""
+    _need(W, "W")
+    if W.dim() != 2:
+        raise ValueError("W must be [N, K]")
+    N, K = W.shape
+    Wq = torch.empty(N, K, dtype=torch.uint8, device=W.device)
+    w_scale = torch.empty(N, dtype=torch.float32, device=W.device)
+    st = lib().fnl_quantize_weight_fp8(h.ptr, _stream_ptr(stream), _p(W), N, K, _p(Wq), _p(w_scale))
+    if st != FNL_OK:
+        h._raise(st, "fnl_quantize_weight_fp8")
+    return Wq, w_scale
+
+
+def add_norm_qkv_fp8(h: Handle, x, residual, gamma, beta, Wq, w_scale, Hq, Hkv, D, norm="rmsnorm", eps=1e-5,
+                     bias=None, residual_out=None, q=None, k=None, v=None, mean_out=None, rstd_out=None,
+                     stream=None):
+    """fnl_add_norm_qkv_fp8: Wq uint8 [N, K] e4m3 codes, w_scale fp32 [N].
+    Returns dict(residual_out, q, k, v, mean, rstd)."""
+    M, K = x.shape
+    _need(x, "x", (M, K))
+    _need(residual, "residual", (M, K))
+    _need(gamma, "gamma", (K,))
+    _need(beta, "beta", (K,))
+    N = (Hq + 2 * Hkv) * D
+    _need(Wq, "Wq", (N, K), torch.uint8)
+    _need(w_scale, "w_scale", (N,), torch.float32)
+    _need(bias, "bias", (N,))
+    if norm not in NORMS:
+        raise ValueError(f"norm must be one of {list(NORMS)}")
+    residual_out = torch.empty_like(x) if residual_out is None else residual_out
+    q = torch.empty(Hq, M, D, dtype=torch.bfloat16, device=x.device) if q is None else q
+    k = torch.empty(Hkv, M, D, dtype=torch.bfloat16, device=x.device) if k is None else k
+    v = torch.empty(Hkv, M, D, dtype=torch.bfloat16, device=x.device) if v is None else v
+    _need(residual_out, "residual_out", (M, K))
+    _need(q, "q", (Hq, M, D)); _need(k, "k", (Hkv, M, D)); _need(v, "v", (Hkv, M, D))
+    if rstd_out is not None:
+        _need(rstd_out, "rstd_out", (M,), torch.float32)
+    if mean_out is not None:
+        _need(mean_out, "mean_out", (M,), torch.float32)
+    st = lib().fnl_add_norm_qkv_fp8(h.ptr, _stream_ptr(stream), _p(x), _p(residual), _p(residual_out), _p(gamma),
+                                    _p(beta), NORMS[norm], float(eps), _p(Wq), _p(w_scale), _p(bias), M, K, Hq,
+                                    Hkv, D, _p(q), _p(k), _p(v), _p(mean_out), _p(rstd_out))
+    if st != FNL_OK:
+        h._raise(st, "fnl_add_norm_qkv_fp8")
+    return {"residual_out": residual_out, "q": q, "k": k, "v": v, "mean": mean_out, "rstd": rstd_out}
+
+
 def run_workload(h: Handle, w, dev: dict, stats: bool = True, stream=None) -> dict:
     """Run a synthetic.Workload on device tensors `dev` (same keys as
     synthetic.make_inputs). Allocates the outputs and statistics buffers."""
     if w.op == "residual":
         return linear_add_residual(h, dev["x"], dev["W"], dev["residual"], bias=dev.get("bias_out"), stream=stream)
     M = dev["x"].shape[0]
+    if w.op == "qkv_fp8":   # dev["W_fp8"]: e4m3 codes (float8_e4m3fn or uint8), dev["w_scale"]: fp32 [N]
+        rstd = torch.empty(M, dtype=torch.float32, device=dev["x"].device) if stats else None
+        mean = (torch.empty(M, dtype=torch.float32, device=dev["x"].device)
+                if stats and w.norm == "layernorm" else None)
+        Wq = dev["W_fp8"]
+        Wq = Wq.view(torch.uint8) if Wq.dtype != torch.uint8 else Wq
+        return add_norm_qkv_fp8(h, dev["x"], dev["residual"], dev["gamma"], dev.get("beta"), Wq, dev["w_scale"],
+                                w.Hq, w.Hkv, w.D, norm=w.norm, eps=w.eps, bias=dev.get("bias_out"), mean_out=mean,
+                                rstd_out=rstd, stream=stream)
     rstd = torch.empty(M, dtype=torch.float32, device=dev["x"].device) if stats else None
     mean = (torch.empty(M, dtype=torch.float32, device=dev["x"].device)
             if stats and w.norm == "layernorm" else None)
