@@ -103,6 +103,29 @@ __device__ __forceinline__ float block_max_256(float v, float* red) {
   return m;
 }
 
+// Sum and max over the block's 256 threads with one shared-memory exchange.
+__device__ __forceinline__ void block_sum_max_256(float& s, float& m, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s += __shfl_xor_sync(0xffffffffu, s, o);
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) {
+    red[warp] = s;
+    red[kK1Threads / 32 + warp] = m;
+  }
+  __syncthreads();
+  s = 0.f;
+  m = 0.f;
+#pragma unroll
+  for (int w = 0; w < kK1Threads / 32; ++w) {
+    s += red[w];
+    m = fmaxf(m, red[kK1Threads / 32 + w]);
+  }
+}
+
 // FP8 pre-pass of the fused ops (per-token dynamic quantisation, TensorRT-LLM
 // 深度工程实践, §3.3 FP4/FP8 动态量化加速: activation ranges from runtime
 // statistics). One CTA per row: h = x + r (+ bias_in) in fp32, residual_out =
@@ -125,13 +148,14 @@ __global__ void __launch_bounds__(kK1Threads) k1_fp8_prepass(const bf16* __restr
                                                              float* __restrict__ rstd_out, int M, int K,
                                                              float eps) {
   pdl_launch_dependents();
-  __shared__ float red[kK1Threads / 32];
+  __shared__ float red[2 * kK1Threads / 32];
   const int row = blockIdx.x;
   if (row >= M) return;
   const int nvec = K >> 3;
   const size_t rbase = static_cast<size_t>(row) * K;
   f32x2 h[MAXV][4];
   float s = 0.f;
+  float amax = 0.f;   // RMSNorm: max |h gamma|, taken in the first pass
 #pragma unroll
   for (int i = 0; i < MAXV; ++i) {
     const int v = threadIdx.x + i * kK1Threads;
@@ -150,6 +174,16 @@ __global__ void __launch_bounds__(kK1Threads) k1_fp8_prepass(const bf16* __restr
         s += RMS ? fmaf(lo, lo, hi * hi) : lo + hi;
         ho[e] = f2_to_bf2(h[i][e]);
       }
+      if (RMS) {   // the value the converters quantise: h * gamma
+        const uint4 gv = ldg16(gamma + v * 8);
+        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float lo, hi;
+          unpk2(mul2(h[i][e], bf2_to_f2(gw[e])), lo, hi);
+          amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+        }
+      }
       *reinterpret_cast<uint4*>(residual_out + rbase + v * 8) = make_uint4(ho[0], ho[1], ho[2], ho[3]);
     } else {
 #pragma unroll
@@ -158,7 +192,8 @@ __global__ void __launch_bounds__(kK1Threads) k1_fp8_prepass(const bf16* __restr
   }
   float mean = 0.f, rstd;
   if (RMS) {
-    rstd = 1.f / sqrtf(block_sum_256(s, red) / static_cast<float>(K) + eps);
+    block_sum_max_256(s, amax, red);
+    rstd = 1.f / sqrtf(s / static_cast<float>(K) + eps);
   } else {
     mean = block_sum_256(s, red) / static_cast<float>(K);
     float s2 = 0.f;
@@ -179,9 +214,8 @@ __global__ void __launch_bounds__(kK1Threads) k1_fp8_prepass(const bf16* __restr
     rstd = 1.f / sqrtf(block_sum_256(s2, red) / static_cast<float>(K) + eps);
   }
   const f32x2 mu2 = pk2(mean, mean), rs2 = pk2(rstd, rstd);
-  float amax = 0.f;
 #pragma unroll
-  for (int i = 0; i < MAXV; ++i) {
+  for (int i = 0; i < MAXV && !RMS; ++i) {   // LayerNorm: amax of the normalised value
     const int v = threadIdx.x + i * kK1Threads;
     if (v < nvec) {
       const uint4 gv = ldg16(gamma + v * 8);
@@ -189,15 +223,14 @@ __global__ void __launch_bounds__(kK1Threads) k1_fp8_prepass(const bf16* __restr
       const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const f32x2 a = RMS ? mul2(h[i][e], bf2_to_f2(gw[e]))
-                            : fma2(mul2(sub2(h[i][e], mu2), rs2), bf2_to_f2(gw[e]), bf2_to_f2(bw[e]));
+        const f32x2 a = fma2(mul2(sub2(h[i][e], mu2), rs2), bf2_to_f2(gw[e]), bf2_to_f2(bw[e]));
         float lo, hi;
         unpk2(a, lo, hi);
         amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
       }
     }
   }
-  amax = block_max_256(amax, red);
+  if (!RMS) amax = block_max_256(amax, red);
   if (threadIdx.x == 0) {
     const float sa = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
     const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;

@@ -52,6 +52,9 @@ constexpr int MAX_MPAD = 128;
 // during it lengthens the chain by more than it saves (decode 32 x 6144 x 4096:
 // 18.7 us per call with 8 stages, 18.2 with 2, 17.7 with none).
 constexpr int PREWAIT_STAGES = 0;
+// The FP8 form's predecessor is always its own light pre-pass (one CTA per
+// token), so its whole first ring of weight stages streams before the wait.
+constexpr int PREWAIT_STAGES_FP8 = MAX_STAGES;
 
 struct Ctrl {
   uint64_t full_w[MAX_STAGES], full_x[MAX_STAGES], conv[MAX_STAGES], empty[MAX_STAGES];
@@ -430,7 +433,8 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
       };
       // Weight stages that may stream before griddepcontrol.wait (weights are
       // never written by the previous kernel; activations are read only after it).
-      const int npre0 = npre < PREWAIT_STAGES ? npre : PREWAIT_STAGES;
+      constexpr int kPre = FP8 ? PREWAIT_STAGES_FP8 : PREWAIT_STAGES;
+      const int npre0 = npre < kPre ? npre : kPre;
       for (int q = 0; q < npre0; ++q) {
         issue_w(cw);
         step(cw);
@@ -629,6 +633,21 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     // to nearest even, saturating).
     const int cw = warp - WARP_CONV0;
     pdl_wait();   // statistics come from the pre-pass
+    // a lane's tasks are rows (lane >> 2) + 8 i, all with chunk j = lane & 3:
+    // their (mean, rstd, 448 / amax) are loaded once
+    constexpr int kRowsPerLane = MAX_MPAD / 8;
+    float smu[kRowsPerLane], srs[kRowsPerLane], sinv[kRowsPerLane];
+#pragma unroll
+    for (int i = 0; i < kRowsPerLane; ++i) {
+      const int row = (lane >> 2) + 8 * i;
+      smu[i] = srs[i] = sinv[i] = 0.f;
+      if (row < M) {
+        const float4 st = p.stats8[row];
+        smu[i] = st.x;
+        srs[i] = st.y;
+        sinv[i] = st.w;
+      }
+    }
     const int P = static_cast<int>(u1 - u0);
     int s = cw;
     uint32_t ph = 0;
@@ -642,10 +661,11 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
       bf16* vec = vecs + s * 3 * kVecElems;
       if (K - kb * BK < BK) zero_vec_tails(vec, kVecElems, K - kb * BK);
       const uint32_t vaddr = smem_u32(vec);
-      for (int task = lane; task < M * 4; task += 32) {
-        const int row = task >> 2, j = task & 3;
-        const float4 st = __ldg(p.stats8 + row);
-        const f32x2 mu2 = pk2(st.x, st.x), rs2 = pk2(st.y, st.y), inv2 = pk2(st.w, st.w);
+#pragma unroll
+      for (int i = 0; i < kRowsPerLane; ++i) {
+        const int row = (lane >> 2) + 8 * i, j = lane & 3;
+        if (row >= M) break;
+        const f32x2 mu2 = pk2(smu[i], smu[i]), rs2 = pk2(srs[i], srs[i]), inv2 = pk2(sinv[i], sinv[i]);
         uint32_t codes[4];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {

@@ -16,9 +16,12 @@
 //
 // Warp roles (14 warps per CTA): 0 TMA producer (own tiles only), 1 TMEM
 // (allocated for the pair) and, in the even CTA, UMMA issuer; 2-5 epilogue
-// (own 128 rows); 6-13 converters. A stage is ready for the UMMA when both
-// CTAs' converters have built their operand and seen their own weight half
-// land: every converter warp of both CTAs arrives on the even CTA's conv[s]
+// (own 128 rows); 6-13 converters, in two groups of four that take alternate
+// stages (the conversion latency of one stage overlaps the next; with one
+// group the fused kernel ran at half the tensor rate of the same pipeline
+// without converters). A stage is ready for the UMMA when both CTAs'
+// converters have built their operand and seen their own weight half land:
+// every converter warp of the stage's group in both CTAs arrives on the even CTA's conv[s]
 // after waiting for its CTA's full_x[s] and full_w[s], so no tensor copy ever
 // signals the other CTA and each CTA drains only its own copies. The UMMA
 // commits arrive on both CTAs' empty[s] / tfull (multicast commit); the
@@ -48,6 +51,9 @@ constexpr int VEC_STAGE_BYTES = 3 * VEC * 2;
 constexpr int VEC_BYTES = STAGES * VEC_STAGE_BYTES;
 constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_EPI0 = 2, NUM_EPI_WARPS = 4;
 constexpr int WARP_CONV0 = 6, NUM_CONV_WARPS = 8;
+constexpr int CONV_GROUPS = 2;                                          // stages converted at once
+constexpr int CONV_GROUP_THREADS = NUM_CONV_WARPS / CONV_GROUPS * 32;   // 128
+constexpr int CONV_ROWS_PER_PASS = CONV_GROUP_THREADS / 4;              // 32 rows x 4 chunks
 constexpr int NUM_THREADS = (WARP_CONV0 + NUM_CONV_WARPS) * 32;   // 448
 constexpr int TMEM_COLS = 512;
 constexpr int GROUP_M = 8;         // pair rows (of 256 tokens) sharing a W tile while it is hot in L2
@@ -57,7 +63,7 @@ struct Ctrl {
   uint64_t tfull, tempty, sfull[2], efree[2], drain;
   uint32_t tmem_base;
   int abort_flag;
-  float rs[2][BM];
+  float rs[2][CONV_GROUPS][BM];   // RMSNorm: per tile buffer, per converter group, sum of h^2 per row
 };
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + VEC_BYTES + static_cast<int>(sizeof(Ctrl)) + 1024;
 
@@ -110,7 +116,7 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&ctrl->full_w[s], 1);
       mbar_init(&ctrl->full_x[s], 1);
-      mbar_init(&ctrl->conv[s], 2 * NUM_CONV_WARPS);   // (even CTA) converter warps of both CTAs
+      mbar_init(&ctrl->conv[s], 2 * NUM_CONV_WARPS / CONV_GROUPS);   // (even CTA) one group's warps of both CTAs
       mbar_init(&ctrl->empty[s], 1);                   // multicast UMMA commit
     }
     mbar_init(&ctrl->tfull, 1);
@@ -304,7 +310,10 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
           if (lane == 0) abort_pair();
           break;
         }
-        scale = ctrl->rs[b][row_local];
+        float ssum = 0.f;
+#pragma unroll
+        for (int g = 0; g < CONV_GROUPS; ++g) ssum += ctrl->rs[b][g][row_local];   // fixed order
+        scale = 1.f / sqrtf(ssum / static_cast<float>(K) + p.eps);
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->efree[b]);   // the converters may refill rs[b]
       }
@@ -313,6 +322,7 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
       tile_coords(t, num_m2, num_n, mb2, nb);
       const int m = mb2 * 2 * BM + static_cast<int>(rank) * BM + row_local;
       const bool row_ok = m < M;
+      if (NORM == kRMSNorm && nb == 0 && row_ok && p.rstd_out != nullptr) p.rstd_out[m] = scale;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
       if (EPI == kEpiSwiGLU) {
 #pragma unroll 1
@@ -373,26 +383,34 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ converters (own 128 rows)
-    // Thread ct: 16-byte chunk c (0..3) of the 64-byte row, rows rbase and
-    // rbase + 64. 64-byte swizzle: chunk c of row r sits at c ^ ((r >> 1) & 3).
+    // Two groups of four warps: group g converts positions q = g, g + 2, ...
+    // of this CTA's (tile, k-block) sequence (stage q % STAGES), so two stages
+    // are converted at once and the conversion latency of one stage overlaps
+    // the next. Thread gt of a group (0..127): 16-byte chunk c = gt & 3 of the
+    // 64-byte row, rows rb + 32 j (rb = gt >> 2, j = 0..3). 64-byte swizzle:
+    // chunk c of row r sits at c ^ ((r >> 1) & 3). RMSNorm: each group sums h^2
+    // over its k-blocks; the epilogue adds the two groups' sums in group order.
     // Without a norm (residual-stream projection) the warps only relay the
     // stage's readiness to the even CTA.
+    constexpr int RPT = BM / CONV_ROWS_PER_PASS;   // rows per thread (4)
     const int ct = threadIdx.x - WARP_CONV0 * 32;   // 0..255
-    const int c = ct & 3;
-    const int rbase = ct >> 2;                       // 0..63
+    const int grp = ct / CONV_GROUP_THREADS;          // 0..CONV_GROUPS-1
+    const int gt = ct - grp * CONV_GROUP_THREADS;     // 0..127
+    const int c = gt & 3;
+    const int rb = gt >> 2;                           // 0..31
     if (NORM == kLayerNorm) pdl_wait();
-    uint32_t s = 0, ph = 0;
     int i = 0;
     bool ok = true;
-    for (int t = pair; t < tiles && ok; t += npairs, ++i) {
+    long long q0 = 0;   // first position of the current tile
+    for (int t = pair; t < tiles && ok; t += npairs, ++i, q0 += nkb) {
       int mb2, nb;
       tile_coords(t, num_m2, num_n, mb2, nb);
       const int mrow0 = mb2 * 2 * BM + static_cast<int>(rank) * BM;
-      float mu[2], rs[2];
-      f32x2 ss[2];
+      float mu[RPT], rs[RPT];
+      f32x2 ss[RPT];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int gm = mrow0 + rbase + 64 * j;
+      for (int j = 0; j < RPT; ++j) {
+        const int gm = mrow0 + rb + CONV_ROWS_PER_PASS * j;
         ss[j] = 0ull;
         mu[j] = 0.f;
         rs[j] = 0.f;
@@ -403,7 +421,12 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
         }
       }
       const bool write_res = (NORM == kRMSNorm) && nb == 0;
-      for (int kb = 0; kb < nkb; ++kb) {
+      // this group's positions of the tile
+      for (long long q = q0 + ((grp - q0 % CONV_GROUPS) + CONV_GROUPS) % CONV_GROUPS; q < q0 + nkb;
+           q += CONV_GROUPS) {
+        const int kb = static_cast<int>(q - q0);
+        const int s = static_cast<int>(q % STAGES);
+        const uint32_t ph = static_cast<uint32_t>(q / STAGES) & 1u;
         if (!warp_wait(&ctrl->full_x[s], ph, abortf, p.status, kStatusWaitFull, p.wait_ns) ||
             !warp_wait(&ctrl->full_w[s], ph, abortf, p.status, kStatusWaitFull, p.wait_ns)) {
           ok = false;
@@ -419,10 +442,10 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
           if (BIAS_IN) vec_pairs(vaddr + 4 * VEC, bi2);
           const uint32_t xs = smem_u32(smem + s * STAGE_BYTES);
           const uint32_t rsm = xs + X_BYTES;
-          uint4 xv[2], rv[2];
+          uint4 xv[RPT], rv[RPT];
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int row = rbase + 64 * j;
+          for (int j = 0; j < RPT; ++j) {
+            const int row = rb + CONV_ROWS_PER_PASS * j;
             const uint32_t off = row * 64 + ((c ^ ((row >> 1) & 3)) << 4);
             xv[j] = ld_shared_v4(xs + off);
             rv[j] = ld_shared_v4(rsm + off);
@@ -431,8 +454,8 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
           auto convert_stage = [&](auto wres_tag) {
             constexpr bool WRES = decltype(wres_tag)::value;
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const int row = rbase + 64 * j;
+            for (int j = 0; j < RPT; ++j) {
+              const int row = rb + CONV_ROWS_PER_PASS * j;
               const uint32_t off = row * 64 + ((c ^ ((row >> 1) & 3)) << 4);
               uint4 hi, lo, hres;
               convert8<(NORM == kNoNorm ? kRMSNorm : NORM), BIAS_IN, SPLIT, WRES>(
@@ -456,19 +479,15 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
           if (leader) mbar_arrive(&ctrl->conv[s]);
           else mbar_arrive_remote(&ctrl->conv[s], 0);
         }
-        if (++s == STAGES) {
-          s = 0;
-          ph ^= 1;
-        }
       }
       if (!ok) {
         if (lane == 0) abort_pair();
         break;
       }
       if (NORM == kRMSNorm) {
-        float sst[2];
+        float sst[RPT];
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
+        for (int j = 0; j < RPT; ++j) {
           float lo_, hi_;
           unpk2(ss[j], lo_, hi_);
           sst[j] = lo_ + hi_;
@@ -482,15 +501,9 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
           if (lane == 0) abort_pair();
           break;
         }
-        if (c == 0) {
+        if (c == 0) {   // this group's sum of h^2 per row over its k-blocks
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int row = rbase + 64 * j;
-            const float r = 1.f / sqrtf(sst[j] / static_cast<float>(K) + p.eps);
-            ctrl->rs[b][row] = r;
-            const int gm = mrow0 + row;
-            if (write_res && p.rstd_out != nullptr && gm < M) p.rstd_out[gm] = r;
-          }
+          for (int j = 0; j < RPT; ++j) ctrl->rs[b][grp][rb + CONV_ROWS_PER_PASS * j] = sst[j];
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->sfull[b]);
