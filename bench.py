@@ -201,7 +201,7 @@ class Bed:
         self.w = w
         self.dev = torch.device("cuda", local)
         self.inputs = synthetic.make_inputs(w, seed=0) if inputs is None else inputs
-        wbytes = 1 if w.op == "qkv_fp8" else 2   # the FP8 form streams one byte per weight
+        wbytes = 1 if w.op in synthetic.FP8_OPS else 2   # the FP8 forms stream one byte per weight
         self.per_copy = sum(t.numel() * (wbytes if k == "W" else t.element_size())
                             for k, t in self.inputs.items() if k in ("x", "residual", "W"))
         self.l2 = torch.cuda.get_device_properties(self.dev).L2_cache_size
@@ -209,7 +209,7 @@ class Bed:
         self.copies = [{k: v.to(self.dev) for k, v in self.inputs.items()} for _ in range(self.R)]
         # shape auto-tuning: the first call below times the candidate plans
         self.h = fnl.Handle(local, max_tokens=w.M, max_n=w.N, tune=tune and path == "auto", path=path)
-        if w.op == "qkv_fp8":   # FP8 weights from the library's own quantiser
+        if w.op in synthetic.FP8_OPS:   # FP8 weights from the library's own quantiser
             for c in self.copies:
                 c["W_fp8"], c["w_scale"] = fnl.quantize_weight_fp8(self.h, c.pop("W"))
         self.outs = [fnl.run_workload(self.h, w, c, stats=True) for c in self.copies]
@@ -226,6 +226,16 @@ class Bed:
                                  w.Hq, w.Hkv, w.D, norm=w.norm, eps=w.eps, bias=c.get("bias_out"),
                                  residual_out=o["residual_out"], q=o["q"], k=o["k"], v=o["v"], mean_out=o["mean"],
                                  rstd_out=o["rstd"])
+        elif w.op == "swiglu_fp8":
+            fnl.add_norm_swiglu_fp8(self.h, c["x"], c["residual"], c["gamma"], c.get("beta"), c["W_fp8"],
+                                    c["w_scale"], w.I, norm=w.norm, eps=w.eps, bias=c.get("bias_out"),
+                                    residual_out=o["residual_out"], out=o["out"], mean_out=o["mean"],
+                                    rstd_out=o["rstd"])
+        elif w.op == "gelu_fp8":
+            fnl.add_bias_norm_gelu_fp8(self.h, c["x"], c["residual"], c["gamma"], c.get("beta"), c["W_fp8"],
+                                       c["w_scale"], bias_in=c.get("bias_in"), bias_out=c.get("bias_out"),
+                                       norm=w.norm, eps=w.eps, residual_out=o["residual_out"], out=o["out"],
+                                       mean_out=o["mean"], rstd_out=o["rstd"])
         elif w.op == "qkv":
             fnl.add_norm_qkv(self.h, c["x"], c["residual"], c["gamma"], c.get("beta"), c["W"], w.Hq, w.Hkv, w.D,
                              norm=w.norm, eps=w.eps, bias=c.get("bias_out"), residual_out=o["residual_out"],
@@ -257,6 +267,16 @@ class Bed:
                                             P(c.get("beta")), norm, eps, P(c["W_fp8"]), P(c["w_scale"]),
                                             P(c.get("bias_out")), w.M, w.K, w.Hq, w.Hkv, w.D, P(o["q"]), P(o["k"]),
                                             P(o["v"]), P(o["mean"]), P(o["rstd"]))
+        if w.op == "swiglu_fp8":
+            return L.fnl_add_norm_swiglu_fp8, (self.h.ptr, st, *common, P(o["residual_out"]), P(c["gamma"]),
+                                               P(c.get("beta")), norm, eps, P(c["W_fp8"]), P(c["w_scale"]),
+                                               P(c.get("bias_out")), w.M, w.K, w.I, P(o["out"]), P(o["mean"]),
+                                               P(o["rstd"]))
+        if w.op == "gelu_fp8":
+            return L.fnl_add_bias_norm_gelu_fp8, (self.h.ptr, st, *common, P(c.get("bias_in")),
+                                                  P(o["residual_out"]), P(c["gamma"]), P(c.get("beta")), norm, eps,
+                                                  P(c["W_fp8"]), P(c["w_scale"]), P(c.get("bias_out")), w.M, w.K,
+                                                  w.N, P(o["out"]), P(o["mean"]), P(o["rstd"]))
         if w.op == "qkv":
             return L.fnl_add_norm_qkv, (self.h.ptr, st, *common, P(o["residual_out"]), P(c["gamma"]),
                                         P(c.get("beta")), norm, eps, P(c["W"]), P(c.get("bias_out")), w.M, w.K,
@@ -390,7 +410,7 @@ def bench_fnl(w, steps, warmup, world, rank, local, tune=True, path="auto"):
 
     unit, per_step, bound = units(w)
     value = per_step * steps * world / (ms_max / 1e3)
-    launches_per_step = 2 if (w.norm == "layernorm" or w.op == "qkv_fp8") else 1   # + the stats pre-pass
+    launches_per_step = 2 if (w.norm == "layernorm" or w.op in synthetic.FP8_OPS) else 1   # + the stats pre-pass
     host_us = bed.host_us_per_call(50 if w.flops() < 1e12 else 10)
 
     # e2e: through the public binding, host buffers, copies inside the timed region
@@ -436,7 +456,7 @@ def bench_fnl(w, steps, warmup, world, rank, local, tune=True, path="auto"):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "e4m3" if w.op == "qkv_fp8" else "bf16",
+        "dtype": "e4m3" if w.op in synthetic.FP8_OPS else "bf16",
         "data": "synthetic (seeded normal draws rounded to bf16; random-init weights)",
         "config": {"workload": w.name, "op": w.op, "norm": w.norm, "M": w.M, "K": w.K, "N": w.N,
                    **({"Hq": w.Hq, "Hkv": w.Hkv, "D": w.D} if w.op in ("qkv", "qkv_fp8") else {}),
@@ -527,7 +547,7 @@ def oracle_rate(w, budget_s=10.0, max_steps=None, rows=None):
     cores = len(os.sched_getaffinity(0))
     rows = min(w.M, 256) if rows is None else rows
     inputs = synthetic.make_inputs(w, rows=rows)
-    if w.op == "qkv_fp8":   # the FP8 weights: an offline step, outside the timed passes
+    if w.op in synthetic.FP8_OPS:   # the FP8 weights: an offline step, outside the timed passes
         codes, scale = oracle.quantize_weight_fp8(inputs["W"].double().numpy())
         inputs["W_fp8"], inputs["w_scale"] = codes, scale
     ws = synthetic.Workload(**{**w.__dict__, "M": rows, "seq_lens": None})
@@ -570,6 +590,22 @@ def bench_reference(w, steps, warmup, world, rank, budget_s=120.0):
     }
 
 
+def eager_calls(w, path: str, n: int):
+    """N plain calls of one workload through the binding, for an ncu launch
+    capture: the launches it makes are exactly those of the product path (the
+    FP8 weight quantiser first, for FP8 workloads), with nothing else on the GPU."""
+    from transformer_layer_residual_b200 import fnl
+    dev = {k: v.cuda() for k, v in synthetic.make_inputs(w).items()}
+    h = fnl.Handle(0, path=path)
+    if w.op in synthetic.FP8_OPS:
+        dev["W_fp8"], dev["w_scale"] = fnl.quantize_weight_fp8(h, dev.pop("W"))
+    for _ in range(n):
+        fnl.run_workload(h, w, dev)
+    h.check()
+    torch.cuda.synchronize()
+    print(w.name, path, h.last_plan(), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -581,7 +617,12 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle time for cpu_baseline")
     ap.add_argument("--no-tune", action="store_true", help="untuned plans (no shape auto-tuning)")
     ap.add_argument("--path", default="auto", help="force a kernel for the headline workload (tests/diagnosis)")
+    ap.add_argument("--calls", type=int, default=0,
+                    help="profiler mode: N eager calls of --workload on --path, no timing and no JSON line")
     a = ap.parse_args()
+    if a.calls > 0:
+        eager_calls(synthetic.workloads()[a.workload], a.path, a.calls)
+        return
     if a.warmup < 3:
         a.warmup = 3
     world, rank, local = dist_setup(a.gpus)

@@ -221,6 +221,26 @@ fnl_status fnl_add_norm_qkv_fp8(fnl_handle* h, fnl_stream stream,
                                 fnl_bf16* q, fnl_bf16* k, fnl_bf16* v,
                                 float* mean_out, float* rstd_out);
 
+/* FP8 (W8A8) forms of fnl_add_norm_swiglu and fnl_add_bias_norm_gelu (M <= 128),
+ * with the same quantisation as fnl_add_norm_qkv_fp8: Wq [2I, K] (gate rows,
+ * then up rows) or [N, K] e4m3 codes with one fp32 scale per row, the
+ * normalised activations coded per token; the epilogue dequantises, then
+ * applies SiLU(gate) * up, or GELU(y + bias_out). bias_in (GELU form) enters h
+ * as in the bf16 op. Requirements and errors as for fnl_add_norm_qkv_fp8. */
+fnl_status fnl_add_norm_swiglu_fp8(fnl_handle* h, fnl_stream stream,
+                                   const fnl_bf16* x, const fnl_bf16* residual, fnl_bf16* residual_out,
+                                   const fnl_bf16* gamma, const fnl_bf16* beta, fnl_norm norm, float eps,
+                                   const uint8_t* Wq, const float* w_scale, const fnl_bf16* bias,
+                                   int M, int K, int I,
+                                   fnl_bf16* out, float* mean_out, float* rstd_out);
+fnl_status fnl_add_bias_norm_gelu_fp8(fnl_handle* h, fnl_stream stream,
+                                      const fnl_bf16* x, const fnl_bf16* residual, const fnl_bf16* bias_in,
+                                      fnl_bf16* residual_out,
+                                      const fnl_bf16* gamma, const fnl_bf16* beta, fnl_norm norm, float eps,
+                                      const uint8_t* Wq, const float* w_scale, const fnl_bf16* bias_out,
+                                      int M, int K, int N,
+                                      fnl_bf16* out, float* mean_out, float* rstd_out);
+
 /* Static per-output-channel FP8 quantisation of a bf16 weight W [N, K] for
  * the FP8 form: w_scale[n] = max_k |W[n, k]| / 448 (1 for an all-zero row) and
  * Wq[n, k] = e4m3(W[n, k] / w_scale[n]), both divisions IEEE fp32, round to

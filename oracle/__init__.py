@@ -86,9 +86,13 @@ from .core import (  # noqa: F401
     e4m3_round,
     fp8_row_scale_and_codes,
     fp8_activation_codes,
+    fp8_h32,
     fp8_normalised32,
     quantize_weight_fp8,
     fp8_linear,
+    fp8_projection,
     add_norm_qkv_fp8,
+    add_norm_swiglu_fp8,
+    add_bias_norm_gelu_fp8,
     run,
 )

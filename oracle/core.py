@@ -215,12 +215,21 @@ def fp8_linear(a32, Wq, w_scale, bias=None):
     return y
 
 
-def fp8_normalised32(h, mean, rstd, gamma, beta):
+def fp8_h32(x, residual, bias_in=None) -> np.ndarray:
+    """h = x + residual (+ bias_in) as the FP8 path forms it for its code
+    decisions (R11): fp32 sums, the bias added to the rounded x + residual."""
+    h = (_f32(x) + _f32(residual)).astype(np.float32)
+    if bias_in is not None:
+        h = (h + _f32(bias_in)[None, :]).astype(np.float32)
+    return h
+
+
+def fp8_normalised32(h32, mean, rstd, gamma, beta):
     """The normalised activation in fp32, as the FP8 path forms it before the
-    code decision (R11): h in fp32, the statistics rounded to fp32,
+    code decision (R11): the statistics rounded to fp32,
     t = fp32(fp32(h - mean) * rstd), a = fp32(t * gamma + beta) with one
     rounding (mean 0 and beta 0 for RMSNorm)."""
-    h32 = _f32(h)
+    h32 = _f32(h32)
     m32 = _f32(np.zeros(h32.shape[0]) if mean is None else mean)
     r32 = _f32(rstd)
     t = ((h32 - m32[:, None]).astype(np.float32) * r32[:, None]).astype(np.float32)
@@ -228,25 +237,44 @@ def fp8_normalised32(h, mean, rstd, gamma, beta):
     return (_f64(t) * _f64(gamma)[None, :] + b[None, :]).astype(np.float32)
 
 
-def add_norm_qkv_fp8(x, residual, gamma, beta, norm, eps, Wq, w_scale, bias, Hq, Hkv, D) -> dict:
-    """The fused QKV op on FP8 tensor cores: residual add -> norm statistics ->
-    the activation in fp32 -> per-token FP8 quantisation -> projection with the
-    FP8 weights and their scales -> head-major Q/K/V split. RMSNorm's 1/rms is
-    a positive per-token factor, so its codes are decided on h * gamma (the same
-    codes as on the normalised row, but for fp32 rounding) and rstd multiplies
-    the token's scale (reading R11)."""
-    h = residual_add(x, residual)
+def fp8_projection(x, residual, bias_in, gamma, beta, norm, eps, Wq, w_scale, bias):
+    """Residual add -> norm statistics -> per-token FP8 codes -> W8A8 projection
+    (+ bias), shared by the three FP8 ops. RMSNorm's 1/rms is a positive
+    per-token factor, so its codes are decided on h * gamma (the same codes as
+    on the normalised row, but for fp32 rounding) and rstd multiplies the
+    token's scale (reading R11). Returns (y, h, mean, rstd)."""
+    h = residual_add(x, residual, bias_in)
     _, mean, rstd = normalize(h, gamma, beta, norm, eps)
+    h32 = fp8_h32(x, residual, bias_in)
     if norm == "rmsnorm":
-        a32 = (_f32(h) * _f32(gamma)[None, :]).astype(np.float32)
+        a32 = (h32 * _f32(gamma)[None, :]).astype(np.float32)
         qa, sa = fp8_activation_codes(a32)
         y = (qa @ _f64(Wq).T) * (_f64(sa) * rstd)[:, None] * _f64(w_scale)[None, :]
         if bias is not None:
             y = y + _f64(bias)[None, :]
     else:
-        y = fp8_linear(fp8_normalised32(h, mean, rstd, gamma, beta), Wq, w_scale, bias)
+        y = fp8_linear(fp8_normalised32(h32, mean, rstd, gamma, beta), Wq, w_scale, bias)
+    return y, h, mean, rstd
+
+
+def add_norm_qkv_fp8(x, residual, gamma, beta, norm, eps, Wq, w_scale, bias, Hq, Hkv, D) -> dict:
+    """The fused QKV op on FP8 tensor cores, then the head-major Q/K/V split."""
+    y, h, mean, rstd = fp8_projection(x, residual, None, gamma, beta, norm, eps, Wq, w_scale, bias)
     q, k, v = split_qkv_head_major(y, Hq, Hkv, D)
     return _stats({"residual_out": bf16_round(h), "q": q, "k": k, "v": v}, mean, rstd)
+
+
+def add_norm_swiglu_fp8(x, residual, gamma, beta, norm, eps, Wq, w_scale, bias, I) -> dict:
+    """The fused gate/up op on FP8 tensor cores (W = [gate; up] rows, one
+    scale per row), then SiLU(gate) * up."""
+    y, h, mean, rstd = fp8_projection(x, residual, None, gamma, beta, norm, eps, Wq, w_scale, bias)
+    return _stats({"residual_out": bf16_round(h), "out": swiglu(y, I)}, mean, rstd)
+
+
+def add_bias_norm_gelu_fp8(x, residual, bias_in, gamma, beta, norm, eps, Wq, w_scale, bias_out) -> dict:
+    """The fused Add + Bias + norm -> Linear + GELU op on FP8 tensor cores."""
+    y, h, mean, rstd = fp8_projection(x, residual, bias_in, gamma, beta, norm, eps, Wq, w_scale, bias_out)
+    return _stats({"residual_out": bf16_round(h), "out": gelu_tanh(y)}, mean, rstd)
 
 
 def run(w, inputs: dict, rows=None) -> dict:
@@ -270,6 +298,12 @@ def run(w, inputs: dict, rows=None) -> dict:
     if w.op == "qkv_fp8":   # "W_fp8" / "w_scale": the FP8 weights (codes as values) and their scales
         return add_norm_qkv_fp8(x, r, g("gamma"), g("beta"), w.norm, w.eps, g("W_fp8"), g("w_scale"),
                                 g("bias_out"), w.Hq, w.Hkv, w.D)
+    if w.op == "swiglu_fp8":
+        return add_norm_swiglu_fp8(x, r, g("gamma"), g("beta"), w.norm, w.eps, g("W_fp8"), g("w_scale"),
+                                   g("bias_out"), w.I)
+    if w.op == "gelu_fp8":
+        return add_bias_norm_gelu_fp8(x, r, g("bias_in"), g("gamma"), g("beta"), w.norm, w.eps, g("W_fp8"),
+                                      g("w_scale"), g("bias_out"))
     if w.op == "qkv":
         return add_norm_qkv(x, r, g("gamma"), g("beta"), w.norm, w.eps, g("W"),
                             g("bias_out"), w.Hq, w.Hkv, w.D)

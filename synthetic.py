@@ -32,6 +32,9 @@ SWIGLU = "swiglu"
 GELU = "gelu"
 RESIDUAL = "residual"   # residual-stream projection: out = residual + a W^T (+ bias)
 QKV_FP8 = "qkv_fp8"     # the QKV op with FP8 (e4m3) weights and activations; W is drawn in bf16
+SWIGLU_FP8 = "swiglu_fp8"
+GELU_FP8 = "gelu_fp8"
+FP8_OPS = (QKV_FP8, SWIGLU_FP8, GELU_FP8)
 NONORM = "none"
 
 
@@ -58,7 +61,7 @@ class Workload:
     @property
     def n_out(self) -> int:
         """Columns of the stored output (I for SwiGLU, N otherwise)."""
-        return self.I if self.op == SWIGLU else self.N
+        return self.I if self.op in (SWIGLU, SWIGLU_FP8) else self.N
 
     def flops(self) -> float:
         return 2.0 * self.M * self.N * self.K
@@ -71,9 +74,10 @@ class Workload:
         M, K, N = self.M, self.K, self.N
         if self.op == RESIDUAL:
             return float(M * K * 2 + 2 * M * N * 2 + N * K * 2 + (N * 2 if self.has_bias_out else 0))
-        if self.op == QKV_FP8:   # one byte per weight plus a 4-byte scale per row
-            b = 2 * M * K * 2 + M * K * 2 + N * K + N * 4 + M * N * 2
-            return float(b + K * 2 * (2 if self.norm == LAYERNORM else 1) + (N * 2 if self.has_bias_out else 0))
+        if self.op in FP8_OPS:   # one byte per weight plus a 4-byte scale per row
+            b = 2 * M * K * 2 + M * K * 2 + N * K + N * 4 + M * self.n_out * 2
+            b += K * 2 * (2 if self.norm == LAYERNORM else 1) + (K * 2 if self.has_bias_in else 0)
+            return float(b + (N * 2 if self.has_bias_out else 0))
         b = 2 * M * K * 2 + M * K * 2 + N * K * 2 + M * self.n_out * 2
         b += K * 2 * (2 if self.norm == LAYERNORM else 1)
         if self.has_bias_in:
@@ -116,15 +120,22 @@ def workloads() -> dict:
 
 
 def fp8_workloads() -> dict:
-    """The decode QKV shapes with FP8 (e4m3) weights and activations: Llama-3-8B
-    (M=32, K=4096, N=6144) and Llama-2-70B (M=32, K=8192, N=10240), RMSNorm.
-    The bf16 W is drawn as for the bf16 op; its FP8 codes and scales are
-    derived from it by the quantiser under test (or the oracle's)."""
+    """Decode shapes (32 tokens) with FP8 (e4m3) weights and activations: the
+    QKV projections of Llama-3-8B (K=4096, N=6144) and Llama-2-70B (K=8192,
+    N=10240) after RMSNorm, the Llama-3-8B gate/up projection (K=4096,
+    I=14336) after RMSNorm, and a GPT-style up-projection (K=4096, N=16384)
+    after LayerNorm with both biases. The bf16 W is drawn as for the bf16 op;
+    its FP8 codes and scales are derived from it by the quantiser under test
+    (or the oracle's)."""
     return {
         "c2_decode_rms_qkv_fp8": Workload("c2_decode_rms_qkv_fp8", QKV_FP8, RMSNORM, 32, 4096, 6144,
                                           Hq=32, Hkv=8, D=128),
         "c5_70b_rms_qkv_m32_fp8": Workload("c5_70b_rms_qkv_m32_fp8", QKV_FP8, RMSNORM, 32, 8192, 10240,
                                            Hq=64, Hkv=8, D=128),
+        "llama3_8b_mlp_decode_swiglu_fp8": Workload("llama3_8b_mlp_decode_swiglu_fp8", SWIGLU_FP8, RMSNORM,
+                                                    32, 4096, 2 * 14336, I=14336),
+        "gpt_mlp_decode_ln_gelu_fp8": Workload("gpt_mlp_decode_ln_gelu_fp8", GELU_FP8, LAYERNORM, 32, 4096,
+                                               16384, has_bias_in=True, has_bias_out=True),
     }
 
 
@@ -189,6 +200,12 @@ def make_custom(op: str, norm: str, M: int, K: int, *, Hq=0, Hkv=0, D=0, I=0, N=
     elif op == QKV_FP8:
         w = Workload(f"custom_qkv_fp8_{M}x{K}", QKV_FP8, norm, M, K, (Hq + 2 * Hkv) * D, Hq=Hq, Hkv=Hkv, D=D,
                      eps=eps, has_bias_in=bias_in, has_bias_out=bias_out, x_loc=x_loc)
+    elif op == SWIGLU_FP8:
+        w = Workload(f"custom_swiglu_fp8_{M}x{K}", SWIGLU_FP8, norm, M, K, 2 * I, I=I, eps=eps,
+                     has_bias_in=bias_in, has_bias_out=bias_out, x_loc=x_loc)
+    elif op == GELU_FP8:
+        w = Workload(f"custom_gelu_fp8_{M}x{K}", GELU_FP8, norm, M, K, N, eps=eps,
+                     has_bias_in=bias_in, has_bias_out=bias_out, x_loc=x_loc)
     elif op == SWIGLU:
         w = Workload(f"custom_swiglu_{M}x{K}", SWIGLU, norm, M, K, 2 * I, I=I, eps=eps,
                      has_bias_in=bias_in, has_bias_out=bias_out, x_loc=x_loc)

@@ -46,7 +46,7 @@ def run_fp8(h, w, inputs):
     return check(w, full, got)
 
 
-@pytest.mark.parametrize("name", ["c2_decode_rms_qkv_fp8", "c5_70b_rms_qkv_m32_fp8"])
+@pytest.mark.parametrize("name", sorted(synthetic.fp8_workloads()))
 def test_fp8_full_compare(handle, name):
     w = WL[name]
     res = run_fp8(handle, w, synthetic.make_inputs(w))
@@ -96,4 +96,31 @@ def test_fp8_errors(cuda_device):
                              torch.zeros(N, 64, dtype=torch.uint8, device="cuda"),
                              torch.ones(N, dtype=torch.float32, device="cuda"), Hq, Hkv, D)
     assert e.value.status == 4
+    h.close()
+
+
+@pytest.mark.parametrize("norm", ["layernorm", "rmsnorm"])
+@pytest.mark.parametrize("M", [1, 16, 33, 128])
+def test_fp8_swiglu_tails(handle, norm, M):
+    w, inputs = synthetic.make_custom("swiglu_fp8", norm, M, 208, I=200, bias_out=True, seed=M + 1)
+    run_fp8(handle, w, inputs)
+
+
+@pytest.mark.parametrize("norm", ["layernorm", "rmsnorm"])
+@pytest.mark.parametrize("M", [1, 16, 33, 128])
+def test_fp8_gelu_tails(handle, norm, M):
+    w, inputs = synthetic.make_custom("gelu_fp8", norm, M, 208, N=328, bias_in=True, bias_out=True, seed=M + 2)
+    run_fp8(handle, w, inputs)
+
+
+@pytest.mark.parametrize("op", ["swiglu_fp8", "gelu_fp8"])
+@pytest.mark.parametrize("path", ["splitk", "cluster"])
+def test_fp8_epilogues_forced_forms(cuda_device, op, path):
+    h = fnl.Handle(0, path=path)
+    for M in (5, 64):
+        if op == "swiglu_fp8":
+            w, inputs = synthetic.make_custom(op, "rmsnorm", M, 528, I=200, bias_out=True, seed=M)
+        else:
+            w, inputs = synthetic.make_custom(op, "layernorm", M, 528, N=328, bias_in=True, bias_out=True, seed=M)
+        run_fp8(h, w, inputs)
     h.close()

@@ -482,12 +482,13 @@ def pin_fp8_activation_codes(ora):
     h = rng.normal(0, 1, (4, 64))
     g, be = 1 + 0.1 * rng.normal(size=64), 0.1 * rng.normal(size=64)
     a64, mean, rstd = ora.layernorm(h, g, be, 1e-5)
-    a32 = ora.fp8_normalised32(h, mean, rstd, g, be)
+    a32 = ora.fp8_normalised32(h.astype(np.float32), mean, rstd, g, be)
     assert a32.dtype == np.float32
-    assert np.all(np.abs(a32 - a64) <= 4 * 2.0 ** -24 * (np.abs(a64) + np.abs(be)[None, :] + 1))
+    # h rounded to fp32 first (as the kernel holds it), then the fp32 steps
+    assert np.all(np.abs(a32 - a64) <= 2.0 ** -20 * (np.abs(a64) + np.abs(be)[None, :] + 1))
     r64, rs = ora.rmsnorm(h, g, 1e-5)
-    r32 = ora.fp8_normalised32(h, None, rs, g, None)
-    assert np.all(np.abs(r32 - r64) <= 4 * 2.0 ** -24 * (np.abs(r64) + 1))
+    r32 = ora.fp8_normalised32(h.astype(np.float32), None, rs, g, None)
+    assert np.all(np.abs(r32 - r64) <= 2.0 ** -20 * (np.abs(r64) + 1))
 
 
 def pin_fp8_fused_qkv(ora):
@@ -511,6 +512,22 @@ def pin_fp8_fused_qkv(ora):
     o16 = ora.add_norm_qkv(xr, rr, g, None, "layernorm", 1e-5, Wd, None, Hq, Hkv, D)
     for key in ("residual_out", "mean", "rstd"):
         assert np.array_equal(o8[key], o16[key])
+    # SwiGLU: one-hot x, W = [gate; up] quantised per row: out = SiLU(y_g) y_u with
+    # y = W~[:, j] gamma_j s rstd
+    I = 5
+    Wsw = rng.normal(0, 0.2, (2 * I, K))
+    Wq2, sw2 = ora.quantize_weight_fp8(Wsw)
+    Wd2 = Wq2 * sw2.astype(np.float64)[:, None]
+    o = ora.add_norm_swiglu_fp8(x, np.zeros((1, K)), g, None, "rmsnorm", eps, Wq2, sw2, None, I)["out"][0]
+    yv = Wd2[:, j] * g[j] * sc / math.sqrt(sc * sc / K + eps)
+    ref = yv[:I] / (1 + np.exp(-yv[:I])) * yv[I:]
+    assert np.max(np.abs(o - ref)) <= 1e-6 * (1 + np.max(np.abs(ref)))
+    # Bias + GELU: bias_in enters h (and the codes), bias_out is added before GELU
+    bi, bo = rng.normal(size=K), 0.02 * rng.normal(size=N)
+    og = ora.add_bias_norm_gelu_fp8(xr, rr, bi, g, None, "layernorm", 1e-5, Wq, sw, bo)
+    y_ln = ora.fp8_linear(ora.fp8_normalised32(ora.fp8_h32(xr, rr, bi), og["mean"], og["rstd"], g, None), Wq, sw, bo)
+    assert np.max(np.abs(og["out"] - ora.gelu_tanh(y_ln))) <= 1e-12
+    assert np.array_equal(og["residual_out"], ora.bf16_round(xr + rr + bi[None, :]))
 
 
 PINS = [pin_layernorm_invariants, pin_rmsnorm_invariant, pin_norms_match_torch,

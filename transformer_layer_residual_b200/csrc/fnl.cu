@@ -553,11 +553,17 @@ fnl_status launch_fp8_prepass(fnl_handle* h, const Call& c, float4* stats8, cuda
   return FNL_OK;
 }
 
-// The small-M kernel's FP8 form (instantiated for the QKV epilogue, the one FP8 entry point).
+// The small-M kernel's FP8 form, for each epilogue.
 fnl_status dispatch_fp8(fnl_handle* h, int epi, int grid, int threads, int smem, bool pdl, cudaStream_t stream,
                         const CUtensorMap& mx, const CUtensorMap& mr, const CUtensorMap& mw, const OpParams& p) {
-  if (epi != fnl::kEpiQKV) return fail(h, FNL_ERR_UNSUPPORTED, "FP8: QKV epilogue only");
-  return launch_gemm(h, fnl::k3_splitk_kernel<fnl::kEpiQKV, fnl::kLayerNorm, false, true>, grid, threads, smem, pdl,
+  using fnl::kLayerNorm;
+  if (epi == fnl::kEpiSwiGLU)
+    return launch_gemm(h, fnl::k3_splitk_kernel<fnl::kEpiSwiGLU, kLayerNorm, false, true>, grid, threads, smem, pdl,
+                       stream, mx, mr, mw, p);
+  if (epi == fnl::kEpiGELU)
+    return launch_gemm(h, fnl::k3_splitk_kernel<fnl::kEpiGELU, kLayerNorm, false, true>, grid, threads, smem, pdl,
+                       stream, mx, mr, mw, p);
+  return launch_gemm(h, fnl::k3_splitk_kernel<fnl::kEpiQKV, kLayerNorm, false, true>, grid, threads, smem, pdl,
                      stream, mx, mr, mw, p);
 }
 
@@ -1143,6 +1149,41 @@ fnl_status fnl_add_norm_qkv_fp8(fnl_handle* h, fnl_stream stream, const fnl_bf16
   c.q = Bm(q); c.k = Bm(k); c.v = Bm(v); c.out = nullptr;
   c.mean_out = mean_out; c.rstd_out = rstd_out;
   if (c.N <= 0 && h) return fail(h, FNL_ERR_INVALID_ARG, "Hq, Hkv, D must be > 0 and (Hq + 2 Hkv) D <= %d", kMaxN);
+  return run(h, c);
+}
+
+fnl_status fnl_add_norm_swiglu_fp8(fnl_handle* h, fnl_stream stream, const fnl_bf16* x, const fnl_bf16* residual,
+                                   fnl_bf16* residual_out, const fnl_bf16* gamma, const fnl_bf16* beta, fnl_norm norm,
+                                   float eps, const uint8_t* Wq, const float* w_scale, const fnl_bf16* bias, int M,
+                                   int K, int I, fnl_bf16* out, float* mean_out, float* rstd_out) {
+  Call c{};
+  c.op = Op::SwiGLU;
+  c.fp8 = true;
+  c.stream = reinterpret_cast<cudaStream_t>(stream);
+  c.x = B(x); c.residual = B(residual); c.bias_in = nullptr; c.gamma = B(gamma); c.beta = B(beta);
+  c.W = reinterpret_cast<const bf16*>(Wq); c.w_scale = w_scale; c.bias = B(bias); c.residual_out = Bm(residual_out);
+  c.norm = norm; c.eps = eps; c.M = M; c.K = K; c.I = I; c.N = (I > 0 && I <= kMaxN / 2) ? 2 * I : 0;
+  c.out = Bm(out);
+  c.mean_out = mean_out; c.rstd_out = rstd_out;
+  if (c.N <= 0 && h) return fail(h, FNL_ERR_INVALID_ARG, "I must be > 0 and 2 I <= %d", kMaxN);
+  return run(h, c);
+}
+
+fnl_status fnl_add_bias_norm_gelu_fp8(fnl_handle* h, fnl_stream stream, const fnl_bf16* x, const fnl_bf16* residual,
+                                      const fnl_bf16* bias_in, fnl_bf16* residual_out, const fnl_bf16* gamma,
+                                      const fnl_bf16* beta, fnl_norm norm, float eps, const uint8_t* Wq,
+                                      const float* w_scale, const fnl_bf16* bias_out, int M, int K, int N,
+                                      fnl_bf16* out, float* mean_out, float* rstd_out) {
+  Call c{};
+  c.op = Op::GELU;
+  c.fp8 = true;
+  c.stream = reinterpret_cast<cudaStream_t>(stream);
+  c.x = B(x); c.residual = B(residual); c.bias_in = B(bias_in); c.gamma = B(gamma); c.beta = B(beta);
+  c.W = reinterpret_cast<const bf16*>(Wq); c.w_scale = w_scale; c.bias = B(bias_out);
+  c.residual_out = Bm(residual_out);
+  c.norm = norm; c.eps = eps; c.M = M; c.K = K; c.N = N;
+  c.out = Bm(out);
+  c.mean_out = mean_out; c.rstd_out = rstd_out;
   return run(h, c);
 }
 

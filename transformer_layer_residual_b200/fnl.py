@@ -26,7 +26,8 @@ PRECISIONS = {"default": 0, "split": 1, "single": 2}
 
 EXPORTED = ("fnl_create", "fnl_destroy", "fnl_status_string", "fnl_last_error", "fnl_last_plan", "fnl_check",
             "fnl_add_norm_qkv", "fnl_add_norm_swiglu", "fnl_add_bias_norm_gelu", "fnl_linear_add_residual",
-            "fnl_add_norm_qkv_fp8", "fnl_quantize_weight_fp8",
+            "fnl_add_norm_qkv_fp8", "fnl_add_norm_swiglu_fp8", "fnl_add_bias_norm_gelu_fp8",
+            "fnl_quantize_weight_fp8",
             "fnl_add_norm_qkv_static", "fnl_check_static")
 
 
@@ -71,6 +72,8 @@ def lib() -> ctypes.CDLL:
     L.fnl_linear_add_residual.argtypes = [P, P, P, P, P, P, P, I, I, I]
     L.fnl_add_norm_qkv_fp8.argtypes = [P, P, P, P, P, P, P, I, F, P, P, P, I, I, I, I, I, P, P, P, P, P]
     L.fnl_quantize_weight_fp8.argtypes = [P, P, P, I, I, P, P]
+    L.fnl_add_norm_swiglu_fp8.argtypes = [P, P, P, P, P, P, P, I, F, P, P, P, I, I, I, P, P, P]
+    L.fnl_add_bias_norm_gelu_fp8.argtypes = [P, P, P, P, P, P, P, P, I, F, P, P, P, I, I, I, P, P, P]
     L.fnl_add_norm_qkv_static.argtypes = [P, P, P, P, P, P, I, F, P, P, I, I, I, I, I, P, P, P, P, P]
     L.fnl_check_static.argtypes = [P]
     for name in EXPORTED:
@@ -300,18 +303,82 @@ def add_norm_qkv_fp8(h: Handle, x, residual, gamma, beta, Wq, w_scale, Hq, Hkv, 
     return {"residual_out": residual_out, "q": q, "k": k, "v": v, "mean": mean_out, "rstd": rstd_out}
 
 
+def _fp8_common(x, residual, gamma, beta, Wq, w_scale, n_rows, norm, residual_out, mean_out, rstd_out):
+    M, K = x.shape
+    _need(x, "x", (M, K))
+    _need(residual, "residual", (M, K))
+    _need(gamma, "gamma", (K,))
+    _need(beta, "beta", (K,))
+    _need(Wq, "Wq", (n_rows, K), torch.uint8)
+    _need(w_scale, "w_scale", (n_rows,), torch.float32)
+    if norm not in NORMS:
+        raise ValueError(f"norm must be one of {list(NORMS)}")
+    residual_out = torch.empty_like(x) if residual_out is None else residual_out
+    _need(residual_out, "residual_out", (M, K))
+    if rstd_out is not None:
+        _need(rstd_out, "rstd_out", (M,), torch.float32)
+    if mean_out is not None:
+        _need(mean_out, "mean_out", (M,), torch.float32)
+    return M, K, residual_out
+
+
+def add_norm_swiglu_fp8(h: Handle, x, residual, gamma, beta, Wq, w_scale, I, norm="rmsnorm", eps=1e-5, bias=None,
+                        residual_out=None, out=None, mean_out=None, rstd_out=None, stream=None):
+    """fnl_add_norm_swiglu_fp8: Wq uint8 [2I, K] e4m3 codes (gate rows, then up
+    rows), w_scale fp32 [2I]. Returns dict(residual_out, out [M, I], mean, rstd)."""
+    M, K, residual_out = _fp8_common(x, residual, gamma, beta, Wq, w_scale, 2 * I, norm, residual_out, mean_out,
+                                     rstd_out)
+    _need(bias, "bias", (2 * I,))
+    out = torch.empty(M, I, dtype=torch.bfloat16, device=x.device) if out is None else out
+    _need(out, "out", (M, I))
+    st = lib().fnl_add_norm_swiglu_fp8(h.ptr, _stream_ptr(stream), _p(x), _p(residual), _p(residual_out),
+                                       _p(gamma), _p(beta), NORMS[norm], float(eps), _p(Wq), _p(w_scale), _p(bias),
+                                       M, K, I, _p(out), _p(mean_out), _p(rstd_out))
+    if st != FNL_OK:
+        h._raise(st, "fnl_add_norm_swiglu_fp8")
+    return {"residual_out": residual_out, "out": out, "mean": mean_out, "rstd": rstd_out}
+
+
+def add_bias_norm_gelu_fp8(h: Handle, x, residual, gamma, beta, Wq, w_scale, bias_in=None, bias_out=None,
+                           norm="layernorm", eps=1e-5, residual_out=None, out=None, mean_out=None, rstd_out=None,
+                           stream=None):
+    """fnl_add_bias_norm_gelu_fp8: Wq uint8 [N, K] e4m3 codes, w_scale fp32 [N].
+    Returns dict(residual_out, out [M, N], mean, rstd)."""
+    N = Wq.shape[0]
+    M, K, residual_out = _fp8_common(x, residual, gamma, beta, Wq, w_scale, N, norm, residual_out, mean_out,
+                                     rstd_out)
+    _need(bias_in, "bias_in", (K,))
+    _need(bias_out, "bias_out", (N,))
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=x.device) if out is None else out
+    _need(out, "out", (M, N))
+    st = lib().fnl_add_bias_norm_gelu_fp8(h.ptr, _stream_ptr(stream), _p(x), _p(residual), _p(bias_in),
+                                          _p(residual_out), _p(gamma), _p(beta), NORMS[norm], float(eps), _p(Wq),
+                                          _p(w_scale), _p(bias_out), M, K, N, _p(out), _p(mean_out), _p(rstd_out))
+    if st != FNL_OK:
+        h._raise(st, "fnl_add_bias_norm_gelu_fp8")
+    return {"residual_out": residual_out, "out": out, "mean": mean_out, "rstd": rstd_out}
+
+
 def run_workload(h: Handle, w, dev: dict, stats: bool = True, stream=None) -> dict:
     """Run a synthetic.Workload on device tensors `dev` (same keys as
     synthetic.make_inputs). Allocates the outputs and statistics buffers."""
     if w.op == "residual":
         return linear_add_residual(h, dev["x"], dev["W"], dev["residual"], bias=dev.get("bias_out"), stream=stream)
     M = dev["x"].shape[0]
-    if w.op == "qkv_fp8":   # dev["W_fp8"]: e4m3 codes (float8_e4m3fn or uint8), dev["w_scale"]: fp32 [N]
+    if w.op.endswith("_fp8"):   # dev["W_fp8"]: e4m3 codes (float8_e4m3fn or uint8), dev["w_scale"]: fp32 [N]
         rstd = torch.empty(M, dtype=torch.float32, device=dev["x"].device) if stats else None
         mean = (torch.empty(M, dtype=torch.float32, device=dev["x"].device)
                 if stats and w.norm == "layernorm" else None)
         Wq = dev["W_fp8"]
         Wq = Wq.view(torch.uint8) if Wq.dtype != torch.uint8 else Wq
+        if w.op == "swiglu_fp8":
+            return add_norm_swiglu_fp8(h, dev["x"], dev["residual"], dev["gamma"], dev.get("beta"), Wq,
+                                       dev["w_scale"], w.I, norm=w.norm, eps=w.eps, bias=dev.get("bias_out"),
+                                       mean_out=mean, rstd_out=rstd, stream=stream)
+        if w.op == "gelu_fp8":
+            return add_bias_norm_gelu_fp8(h, dev["x"], dev["residual"], dev["gamma"], dev.get("beta"), Wq,
+                                          dev["w_scale"], bias_in=dev.get("bias_in"), bias_out=dev.get("bias_out"),
+                                          norm=w.norm, eps=w.eps, mean_out=mean, rstd_out=rstd, stream=stream)
         return add_norm_qkv_fp8(h, dev["x"], dev["residual"], dev["gamma"], dev.get("beta"), Wq, dev["w_scale"],
                                 w.Hq, w.Hkv, w.D, norm=w.norm, eps=w.eps, bias=dev.get("bias_out"), mean_out=mean,
                                 rstd_out=rstd, stream=stream)
