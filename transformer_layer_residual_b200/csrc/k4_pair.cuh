@@ -1,9 +1,9 @@
 // K4: large-M fused norm + GEMM + epilogue on CTA pairs (tcgen05 cta_group::2).
 //
 // Same dataflow as the 128 x 512 kernel (TMA x / residual / W tiles ->
-// converter warps build the normalised bf16 operand in place in shared memory
-// -> tcgen05.mma into TMEM -> fused epilogue), with the pair tile spread over
-// two CTAs of a cluster: 256 tokens x 512 W rows (SwiGLU: 256 gate rows + the
+// converter warps build the normalised bf16 operand in shared memory ->
+// tcgen05.mma into TMEM -> fused epilogue), with the pair tile spread over two
+// CTAs of a cluster: 256 tokens x 512 W rows (SwiGLU: 256 gate rows + the
 // matching 256 up rows). Each CTA holds its 128 tokens' x, residual and
 // normalised operand, and half of each weight operand; the pair's even CTA
 // issues tcgen05.mma.cta_group::2 M=256 N=256 K=16, which reads A from both
@@ -14,24 +14,35 @@
 // 48 KB in the single-CTA 128 x 512 kernel: shared-memory bytes per FLOP, the
 // bound of the fused operand's pipeline, drop by about a quarter.
 //
-// Warp roles (14 warps per CTA): 0 TMA producer (own tiles only), 1 TMEM
-// (allocated for the pair) and, in the even CTA, UMMA issuer; 2-5 epilogue
-// (own 128 rows); 6-13 converters, in two groups of four that take alternate
-// stages (the conversion latency of one stage overlaps the next; with one
-// group the fused kernel ran at half the tensor rate of the same pipeline
-// without converters). A stage is ready for the UMMA when both CTAs'
-// converters have built their operand and seen their own weight half land:
-// every converter warp of the stage's group in both CTAs arrives on the even CTA's conv[s]
-// after waiting for its CTA's full_x[s] and full_w[s], so no tensor copy ever
-// signals the other CTA and each CTA drains only its own copies. The UMMA
-// commits arrive on both CTAs' empty[s] / tfull (multicast commit); the
-// epilogue warps of both CTAs arrive on the even CTA's tempty. RMSNorm uses the
-// deferred scale of the other kernels (each CTA's converters sum h^2 of its
-// rows for its own epilogue); LayerNorm statistics come from the statistics
-// kernel. A wait that gives up raises the abort flag of both CTAs; both CTAs
-// meet at a cluster barrier after their role loops (and after the last UMMA
-// completed), so neither leaves while the other may still touch its shared
-// memory.
+// Two rings per CTA. The operand ring (OST slots: normalised A [+ its lo part
+// for the split form], W half 0, W half 1) holds what the UMMA reads; a slot is
+// refilled once the UMMA that read it has completed. The raw ring (RST slots:
+// x, residual and the gamma / beta / bias_in slices) only feeds the
+// converters, and a raw slot is refilled as soon as its converters have read
+// it. So the activation copies run ahead of the UMMA, and an operand slot's
+// turnaround (UMMA done -> W copy and conversion -> next UMMA) no longer
+// includes the activation copy's latency: on B200 that turnaround was about
+// 1.1 us against 6 x 0.31 us of tensor work buffered, and the tensor pipe
+// waited on the ring for about 40% of the time when both copies sat in one slot.
+//
+// Warp roles (15 warps per CTA): 0 raw-ring producer (x, residual, vectors),
+// 1 TMEM (allocated for the pair) and, in the even CTA, UMMA issuer; 2-5
+// epilogue (own 128 rows); 6-13 converters, in two groups of four that take
+// alternate positions (the conversion latency of one position overlaps the
+// next); 14 operand-ring producer (W halves; without a norm also the
+// activation tile, which is the operand as loaded). An operand slot is ready
+// for the UMMA when both CTAs' converters have built their operand and seen
+// their own weight halves land: every converter warp of the position's group in
+// both CTAs arrives on the even CTA's conv[s] after waiting for its CTA's
+// full_w[s], so no tensor copy ever signals the other CTA and each CTA drains
+// only its own copies. The UMMA commits arrive on both CTAs' empty[s] / tfull
+// (multicast commit); the epilogue warps of both CTAs arrive on the even
+// CTA's tempty. RMSNorm uses the deferred scale of the other kernels (each
+// CTA's converters sum h^2 of its rows for its own epilogue); LayerNorm
+// statistics come from the statistics kernel. A wait that gives up raises the
+// abort flag of both CTAs; both CTAs meet at a cluster barrier after their role
+// loops (and after the last UMMA completed), so neither leaves while the other
+// may still touch its shared memory.
 #pragma once
 
 #include "common.cuh"
@@ -42,30 +53,41 @@ namespace k4 {
 constexpr int BM = 128;            // tokens per CTA (256 per pair)
 constexpr int BN = 512;            // W rows per pair tile (all in each CTA's TMEM)
 constexpr int BK = 32;             // k-block: 64-byte rows, 64-byte swizzle
-constexpr int STAGES = 6;
-constexpr int X_BYTES = BM * BK * 2;              // 8 KB
+constexpr int X_BYTES = BM * BK * 2;              // 8 KB: x, residual, A or lo(A) of one k-block
 constexpr int WH_BYTES = 128 * BK * 2;            // 8 KB: one 128-row half of an N=256 operand
-constexpr int STAGE_BYTES = 2 * X_BYTES + 2 * WH_BYTES;   // 32 KB: x, residual, W half 0, W half 1
+constexpr int RAW_BYTES = 2 * X_BYTES;            // raw slot: x, residual
+// operand ring: A [lo(A)] W0 W1; the split form's larger slots leave room for fewer
+__host__ __device__ constexpr int op_stages(bool split) { return split ? 5 : 6; }
+__host__ __device__ constexpr int raw_stages(bool split) { return split ? 3 : 4; }
+__host__ __device__ constexpr int op_a_bytes(bool split) { return (split ? 2 : 1) * X_BYTES; }
+__host__ __device__ constexpr int op_bytes(bool split) { return op_a_bytes(split) + 2 * WH_BYTES; }
+constexpr int MAX_OST = 6, MAX_RST = 4;
+constexpr int RINGS_BYTES = 6 * (X_BYTES + 2 * WH_BYTES) + 4 * RAW_BYTES;   // 208 KB (the split form: the same)
+static_assert(op_stages(true) * op_bytes(true) + raw_stages(true) * RAW_BYTES == RINGS_BYTES, "ring sizes");
+static_assert(op_stages(false) * op_bytes(false) + raw_stages(false) * RAW_BYTES == RINGS_BYTES, "ring sizes");
 constexpr int VEC = BK;
 constexpr int VEC_STAGE_BYTES = 3 * VEC * 2;
-constexpr int VEC_BYTES = STAGES * VEC_STAGE_BYTES;
+constexpr int VEC_BYTES = MAX_RST * VEC_STAGE_BYTES;
 constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_EPI0 = 2, NUM_EPI_WARPS = 4;
 constexpr int WARP_CONV0 = 6, NUM_CONV_WARPS = 8;
-constexpr int CONV_GROUPS = 2;                                          // stages converted at once
-constexpr int CONV_GROUP_THREADS = NUM_CONV_WARPS / CONV_GROUPS * 32;   // 128
+constexpr int WARP_WTMA = WARP_CONV0 + NUM_CONV_WARPS;                  // 14
+constexpr int CONV_GROUPS = 2;                                          // positions converted at once
+constexpr int CONV_GROUP_WARPS = NUM_CONV_WARPS / CONV_GROUPS;          // 4
+constexpr int CONV_GROUP_THREADS = CONV_GROUP_WARPS * 32;               // 128
 constexpr int CONV_ROWS_PER_PASS = CONV_GROUP_THREADS / 4;              // 32 rows x 4 chunks
-constexpr int NUM_THREADS = (WARP_CONV0 + NUM_CONV_WARPS) * 32;   // 448
+constexpr int NUM_THREADS = (WARP_WTMA + 1) * 32;   // 480
 constexpr int TMEM_COLS = 512;
 constexpr int GROUP_M = 8;         // pair rows (of 256 tokens) sharing a W tile while it is hot in L2
 
 struct Ctrl {
-  uint64_t full_w[STAGES], full_x[STAGES], conv[STAGES], empty[STAGES];
+  uint64_t full_w[MAX_OST], conv[MAX_OST], empty[MAX_OST];   // operand ring
+  uint64_t raw_full[MAX_RST], raw_empty[MAX_RST];            // raw ring
   uint64_t tfull, tempty, sfull[2], efree[2], drain;
   uint32_t tmem_base;
   int abort_flag;
   float rs[2][CONV_GROUPS][BM];   // RMSNorm: per tile buffer, per converter group, sum of h^2 per row
 };
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + VEC_BYTES + static_cast<int>(sizeof(Ctrl)) + 1024;
+constexpr int SMEM_BYTES = RINGS_BYTES + VEC_BYTES + static_cast<int>(sizeof(Ctrl)) + 1024;
 
 __device__ __forceinline__ void tile_coords(int t, int num_m2, int num_n, int& mb2, int& nb) {
   const int per_group = GROUP_M * num_n;
@@ -92,10 +114,13 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
     k4_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_r,
                    const __grid_constant__ CUtensorMap tm_w, const OpParams p) {
   using namespace k4;
+  constexpr int OST = op_stages(SPLIT), RST = raw_stages(SPLIT);
+  constexpr int OPB = op_bytes(SPLIT), OPA = op_a_bytes(SPLIT);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  bf16* vecs = reinterpret_cast<bf16*>(smem + STAGES * STAGE_BYTES);   // [STAGES][3][32]
-  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + STAGES * STAGE_BYTES + VEC_BYTES);
+  uint8_t* raw = smem + OST * OPB;                                        // [RST][x | residual]
+  bf16* vecs = reinterpret_cast<bf16*>(smem + RINGS_BYTES);               // [RST][3][32]
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + RINGS_BYTES + VEC_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();       // 0: the pair's UMMA issuer
   const uint32_t peer = rank ^ 1u;
@@ -110,14 +135,19 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
   const int tiles = num_m2 * num_n;
   const int nkb = (K + BK - 1) / BK;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int my_tiles = pair < tiles ? (tiles - 1 - pair) / npairs + 1 : 0;
+  const int P = my_tiles * nkb;   // positions (tile, k-block) of this CTA
 
   if (threadIdx.x == 0) {
     pdl_launch_dependents();
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < OST; ++s) {
       mbar_init(&ctrl->full_w[s], 1);
-      mbar_init(&ctrl->full_x[s], 1);
-      mbar_init(&ctrl->conv[s], 2 * NUM_CONV_WARPS / CONV_GROUPS);   // (even CTA) one group's warps of both CTAs
-      mbar_init(&ctrl->empty[s], 1);                   // multicast UMMA commit
+      mbar_init(&ctrl->conv[s], 2 * CONV_GROUP_WARPS);   // (even CTA) one group's warps of both CTAs
+      mbar_init(&ctrl->empty[s], 1);                     // multicast UMMA commit
+    }
+    for (int r = 0; r < RST; ++r) {
+      mbar_init(&ctrl->raw_full[r], 1);
+      mbar_init(&ctrl->raw_empty[r], CONV_GROUP_WARPS);  // the warps of the group that converted it
     }
     mbar_init(&ctrl->tfull, 1);
     mbar_init(&ctrl->tempty, 2 * NUM_EPI_WARPS);       // (even CTA) epilogue warps of both CTAs
@@ -132,13 +162,13 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
   if (warp == WARP_TMA && lane == 0) {
     prefetch_tmap(&tm_x);
     prefetch_tmap(&tm_r);
-    prefetch_tmap(&tm_w);
   }
+  if (warp == WARP_WTMA && lane == 0) prefetch_tmap(&tm_w);
   if (warp == WARP_MMA) {
     tmem_alloc_pair(&ctrl->tmem_base, TMEM_COLS);
     tmem_relinquish_pair();
   }
-  zero_vec_slices(vecs, STAGES * 3 * VEC);
+  zero_vec_slices(vecs, RST * 3 * VEC);
   tc_fence_before();
   __syncthreads();
   cluster_sync();   // both CTAs' barriers are initialised before any remote arrive
@@ -149,19 +179,59 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
   auto abort_pair = [&]() { st_remote_u32(&ctrl->abort_flag, peer, 1u); };
 
   if (warp == WARP_TMA) {
-    // ------------------------------------------------------------ producer (own tiles)
-    if (lane == 0) {
-      const int my_tiles = pair < tiles ? (tiles - 1 - pair) / npairs + 1 : 0;
-      const int P = my_tiles * nkb;
-      const int npre = P < STAGES ? P : STAGES;
-      uint32_t armed_w = 0, armed_x = 0, par_w = 0, par_x = 0;
+    // ------------------------------------------------------------ raw-ring producer (own rows)
+    if (lane == 0 && NORM != kNoNorm) {
+      uint32_t armed = 0, par = 0;
       bool ok = true;
-      bool withhold = p.stall != 0 && blockIdx.x == 0;   // fault injection (status-path tests only)
+      int t = pair, mb2 = 0, nb = 0, kb = 0;
+      if (P > 0) tile_coords(t, num_m2, num_n, mb2, nb);
+      pdl_wait();   // activations may be written by the previous kernel
+      for (int q = 0; q < P; ++q) {
+        const int r = q % RST;
+        const uint32_t ph = static_cast<uint32_t>(q / RST) & 1u;
+        if (q >= RST &&
+            !mbar_wait(&ctrl->raw_empty[r], ph ^ 1u, abortf, p.status, kStatusWaitEmpty, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = raw + r * RAW_BYTES;
+        const int k0 = kb * BK;
+        const int row0 = mb2 * 2 * BM + static_cast<int>(rank) * BM;
+        bf16* vec = vecs + r * 3 * VEC;
+        const uint32_t vb = static_cast<uint32_t>(min(VEC, K - k0)) * 2;
+        const uint32_t nvec = 1 + (has_beta ? 1 : 0) + (has_bias_in ? 1 : 0);
+        mbar_arrive_expect_tx(&ctrl->raw_full[r], 2 * X_BYTES + vb * nvec);
+        bulk_load(vec, p.gamma + k0, vb, &ctrl->raw_full[r]);
+        if (has_beta) bulk_load(vec + VEC, p.beta + k0, vb, &ctrl->raw_full[r]);
+        if (has_bias_in) bulk_load(vec + 2 * VEC, p.bias_in + k0, vb, &ctrl->raw_full[r]);
+        tma_load_2d(st, &tm_x, &ctrl->raw_full[r], k0, row0);
+        tma_load_2d(st + X_BYTES, &tm_r, &ctrl->raw_full[r], k0, row0);
+        armed |= 1u << r;
+        par = (par & ~(1u << r)) | (ph << r);
+        if (++kb == nkb) {
+          kb = 0;
+          t += npairs;
+          if (t < tiles) tile_coords(t, num_m2, num_n, mb2, nb);
+        }
+      }
+      if (!ok) {
+        abort_pair();
+        for (int i = 0; i < RST; ++i)   // let every issued copy land before the CTA can exit
+          if (armed & (1u << i)) drain_wait(&ctrl->raw_full[i], (par >> i) & 1);
+      }
+    }
+  } else if (warp == WARP_WTMA) {
+    // ------------------------------------------------------------ operand-ring producer (own halves)
+    if (lane == 0) {
+      const int npre = P < OST ? P : OST;
+      uint32_t armed = 0, par = 0;
+      bool ok = true;
+      // fault injection (status-path tests only): CTA 0 withholds position 0's copies
+      const int skip = (p.stall != 0 && blockIdx.x == 0) ? 0 : -1;
       struct Cur {
-        int t, mb2, nb, kb, s;
-        uint32_t ph;
+        int t, mb2, nb, kb;
       };
-      Cur cw{pair, 0, 0, 0, 0, 0u};
+      Cur cw{pair, 0, 0, 0};
       if (P > 0) tile_coords(cw.t, num_m2, num_n, cw.mb2, cw.nb);
       Cur cx = cw;
       auto step = [&](Cur& c) {
@@ -170,18 +240,20 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
           c.t += npairs;
           if (c.t < tiles) tile_coords(c.t, num_m2, num_n, c.mb2, c.nb);
         }
-        if (++c.s == STAGES) {
-          c.s = 0;
-          c.ph ^= 1u;
-        }
       };
-      auto issue_w = [&](const Cur& c) {
-        if (withhold) {
-          withhold = false;
-          return;
-        }
-        uint8_t* st = smem + c.s * STAGE_BYTES + 2 * X_BYTES;
-        mbar_arrive_expect_tx(&ctrl->full_w[c.s], 2 * WH_BYTES);
+      // one arrive_expect_tx per slot use: the W halves (+ the activation tile without a norm)
+      auto arm = [&](int q) {
+        if (q == skip) return;
+        const int s = q % OST;
+        const uint32_t ph = static_cast<uint32_t>(q / OST) & 1u;
+        mbar_arrive_expect_tx(&ctrl->full_w[s], 2 * WH_BYTES + (NORM == kNoNorm ? X_BYTES : 0));
+        armed |= 1u << s;
+        par = (par & ~(1u << s)) | (ph << s);
+      };
+      auto issue_w = [&](int q, const Cur& c) {
+        if (q == skip) return;
+        const int s = q % OST;
+        uint8_t* st = smem + s * OPB + OPA;
         // this CTA's 128-row halves of the two N=256 operands
         int r0, r1;
         if (EPI == kEpiSwiGLU) {
@@ -191,55 +263,46 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
           r0 = c.nb * BN + static_cast<int>(rank) * 128;
           r1 = c.nb * BN + 256 + static_cast<int>(rank) * 128;
         }
-        tma_load_2d(st, &tm_w, &ctrl->full_w[c.s], c.kb * BK, r0);
-        tma_load_2d(st + WH_BYTES, &tm_w, &ctrl->full_w[c.s], c.kb * BK, r1);
-        armed_w |= 1u << c.s;
-        par_w = (par_w & ~(1u << c.s)) | (c.ph << c.s);
+        tma_load_2d(st, &tm_w, &ctrl->full_w[s], c.kb * BK, r0);
+        tma_load_2d(st + WH_BYTES, &tm_w, &ctrl->full_w[s], c.kb * BK, r1);
       };
-      auto issue_x = [&](const Cur& c) {
-        uint8_t* st = smem + c.s * STAGE_BYTES;
-        const int k0 = c.kb * BK;
-        const int row0 = c.mb2 * 2 * BM + static_cast<int>(rank) * BM;
-        if (NORM == kNoNorm) {
-          mbar_arrive_expect_tx(&ctrl->full_x[c.s], X_BYTES);
-          tma_load_2d(st, &tm_x, &ctrl->full_x[c.s], k0, row0);
-        } else {
-          bf16* vec = vecs + c.s * 3 * VEC;
-          const uint32_t vb = static_cast<uint32_t>(min(VEC, K - k0)) * 2;
-          const uint32_t nvec = 1 + (has_beta ? 1 : 0) + (has_bias_in ? 1 : 0);
-          mbar_arrive_expect_tx(&ctrl->full_x[c.s], 2 * X_BYTES + vb * nvec);
-          bulk_load(vec, p.gamma + k0, vb, &ctrl->full_x[c.s]);
-          if (has_beta) bulk_load(vec + VEC, p.beta + k0, vb, &ctrl->full_x[c.s]);
-          if (has_bias_in) bulk_load(vec + 2 * VEC, p.bias_in + k0, vb, &ctrl->full_x[c.s]);
-          tma_load_2d(st, &tm_x, &ctrl->full_x[c.s], k0, row0);
-          tma_load_2d(st + X_BYTES, &tm_r, &ctrl->full_x[c.s], k0, row0);
-        }
-        armed_x |= 1u << c.s;
-        par_x = (par_x & ~(1u << c.s)) | (c.ph << c.s);
+      auto issue_x = [&](int q, const Cur& c) {   // no norm: the activation tile is the operand
+        if (q == skip) return;
+        const int s = q % OST;
+        tma_load_2d(smem + s * OPB, &tm_x, &ctrl->full_w[s], c.kb * BK,
+                    c.mb2 * 2 * BM + static_cast<int>(rank) * BM);
       };
       for (int q = 0; q < npre; ++q) {   // weights stream before the dependency wait
-        issue_w(cw);
+        arm(q);
+        issue_w(q, cw);
         step(cw);
       }
-      pdl_wait();
-      for (int q = 0; q < P; ++q) {
-        if (q >= npre) {
-          if (!mbar_wait(&ctrl->empty[cw.s], cw.ph ^ 1, abortf, p.status, kStatusWaitEmpty, p.wait_ns)) {
-            ok = false;
-            break;
-          }
-          issue_w(cw);
-          step(cw);
+      if (NORM == kNoNorm) {
+        pdl_wait();
+        for (int q = 0; q < npre; ++q) {
+          issue_x(q, cx);
+          step(cx);
         }
-        issue_x(cx);
-        step(cx);
+      }
+      for (int q = npre; q < P; ++q) {
+        const int s = q % OST;
+        const uint32_t ph = static_cast<uint32_t>(q / OST) & 1u;
+        if (!mbar_wait(&ctrl->empty[s], ph ^ 1u, abortf, p.status, kStatusWaitEmpty, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        arm(q);
+        issue_w(q, cw);
+        step(cw);
+        if (NORM == kNoNorm) {
+          issue_x(q, cx);
+          step(cx);
+        }
       }
       if (!ok) {
         abort_pair();
-        for (int i = 0; i < STAGES; ++i) {   // let every issued copy land before the CTA can exit
-          if (armed_w & (1u << i)) drain_wait(&ctrl->full_w[i], (par_w >> i) & 1);
-          if (armed_x & (1u << i)) drain_wait(&ctrl->full_x[i], (par_x >> i) & 1);
-        }
+        for (int i = 0; i < OST; ++i)   // let every issued copy land before the CTA can exit
+          if (armed & (1u << i)) drain_wait(&ctrl->full_w[i], (par >> i) & 1);
       }
     }
   } else if (warp == WARP_MMA) {
@@ -262,11 +325,11 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t xa = smem_u32(smem + s * STAGE_BYTES);
+          const uint32_t xa = smem_u32(smem + s * OPB);
           const uint64_t ad = sw64_desc(xa);
           const uint64_t ld = sw64_desc(xa + X_BYTES);
-          const uint64_t bd0 = sw64_desc(xa + 2 * X_BYTES);
-          const uint64_t bd1 = sw64_desc(xa + 2 * X_BYTES + WH_BYTES);
+          const uint64_t bd0 = sw64_desc(xa + OPA);
+          const uint64_t bd1 = sw64_desc(xa + OPA + WH_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
@@ -277,8 +340,8 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
               umma_bf16_pair(tmem + 256, ld + 2 * kk, bd1 + 2 * kk, idesc, 1u);
             }
           }
-          umma_commit_pair(&ctrl->empty[s], 0x3);   // the stage is free in both CTAs
-          if (++s == STAGES) {
+          umma_commit_pair(&ctrl->empty[s], 0x3);   // the slot is free in both CTAs
+          if (++s == static_cast<uint32_t>(OST)) {
             s = 0;
             ph ^= 1;
           }
@@ -384,14 +447,15 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
   } else {
     // ------------------------------------------------------------ converters (own 128 rows)
     // Two groups of four warps: group g converts positions q = g, g + 2, ...
-    // of this CTA's (tile, k-block) sequence (stage q % STAGES), so two stages
-    // are converted at once and the conversion latency of one stage overlaps
-    // the next. Thread gt of a group (0..127): 16-byte chunk c = gt & 3 of the
-    // 64-byte row, rows rb + 32 j (rb = gt >> 2, j = 0..3). 64-byte swizzle:
-    // chunk c of row r sits at c ^ ((r >> 1) & 3). RMSNorm: each group sums h^2
-    // over its k-blocks; the epilogue adds the two groups' sums in group order.
-    // Without a norm (residual-stream projection) the warps only relay the
-    // stage's readiness to the even CTA.
+    // of this CTA's (tile, k-block) sequence, reading raw slot q % RST and
+    // writing operand slot q % OST, so two positions are converted at once and
+    // the conversion latency of one overlaps the next. Thread gt of a group
+    // (0..127): 16-byte chunk c = gt & 3 of the 64-byte row, rows rb + 32 j
+    // (rb = gt >> 2, j = 0..3). 64-byte swizzle: chunk c of row r sits at
+    // c ^ ((r >> 1) & 3). RMSNorm: each group sums h^2 over its k-blocks; the
+    // epilogue adds the two groups' sums in group order. Without a norm
+    // (residual-stream projection) the warps only relay the slot's readiness
+    // to the even CTA.
     constexpr int RPT = BM / CONV_ROWS_PER_PASS;   // rows per thread (4)
     const int ct = threadIdx.x - WARP_CONV0 * 32;   // 0..255
     const int grp = ct / CONV_GROUP_THREADS;          // 0..CONV_GROUPS-1
@@ -425,23 +489,28 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
       for (long long q = q0 + ((grp - q0 % CONV_GROUPS) + CONV_GROUPS) % CONV_GROUPS; q < q0 + nkb;
            q += CONV_GROUPS) {
         const int kb = static_cast<int>(q - q0);
-        const int s = static_cast<int>(q % STAGES);
-        const uint32_t ph = static_cast<uint32_t>(q / STAGES) & 1u;
-        if (!warp_wait(&ctrl->full_x[s], ph, abortf, p.status, kStatusWaitFull, p.wait_ns) ||
-            !warp_wait(&ctrl->full_w[s], ph, abortf, p.status, kStatusWaitFull, p.wait_ns)) {
-          ok = false;
-          break;
-        }
+        const int s = static_cast<int>(q % OST);
+        const uint32_t ph = static_cast<uint32_t>(q / OST) & 1u;
         if (NORM != kNoNorm) {
-          bf16* vec = vecs + s * 3 * VEC;
+          const int r = static_cast<int>(q % RST);
+          const uint32_t rph = static_cast<uint32_t>(q / RST) & 1u;
+          // the raw tiles have landed, and the UMMA that last read operand slot s is done
+          if (!warp_wait(&ctrl->raw_full[r], rph, abortf, p.status, kStatusWaitFull, p.wait_ns) ||
+              (q >= OST &&
+               !warp_wait(&ctrl->empty[s], ph ^ 1u, abortf, p.status, kStatusWaitEmpty, p.wait_ns))) {
+            ok = false;
+            break;
+          }
+          bf16* vec = vecs + r * 3 * VEC;
           if (K - kb * BK < BK) zero_vec_tails(vec, VEC, K - kb * BK);
           const uint32_t vaddr = smem_u32(vec) + c * 16;
           f32x2 g2[4], be2[4] = {}, bi2[4] = {};
           vec_pairs(vaddr, g2);
           if (NORM == kLayerNorm) vec_pairs(vaddr + 2 * VEC, be2);
           if (BIAS_IN) vec_pairs(vaddr + 4 * VEC, bi2);
-          const uint32_t xs = smem_u32(smem + s * STAGE_BYTES);
+          const uint32_t xs = smem_u32(raw + r * RAW_BYTES);
           const uint32_t rsm = xs + X_BYTES;
+          const uint32_t as = smem_u32(smem + s * OPB);
           uint4 xv[RPT], rv[RPT];
 #pragma unroll
           for (int j = 0; j < RPT; ++j) {
@@ -450,6 +519,9 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
             xv[j] = ld_shared_v4(xs + off);
             rv[j] = ld_shared_v4(rsm + off);
           }
+          // the raw slot is read: its next copies may start
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctrl->raw_empty[r]);
           // instantiated with and without the residual_out store (first N column)
           auto convert_stage = [&](auto wres_tag) {
             constexpr bool WRES = decltype(wres_tag)::value;
@@ -460,8 +532,8 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
               uint4 hi, lo, hres;
               convert8<(NORM == kNoNorm ? kRMSNorm : NORM), BIAS_IN, SPLIT, WRES>(
                   xv[j], rv[j], g2, be2, bi2, mu[j], rs[j], ss[j], hi, lo, hres);
-              st_shared_v4(xs + off, hi);
-              if (SPLIT) st_shared_v4(rsm + off, lo);
+              st_shared_v4(as + off, hi);
+              if (SPLIT) st_shared_v4(as + X_BYTES + off, lo);
               if (WRES) {
                 const int gm = mrow0 + row;
                 const int k0 = kb * BK + c * 8;
@@ -474,8 +546,13 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
           else convert_stage(BoolC<false>{});
           fence_proxy_async_smem();
         }
+        // this CTA's weight halves (and, without a norm, its activation tile) have landed
+        if (!warp_wait(&ctrl->full_w[s], ph, abortf, p.status, kStatusWaitFull, p.wait_ns)) {
+          ok = false;
+          break;
+        }
         __syncwarp();
-        if (lane == 0) {   // this CTA's half of stage s is ready for the pair's UMMA
+        if (lane == 0) {   // this CTA's half of slot s is ready for the pair's UMMA
           if (leader) mbar_arrive(&ctrl->conv[s]);
           else mbar_arrive_remote(&ctrl->conv[s], 0);
         }
