@@ -68,23 +68,33 @@ def _code_only(text: str) -> str:
     return " ".join(text.split())
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(files) -> str:
+    """Hash of the device code a kernel is built from (its own header plus the
+    shared device headers), comments and whitespace stripped."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "transformer_layer_residual_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(files):
         h.update(f.encode())
         h.update(_code_only(open(os.path.join(csrc, f), encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """dram bytes per launch of the dominant kernel from the committed ncu
-    summary, only if it was taken on the current kernel sources."""
+def plan_shape(plan: str) -> str:
+    """The kernel and launch shape of a plan description, without the tuner's note."""
+    return plan.split(" (")[0].strip()
+
+
+def recorded_traffic(workload: str, plan: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, only if it was taken on the current device code of that kernel
+    and with the same kernel and launch shape as the plan being timed."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p)).get(workload)
-    if not d or d.get("kernel_source_hash") != kernel_source_hash():
+    if not d or d.get("kernel_source_hash") != kernel_source_hash(d.get("kernel_files", [])):
+        return None
+    if d.get("plan") != plan_shape(plan):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -472,7 +482,7 @@ def bench_fnl(w, steps, warmup, world, rank, local, tune=True, path="auto"):
         "tokens_per_s_layer": round(w.M * steps * world / (ms_max / 1e3), 1),
         "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": runit,
                      "frac": round(achieved / peak, 4), "peak_source": peak_src,
-                     "traffic": recorded_traffic(w.name),
+                     "traffic": recorded_traffic(w.name, bed.plan),
                      "algorithmic_per_launch": w.algorithmic_bytes() if bound == "hbm" else w.flops(),
                      "kernel": "fused GEMM kernel" + (" + LayerNorm stats kernel (PDL)" if w.norm == "layernorm" else "")},
         "e2e": {"value": round(e2e_value, 3), "unit": unit, "h2d_bytes_per_step": h2d,

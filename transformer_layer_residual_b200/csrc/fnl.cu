@@ -524,9 +524,9 @@ int epi_of(const Call& c) {
   return c.op == Op::QKV ? fnl::kEpiQKV : (c.op == Op::SwiGLU ? fnl::kEpiSwiGLU : fnl::kEpiGELU);
 }
 
-// FP8 pre-pass: residual_out, statistics outputs and the per-token (mean,
-// rstd, s_a, 448 / amax) for the converters.
-fnl_status launch_fp8_prepass(fnl_handle* h, const Call& c, float4* stats8, cudaStream_t stream) {
+// FP8 pre-pass: residual_out, statistics outputs, the per-token (mean, rstd,
+// s_a, 448 / amax) and the activation codes q8 [M][K] that the GEMM loads.
+fnl_status launch_fp8_prepass(fnl_handle* h, const Call& c, float4* stats8, uint8_t* q8, cudaStream_t stream) {
   const int nvec = c.K / 8;
   const int v = (nvec + fnl::kK1Threads - 1) / fnl::kK1Threads;
   const bool rms = c.norm == FNL_NORM_RMSNORM;
@@ -535,11 +535,12 @@ fnl_status launch_fp8_prepass(fnl_handle* h, const Call& c, float4* stats8, cuda
   do {                                                                                                             \
     if (rms)                                                                                                       \
       fnl::k1_fp8_prepass<MAXV, true><<<grid, block, 0, stream>>>(c.x, c.residual, c.bias_in, c.gamma, nullptr,   \
-                                                                  c.residual_out, stats8, nullptr, c.rstd_out,    \
+                                                                  c.residual_out, stats8, q8, nullptr, c.rstd_out, \
                                                                   c.M, c.K, c.eps);                                \
     else                                                                                                           \
       fnl::k1_fp8_prepass<MAXV, false><<<grid, block, 0, stream>>>(c.x, c.residual, c.bias_in, c.gamma, c.beta,   \
-                                                                   c.residual_out, stats8, c.mean_out, c.rstd_out, \
+                                                                   c.residual_out, stats8, q8, c.mean_out,         \
+                                                                   c.rstd_out,                                     \
                                                                    c.M, c.K, c.eps);                               \
   } while (0)
   if (v <= 1) FNL_PP(1);
@@ -623,7 +624,7 @@ fnl_status plan_kernel(fnl_handle* h, const Call& c, Kern kern, int cls_req, Pla
     const long long U = static_cast<long long>(q.T) * nkb;
     q.grid = static_cast<int>(std::min<long long>(max_ctas, U));
     const int sb = c.fp8 ? fnl::k3::stage_bytes8(q.mpad) : fnl::k3::stage_bytes(q.mpad);
-    q.stages = std::min(fnl::k3::MAX_STAGES, (200 * 1024) / sb);
+    q.stages = std::min(c.fp8 ? fnl::k3::MAX_STAGES_FP8 : fnl::k3::MAX_STAGES, (200 * 1024) / sb);
     q.smem = fnl::k3::smem_bytes(q.mpad, q.stages, c.fp8);
     q.threads = fnl::k3::NUM_THREADS;
     if (cls_req >= 2) {
@@ -728,7 +729,8 @@ fnl_status default_plan(fnl_handle* h, const Call& c, Plan* pl) {
 }
 
 size_t stats_bytes_of(const Call& c) {
-  if (c.fp8) return align256(static_cast<size_t>(c.M) * 16);   // (mean, rstd, s_a, 448 / amax) per token
+  // FP8: (mean, rstd, s_a, 448 / amax) per token, then the tokens' e4m3 activation codes
+  if (c.fp8) return align256(static_cast<size_t>(c.M) * 16) + align256(static_cast<size_t>(c.M) * c.K);
   const bool ln = c.op != Op::Residual && c.norm == FNL_NORM_LAYERNORM;
   return ln ? align256(static_cast<size_t>(c.M) * 8) : 0;
 }
@@ -805,8 +807,15 @@ fnl_status launch_plan(fnl_handle* h, const Call& c, const Plan& q) {
   else if (pair) w_rows = 128;   // one CTA's half of an N = 256 operand
   else w_rows = c.op == Op::SwiGLU ? 128 : fnl::k2::BN;
   const int box_cols = wide ? fnl::k2w::BK : (pair ? fnl::k4::BK : 64);
-  if ((st = make_map(h, &mx, c.x, c.M, c.K, act_rows, box_cols)) != FNL_OK) return st;
-  if (!nonorm && (st = make_map(h, &mr, c.residual, c.M, c.K, act_rows, box_cols)) != FNL_OK) return st;
+  // FP8: the activation operand is the pre-pass's codes (one byte each), after the per-token scales
+  uint8_t* q8 = c.fp8 ? ws + kFixedBytes + align256(static_cast<size_t>(c.M) * 16) : nullptr;
+  if (c.fp8) {
+    if ((st = make_map(h, &mx, q8, c.M, c.K, act_rows, 64, 1)) != FNL_OK) return st;
+    mr = mx;   // unused
+  } else {
+    if ((st = make_map(h, &mx, c.x, c.M, c.K, act_rows, box_cols)) != FNL_OK) return st;
+    if (!nonorm && (st = make_map(h, &mr, c.residual, c.M, c.K, act_rows, box_cols)) != FNL_OK) return st;
+  }
   if ((st = make_map(h, &mw, c.W, c.N, c.K, w_rows, box_cols, c.fp8 ? 1 : 2)) != FNL_OK) return st;
   // Every GEMM kernel is a programmatic dependent of its predecessor: it
   // streams its first weight tiles before griddepcontrol.wait and touches
@@ -814,7 +823,7 @@ fnl_status launch_plan(fnl_handle* h, const Call& c, const Plan& q) {
   const bool pdl = true;
   if (nonorm) return dispatch_residual(h, small, wide, pair, q.grid, q.threads, q.smem, pdl, c.stream, mx, mw, p);
   if (c.fp8) {
-    if ((st = launch_fp8_prepass(h, c, reinterpret_cast<float4*>(stats), c.stream)) != FNL_OK) return st;
+    if ((st = launch_fp8_prepass(h, c, reinterpret_cast<float4*>(stats), q8, c.stream)) != FNL_OK) return st;
     return dispatch_fp8(h, epi_of(c), q.grid, q.threads, q.smem, pdl, c.stream, mx, mr, mw, p);
   }
   if (!rms) {

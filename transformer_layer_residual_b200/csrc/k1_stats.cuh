@@ -135,7 +135,10 @@ __device__ __forceinline__ void block_sum_max_256(float& s, float& m, float* red
 // gamma + beta; RMSNorm a = h gamma (1/rms is a positive per-token factor, so
 // it joins the token's dequantisation scale instead). Writes stats8[row] =
 // (mean, rstd, dequantisation scale, 448 / amax) with the scale amax / 448
-// (times rstd for RMSNorm); 1 and 1 for a zero row.
+// (times rstd for RMSNorm); 1 and 1 for a zero row; and the row's activation
+// codes q8[row][k] = e4m3(a * 448 / amax) (round to nearest even, saturating),
+// which the GEMM loads as its operand: the row is quantised once, not once per
+// weight tile.
 template <int MAXV, bool RMS>
 __global__ void __launch_bounds__(kK1Threads) k1_fp8_prepass(const bf16* __restrict__ x,
                                                              const bf16* __restrict__ residual,
@@ -144,6 +147,7 @@ __global__ void __launch_bounds__(kK1Threads) k1_fp8_prepass(const bf16* __restr
                                                              const bf16* __restrict__ beta,
                                                              bf16* __restrict__ residual_out,
                                                              float4* __restrict__ stats8,
+                                                             uint8_t* __restrict__ q8,
                                                              float* __restrict__ mean_out,
                                                              float* __restrict__ rstd_out, int M, int K,
                                                              float eps) {
@@ -231,12 +235,31 @@ __global__ void __launch_bounds__(kK1Threads) k1_fp8_prepass(const bf16* __restr
     }
   }
   if (!RMS) amax = block_max_256(amax, red);
+  const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
   if (threadIdx.x == 0) {
     const float sa = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-    const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
     stats8[row] = make_float4(mean, rstd, RMS ? rstd * sa : sa, inv);
     if (mean_out) mean_out[row] = mean;
     if (rstd_out) rstd_out[row] = rstd;
+  }
+  // the codes: the same fp32 operations, in the same order, as the amax above
+  const f32x2 inv2 = pk2(inv, inv);
+#pragma unroll
+  for (int i = 0; i < MAXV; ++i) {
+    const int v = threadIdx.x + i * kK1Threads;
+    if (v < nvec) {
+      const uint4 gv = ldg16(gamma + v * 8);
+      const uint4 bv = (!RMS && beta != nullptr) ? ldg16(beta + v * 8) : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, bw[4] = {bv.x, bv.y, bv.z, bv.w};
+      f32x2 a[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const f32x2 y = RMS ? mul2(h[i][e], bf2_to_f2(gw[e]))
+                            : fma2(mul2(sub2(h[i][e], mu2), rs2), bf2_to_f2(gw[e]), bf2_to_f2(bw[e]));
+        a[e] = mul2(y, inv2);
+      }
+      *reinterpret_cast<uint2*>(q8 + rbase + v * 8) = make_uint2(e4m3x4(a[0], a[1]), e4m3x4(a[2], a[3]));
+    }
   }
 }
 

@@ -40,7 +40,9 @@ namespace k3 {
 
 constexpr int BW = 128;   // W rows per tile (UMMA M)
 constexpr int BK = 64;
-constexpr int MAX_STAGES = 8;
+constexpr int MAX_STAGES = 8;        // bf16 forms
+constexpr int MAX_STAGES_FP8 = 16;   // FP8 form: 8 KB weight stages, so twice as many for the same bytes in flight
+constexpr int RING = MAX_STAGES_FP8;
 constexpr int W_BYTES = BW * BK * 2;   // 16 KB
 constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_EPI0 = 2, NUM_EPI_WARPS = 4;
 constexpr int WARP_CONV0 = 6, NUM_CONV_WARPS = 4;
@@ -54,10 +56,10 @@ constexpr int MAX_MPAD = 128;
 constexpr int PREWAIT_STAGES = 0;
 // The FP8 form's predecessor is always its own light pre-pass (one CTA per
 // token), so its whole first ring of weight stages streams before the wait.
-constexpr int PREWAIT_STAGES_FP8 = MAX_STAGES;
+constexpr int PREWAIT_STAGES_FP8 = MAX_STAGES_FP8;
 
 struct Ctrl {
-  uint64_t full_w[MAX_STAGES], full_x[MAX_STAGES], conv[MAX_STAGES], empty[MAX_STAGES];
+  uint64_t full_w[RING], full_x[RING], conv[RING], empty[RING];
   uint64_t tfull[2], tempty[2], sfull[2], drain, esync, rbar;
   long long u0, u1;   // this CTA's unit range
   uint32_t tmem_base;
@@ -69,12 +71,12 @@ struct Ctrl {
 };
 
 __host__ __device__ inline int stage_bytes(int mpad) { return W_BYTES + 2 * mpad * BK * 2; }
-// FP8 form: the W tile is 128 rows x 64 e4m3 (8 KB, 64-byte swizzle), the x and
-// residual tiles stay bf16, and the converters write the e4m3 activation
-// operand [mpad][64] (64-byte swizzle) after them.
+// FP8 form: the W tile is 128 rows x 64 e4m3 (8 KB, 64-byte swizzle) and the
+// activation operand [mpad][64] e4m3 codes (64-byte swizzle), both as loaded:
+// the pre-pass has quantised each token's row once, so no W tile re-does it.
 constexpr int W8_BYTES = BW * BK;   // 8 KB
-__host__ __device__ inline int stage_bytes8(int mpad) { return W8_BYTES + 2 * mpad * BK * 2 + mpad * BK; }
-constexpr int VEC_BYTES = MAX_STAGES * kVecStageBytes;   // 3 KB
+__host__ __device__ inline int stage_bytes8(int mpad) { return W8_BYTES + mpad * BK; }
+constexpr int VEC_BYTES = MAX_STAGES * kVecStageBytes;   // 3 KB (the bf16 forms' gamma / beta / bias_in slices)
 __host__ __device__ inline int smem_bytes(int mpad, int stages, bool fp8 = false) {
   return stages * (fp8 ? stage_bytes8(mpad) : stage_bytes(mpad)) + VEC_BYTES + static_cast<int>(sizeof(Ctrl)) + 1024;
 }
@@ -296,10 +298,11 @@ __device__ __forceinline__ void k3_cluster_reduce(const OpParams& p, uint32_t pa
   }
 }
 
-// FP8 (e4m3 weights and activations, kind::f8f6f4 UMMA): the normalisation uses
-// the pre-pass statistics (p.stats8: mean, rstd and the token's quantisation
-// scale) for both norms, so it is instantiated with NORM = kLayerNorm (beta
-// absent and mean 0 for RMSNorm); the epilogue multiplies by s_a[m] s_w[n].
+// FP8 (e4m3 weights and activations, kind::f8f6f4 UMMA): the pre-pass has
+// normalised and quantised each token's row once (e4m3 codes [M][K] in the
+// workspace, tm_x maps them), so the codes tile is the UMMA's B operand as
+// loaded and the converter warps have nothing to do; the epilogue multiplies by
+// s_a[m] s_w[n] (p.stats8, p.w_scale). Instantiated with NORM = kLayerNorm.
 template <int EPI, int NORM, bool SPLIT, bool FP8 = false>
 __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     k3_splitk_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_r,
@@ -310,6 +313,9 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
   const int mpad = p.mpad, S = p.stages;
   const int SB = FP8 ? stage_bytes8(mpad) : stage_bytes(mpad);
   const int WB = FP8 ? W8_BYTES : W_BYTES;   // x tile offset within a stage
+  // the activation tile is the UMMA operand as loaded: no norm (residual-stream
+  // projection), or the FP8 form's pre-quantised codes
+  constexpr bool DIRECT = NORM == kNoNorm || FP8;
   const int XB = mpad * BK * 2;
   bf16* vecs = reinterpret_cast<bf16*>(smem + S * SB);   // [S][3][64]
   Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + S * SB + VEC_BYTES);
@@ -363,7 +369,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
     tmem_alloc(&ctrl->tmem_base, ncols);
     tmem_relinquish();
   }
-  zero_vec_slices(vecs, S * 3 * kVecElems);
+  if (!DIRECT) zero_vec_slices(vecs, S * 3 * kVecElems);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -417,8 +423,8 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
       };
       auto issue_x = [&](const Cur& c) {
         uint8_t* st = smem + c.s * SB;
-        if (NORM == kNoNorm) {   // the activation tile is the operand as loaded
-          mbar_arrive_expect_tx(&ctrl->full_x[c.s], XB);
+        if (DIRECT) {   // the activation tile is the operand as loaded
+          mbar_arrive_expect_tx(&ctrl->full_x[c.s], FP8 ? mpad * BK : XB);
           tma_load_2d(st + WB, &tm_x, &ctrl->full_x[c.s], c.kb * BK, 0);
           armed_x |= 1u << c.s;
           par_x = (par_x & ~(1u << c.s)) | (c.ph << c.s);
@@ -479,7 +485,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
         const uint32_t d = tmem + b * mpad;
         for (int kb = 0; kb < nk; ++kb) {
           // the converted operand (or, without a norm, the activation tile as loaded)
-          uint64_t* ready = NORM == kNoNorm ? &ctrl->full_x[s] : &ctrl->conv[s];
+          uint64_t* ready = DIRECT ? &ctrl->full_x[s] : &ctrl->conv[s];
           if (!mbar_wait(ready, ph, abortf, p.status, kStatusWaitConv, p.wait_ns) ||
               !mbar_wait(&ctrl->full_w[s], ph, abortf, p.status, kStatusWaitFull, p.wait_ns)) {
             ok = false;
@@ -489,7 +495,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
           const uint32_t wa = smem_u32(smem + s * SB);
           if (FP8) {   // 64 e4m3 per row: two K = 32 steps of 32 bytes
             const uint64_t ad = sw64_desc(wa);
-            const uint64_t bd = sw64_desc(wa + WB + 2 * XB);
+            const uint64_t bd = sw64_desc(wa + WB);
 #pragma unroll
             for (int kk = 0; kk < BK / 32; ++kk)
               umma_f8(d, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
@@ -622,89 +628,7 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
         }
       }
     }
-  } else if (FP8) {
-    // ------------------------------------------------------------ converters (FP8)
-    // Converter warp cw owns positions cw, cw + 4, ... as below. A lane task is
-    // (token row, 16-byte e4m3 chunk j of the row's 64): it reads the bf16
-    // chunks 2j and 2j + 1 of x and the residual, forms h (+ bias_in), normalises
-    // with the pre-pass statistics, a = (h - mean) rstd gamma + beta for
-    // LayerNorm, a = h gamma for RMSNorm (the pre-pass computes the same
-    // expression for the token's amax), and stores e4m3(a * 448 / amax) (round
-    // to nearest even, saturating).
-    const int cw = warp - WARP_CONV0;
-    pdl_wait();   // statistics come from the pre-pass
-    // a lane's tasks are rows (lane >> 2) + 8 i, all with chunk j = lane & 3:
-    // their (mean, rstd, 448 / amax) are loaded once
-    constexpr int kRowsPerLane = MAX_MPAD / 8;
-    float smu[kRowsPerLane], srs[kRowsPerLane], sinv[kRowsPerLane];
-#pragma unroll
-    for (int i = 0; i < kRowsPerLane; ++i) {
-      const int row = (lane >> 2) + 8 * i;
-      smu[i] = srs[i] = sinv[i] = 0.f;
-      if (row < M) {
-        const float4 st = p.stats8[row];
-        smu[i] = st.x;
-        srs[i] = st.y;
-        sinv[i] = st.w;
-      }
-    }
-    const int P = static_cast<int>(u1 - u0);
-    int s = cw;
-    uint32_t ph = 0;
-    for (int q = cw; q < P; q += NUM_CONV_WARPS) {
-      const long long u = u0 + q;
-      const int kb = static_cast<int>(u % nkb);
-      if (!warp_wait(&ctrl->full_x[s], ph, abortf, p.status, kStatusWaitFull, p.wait_ns)) break;
-      const uint32_t xs = smem_u32(smem + s * SB) + WB;
-      const uint32_t rsm = xs + XB;
-      const uint32_t qs = rsm + XB;
-      bf16* vec = vecs + s * 3 * kVecElems;
-      if (K - kb * BK < BK) zero_vec_tails(vec, kVecElems, K - kb * BK);
-      const uint32_t vaddr = smem_u32(vec);
-#pragma unroll
-      for (int i = 0; i < kRowsPerLane; ++i) {
-        const int row = (lane >> 2) + 8 * i, j = lane & 3;
-        if (row >= M) break;
-        const f32x2 mu2 = pk2(smu[i], smu[i]), rs2 = pk2(srs[i], srs[i]), inv2 = pk2(sinv[i], sinv[i]);
-        uint32_t codes[4];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int c = 2 * j + hh;
-          const uint32_t off = row * 128 + ((c ^ (row & 7)) << 4);
-          const uint4 xv = ld_shared_v4(xs + off), rv = ld_shared_v4(rsm + off);
-          f32x2 g2[4], be2[4] = {}, bi2[4] = {};
-          vec_pairs(vaddr + c * 16, g2);
-          if (p.beta != nullptr) vec_pairs(vaddr + 2 * kVecElems + c * 16, be2);
-          if (BIAS_IN) vec_pairs(vaddr + 4 * kVecElems + c * 16, bi2);
-          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, rw[4] = {rv.x, rv.y, rv.z, rv.w};
-#pragma unroll
-          for (int i = 0; i < 4; i += 2) {
-            f32x2 h0 = add2(bf2_to_f2(xw[i]), bf2_to_f2(rw[i]));
-            f32x2 h1 = add2(bf2_to_f2(xw[i + 1]), bf2_to_f2(rw[i + 1]));
-            if (BIAS_IN) {
-              h0 = add2(h0, bi2[i]);
-              h1 = add2(h1, bi2[i + 1]);
-            }
-            // RMSNorm: codes of h * gamma (rstd joins the token's scale); LayerNorm:
-            // of the normalised value
-            const f32x2 a0 = mul2(p.fp8_rms ? mul2(h0, g2[i]) : fma2(mul2(sub2(h0, mu2), rs2), g2[i], be2[i]), inv2);
-            const f32x2 a1 =
-                mul2(p.fp8_rms ? mul2(h1, g2[i + 1]) : fma2(mul2(sub2(h1, mu2), rs2), g2[i + 1], be2[i + 1]), inv2);
-            codes[hh * 2 + i / 2] = e4m3x4(a0, a1);
-          }
-        }
-        st_shared_v4(qs + row * 64 + ((j ^ ((row >> 1) & 3)) << 4), make_uint4(codes[0], codes[1], codes[2], codes[3]));
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctrl->conv[s]);
-      s += NUM_CONV_WARPS;
-      if (s >= S) {
-        s -= S;
-        ph ^= 1u;
-      }
-    }
-  } else if (NORM != kNoNorm) {
+  } else if (!DIRECT) {
     // ------------------------------------------------------------ converters
     // Converter warp cw owns pipeline positions cw, cw + 4, cw + 8, ... of this
     // CTA's unit sequence, so up to four stages are converted at once. Lanes
