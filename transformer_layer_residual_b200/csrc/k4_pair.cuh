@@ -76,6 +76,16 @@ constexpr int CONV_GROUP_WARPS = NUM_CONV_WARPS / CONV_GROUPS;          // 4
 constexpr int CONV_GROUP_THREADS = CONV_GROUP_WARPS * 32;               // 128
 constexpr int CONV_ROWS_PER_PASS = CONV_GROUP_THREADS / 4;              // 32 rows x 4 chunks
 constexpr int NUM_THREADS = (WARP_WTMA + 1) * 32;   // 480
+// The epilogue is shared by the epilogue warps and each converter group for
+// LayerNorm and for the no-norm projection (on B200: LayerNorm + GELU 0.60 ->
+// 0.64 of the sustained tensor peak, the down projection 0.96 -> 0.99). Not with
+// RMSNorm: there the converters also carry the h^2 sums, the shared form needs
+// more registers than the 128 a thread of this 480-thread CTA can have, and in
+// the long power-capped runs the busier SM clocked lower and lost 2-3%. Nor in
+// the split form, which is bound by the tensor pipe (two UMMAs per operand).
+__host__ __device__ constexpr int epi_shares(bool split, int norm) {
+  return (split || norm == kRMSNorm) ? 1 : 1 + CONV_GROUPS;
+}
 constexpr int TMEM_COLS = 512;
 constexpr int GROUP_M = 8;         // pair rows (of 256 tokens) sharing a W tile while it is hot in L2
 
@@ -116,6 +126,7 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
   using namespace k4;
   constexpr int OST = op_stages(SPLIT), RST = raw_stages(SPLIT);
   constexpr int OPB = op_bytes(SPLIT), OPA = op_a_bytes(SPLIT);
+  constexpr int EPI_SHARES = epi_shares(SPLIT, NORM);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* raw = smem + OST * OPB;                                        // [RST][x | residual]
@@ -150,7 +161,7 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
       mbar_init(&ctrl->raw_empty[r], CONV_GROUP_WARPS);  // the warps of the group that converted it
     }
     mbar_init(&ctrl->tfull, 1);
-    mbar_init(&ctrl->tempty, 2 * NUM_EPI_WARPS);       // (even CTA) epilogue warps of both CTAs
+    mbar_init(&ctrl->tempty, 2 * NUM_EPI_WARPS * EPI_SHARES);   // (even CTA) every epilogue share of both CTAs
     for (int b = 0; b < 2; ++b) {
       mbar_init(&ctrl->sfull[b], NUM_CONV_WARPS);
       mbar_init(&ctrl->efree[b], NUM_EPI_WARPS);
@@ -177,6 +188,95 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
   volatile int* abortf = &ctrl->abort_flag;
   // a wait that gave up (or saw the flag) also stops the other CTA of the pair
   auto abort_pair = [&]() { st_remote_u32(&ctrl->abort_flag, peer, 1u); };
+
+  // The epilogue of the pair's i-th tile t for this warp's TMEM lane quarter
+  // (rows q32 .. q32 + 31 of the CTA's 128): share j of EPI_SHARES, 16-column
+  // chunks cc = j, j + EPI_SHARES, ... The epilogue warps take share 0; the
+  // converter warps, idle while the UMMA waits for the accumulator, take shares
+  // 1 and 2 (group 0 and 1) before they start on the next tile. Every taking
+  // warp of both CTAs arrives on the even CTA's tempty.
+  auto epilogue_share = [&](int i, int t, int j) -> bool {
+    const int q32 = (warp & 3) * 32;
+    const int row_local = q32 + lane;
+    if (!warp_wait(&ctrl->tfull, static_cast<uint32_t>(i) & 1, abortf, p.status, kStatusWaitTmemFull,
+                   p.wait_ns)) {
+      if (lane == 0) abort_pair();
+      return false;
+    }
+    float scale = 1.f;
+    if (NORM == kRMSNorm) {
+      const int b = i & 1;
+      if (!warp_wait(&ctrl->sfull[b], static_cast<uint32_t>(i >> 1) & 1, abortf, p.status, kStatusWaitStats,
+                     p.wait_ns)) {
+        if (lane == 0) abort_pair();
+        return false;
+      }
+      float ssum = 0.f;
+#pragma unroll
+      for (int g = 0; g < CONV_GROUPS; ++g) ssum += ctrl->rs[b][g][row_local];   // fixed order
+      scale = 1.f / sqrtf(ssum / static_cast<float>(K) + p.eps);
+      __syncwarp();
+      if (j == 0 && lane == 0) mbar_arrive(&ctrl->efree[b]);   // the converters may refill rs[b] (see below)
+    }
+    tc_fence_after();
+    int mb2, nb;
+    tile_coords(t, num_m2, num_n, mb2, nb);
+    const int m = mb2 * 2 * BM + static_cast<int>(rank) * BM + row_local;
+    const bool row_ok = m < M;
+    if (NORM == kRMSNorm && j == 0 && nb == 0 && row_ok && p.rstd_out != nullptr) p.rstd_out[m] = scale;
+    const uint32_t tbase = tmem + (static_cast<uint32_t>(q32) << 16);
+    // 16-column chunks: few registers held, so the converter warps can take shares without spilling
+    if (EPI == kEpiSwiGLU) {
+#pragma unroll 1
+      for (int cc = j; cc < 16; cc += EPI_SHARES) {
+        uint32_t g0[16], u0[16];
+        tmem_ld16(tbase + cc * 16, g0);
+        tmem_ld16(tbase + 256 + cc * 16, u0);
+        tmem_ld_wait();
+        if (row_ok) {
+#pragma unroll
+          for (int g8 = 0; g8 < 2; ++g8) {
+            const int jj = nb * 256 + cc * 16 + g8 * 8;
+            if (jj < p.I) {
+              float gv[8], uv[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                gv[e] = __uint_as_float(g0[g8 * 8 + e]);
+                uv[e] = __uint_as_float(u0[g8 * 8 + e]);
+              }
+              store_swiglu8(p, m, jj, gv, uv, scale);
+            }
+          }
+        }
+      }
+    } else {
+#pragma unroll 1
+      for (int cc = j; cc < BN / 16; cc += EPI_SHARES) {
+        uint32_t a0[16];
+        tmem_ld16(tbase + cc * 16, a0);
+        tmem_ld_wait();
+        if (row_ok) {
+#pragma unroll
+          for (int g8 = 0; g8 < 2; ++g8) {
+            const int n = nb * BN + cc * 16 + g8 * 8;
+            if (n < p.N) {
+              float av[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) av[e] = __uint_as_float(a0[g8 * 8 + e]);
+              store_out8<EPI>(p, m, n, av, scale);
+            }
+          }
+        }
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {   // the pair's accumulator may be overwritten once every share of both CTAs is read
+      if (leader) mbar_arrive(&ctrl->tempty);
+      else mbar_arrive_remote(&ctrl->tempty, 0);
+    }
+    return true;
+  };
 
   if (warp == WARP_TMA) {
     // ------------------------------------------------------------ raw-ring producer (own rows)
@@ -354,96 +454,11 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
       drain_wait(&ctrl->drain, 0);
     }
   } else if (warp < WARP_CONV0) {
-    // ------------------------------------------------------------ epilogue (own 128 rows)
-    const int q = warp & 3;
-    const int row_local = q * 32 + lane;
+    // ------------------------------------------------------------ epilogue (own 128 rows, share 0)
     pdl_wait();
     int i = 0;
-    for (int t = pair; t < tiles; t += npairs, ++i) {
-      const uint32_t par = static_cast<uint32_t>(i) & 1;
-      if (!warp_wait(&ctrl->tfull, par, abortf, p.status, kStatusWaitTmemFull, p.wait_ns)) {
-        if (lane == 0) abort_pair();
-        break;
-      }
-      float scale = 1.f;
-      if (NORM == kRMSNorm) {
-        const int b = i & 1;
-        if (!warp_wait(&ctrl->sfull[b], static_cast<uint32_t>(i >> 1) & 1, abortf, p.status, kStatusWaitStats,
-                       p.wait_ns)) {
-          if (lane == 0) abort_pair();
-          break;
-        }
-        float ssum = 0.f;
-#pragma unroll
-        for (int g = 0; g < CONV_GROUPS; ++g) ssum += ctrl->rs[b][g][row_local];   // fixed order
-        scale = 1.f / sqrtf(ssum / static_cast<float>(K) + p.eps);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctrl->efree[b]);   // the converters may refill rs[b]
-      }
-      tc_fence_after();
-      int mb2, nb;
-      tile_coords(t, num_m2, num_n, mb2, nb);
-      const int m = mb2 * 2 * BM + static_cast<int>(rank) * BM + row_local;
-      const bool row_ok = m < M;
-      if (NORM == kRMSNorm && nb == 0 && row_ok && p.rstd_out != nullptr) p.rstd_out[m] = scale;
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      if (EPI == kEpiSwiGLU) {
-#pragma unroll 1
-        for (int cc = 0; cc < 8; ++cc) {
-          uint32_t g0[16], g1[16], u0[16], u1[16];
-          tmem_ld16(tbase + cc * 32, g0);
-          tmem_ld16(tbase + cc * 32 + 16, g1);
-          tmem_ld16(tbase + 256 + cc * 32, u0);
-          tmem_ld16(tbase + 256 + cc * 32 + 16, u1);
-          tmem_ld_wait();
-          if (row_ok) {
-#pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) {
-              const int j = nb * 256 + cc * 32 + g8 * 8;
-              if (j < p.I) {
-                float gv[8], uv[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  const int c = g8 * 8 + e;
-                  gv[e] = __uint_as_float(c < 16 ? g0[c] : g1[c - 16]);
-                  uv[e] = __uint_as_float(c < 16 ? u0[c] : u1[c - 16]);
-                }
-                store_swiglu8(p, m, j, gv, uv, scale);
-              }
-            }
-          }
-        }
-      } else {
-#pragma unroll 1
-        for (int cc = 0; cc < BN / 32; ++cc) {
-          uint32_t a0[16], a1[16];
-          tmem_ld16(tbase + cc * 32, a0);
-          tmem_ld16(tbase + cc * 32 + 16, a1);
-          tmem_ld_wait();
-          if (row_ok) {
-#pragma unroll
-            for (int g8 = 0; g8 < 4; ++g8) {
-              const int n = nb * BN + cc * 32 + g8 * 8;
-              if (n < p.N) {
-                float av[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                  const int c = g8 * 8 + e;
-                  av[e] = __uint_as_float(c < 16 ? a0[c] : a1[c - 16]);
-                }
-                store_out8<EPI>(p, m, n, av, scale);
-              }
-            }
-          }
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {   // the pair's accumulator may be overwritten once both CTAs read it
-        if (leader) mbar_arrive(&ctrl->tempty);
-        else mbar_arrive_remote(&ctrl->tempty, 0);
-      }
-    }
+    for (int t = pair; t < tiles; t += npairs, ++i)
+      if (!epilogue_share(i, t, 0)) break;
   } else {
     // ------------------------------------------------------------ converters (own 128 rows)
     // Two groups of four warps: group g converts positions q = g, g + 2, ...
@@ -455,7 +470,9 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
     // c ^ ((r >> 1) & 3). RMSNorm: each group sums h^2 over its k-blocks; the
     // epilogue adds the two groups' sums in group order. Without a norm
     // (residual-stream projection) the warps only relay the slot's readiness
-    // to the even CTA.
+    // to the even CTA. Before tile i + 1 each group takes its share of tile i's
+    // epilogue: the UMMA cannot start tile i + 1 before the accumulator is
+    // read, so the shares shorten the gap between tiles.
     constexpr int RPT = BM / CONV_ROWS_PER_PASS;   // rows per thread (4)
     const int ct = threadIdx.x - WARP_CONV0 * 32;   // 0..255
     const int grp = ct / CONV_GROUP_THREADS;          // 0..CONV_GROUPS-1
@@ -467,6 +484,11 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
     bool ok = true;
     long long q0 = 0;   // first position of the current tile
     for (int t = pair; t < tiles && ok; t += npairs, ++i, q0 += nkb) {
+      // this group's share of the previous tile's epilogue, before any of this tile's state is live
+      if (EPI_SHARES > 1 && i > 0 && !epilogue_share(i - 1, t - npairs, 1 + grp)) {
+        ok = false;
+        break;
+      }
       int mb2, nb;
       tile_coords(t, num_m2, num_n, mb2, nb);
       const int mrow0 = mb2 * 2 * BM + static_cast<int>(rank) * BM;
@@ -586,6 +608,8 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
         if (lane == 0) mbar_arrive(&ctrl->sfull[b]);
       }
     }
+    // the last tile's share (its epilogue has no next tile to wait behind)
+    if (EPI_SHARES > 1 && ok && i > 0) epilogue_share(i - 1, pair + (i - 1) * npairs, 1 + grp);
   }
 
   // Every role's loop is over and the even CTA's last UMMA has completed (its
