@@ -84,7 +84,8 @@ def test_binding_codes_match_the_header():
     the header's enum values (a mismatch would silently pick another kernel)."""
     e = _header_enum_values()
     paths = {"auto": "FNL_PATH_AUTO", "tile": "FNL_PATH_TILE", "splitk": "FNL_PATH_SPLITK",
-             "wide": "FNL_PATH_TILE_WIDE", "cluster": "FNL_PATH_SPLITK_CLUSTER", "pair": "FNL_PATH_TILE_PAIR"}
+             "wide": "FNL_PATH_TILE_WIDE", "cluster": "FNL_PATH_SPLITK_CLUSTER", "pair": "FNL_PATH_TILE_PAIR",
+             "pair_sk": "FNL_PATH_TILE_PAIR_SPLIT"}
     assert {k: e[v] for k, v in paths.items()} == fnl.PATHS
     assert {"layernorm": e["FNL_NORM_LAYERNORM"], "rmsnorm": e["FNL_NORM_RMSNORM"]} == fnl.NORMS
     precisions = {"default": "FNL_PRECISION_DEFAULT", "split": "FNL_PRECISION_SPLIT",

@@ -316,3 +316,56 @@ def test_pair_kernel_row_tails(cuda_device, M, op, norm):
     w, inputs = _tail_workload(op, norm, M, K=328, seed=M)
     run_and_check(h, w, inputs)
     h.close()
+
+
+# Pair kernel, stream-K form (forced): few tiles for the 74 pairs, so the (tile,
+# k-block) units are dealt over all pairs and each tile is summed from several
+# pairs' partial sums (K not a multiple of the 32-wide k-block in two cases).
+STREAM_K_CASES = [
+    ("qkv", "rmsnorm", 300, 2048, dict(Hq=6, Hkv=2, D=128, bias_out=True)),
+    ("qkv", "layernorm", 513, 2000, dict(Hq=4, Hkv=2, D=128)),
+    ("swiglu", "rmsnorm", 260, 1536, dict(I=600, bias_out=True)),
+    ("swiglu", "layernorm", 256, 4096, dict(I=256)),   # one tile over every pair
+    ("gelu", "layernorm", 256, 2600, dict(N=1000, bias_in=True, bias_out=True)),
+    ("residual", "none", 384, 2048, dict(N=704, bias_out=True)),
+]
+
+
+@pytest.mark.parametrize("op,norm,M,K,kw", STREAM_K_CASES)
+def test_pair_kernel_stream_k(cuda_device, op, norm, M, K, kw):
+    h = fnl.Handle(0, path="pair_sk")
+    w, inputs = synthetic.make_custom(op, norm, M, K, seed=M + K, **kw)
+    _, got = run_and_check(h, w, inputs)
+    assert "stream-K" in h.last_plan(), h.last_plan()
+    # the slot-order sum makes the result independent of which pair arrives last
+    _, again = run_and_check(h, w, inputs)
+    for k, v in got.items():
+        if v is not None:
+            assert torch.equal(v, again[k]), k
+    h.close()
+
+
+@pytest.mark.parametrize("kind", ["whole tiles", "stream-K", "whole waves + stream-K"])
+def test_pair_kernel_repeat_full_compare(cuda_device, kind):
+    """Every row against the oracle, and bitwise-equal repeats, with the
+    activation tiles resident in L2 (copies land fast, so a ring slot released
+    too early would be overwritten before its reads): 72 pair tiles for 74
+    pairs (whole tiles), the 70B QKV at M = 256 (20 tiles, all split), and 80
+    tiles (one whole wave of 74, the other 6 split)."""
+    if kind == "whole tiles":
+        w, inputs = synthetic.make_custom("qkv", "rmsnorm", 2304, 1024, Hq=24, Hkv=4, D=128, seed=11)
+    elif kind == "stream-K":
+        w = WL["c5_70b_rms_qkv_m256"]
+        inputs = synthetic.make_inputs(w)
+    else:
+        w, inputs = synthetic.make_custom("qkv", "rmsnorm", 2560, 1024, Hq=24, Hkv=4, D=128, seed=12)
+    h = fnl.Handle(0, path="pair" if kind == "whole tiles" else "pair_sk")
+    _, first = run_and_check(h, w, inputs)
+    assert ("stream-K" in h.last_plan()) == (kind != "whole tiles"), h.last_plan()
+    dev = {k: v.cuda() for k, v in inputs.items()}
+    for _ in range(3):
+        again = fnl.run_workload(h, w, dev)
+        h.check()
+        for k in ("q", "k", "v"):
+            assert torch.equal(first[k], again[k]), k
+    h.close()

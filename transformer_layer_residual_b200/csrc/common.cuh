@@ -45,7 +45,8 @@ struct OpParams {
   int mpad;
   int stages;
   int cls;               // small-M kernel: CTAs per cluster (one W tile per cluster), 0 = stream-K form
-  int sk;                // 128x256 tile kernel: 1 = stream-K over (tile, k-block) units, 0 = whole tiles
+  int sk;                // 128x256 tile and pair kernels: 1 = stream-K over (tile, k-block) units, 0 = whole tiles
+  int sk_full;           // pair kernel, stream-K: tiles [0, sk_full) whole, round robin; the rest split
   int split;             // 1: operand = bf16 hi + bf16 lo (two UMMAs), 0: single bf16 rounding
   int* status;           // device status word (bounded-wait failures)
   unsigned long long wait_ns;   // limit of the main-loop waits (the drain waits keep FNL_WAIT_NS)

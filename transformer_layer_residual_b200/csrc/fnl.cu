@@ -30,11 +30,12 @@ using fnl::OpParams;
 
 namespace fnlh {
 // A plan: which kernel runs a call, in which form, on how many CTAs.
-enum class Kern { K3, K2, K2W, K4 };
+enum class Kern { K3, K2, K2W, K4, K4S };   // K4S: the pair kernel's stream-K form
 
 struct Plan {
   Kern kern = Kern::K3;
   int grid = 1, threads = 0, smem = 0, mpad = 0, stages = 0, max_seg = 1, T = 0, cls = 0, sk = 0;
+  int sk_full = 0;   // pair kernel, stream-K: tiles processed whole before the split ones
 };
 
 // Key of the shape auto-tuning cache (see tune()).
@@ -645,7 +646,7 @@ fnl_status plan_kernel(fnl_handle* h, const Call& c, Kern kern, int cls_req, Pla
     else q.max_seg = max_segments(q.T, nkb, q.grid);
   } else if (c.fp8) {
     return fail(h, FNL_ERR_UNSUPPORTED, "the FP8 form runs the small-M kernel only");
-  } else if (kern == Kern::K4) {
+  } else if (kern == Kern::K4 || kern == Kern::K4S) {
     // CTA pairs, 256 tokens x 512 W rows per pair tile, one pair tile at a time per pair
     const int pairs_max = std::min(resident_pairs(h), max_ctas / 2);
     if (pairs_max <= 0) return fail(h, FNL_ERR_UNSUPPORTED, "the pair kernel cannot be resident");
@@ -653,6 +654,25 @@ fnl_status plan_kernel(fnl_handle* h, const Call& c, Kern kern, int cls_req, Pla
     const long long tiles = static_cast<long long>(num_m2) *
                             (c.op == Op::SwiGLU ? (c.I + 255) / 256 : (c.N + fnl::k4::BN - 1) / fnl::k4::BN);
     q.grid = 2 * static_cast<int>(std::min<long long>(pairs_max, tiles));
+    // Stream-K form: the whole waves stay whole tiles, and the (tile, 32-wide
+    // k-block) units of the tiles left over are dealt evenly over all pairs.
+    // Measured on B200 it lost to the plain forms (70B QKV at M = 256: 187 us
+    // against 85 us for the 128x256 stream-K kernel; M = 2048: 472 against 395
+    // us with whole tiles): the last pair to arrive at a split tile reads the
+    // others' 128 x 512 fp32 partial sums back through L2. So it is a tuner
+    // candidate and a forced path, not the default.
+    const long long nkb4 = (c.K + fnl::k4::BK - 1) / fnl::k4::BK;
+    if (kern == Kern::K4S) {
+      if (tiles * nkb4 < pairs_max)
+        return fail(h, FNL_ERR_UNSUPPORTED, "the pair kernel's stream-K form needs a unit per pair");
+      const long long full = (tiles / pairs_max) * pairs_max;
+      if (2 * (tiles - full) > kMaxTiles) return fail(h, FNL_ERR_UNSUPPORTED, "too many W tiles");
+      q.sk = 1;
+      q.sk_full = static_cast<int>(full);
+      q.T = static_cast<int>(tiles - full);   // the split tiles (partial-sum slots, counters)
+      q.grid = 2 * pairs_max;
+      q.max_seg = max_segments(q.T, static_cast<int>(nkb4), pairs_max);
+    }
     q.cls = 2;
     q.smem = fnl::k4::SMEM_BYTES;
     q.threads = fnl::k4::NUM_THREADS;
@@ -687,6 +707,7 @@ fnl_status default_plan(fnl_handle* h, const Call& c, Plan* pl) {
     case FNL_PATH_TILE: return plan_kernel(h, c, Kern::K2, -1, pl);
     case FNL_PATH_TILE_WIDE: return plan_kernel(h, c, Kern::K2W, -1, pl);
     case FNL_PATH_TILE_PAIR: return plan_kernel(h, c, Kern::K4, -1, pl);
+    case FNL_PATH_TILE_PAIR_SPLIT: return plan_kernel(h, c, Kern::K4S, -1, pl);
     case FNL_PATH_SPLITK: return plan_kernel(h, c, Kern::K3, 0, pl);
     case FNL_PATH_SPLITK_CLUSTER: {
       // the largest cluster size whose clusters are all resident
@@ -721,7 +742,12 @@ fnl_status default_plan(fnl_handle* h, const Call& c, Plan* pl) {
     const long long g = std::min<long long>(slots, tiles);
     return static_cast<double>((tiles + g - 1) / g);
   };
-  const double t_n = waves(tiles_n, max_ctas), t_w = 1.6 * waves(tiles_w, max_ctas);
+  // the stream-K forms (plan_kernel's rules) spread the units evenly: fractional
+  // waves, plus the partial-sum exchange
+  auto sk_waves = [](long long tiles, long long slots) { return static_cast<double>(tiles) / slots + 0.15; };
+  const double t_n =
+      tiles_n * 5 <= static_cast<long long>(max_ctas) * 4 ? sk_waves(tiles_n, max_ctas) : waves(tiles_n, max_ctas);
+  const double t_w = 1.6 * waves(tiles_w, max_ctas);
   const int pairs = h->opt.max_ctas == 0 ? resident_pairs(h) : 0;
   const double t_p = pairs > 0 ? 1.45 * waves(tiles_p, pairs) : 1e30;
   if (t_p <= t_w && t_p <= t_n) return plan_kernel(h, c, Kern::K4, -1, pl);
@@ -735,10 +761,15 @@ size_t stats_bytes_of(const Call& c) {
   return ln ? align256(static_cast<size_t>(c.M) * 8) : 0;
 }
 size_t ss_bytes_of(const Plan& q) {
+  // pair kernel, stream-K: per (tile, slot, CTA half) 128 rows' partial sums of h^2
+  if (q.kern == Kern::K4 || q.kern == Kern::K4S)
+    return q.sk ? align256(static_cast<size_t>(q.T) * q.max_seg * 2 * 128 * 4) : 0;
   return q.kern == Kern::K3 && q.cls == 0 ? align256(static_cast<size_t>(q.T) * q.max_seg * q.mpad * 4) : 0;
 }
 size_t part_bytes_of(const Plan& q) {
-  if (q.kern == Kern::K4) return 0;
+  // pair kernel, stream-K: per (tile, slot, CTA half) 128 x 512 fp32 partial sums
+  if (q.kern == Kern::K4 || q.kern == Kern::K4S)
+    return q.sk ? align256(static_cast<size_t>(q.T) * q.max_seg * 2 * 128 * 512 * 4) : 0;
   if (q.kern == Kern::K3) return q.cls == 0 ? align256(static_cast<size_t>(q.T) * q.max_seg * q.mpad * 128 * 4) : 0;
   if (q.sk) return align256(static_cast<size_t>(q.T) * q.max_seg * fnl::k2::SLOT_FLOATS * 4);
   return 0;
@@ -751,7 +782,8 @@ const char* kern_name(const Plan& q) {
   switch (q.kern) {
     case Kern::K3: return q.cls > 0 ? "small-M split-K kernel, cluster form" : "small-M split-K kernel, stream-K form";
     case Kern::K2: return q.sk ? "128x256 tile kernel, stream-K" : "128x256 tile kernel";
-    case Kern::K4: return "256x512 CTA-pair kernel";
+    case Kern::K4:
+    case Kern::K4S: return q.sk ? "256x512 CTA-pair kernel, stream-K" : "256x512 CTA-pair kernel";
     default: return "128x512 tile kernel";
   }
 }
@@ -761,7 +793,8 @@ fnl_status launch_plan(fnl_handle* h, const Call& c, const Plan& q) {
   fnl_status st;
   const bool nonorm = c.op == Op::Residual;   // residual-stream projection: no add, no norm
   const bool rms = !nonorm && c.norm == FNL_NORM_RMSNORM;
-  const bool small = q.kern == Kern::K3, wide = q.kern == Kern::K2W, pair = q.kern == Kern::K4;
+  const bool small = q.kern == Kern::K3, wide = q.kern == Kern::K2W,
+             pair = q.kern == Kern::K4 || q.kern == Kern::K4S;
   const size_t sb = stats_bytes_of(c), ssb = ss_bytes_of(q);
   uint8_t* ws = h->ws;
   int* status = reinterpret_cast<int*>(ws);
@@ -786,7 +819,7 @@ fnl_status launch_plan(fnl_handle* h, const Call& c, const Plan& q) {
     p.beta = rms ? nullptr : c.beta;
   }
   p.part = part; p.part_ss = part_ss; p.counters = counters; p.max_seg = q.max_seg; p.mpad = q.mpad;
-  p.stages = q.stages; p.status = status; p.cls = q.cls; p.sk = q.sk;
+  p.stages = q.stages; p.status = status; p.cls = q.cls; p.sk = q.sk; p.sk_full = q.sk_full;
   p.wait_ns = h->opt.wait_ns > 0 ? static_cast<unsigned long long>(h->opt.wait_ns) : FNL_WAIT_NS;
   p.stall = 0;
   if (h->opt.debug_stall_calls > 0) {   // one-shot fault injection for the status-path tests
@@ -882,7 +915,7 @@ fnl_status time_once(fnl_handle* h, const Call& c, const Plan& q, void* flush, s
 
 // Same kernel, form and grid.
 bool same_plan(const Plan& a, const Plan& b) {
-  return a.kern == b.kern && a.cls == b.cls && a.sk == b.sk && a.grid == b.grid;
+  return a.kern == b.kern && a.cls == b.cls && a.sk == b.sk && a.sk_full == b.sk_full && a.grid == b.grid;
 }
 
 fnl_status tune(fnl_handle* h, const Call& c, Plan* best) {
@@ -902,6 +935,7 @@ fnl_status tune(fnl_handle* h, const Call& c, Plan* best) {
   if (!c.fp8 && plan_kernel(h, c, Kern::K2, -1, &q) == FNL_OK) cand[n++] = q;
   if (!small_ok && plan_kernel(h, c, Kern::K2W, -1, &q) == FNL_OK) cand[n++] = q;
   if (!small_ok && plan_kernel(h, c, Kern::K4, -1, &q) == FNL_OK) cand[n++] = q;
+  if (!small_ok && plan_kernel(h, c, Kern::K4S, -1, &q) == FNL_OK) cand[n++] = q;
   h->err.clear();   // refused candidates are not errors of the call
   if (n == 0) return default_plan(h, c, best);
   size_t need = 0;
@@ -1010,7 +1044,7 @@ fnl_status fnl_create(fnl_handle** out, int device, const fnl_options* opt) {
   *out = nullptr;
   fnl_handle* h = new fnl_handle();
   if (opt) h->opt = *opt;
-  if (h->opt.path < FNL_PATH_AUTO || h->opt.path > FNL_PATH_TILE_PAIR || h->opt.max_tokens < 0 || h->opt.max_n < 0 ||
+  if (h->opt.path < FNL_PATH_AUTO || h->opt.path > FNL_PATH_TILE_PAIR_SPLIT || h->opt.max_tokens < 0 || h->opt.max_n < 0 ||
       h->opt.precision < FNL_PRECISION_DEFAULT || h->opt.precision > FNL_PRECISION_SINGLE || h->opt.wait_ns < 0 ||
       h->opt.debug_stall_calls < 0 || h->opt.tune < 0 || h->opt.tune > 1) {
     delete h;

@@ -43,6 +43,12 @@
 // abort flag of both CTAs; both CTAs meet at a cluster barrier after their role
 // loops (and after the last UMMA completed), so neither leaves while the other
 // may still touch its shared memory.
+//
+// Work split: each pair takes whole tiles in turn, or, when the tiles fill the
+// pairs' waves poorly (70B QKV at M = 256: 20 tiles for 74 pairs; M = 2048: 2.2
+// waves), stream-K: the (tile, k-block) units are dealt evenly over the pairs
+// and a tile shared by several pairs is summed by the last to arrive (see the
+// epilogue).
 #pragma once
 
 #include "common.cuh"
@@ -92,10 +98,11 @@ constexpr int GROUP_M = 8;         // pair rows (of 256 tokens) sharing a W tile
 struct Ctrl {
   uint64_t full_w[MAX_OST], conv[MAX_OST], empty[MAX_OST];   // operand ring
   uint64_t raw_full[MAX_RST], raw_empty[MAX_RST];            // raw ring
-  uint64_t tfull, tempty, sfull[2], efree[2], drain;
+  uint64_t tfull, tempty, sfull[2], efree[2], drain, esync;
   uint32_t tmem_base;
   int abort_flag;
-  float rs[2][CONV_GROUPS][BM];   // RMSNorm: per tile buffer, per converter group, sum of h^2 per row
+  int last_flag;   // stream-K: this CTA arrived last at the current partial tile
+  float rs[2][CONV_GROUPS][BM];   // RMSNorm: per segment buffer, per converter group, sum of h^2 per row
 };
 constexpr int SMEM_BYTES = RINGS_BYTES + VEC_BYTES + static_cast<int>(sizeof(Ctrl)) + 1024;
 
@@ -116,6 +123,77 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
   }
   return true;
 }
+
+// The pair's work as segments (tile t, k-blocks [kb0, kb0 + nk), slot, nseg):
+// whole tiles t = pair, pair + npairs, ... below `full` (nseg = 1), then, with
+// stream-K, the contiguous units [pair U / G, (pair + 1) U / G) of the U =
+// (tiles - full) x nkb (tile, k-block) units of the remaining tiles, cut at tile
+// boundaries, where slot is this pair's index among the nseg pairs that share
+// tile t. The whole waves keep the pairs on neighbouring tiles (their W and
+// activation tiles stay in L2); only the last, partial wave is split.
+struct PairSegs {
+  long long u, u1, U;
+  int nkb, G, g, t, full;
+  bool sk;
+  __device__ PairSegs(bool sk_, int full_, int tiles, int nkb_, int G_, int g_)
+      : u(0), u1(0), U(static_cast<long long>(tiles - full_) * nkb_), nkb(nkb_), G(G_), g(g_), t(g_),
+        full(full_), sk(sk_) {
+    if (sk) {
+      u = static_cast<long long>(g) * U / G;
+      u1 = static_cast<long long>(g + 1) * U / G;
+    }
+  }
+  __device__ int positions() const {
+    const int whole = g < full ? ((full - 1 - g) / G + 1) * nkb : 0;
+    return whole + static_cast<int>(u1 - u);
+  }
+  // slot storage index of tile t (stream-K tiles only)
+  __device__ int sk_tile(int tt) const { return tt - full; }
+  __device__ bool next(int& tt, int& kb0, int& nk, int& slot, int& nseg) {
+    if (t < full) {
+      tt = t;
+      kb0 = 0;
+      nk = nkb;
+      slot = 0;
+      nseg = 1;
+      t += G;
+      return true;
+    }
+    if (u >= u1) return false;
+    const int ts = static_cast<int>(u / nkb);   // index among the split tiles
+    tt = full + ts;
+    kb0 = static_cast<int>(u - static_cast<long long>(ts) * nkb);
+    const long long tile_end = static_cast<long long>(ts + 1) * nkb;
+    const long long e = tile_end < u1 ? tile_end : u1;
+    nk = static_cast<int>(e - u);
+    const int first = unit_owner_fast(static_cast<long long>(ts) * nkb, G, U);
+    const int last = unit_owner_fast(tile_end - 1, G, U);
+    slot = g - first;
+    nseg = last - first + 1;
+    u = e;
+    return true;
+  }
+};
+
+// The producers' walk over the pair's positions: tile coordinates and k-block
+// of each (tile, k-block) unit in order.
+struct PosCur {
+  PairSegs segs;
+  int num_m2, num_n, t, kb, kb_end, mb2, nb;
+  __device__ PosCur(const PairSegs& s_, int num_m2_, int num_n_) : segs(s_), num_m2(num_m2_), num_n(num_n_) {
+    kb = kb_end = 0;
+    step();
+  }
+  __device__ void step() {
+    if (++kb < kb_end) return;
+    int kb0, nk, slot, nseg;
+    if (segs.next(t, kb0, nk, slot, nseg)) {
+      kb = kb0;
+      kb_end = kb0 + nk;
+      tile_coords(t, num_m2, num_n, mb2, nb);
+    }
+  }
+};
 
 }  // namespace k4
 
@@ -146,8 +224,8 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
   const int tiles = num_m2 * num_n;
   const int nkb = (K + BK - 1) / BK;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const int my_tiles = pair < tiles ? (tiles - 1 - pair) / npairs + 1 : 0;
-  const int P = my_tiles * nkb;   // positions (tile, k-block) of this CTA
+  const PairSegs segs0(p.sk != 0, p.sk != 0 ? p.sk_full : tiles, tiles, nkb, npairs, pair);
+  const int P = segs0.positions();   // positions (tile, k-block) of this CTA
 
   if (threadIdx.x == 0) {
     pdl_launch_dependents();
@@ -167,7 +245,9 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
       mbar_init(&ctrl->efree[b], NUM_EPI_WARPS);
     }
     mbar_init(&ctrl->drain, 1);
+    mbar_init(&ctrl->esync, NUM_EPI_WARPS * EPI_SHARES);   // every epilogue share of this CTA
     ctrl->abort_flag = 0;
+    ctrl->last_flag = 0;
     fence_mbar_init();
   }
   if (warp == WARP_TMA && lane == 0) {
@@ -189,13 +269,21 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
   // a wait that gave up (or saw the flag) also stops the other CTA of the pair
   auto abort_pair = [&]() { st_remote_u32(&ctrl->abort_flag, peer, 1u); };
 
-  // The epilogue of the pair's i-th tile t for this warp's TMEM lane quarter
-  // (rows q32 .. q32 + 31 of the CTA's 128): share j of EPI_SHARES, 16-column
-  // chunks cc = j, j + EPI_SHARES, ... The epilogue warps take share 0; the
-  // converter warps, idle while the UMMA waits for the accumulator, take shares
-  // 1 and 2 (group 0 and 1) before they start on the next tile. Every taking
-  // warp of both CTAs arrives on the even CTA's tempty.
-  auto epilogue_share = [&](int i, int t, int j) -> bool {
+  // The epilogue of the pair's i-th segment (tile t, slot of nseg) for this
+  // warp's TMEM lane quarter (rows q32 .. q32 + 31 of the CTA's 128): share j of
+  // EPI_SHARES, 16-column chunks cc = j, j + EPI_SHARES, ... The epilogue warps
+  // take share 0; with EPI_SHARES > 1 the converter warps, idle while the UMMA
+  // waits for the accumulator, take shares 1 and 2 (group 0 and 1) before they
+  // start on the next segment. Every taking warp of both CTAs arrives on the
+  // even CTA's tempty.
+  // A segment that is only part of its tile's k-blocks (stream-K, nseg > 1)
+  // first stores this CTA's 128 rows of partial sums (fp32 [128][512], and the
+  // rows' partial sums of h^2) in its slot; one thread's acquire-release arrival
+  // on the tile half's counter then elects the CTA that arrives last, which sums
+  // the nseg slots in slot order (its own from TMEM), so the result does not
+  // depend on the arrival order, runs the epilogue and resets the counter.
+  uint32_t esync_phase = 0;
+  auto epilogue_share = [&](int i, int t, int slot, int nseg, int j) -> bool {
     const int q32 = (warp & 3) * 32;
     const int row_local = q32 + lane;
     if (!warp_wait(&ctrl->tfull, static_cast<uint32_t>(i) & 1, abortf, p.status, kStatusWaitTmemFull,
@@ -203,7 +291,7 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
       if (lane == 0) abort_pair();
       return false;
     }
-    float scale = 1.f;
+    float ssum = 0.f;   // RMSNorm: this segment's sum of h^2 of the row
     if (NORM == kRMSNorm) {
       const int b = i & 1;
       if (!warp_wait(&ctrl->sfull[b], static_cast<uint32_t>(i >> 1) & 1, abortf, p.status, kStatusWaitStats,
@@ -211,10 +299,8 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
         if (lane == 0) abort_pair();
         return false;
       }
-      float ssum = 0.f;
 #pragma unroll
       for (int g = 0; g < CONV_GROUPS; ++g) ssum += ctrl->rs[b][g][row_local];   // fixed order
-      scale = 1.f / sqrtf(ssum / static_cast<float>(K) + p.eps);
       __syncwarp();
       if (j == 0 && lane == 0) mbar_arrive(&ctrl->efree[b]);   // the converters may refill rs[b] (see below)
     }
@@ -223,47 +309,140 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
     tile_coords(t, num_m2, num_n, mb2, nb);
     const int m = mb2 * 2 * BM + static_cast<int>(rank) * BM + row_local;
     const bool row_ok = m < M;
-    if (NORM == kRMSNorm && j == 0 && nb == 0 && row_ok && p.rstd_out != nullptr) p.rstd_out[m] = scale;
     const uint32_t tbase = tmem + (static_cast<uint32_t>(q32) << 16);
-    // 16-column chunks: few registers held, so the converter warps can take shares without spilling
-    if (EPI == kEpiSwiGLU) {
+    // TMEM column of 16-column chunk cc: the gate and up halves for SwiGLU
+    constexpr int NCH = EPI == kEpiSwiGLU ? 16 : BN / 16;
+    const bool partial = nseg > 1;
+    // slot sl of this tile half: 128 rows x 512 fp32 partial sums, 128 partial sums of h^2
+    const size_t half0 = static_cast<size_t>(partial ? segs0.sk_tile(t) : 0) * p.max_seg * 2 + rank;
+    auto part_row = [&](int sl) { return p.part + ((half0 + static_cast<size_t>(sl) * 2) * BM + row_local) * 512; };
+    bool last = true;
+    if (partial) {
+      float* own = part_row(slot);
 #pragma unroll 1
-      for (int cc = j; cc < 16; cc += EPI_SHARES) {
-        uint32_t g0[16], u0[16];
-        tmem_ld16(tbase + cc * 16, g0);
-        tmem_ld16(tbase + 256 + cc * 16, u0);
+      for (int cc = j; cc < NCH; cc += EPI_SHARES) {
+        uint32_t a0[16];
+        tmem_ld16(tbase + cc * 16, a0);
+        if (EPI == kEpiSwiGLU) {
+          uint32_t u0[16];
+          tmem_ld16(tbase + 256 + cc * 16, u0);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; e += 4) {
+            *reinterpret_cast<uint4*>(own + cc * 16 + e) = make_uint4(a0[e], a0[e + 1], a0[e + 2], a0[e + 3]);
+            *reinterpret_cast<uint4*>(own + 256 + cc * 16 + e) = make_uint4(u0[e], u0[e + 1], u0[e + 2], u0[e + 3]);
+          }
+        } else {
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; e += 4)
+            *reinterpret_cast<uint4*>(own + cc * 16 + e) = make_uint4(a0[e], a0[e + 1], a0[e + 2], a0[e + 3]);
+        }
+      }
+      if (NORM == kRMSNorm && j == 0) p.part_ss[(half0 + static_cast<size_t>(slot) * 2) * BM + row_local] = ssum;
+      // every share of this CTA has stored its part; then the arrival (one thread), then its result
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctrl->esync);
+      if (!warp_wait(&ctrl->esync, esync_phase, abortf, p.status, kStatusWaitDrain, p.wait_ns)) {
+        if (lane == 0) abort_pair();
+        return false;
+      }
+      esync_phase ^= 1u;
+      if (j == 0 && (warp & 3) == 0 && lane == 0) {
+        unsigned* cnt = p.counters + static_cast<size_t>(segs0.sk_tile(t)) * 2 + rank;
+        const unsigned old = atom_add_acq_rel_gpu(cnt, 1u);
+        const int is_last = old == static_cast<unsigned>(nseg - 1) ? 1 : 0;
+        ctrl->last_flag = is_last;
+        if (is_last) *cnt = 0u;   // no other CTA touches it again in this launch
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctrl->esync);
+      if (!warp_wait(&ctrl->esync, esync_phase, abortf, p.status, kStatusWaitDrain, p.wait_ns)) {
+        if (lane == 0) abort_pair();
+        return false;
+      }
+      esync_phase ^= 1u;
+      last = ctrl->last_flag != 0;
+    }
+    if (last) {
+      float scale = 1.f;
+      if (NORM == kRMSNorm) {
+        float tot = ssum;
+        if (partial) {
+          tot = 0.f;
+          for (int sl = 0; sl < nseg; ++sl)
+            tot += sl == slot ? ssum : __ldcg(p.part_ss + (half0 + static_cast<size_t>(sl) * 2) * BM + row_local);
+        }
+        scale = 1.f / sqrtf(tot / static_cast<float>(K) + p.eps);
+      }
+      if (NORM == kRMSNorm && j == 0 && nb == 0 && row_ok && p.rstd_out != nullptr) p.rstd_out[m] = scale;
+      // 16 columns at TMEM column `col`: this CTA's own value, plus (partial) the other slots in slot order
+      auto gather16 = [&](int col, float (&v)[16]) {
+        uint32_t a0[16];
+        tmem_ld16(tbase + col, a0);
         tmem_ld_wait();
-        if (row_ok) {
+        if (!partial) {
 #pragma unroll
-          for (int g8 = 0; g8 < 2; ++g8) {
-            const int jj = nb * 256 + cc * 16 + g8 * 8;
-            if (jj < p.I) {
-              float gv[8], uv[8];
+          for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(a0[e]);
+          return;
+        }
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                gv[e] = __uint_as_float(g0[g8 * 8 + e]);
-                uv[e] = __uint_as_float(u0[g8 * 8 + e]);
-              }
-              store_swiglu8(p, m, jj, gv, uv, scale);
+        for (int e = 0; e < 16; ++e) v[e] = 0.f;
+        for (int sl = 0; sl < nseg; ++sl) {
+          if (sl == slot) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] += __uint_as_float(a0[e]);
+          } else {
+            const float* src = part_row(sl) + col;
+#pragma unroll
+            for (int e = 0; e < 16; e += 4) {
+              const float4 w = __ldcg(reinterpret_cast<const float4*>(src + e));
+              v[e] += w.x;
+              v[e + 1] += w.y;
+              v[e + 2] += w.z;
+              v[e + 3] += w.w;
             }
           }
         }
-      }
-    } else {
+      };
+      // 16-column chunks: few registers held, so the converter warps can take shares without spilling
+      if (EPI == kEpiSwiGLU) {
 #pragma unroll 1
-      for (int cc = j; cc < BN / 16; cc += EPI_SHARES) {
-        uint32_t a0[16];
-        tmem_ld16(tbase + cc * 16, a0);
-        tmem_ld_wait();
-        if (row_ok) {
+        for (int cc = j; cc < NCH; cc += EPI_SHARES) {
+          float g0[16], u0[16];
+          gather16(cc * 16, g0);
+          gather16(256 + cc * 16, u0);
+          if (row_ok) {
 #pragma unroll
-          for (int g8 = 0; g8 < 2; ++g8) {
-            const int n = nb * BN + cc * 16 + g8 * 8;
-            if (n < p.N) {
-              float av[8];
+            for (int g8 = 0; g8 < 2; ++g8) {
+              const int jj = nb * 256 + cc * 16 + g8 * 8;
+              if (jj < p.I) {
+                float gv[8], uv[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) av[e] = __uint_as_float(a0[g8 * 8 + e]);
-              store_out8<EPI>(p, m, n, av, scale);
+                for (int e = 0; e < 8; ++e) {
+                  gv[e] = g0[g8 * 8 + e];
+                  uv[e] = u0[g8 * 8 + e];
+                }
+                store_swiglu8(p, m, jj, gv, uv, scale);
+              }
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int cc = j; cc < NCH; cc += EPI_SHARES) {
+          float a0[16];
+          gather16(cc * 16, a0);
+          if (row_ok) {
+#pragma unroll
+            for (int g8 = 0; g8 < 2; ++g8) {
+              const int n = nb * BN + cc * 16 + g8 * 8;
+              if (n < p.N) {
+                float av[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) av[e] = a0[g8 * 8 + e];
+                store_out8<EPI>(p, m, n, av, scale);
+              }
             }
           }
         }
@@ -271,7 +450,7 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) {   // the pair's accumulator may be overwritten once every share of both CTAs is read
+    if (lane == 0) {   // the pair's accumulator may be overwritten once every share of both CTAs is done
       if (leader) mbar_arrive(&ctrl->tempty);
       else mbar_arrive_remote(&ctrl->tempty, 0);
     }
@@ -283,10 +462,9 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
     if (lane == 0 && NORM != kNoNorm) {
       uint32_t armed = 0, par = 0;
       bool ok = true;
-      int t = pair, mb2 = 0, nb = 0, kb = 0;
-      if (P > 0) tile_coords(t, num_m2, num_n, mb2, nb);
+      PosCur c(segs0, num_m2, num_n);
       pdl_wait();   // activations may be written by the previous kernel
-      for (int q = 0; q < P; ++q) {
+      for (int q = 0; q < P; ++q, c.step()) {
         const int r = q % RST;
         const uint32_t ph = static_cast<uint32_t>(q / RST) & 1u;
         if (q >= RST &&
@@ -295,8 +473,8 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
           break;
         }
         uint8_t* st = raw + r * RAW_BYTES;
-        const int k0 = kb * BK;
-        const int row0 = mb2 * 2 * BM + static_cast<int>(rank) * BM;
+        const int k0 = c.kb * BK;
+        const int row0 = c.mb2 * 2 * BM + static_cast<int>(rank) * BM;
         bf16* vec = vecs + r * 3 * VEC;
         const uint32_t vb = static_cast<uint32_t>(min(VEC, K - k0)) * 2;
         const uint32_t nvec = 1 + (has_beta ? 1 : 0) + (has_bias_in ? 1 : 0);
@@ -308,11 +486,6 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
         tma_load_2d(st + X_BYTES, &tm_r, &ctrl->raw_full[r], k0, row0);
         armed |= 1u << r;
         par = (par & ~(1u << r)) | (ph << r);
-        if (++kb == nkb) {
-          kb = 0;
-          t += npairs;
-          if (t < tiles) tile_coords(t, num_m2, num_n, mb2, nb);
-        }
       }
       if (!ok) {
         abort_pair();
@@ -328,19 +501,8 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
       bool ok = true;
       // fault injection (status-path tests only): CTA 0 withholds position 0's copies
       const int skip = (p.stall != 0 && blockIdx.x == 0) ? 0 : -1;
-      struct Cur {
-        int t, mb2, nb, kb;
-      };
-      Cur cw{pair, 0, 0, 0};
-      if (P > 0) tile_coords(cw.t, num_m2, num_n, cw.mb2, cw.nb);
-      Cur cx = cw;
-      auto step = [&](Cur& c) {
-        if (++c.kb == nkb) {
-          c.kb = 0;
-          c.t += npairs;
-          if (c.t < tiles) tile_coords(c.t, num_m2, num_n, c.mb2, c.nb);
-        }
-      };
+      PosCur cw(segs0, num_m2, num_n), cx = cw;
+      auto step = [&](PosCur& c) { c.step(); };
       // one arrive_expect_tx per slot use: the W halves (+ the activation tile without a norm)
       auto arm = [&](int q) {
         if (q == skip) return;
@@ -350,7 +512,7 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
         armed |= 1u << s;
         par = (par & ~(1u << s)) | (ph << s);
       };
-      auto issue_w = [&](int q, const Cur& c) {
+      auto issue_w = [&](int q, const PosCur& c) {
         if (q == skip) return;
         const int s = q % OST;
         uint8_t* st = smem + s * OPB + OPA;
@@ -366,7 +528,7 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
         tma_load_2d(st, &tm_w, &ctrl->full_w[s], c.kb * BK, r0);
         tma_load_2d(st + WH_BYTES, &tm_w, &ctrl->full_w[s], c.kb * BK, r1);
       };
-      auto issue_x = [&](int q, const Cur& c) {   // no norm: the activation tile is the operand
+      auto issue_x = [&](int q, const PosCur& c) {   // no norm: the activation tile is the operand
         if (q == skip) return;
         const int s = q % OST;
         tma_load_2d(smem + s * OPB, &tm_x, &ctrl->full_w[s], c.kb * BK,
@@ -411,15 +573,16 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
       uint32_t s = 0, ph = 0;
       bool ok = true;
       const uint32_t idesc = idesc_bf16(2 * BM, 256);
-      int i = 0;
-      for (int t = pair; t < tiles && ok; t += npairs, ++i) {
+      PairSegs segs = segs0;
+      int t, kb0, nk, slot, nseg;
+      for (int i = 0; ok && segs.next(t, kb0, nk, slot, nseg); ++i) {
         if (!mbar_wait_cluster(&ctrl->tempty, (static_cast<uint32_t>(i) & 1) ^ 1, abortf, p.status,
                                kStatusWaitTmemEmpty, p.wait_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = 0; kb < nk; ++kb) {   // accumulate from the segment's first k-block
           if (!mbar_wait_cluster(&ctrl->conv[s], ph, abortf, p.status, kStatusWaitConv, p.wait_ns)) {
             ok = false;
             break;
@@ -456,9 +619,10 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
   } else if (warp < WARP_CONV0) {
     // ------------------------------------------------------------ epilogue (own 128 rows, share 0)
     pdl_wait();
-    int i = 0;
-    for (int t = pair; t < tiles; t += npairs, ++i)
-      if (!epilogue_share(i, t, 0)) break;
+    PairSegs segs = segs0;
+    int t, kb0, nk, slot, nseg;
+    for (int i = 0; segs.next(t, kb0, nk, slot, nseg); ++i)
+      if (!epilogue_share(i, t, slot, nseg, 0)) break;
   } else {
     // ------------------------------------------------------------ converters (own 128 rows)
     // Two groups of four warps: group g converts positions q = g, g + 2, ...
@@ -470,9 +634,9 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
     // c ^ ((r >> 1) & 3). RMSNorm: each group sums h^2 over its k-blocks; the
     // epilogue adds the two groups' sums in group order. Without a norm
     // (residual-stream projection) the warps only relay the slot's readiness
-    // to the even CTA. Before tile i + 1 each group takes its share of tile i's
-    // epilogue: the UMMA cannot start tile i + 1 before the accumulator is
-    // read, so the shares shorten the gap between tiles.
+    // to the even CTA. Before segment i + 1 each group takes its share of
+    // segment i's epilogue: the UMMA cannot start segment i + 1 before the
+    // accumulator is read, so the shares shorten the gap between segments.
     constexpr int RPT = BM / CONV_ROWS_PER_PASS;   // rows per thread (4)
     const int ct = threadIdx.x - WARP_CONV0 * 32;   // 0..255
     const int grp = ct / CONV_GROUP_THREADS;          // 0..CONV_GROUPS-1
@@ -482,13 +646,19 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
     if (NORM == kLayerNorm) pdl_wait();
     int i = 0;
     bool ok = true;
-    long long q0 = 0;   // first position of the current tile
-    for (int t = pair; t < tiles && ok; t += npairs, ++i, q0 += nkb) {
-      // this group's share of the previous tile's epilogue, before any of this tile's state is live
-      if (EPI_SHARES > 1 && i > 0 && !epilogue_share(i - 1, t - npairs, 1 + grp)) {
+    long long q0 = 0;   // first position of the current segment
+    PairSegs segs = segs0;
+    int t, kb0, nk, slot, nseg;
+    int pt = 0, pslot = 0, pnseg = 1;   // the previous segment, for its epilogue share
+    for (; ok && segs.next(t, kb0, nk, slot, nseg); ++i, q0 += nk) {
+      // this group's share of the previous segment's epilogue, before any of this segment's state is live
+      if (EPI_SHARES > 1 && i > 0 && !epilogue_share(i - 1, pt, pslot, pnseg, 1 + grp)) {
         ok = false;
         break;
       }
+      pt = t;
+      pslot = slot;
+      pnseg = nseg;
       int mb2, nb;
       tile_coords(t, num_m2, num_n, mb2, nb);
       const int mrow0 = mb2 * 2 * BM + static_cast<int>(rank) * BM;
@@ -507,19 +677,17 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
         }
       }
       const bool write_res = (NORM == kRMSNorm) && nb == 0;
-      // this group's positions of the tile
-      for (long long q = q0 + ((grp - q0 % CONV_GROUPS) + CONV_GROUPS) % CONV_GROUPS; q < q0 + nkb;
+      // this group's positions of the segment
+      for (long long q = q0 + ((grp - q0 % CONV_GROUPS) + CONV_GROUPS) % CONV_GROUPS; q < q0 + nk;
            q += CONV_GROUPS) {
-        const int kb = static_cast<int>(q - q0);
+        const int kb = kb0 + static_cast<int>(q - q0);
         const int s = static_cast<int>(q % OST);
         const uint32_t ph = static_cast<uint32_t>(q / OST) & 1u;
         if (NORM != kNoNorm) {
           const int r = static_cast<int>(q % RST);
           const uint32_t rph = static_cast<uint32_t>(q / RST) & 1u;
-          // the raw tiles have landed, and the UMMA that last read operand slot s is done
-          if (!warp_wait(&ctrl->raw_full[r], rph, abortf, p.status, kStatusWaitFull, p.wait_ns) ||
-              (q >= OST &&
-               !warp_wait(&ctrl->empty[s], ph ^ 1u, abortf, p.status, kStatusWaitEmpty, p.wait_ns))) {
+          // the raw tiles have landed
+          if (!warp_wait(&ctrl->raw_full[r], rph, abortf, p.status, kStatusWaitFull, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -532,7 +700,6 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
           if (BIAS_IN) vec_pairs(vaddr + 4 * VEC, bi2);
           const uint32_t xs = smem_u32(raw + r * RAW_BYTES);
           const uint32_t rsm = xs + X_BYTES;
-          const uint32_t as = smem_u32(smem + s * OPB);
           uint4 xv[RPT], rv[RPT];
 #pragma unroll
           for (int j = 0; j < RPT; ++j) {
@@ -541,31 +708,50 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
             xv[j] = ld_shared_v4(xs + off);
             rv[j] = ld_shared_v4(rsm + off);
           }
-          // the raw slot is read: its next copies may start
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&ctrl->raw_empty[r]);
-          // instantiated with and without the residual_out store (first N column)
-          auto convert_stage = [&](auto wres_tag) {
+          // the operand into registers (instantiated with and without the
+          // residual_out store of the first N column)
+          uint4 hi[RPT], lo[RPT];
+          auto convert_rows = [&](auto wres_tag) {
             constexpr bool WRES = decltype(wres_tag)::value;
 #pragma unroll
             for (int j = 0; j < RPT; ++j) {
-              const int row = rb + CONV_ROWS_PER_PASS * j;
-              const uint32_t off = row * 64 + ((c ^ ((row >> 1) & 3)) << 4);
-              uint4 hi, lo, hres;
+              uint4 hres;
               convert8<(NORM == kNoNorm ? kRMSNorm : NORM), BIAS_IN, SPLIT, WRES>(
-                  xv[j], rv[j], g2, be2, bi2, mu[j], rs[j], ss[j], hi, lo, hres);
-              st_shared_v4(as + off, hi);
-              if (SPLIT) st_shared_v4(as + X_BYTES + off, lo);
+                  xv[j], rv[j], g2, be2, bi2, mu[j], rs[j], ss[j], hi[j], lo[j], hres);
               if (WRES) {
-                const int gm = mrow0 + row;
+                const int gm = mrow0 + rb + CONV_ROWS_PER_PASS * j;
                 const int k0 = kb * BK + c * 8;
                 if (gm < M && k0 < K)
                   *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(gm) * K + k0) = hres;
               }
             }
           };
-          if (write_res) convert_stage(BoolC<true>{});
-          else convert_stage(BoolC<false>{});
+          if (write_res) convert_rows(BoolC<true>{});
+          else convert_rows(BoolC<false>{});
+          // The raw slot may take its next copies now, behind a proxy fence: the
+          // fence completes this thread's reads of the slot (the conversion has
+          // consumed them) before the tensor copies, which write through the
+          // async proxy, can be issued against it. (Released right after the
+          // loads were issued and with no fence, the next x tile landed before
+          // some loads had read the current one: rows of the operand mixed the
+          // next k-block's x with this one's residual.) The slot no longer
+          // waits for the UMMA to free an operand slot.
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctrl->raw_empty[r]);
+          // the UMMA that last read operand slot s is done: store the operand
+          if (q >= OST && !warp_wait(&ctrl->empty[s], ph ^ 1u, abortf, p.status, kStatusWaitEmpty, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          const uint32_t as = smem_u32(smem + s * OPB);
+#pragma unroll
+          for (int j = 0; j < RPT; ++j) {
+            const int row = rb + CONV_ROWS_PER_PASS * j;
+            const uint32_t off = row * 64 + ((c ^ ((row >> 1) & 3)) << 4);
+            st_shared_v4(as + off, hi[j]);
+            if (SPLIT) st_shared_v4(as + X_BYTES + off, lo[j]);
+          }
           fence_proxy_async_smem();
         }
         // this CTA's weight halves (and, without a norm, its activation tile) have landed
@@ -594,13 +780,13 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
           sst[j] += __shfl_xor_sync(0xffffffffu, sst[j], 2);
         }
         const int b = i & 1;
-        // the epilogue of the tile two back has read rs[b]
+        // the epilogue of the segment two back has read rs[b]
         if (!warp_wait(&ctrl->efree[b], (static_cast<uint32_t>(i >> 1) & 1) ^ 1, abortf, p.status,
                        kStatusWaitTmemEmpty, p.wait_ns)) {
           if (lane == 0) abort_pair();
           break;
         }
-        if (c == 0) {   // this group's sum of h^2 per row over its k-blocks
+        if (c == 0) {   // this group's sum of h^2 per row over its k-blocks of the segment
 #pragma unroll
           for (int j = 0; j < RPT; ++j) ctrl->rs[b][grp][rb + CONV_ROWS_PER_PASS * j] = sst[j];
         }
@@ -608,8 +794,8 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
         if (lane == 0) mbar_arrive(&ctrl->sfull[b]);
       }
     }
-    // the last tile's share (its epilogue has no next tile to wait behind)
-    if (EPI_SHARES > 1 && ok && i > 0) epilogue_share(i - 1, pair + (i - 1) * npairs, 1 + grp);
+    // the last segment's share (its epilogue has no next segment to wait behind)
+    if (EPI_SHARES > 1 && ok && i > 0) epilogue_share(i - 1, pt, pslot, pnseg, 1 + grp);
   }
 
   // Every role's loop is over and the even CTA's last UMMA has completed (its

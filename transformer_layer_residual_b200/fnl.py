@@ -21,7 +21,7 @@ FNL_OK = 0
 STATUS_NAMES = {0: "FNL_OK", 1: "FNL_ERR_INVALID_ARG", 2: "FNL_ERR_ALIGNMENT", 3: "FNL_ERR_ALIAS",
                 4: "FNL_ERR_UNSUPPORTED", 5: "FNL_ERR_CUDA", 6: "FNL_ERR_DEVICE_STATUS"}
 NORMS = {"layernorm": 0, "rmsnorm": 1}
-PATHS = {"auto": 0, "tile": 1, "splitk": 2, "wide": 3, "cluster": 4, "pair": 5}
+PATHS = {"auto": 0, "tile": 1, "splitk": 2, "wide": 3, "cluster": 4, "pair": 5, "pair_sk": 6}
 PRECISIONS = {"default": 0, "split": 1, "single": 2}
 
 EXPORTED = ("fnl_create", "fnl_destroy", "fnl_status_string", "fnl_last_error", "fnl_last_plan", "fnl_check",
