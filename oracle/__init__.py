@@ -65,6 +65,11 @@ Readings taken where the pages are silent:
      but give no formula for the residual connection; this is the pre-norm
      transformer's plain reading.
 
+  R13 tensor parallelism (the pages split the output and down projections by
+     rows and all-reduce their partial outputs; they give no precision): the
+     P ranks' bf16 partial activations are summed exactly and rounded once to
+     bf16, and that sum is the x of the next fused add + norm + projection.
+
 Parity pins live in tests/test_oracle_pins.py; every function here is pinned.
 """
 from .core import (  # noqa: F401
@@ -82,6 +87,8 @@ from .core import (  # noqa: F401
     add_norm_swiglu,
     add_bias_norm_gelu,
     linear_add_residual,
+    tp_allreduce,
+    add_norm_qkv_tp,
     E4M3_MAX,
     e4m3_round,
     fp8_row_scale_and_codes,

@@ -142,6 +142,22 @@ def add_bias_norm_gelu(x, residual, bias_in, gamma, beta, norm, eps, W, bias_out
     return _stats({"residual_out": bf16_round(h), "out": gelu_tanh(z)}, mean, rstd)
 
 
+def tp_allreduce(parts) -> np.ndarray:
+    """Tensor-parallel all-reduce of the row-parallel projection's partial
+    outputs (TensorRT-LLM 深度工程实践, §4.1 Tensor Parallelism: the output and
+    down projections are split by rows, and each rank's partial result is
+    summed across ranks before the next add and norm). Reading R13: the P
+    ranks' bf16 partials summed exactly, then rounded once to bf16, because the
+    reduced tensor is bf16 like its inputs."""
+    return bf16_round(np.sum(np.stack([_f64(v) for v in parts]), axis=0))
+
+
+def add_norm_qkv_tp(parts, residual, gamma, beta, norm, eps, W, bias, Hq, Hkv, D) -> dict:
+    """The fused QKV op fed by the all-reduce: x = tp_allreduce(parts), then
+    add_norm_qkv(x, residual, ...) (reading R13)."""
+    return add_norm_qkv(tp_allreduce(parts), residual, gamma, beta, norm, eps, W, bias, Hq, Hkv, D)
+
+
 def linear_add_residual(a, W, bias, residual) -> dict:
     """Residual-stream projection (o_proj / down_proj) with the residual add
     fused after it: out = residual + a W^T (+ bias), in fp64 (reading R9).

@@ -530,11 +530,45 @@ def pin_fp8_fused_qkv(ora):
     assert np.array_equal(og["residual_out"], ora.bf16_round(xr + rr + bi[None, :]))
 
 
+def pin_tp_allreduce(ora):
+    """Tensor-parallel all-reduce (reading R13): integer partials sum exactly;
+    one rank is the identity; the sum is rounded once (ties to even) after an
+    exact sum, not after each addition; a row-parallel projection split over
+    ranks all-reduces to the unsplit one; the composed QKV op on a one-hot row
+    split over two ranks has the RMSNorm closed form."""
+    rng = np.random.default_rng(91)
+    parts = [rng.integers(-20, 21, size=(3, 8)).astype(np.float64) for _ in range(4)]
+    assert np.array_equal(ora.tp_allreduce(parts), np.sum(parts, axis=0))
+    one = ora.bf16_round(rng.normal(size=(2, 5)))
+    assert np.array_equal(ora.tp_allreduce([one]), one)
+    t = 2.0 ** -8
+    assert ora.tp_allreduce([np.array([1.0]), np.array([t])])[0] == 1.0                    # tie -> even
+    assert ora.tp_allreduce([np.array([1.0]), np.array([3 * t])])[0] == 1.0 + 2 * 2.0 ** -7   # tie -> even
+    assert ora.tp_allreduce([np.array([1.0]), np.array([t]), np.array([t])])[0] == 1.0 + 2.0 ** -7
+    assert ora.tp_allreduce([np.array([2.0 ** 30]), np.array([1.0]), np.array([-2.0 ** 30])])[0] == 1.0
+    # row-parallel projection: K split over 2 ranks, small integers (exact)
+    a = rng.integers(-3, 4, size=(4, 12)).astype(np.float64)
+    W = rng.integers(-3, 4, size=(6, 12)).astype(np.float64)
+    ranks = [ora.projection(a[:, :5], W[:, :5]), ora.projection(a[:, 5:], W[:, 5:])]
+    assert np.array_equal(ora.tp_allreduce(ranks), a @ W.T)
+    # the composed QKV op: x = e_j s arrives as two ranks' parts (1 and 2)
+    Hq, Hkv, D, K, j, eps = 2, 1, 4, 16, 5, 1e-3
+    g = 1.0 + 0.1 * rng.normal(size=K)
+    Wq = rng.normal(0, 0.2, ((Hq + 2 * Hkv) * D, K))
+    p0, p1 = np.zeros((1, K)), np.zeros((1, K))
+    p0[0, j], p1[0, j] = 1.0, 2.0
+    out = ora.add_norm_qkv_tp([p0, p1], np.zeros((1, K)), g, None, "rmsnorm", eps, Wq, None, Hq, Hkv, D)
+    y = np.concatenate([out["q"][:, 0, :].reshape(-1), out["k"][:, 0, :].reshape(-1), out["v"][:, 0, :].reshape(-1)])
+    ref = Wq[:, j] * g[j] * 3.0 / math.sqrt(9.0 / K + eps)
+    assert np.max(np.abs(y - ref)) <= 1e-12 * np.max(np.abs(ref))
+    assert np.array_equal(out["residual_out"][0], np.where(np.arange(K) == j, 3.0, 0.0))
+
+
 PINS = [pin_layernorm_invariants, pin_rmsnorm_invariant, pin_norms_match_torch,
         pin_identity_weight, pin_one_hot, pin_brute_force, pin_epilogue_values,
         pin_qkv_bijection, pin_bf16_round, pin_residual_out,
         pin_run_maps_workload_inputs, pin_residual_projection, pin_e4m3_format, pin_fp8_quantisers,
-        pin_fp8_linear, pin_fp8_activation_codes, pin_fp8_fused_qkv]
+        pin_fp8_linear, pin_fp8_activation_codes, pin_fp8_fused_qkv, pin_tp_allreduce]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
@@ -548,7 +582,7 @@ def test_pin_holds(pin):
 
 ORIG = {name: getattr(core, name) for name in ("layernorm", "rmsnorm", "split_qkv_head_major", "run",
                                                "e4m3_round", "fp8_row_scale_and_codes", "fp8_activation_codes",
-                                               "fp8_linear", "fp8_normalised32")}
+                                               "fp8_linear", "fp8_normalised32", "tp_allreduce")}
 
 
 def _ln_unbiased(h, gamma, beta, eps):
@@ -743,6 +777,21 @@ def _fp8_norm32_drops_beta(h, mean, rstd, gamma, beta):
     return ORIG["fp8_normalised32"](h, mean, rstd, gamma, None)
 
 
+def _tp_rounds_each_addition(parts):
+    acc = core.bf16_round(np.asarray(parts[0], dtype=np.float64))
+    for v in parts[1:]:
+        acc = core.bf16_round(acc + np.asarray(v, dtype=np.float64))
+    return acc
+
+
+def _tp_drops_last_rank(parts):
+    return ORIG["tp_allreduce"](list(parts)[:-1]) if len(parts) > 1 else ORIG["tp_allreduce"](parts)
+
+
+def _tp_mean(parts):
+    return ORIG["tp_allreduce"](parts) / len(parts)
+
+
 MUTANTS = {
     "variance_divides_by_K_minus_1": ("layernorm", _ln_unbiased),
     "eps_outside_sqrt": ("layernorm", _ln_eps_outside),
@@ -778,6 +827,9 @@ MUTANTS = {
     "fp8_activation_scale_per_tensor": ("fp8_activation_codes", _fp8_act_per_tensor),
     "fp8_activation_scale_dropped": ("fp8_activation_codes", _fp8_act_no_dequant),
     "fp8_normalisation_drops_beta": ("fp8_normalised32", _fp8_norm32_drops_beta),
+    "tp_allreduce_rounds_each_addition": ("tp_allreduce", _tp_rounds_each_addition),
+    "tp_allreduce_drops_last_rank": ("tp_allreduce", _tp_drops_last_rank),
+    "tp_allreduce_averages": ("tp_allreduce", _tp_mean),
 }
 
 
