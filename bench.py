@@ -600,6 +600,60 @@ def bench_reference(w, steps, warmup, world, rank, budget_s=120.0):
     }
 
 
+def tp_entry(local, P: int, M: int, K: int, min_ms: float = 100.0):
+    """The tensor-parallel all-reduce (fnl_tp_allreduce) of P ranks' partial
+    outputs [M, K], on one GPU: the P parts are local buffers standing in for the
+    peers' (on a node the same loads cross NVLink). HBM-bound: (P + 1) M K 2
+    bytes per call; CUDA-graph replays over rotating copies larger than L2."""
+    from transformer_layer_residual_b200 import fnl
+    dev = torch.device("cuda", local)
+    n = M * K
+    per = (P + 1) * n * 2
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = max(1, min(64, -(-3 * l2 // per)))
+    gen = torch.Generator(device=dev).manual_seed(0)
+    sets = [([torch.randn(n, device=dev, generator=gen).to(torch.bfloat16) for _ in range(P)],
+             torch.empty(n, dtype=torch.bfloat16, device=dev)) for _ in range(R)]
+    h = fnl.Handle(local)
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        for parts, out in sets:
+            fnl.tp_allreduce(h, parts, out=out, stream=stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for parts, out in sets:
+            fnl.tp_allreduce(h, parts, out=out, stream=stream)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+        ev0.record(stream)
+        g.replay()
+        ev1.record(stream)
+    ev1.synchronize()
+    one = ev0.elapsed_time(ev1)
+    reps = max(1, int(np.ceil(min_ms / max(one, 1e-3))))
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        ev1.record(stream)
+    ev1.synchronize()
+    h.check()
+    per_ms = ev0.elapsed_time(ev1) / (reps * R)
+    pk, pk_src = peaks()
+    gbps = per / (per_ms / 1e3) / 1e9
+    e = {"us_per_call": round(per_ms * 1e3, 2), "calls": reps * R, "plan": f"tensor-parallel all-reduce, P={P}",
+         "M": M, "K": K, "P": P, "op": "tp_allreduce", "bound": "hbm", "achieved": round(gbps, 2),
+         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gbps / pk["hbm_gbs"], 4),
+         "peak_source": f"{pk_src} hbm_gbs"}
+    del g, sets
+    h.close()
+    torch.cuda.empty_cache()
+    return e
+
+
 def eager_calls(w, path: str, n: int):
     """N plain calls of one workload through the binding, for an ncu launch
     capture: the launches it makes are exactly those of the product path (the
@@ -652,6 +706,10 @@ def main():
         sweep = {}
         for name, ws in synthetic.workloads().items():
             sweep[name] = sweep_entry(ws, local, tune=not a.no_tune)
+            barrier(world)
+        # the tensor-parallel all-reduce that feeds the fused op (8 ranks, 70B hidden size)
+        for M in (32, 2048):
+            sweep[f"tp8_allreduce_m{M}_k8192"] = tp_entry(local, 8, M, 8192)
             barrier(world)
         line["sweep"] = sweep
     if rank == 0 and world == 1:

@@ -201,6 +201,23 @@ fnl_status fnl_add_bias_norm_gelu(fnl_handle* h, fnl_stream stream,
                                   int M, int K, int N,
                                   fnl_bf16* out, float* mean_out, float* rstd_out);
 
+/* Tensor-parallel all-reduce of the row-parallel projection's partial
+ * outputs, the input of the next fused op (TensorRT-LLM 深度工程实践, §4.1
+ * Tensor Parallelism: the output and down projections are split by rows, and
+ * the ranks' partial results are summed before the next add + norm).
+ * out[i] = bf16(sum over p = 0..P-1 of parts[p][i]), the sum in fp32 in rank
+ * order (every rank that runs it gets the same bits), one round-to-nearest-even.
+ * parts: host array of P device pointers, each n bf16 (16-byte aligned); on a
+ * node they are the P ranks' buffers, the peers' mapped into this device's
+ * address space (CUDA IPC / peer access), read with plain loads. The call does
+ * not wait for the other ranks: order it after every partial is complete (a
+ * host barrier or stream events). out: n bf16 (16-byte aligned), then passed as
+ * x to fnl_add_norm_* with the residual stream as residual. 1 <= P <= 16.
+ * Errors: FNL_ERR_INVALID_ARG (P out of range, n < 0, NULL), FNL_ERR_ALIGNMENT,
+ * FNL_ERR_ALIAS (out overlaps a part). */
+fnl_status fnl_tp_allreduce(fnl_handle* h, fnl_stream stream, const fnl_bf16* const* parts, int P, fnl_bf16* out,
+                            long long n);
+
 /* FP8 (W8A8) form of fnl_add_norm_qkv for decode-sized batches (M <= 128),
  * on the e4m3 tensor cores (tcgen05.mma kind::f8f6f4). TensorRT-LLM
  * 深度工程实践, §3.3 FP4/FP8 动态量化加速: W8A8_FP8 with activation ranges taken

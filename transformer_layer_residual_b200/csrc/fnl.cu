@@ -24,6 +24,7 @@
 #include "k2_wide.cuh"
 #include "k3_splitk.cuh"
 #include "k4_pair.cuh"
+#include "k5_tp.cuh"
 
 using fnl::bf16;
 using fnl::OpParams;
@@ -1228,6 +1229,35 @@ fnl_status fnl_add_bias_norm_gelu_fp8(fnl_handle* h, fnl_stream stream, const fn
   c.out = Bm(out);
   c.mean_out = mean_out; c.rstd_out = rstd_out;
   return run(h, c);
+}
+
+fnl_status fnl_tp_allreduce(fnl_handle* h, fnl_stream stream, const fnl_bf16* const* parts, int P, fnl_bf16* out,
+                            long long n) {
+  if (!h) return FNL_ERR_INVALID_ARG;
+  if (P < 1 || P > fnl::kMaxTpRanks || n < 0)
+    return fail(h, FNL_ERR_INVALID_ARG, "need 1 <= P <= %d and n >= 0 (P=%d)", fnl::kMaxTpRanks, P);
+  if (n == 0) return FNL_OK;
+  if (!parts || !out) return fail(h, FNL_ERR_INVALID_ARG, "parts and out are required");
+  fnl::TpParts tp{};
+  const Range o{out, static_cast<size_t>(n) * 2, "out"};
+  if (!al16(out)) return fail(h, FNL_ERR_ALIGNMENT, "out must be 16-byte aligned");
+  for (int q = 0; q < P; ++q) {
+    if (!parts[q]) return fail(h, FNL_ERR_INVALID_ARG, "parts[%d] is NULL", q);
+    if (!al16(parts[q])) return fail(h, FNL_ERR_ALIGNMENT, "parts[%d] must be 16-byte aligned", q);
+    if (overlap(o, Range{parts[q], static_cast<size_t>(n) * 2, "part"}))
+      return fail(h, FNL_ERR_ALIAS, "out overlaps parts[%d]", q);
+    tp.p[q] = B(parts[q]);
+  }
+  cudaError_t e = cudaSetDevice(h->device);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaSetDevice");
+  const long long n8 = std::max<long long>(n / 8, 1);
+  const int grid = static_cast<int>(std::min<long long>((n8 + fnl::kTpThreads - 1) / fnl::kTpThreads,
+                                                        static_cast<long long>(h->num_sms) * 4));
+  fnl::k5_tp_allreduce<<<grid, fnl::kTpThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      tp, P, reinterpret_cast<bf16*>(out), n);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(h, e, "launch of the tensor-parallel all-reduce");
+  return FNL_OK;
 }
 
 fnl_status fnl_quantize_weight_fp8(fnl_handle* h, fnl_stream stream, const fnl_bf16* W, int N, int K, uint8_t* Wq,

@@ -27,7 +27,7 @@ PRECISIONS = {"default": 0, "split": 1, "single": 2}
 EXPORTED = ("fnl_create", "fnl_destroy", "fnl_status_string", "fnl_last_error", "fnl_last_plan", "fnl_check",
             "fnl_add_norm_qkv", "fnl_add_norm_swiglu", "fnl_add_bias_norm_gelu", "fnl_linear_add_residual",
             "fnl_add_norm_qkv_fp8", "fnl_add_norm_swiglu_fp8", "fnl_add_bias_norm_gelu_fp8",
-            "fnl_quantize_weight_fp8",
+            "fnl_quantize_weight_fp8", "fnl_tp_allreduce",
             "fnl_add_norm_qkv_static", "fnl_check_static")
 
 
@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
     L.fnl_linear_add_residual.argtypes = [P, P, P, P, P, P, P, I, I, I]
     L.fnl_add_norm_qkv_fp8.argtypes = [P, P, P, P, P, P, P, I, F, P, P, P, I, I, I, I, I, P, P, P, P, P]
     L.fnl_quantize_weight_fp8.argtypes = [P, P, P, I, I, P, P]
+    L.fnl_tp_allreduce.argtypes = [P, P, ctypes.POINTER(P), I, P, ctypes.c_longlong]
     L.fnl_add_norm_swiglu_fp8.argtypes = [P, P, P, P, P, P, P, I, F, P, P, P, I, I, I, P, P, P]
     L.fnl_add_bias_norm_gelu_fp8.argtypes = [P, P, P, P, P, P, P, P, I, F, P, P, P, I, I, I, P, P, P]
     L.fnl_add_norm_qkv_static.argtypes = [P, P, P, P, P, P, I, F, P, P, I, I, I, I, I, P, P, P, P, P]
@@ -232,6 +233,36 @@ def add_bias_norm_gelu(h: Handle, x, residual, gamma, beta, W, bias_in=None, bia
     if st != FNL_OK:
         h._raise(st, "fnl_add_bias_norm_gelu")
     return {"residual_out": residual_out, "out": out, "mean": mean_out, "rstd": rstd_out}
+
+
+def tp_allreduce(h: Handle, parts, out=None, stream=None):
+    """fnl_tp_allreduce: out = bf16(sum of the P same-shape bf16 tensors in
+    `parts`, in list order). On a node the parts are the ranks' partial outputs
+    (the peers' as tensors over their mapped memory); here any device tensors.
+    Returns out."""
+    parts = list(parts)
+    if not parts:
+        raise ValueError("tp_allreduce needs at least one part")
+    shape = tuple(parts[0].shape)
+    for t in parts:
+        _need(t, "part", shape)
+    out = torch.empty(shape, dtype=torch.bfloat16, device=parts[0].device) if out is None else out
+    _need(out, "out", shape)
+    arr = (ctypes.c_void_p * len(parts))(*[t.data_ptr() for t in parts])
+    st = lib().fnl_tp_allreduce(h.ptr, _stream_ptr(stream), arr, len(parts), _p(out), out.numel())
+    if st != FNL_OK:
+        h._raise(st, "fnl_tp_allreduce")
+    return out
+
+
+def add_norm_qkv_tp(h: Handle, parts, residual, gamma, beta, W, Hq, Hkv, D, norm="rmsnorm", eps=1e-5, bias=None,
+                    x_buf=None, stream=None, **outs):
+    """The QKV op fed by the tensor-parallel all-reduce: x = tp_allreduce(parts)
+    (into x_buf if given), then add_norm_qkv(x, residual, ...). Two launches on
+    the stream; the fused op is a programmatic dependent of the all-reduce."""
+    x = tp_allreduce(h, parts, out=x_buf, stream=stream)
+    return add_norm_qkv(h, x, residual, gamma, beta, W, Hq, Hkv, D, norm=norm, eps=eps, bias=bias, stream=stream,
+                        **outs)
 
 
 def linear_add_residual(h: Handle, a, W, residual, bias=None, out=None, stream=None):
