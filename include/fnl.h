@@ -159,8 +159,11 @@ const char* fnl_last_error(const fnl_handle* h);
 const char* fnl_last_plan(const fnl_handle* h);
 
 /* Synchronise `stream`, read and clear the device status word. Returns
- * FNL_ERR_DEVICE_STATUS if a kernel since the last check gave up a wait; the
- * outputs of the calls since the last check are then not to be trusted. It
+ * FNL_ERR_DEVICE_STATUS if a kernel since the last check gave up a wait
+ * (device codes 1-7) or, in the debug build libfnl_debug.so (compiled with
+ * FNL_DEBUG_CHECKS), skipped an output store that would have left its buffer
+ * (device code 8); fnl_last_error() names the code. The outputs of the calls
+ * since the last check are then not to be trusted. It
  * also resets the handle's split-K arrival counters (an aborted CTA leaves its
  * tiles' counters part-way), so later calls on the handle compute correctly. */
 fnl_status fnl_check(fnl_handle* h, fnl_stream stream);

@@ -36,6 +36,15 @@ def test_library_exports_every_declared_symbol():
     assert set(declared_symbols()) <= exported
 
 
+def test_debug_build_exports_the_same_symbols():
+    """libfnl_debug.so (output stores bounds-checked) is a drop-in for libfnl.so."""
+    path = os.path.join(os.path.dirname(fnl.lib_path()), "libfnl_debug.so")
+    if not os.path.exists(path):
+        pytest.skip("debug build not built")
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
+    assert set(declared_symbols()) <= set(re.findall(r" T (fnl_\w+)", out))
+
+
 def test_library_is_sm100a_only_and_self_contained():
     out = subprocess.run(["ldd", fnl.lib_path()], capture_output=True, text=True).stdout
     assert "libcudart" not in out          # runtime linked statically

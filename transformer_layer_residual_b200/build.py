@@ -1,9 +1,13 @@
 """Builds libfnl.so (the C-ABI CUDA library) in-tree for sm_100a.
 
-    python -m transformer_layer_residual_b200.build [--verbose]
+    python -m transformer_layer_residual_b200.build [--verbose] [--force] [--debug]
 
 The library is one translation unit (csrc/fnl.cu) compiled by nvcc with the
 CUDA runtime linked statically, so the .so depends only on the driver.
+--debug builds libfnl_debug.so instead: the same code with FNL_DEBUG_CHECKS,
+which checks every output store against its buffer (an out-of-range store is
+skipped and reported through fnl_check as device status 8). The binding loads
+it when FNL_LIBRARY=debug is set.
 """
 from __future__ import annotations
 
@@ -17,6 +21,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfnl.so")
+LIB_DEBUG = os.path.join(PKG, "libfnl_debug.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -38,19 +43,20 @@ def sources() -> list:
     return [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC))]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + [os.path.join(INCLUDE, "fnl.h"), os.path.abspath(__file__)]
     return all(os.path.getmtime(d) <= t for d in deps)
 
 
-def build(verbose: bool = False, force: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    cmd = [nvcc()] + NVCC_FLAGS + ["-I", INCLUDE, "-I", CSRC, "-o", LIB + ".tmp",
-                                  os.path.join(CSRC, "fnl.cu")]
+def build(verbose: bool = False, force: bool = False, debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    cmd = [nvcc()] + NVCC_FLAGS + (["-DFNL_DEBUG_CHECKS"] if debug else []) + \
+        ["-I", INCLUDE, "-I", CSRC, "-o", lib + ".tmp", os.path.join(CSRC, "fnl.cu")]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd))
@@ -59,9 +65,9 @@ def build(verbose: bool = False, force: bool = False) -> str:
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     if verbose:
         sys.stdout.write(res.stdout + res.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose="--verbose" in sys.argv, force="--force" in sys.argv))
+    print(build(verbose="--verbose" in sys.argv, force="--force" in sys.argv, debug="--debug" in sys.argv))

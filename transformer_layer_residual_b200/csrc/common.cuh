@@ -219,6 +219,22 @@ __device__ __forceinline__ void fp8_dequant8(const OpParams& p, int m, int n, fl
   for (int e = 0; e < 8; ++e) y[e] *= sa * ws[e];
 }
 
+// Debug builds (FNL_DEBUG_CHECKS: libfnl_debug.so, built beside libfnl.so) check
+// every output store against its buffer: an out-of-range store is skipped and
+// the status word records kStatusBounds, which fnl_check reports. It stands in
+// for compute-sanitizer on the outputs, where a wrong index would otherwise
+// corrupt memory silently. Release builds compile the check away.
+__device__ __forceinline__ bool store_in_bounds(const OpParams& p, const bf16* dst, const bf16* base,
+                                                size_t elems) {
+#ifdef FNL_DEBUG_CHECKS
+  if (base == nullptr || dst < base || dst + 8 > base + elems) {
+    if (p.status != nullptr) atomicCAS(p.status, 0, kStatusBounds);
+    return false;
+  }
+#endif
+  return true;
+}
+
 template <int EPI>
 __device__ __forceinline__ void store_out8(const OpParams& p, int m, int n, const float (&acc)[8], float scale) {
   float y[8];
@@ -232,6 +248,8 @@ __device__ __forceinline__ void store_out8(const OpParams& p, int m, int n, cons
     for (int e = 0; e < 8; ++e) y[e] += b[e];
   }
   bf16* dst;
+  const bf16* base = p.out;
+  size_t elems = static_cast<size_t>(p.M) * p.N;
   if (EPI == kEpiResidual) {
     const size_t off = static_cast<size_t>(m) * p.N + n;
     float r[8];
@@ -250,14 +268,21 @@ __device__ __forceinline__ void store_out8(const OpParams& p, int m, int n, cons
     if (n < nq) {
       const int h = n / D;
       dst = p.q + (static_cast<size_t>(h) * p.M + m) * D + (n - h * D);
+      base = p.q;
+      elems = static_cast<size_t>(p.Hq) * p.M * D;
     } else if (n < nk) {
       const int n2 = n - nq, h = n2 / D;
       dst = p.k + (static_cast<size_t>(h) * p.M + m) * D + (n2 - h * D);
+      base = p.k;
+      elems = static_cast<size_t>(p.Hkv) * p.M * D;
     } else {
       const int n2 = n - nk, h = n2 / D;
       dst = p.v + (static_cast<size_t>(h) * p.M + m) * D + (n2 - h * D);
+      base = p.v;
+      elems = static_cast<size_t>(p.Hkv) * p.M * D;
     }
   }
+  if (!store_in_bounds(p, dst, base, elems)) return;
   *reinterpret_cast<uint4*>(dst) = pack8(y);
 }
 
@@ -287,7 +312,9 @@ __device__ __forceinline__ void store_swiglu8(const OpParams& p, int m, int j, c
   float y[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) y[e] = silu_f(g[e]) * u[e];
-  *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(m) * p.I + j) = pack8(y);
+  bf16* dst = p.out + static_cast<size_t>(m) * p.I + j;
+  if (!store_in_bounds(p, dst, p.out, static_cast<size_t>(p.M) * p.I)) return;
+  *reinterpret_cast<uint4*>(dst) = pack8(y);
 }
 
 }  // namespace fnl

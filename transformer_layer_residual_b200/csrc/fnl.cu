@@ -1123,7 +1123,9 @@ fnl_status fnl_check(fnl_handle* h, fnl_stream stream) {
     e = cudaMemset(h->ws, 0, kFixedBytes);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemset(status, counters)");
-    return fail(h, FNL_ERR_DEVICE_STATUS, "a kernel gave up a bounded wait (code %d)", status);
+    return fail(h, FNL_ERR_DEVICE_STATUS,
+                "device status %d (1-7: a kernel gave up a bounded wait; 8: a debug build refused an out-of-range "
+                "store)", status);
   }
   return FNL_OK;
 }

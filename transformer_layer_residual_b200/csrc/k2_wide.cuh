@@ -393,8 +393,11 @@ __global__ void __launch_bounds__(k2w::NUM_THREADS, 1)
             if (WRES) {
               const int gm = mb * BM + row;
               const int k0 = kb * BK + c * 8;
-              if (gm < M && k0 < K)
-                *reinterpret_cast<uint4*>(p.residual_out + static_cast<size_t>(gm) * K + k0) = hres;
+              if (gm < M && k0 < K) {
+                bf16* dst = p.residual_out + static_cast<size_t>(gm) * K + k0;
+                if (store_in_bounds(p, dst, p.residual_out, static_cast<size_t>(M) * K))
+                  *reinterpret_cast<uint4*>(dst) = hres;
+              }
             }
           }
         };

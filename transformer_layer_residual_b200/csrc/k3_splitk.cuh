@@ -552,7 +552,8 @@ __global__ void __launch_bounds__(k3::NUM_THREADS, 1)
           if (BIAS_IN) h = add2(h, bf2_to_f2(bw[e]));
           hw[e] = f2_to_bf2(h);
         }
-        *reinterpret_cast<uint4*>(p.residual_out + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        if (store_in_bounds(p, p.residual_out + off, p.residual_out, static_cast<size_t>(p.M) * p.K))
+          *reinterpret_cast<uint4*>(p.residual_out + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
       }
     }
     SegIter it(u0, u1, U, nkb, gridDim.x, blockIdx.x);

@@ -28,6 +28,7 @@ enum : int {
   kStatusWaitTmemEmpty = 5,
   kStatusWaitStats = 6,
   kStatusWaitDrain = 7,
+  kStatusBounds = 8,   // debug build (FNL_DEBUG_CHECKS): an output store fell outside its buffer
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -14,7 +14,9 @@ from typing import Optional
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfnl.so")
+# FNL_LIBRARY=debug selects the debug build (output stores checked against their buffers)
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                         "libfnl_debug.so" if os.environ.get("FNL_LIBRARY") == "debug" else "libfnl.so")
 _lib = None
 
 FNL_OK = 0
