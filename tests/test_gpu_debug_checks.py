@@ -27,12 +27,13 @@ FORMS = {
     "wide": [("qkv", "layernorm", 300, 520), ("swiglu", "rmsnorm", 64, 200), ("residual", "none", 7, 328)],
     "pair": [("qkv", "rmsnorm", 600, 328), ("swiglu", "layernorm", 257, 520), ("gelu", "layernorm", 129, 200),
              ("residual", "none", 255, 328)],
-    "pair_sk": [("qkv", "rmsnorm", 300, 2048), ("swiglu", "layernorm", 256, 1536), ("gelu", "layernorm", 260, 2000),
+    # stream-K needs at least one (tile, k-block) unit per pair: 74 pairs
+    "pair_sk": [("qkv", "rmsnorm", 300, 2048), ("swiglu", "layernorm", 260, 4096), ("gelu", "layernorm", 260, 2000),
                 ("residual", "none", 384, 2048)],
     "splitk": [("qkv", "layernorm", 33, 1024), ("swiglu", "rmsnorm", 1, 200), ("gelu", "rmsnorm", 128, 520),
                ("residual", "none", 16, 520), ("qkv_fp8", "rmsnorm", 16, 528), ("swiglu_fp8", "layernorm", 33, 208)],
-    "cluster": [("qkv", "rmsnorm", 8, 4096), ("swiglu", "layernorm", 64, 520), ("gelu", "layernorm", 5, 200),
-                ("residual", "none", 128, 328), ("gelu_fp8", "rmsnorm", 7, 528), ("qkv_fp8", "layernorm", 128, 208)],
+    "cluster": [("qkv", "rmsnorm", 8, 4096), ("swiglu", "layernorm", 64, 520), ("gelu", "layernorm", 5, 520),
+                ("residual", "none", 128, 328), ("gelu_fp8", "rmsnorm", 7, 528), ("qkv_fp8", "layernorm", 128, 528)],
 }
 
 
