@@ -421,6 +421,8 @@ def bench_fnl(w, steps, warmup, world, rank, local, tune=True, path="auto"):
     unit, per_step, bound = units(w)
     value = per_step * steps * world / (ms_max / 1e3)
     launches_per_step = 2 if (w.norm == "layernorm" or w.op in synthetic.FP8_OPS) else 1   # + the stats pre-pass
+    if "stream-K" in bed.plan and "CTA-pair" in bed.plan:
+        launches_per_step += 1   # the pair kernel's fix-up of its split tiles
     host_us = bed.host_us_per_call(50 if w.flops() < 1e12 else 10)
 
     # e2e: through the public binding, host buffers, copies inside the timed region

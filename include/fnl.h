@@ -99,8 +99,9 @@ typedef enum {
                                   the tiles cannot all run at once as clusters of 2..8 CTAs) */
   FNL_PATH_TILE_PAIR = 5,      /* force the large-M kernel on CTA pairs (tcgen05 cta_group::2), 256 x 512 tiles */
   FNL_PATH_TILE_PAIR_SPLIT = 6 /* the pair kernel's stream-K form: whole waves of tiles as above, the tiles left
-                                  over dealt to all pairs as (tile, k-block) units, their partial sums added by
-                                  the last pair to arrive, in a fixed order (a candidate of the shape tuner) */
+                                  over dealt to all pairs as (tile, k-block) units; a fix-up kernel launched
+                                  after it adds each split tile's partial sums in a fixed order and runs the
+                                  epilogue (a candidate of the shape tuner) */
 } fnl_path;
 
 /* How the normalised activation a is rounded for the bf16 tensor cores.

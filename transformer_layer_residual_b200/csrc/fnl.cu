@@ -474,6 +474,43 @@ fnl_status dispatch_residual(fnl_handle* h, bool small, bool wide, bool pair, in
                      mw, p);
 }
 
+// The fix-up of the pair kernel's split tiles (stream-K form), a programmatic
+// dependent of the pair kernel: one CTA per (split tile, CTA half, 16 rows).
+template <int EPI, int NORM>
+fnl_status launch_fixup_t(fnl_handle* h, int T, int pairs, cudaStream_t stream, const OpParams& p) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(T) * 2 * fnl::k6::GROUPS);
+  cfg.blockDim = dim3(fnl::k6::THREADS);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, fnl::k6_pair_fixup<EPI, NORM>, p, pairs);
+  if (e != cudaSuccess) return cuda_fail(h, e, "launch of the pair kernel's fix-up kernel");
+  return FNL_OK;
+}
+
+fnl_status launch_fixup(fnl_handle* h, int epi, int norm, int T, int pairs, cudaStream_t stream,
+                        const OpParams& p) {
+  using namespace fnl;
+  if (epi == kEpiResidual) return launch_fixup_t<kEpiResidual, kNoNorm>(h, T, pairs, stream, p);
+  const bool rms = norm == kRMSNorm;
+  switch (epi) {
+    case kEpiQKV:
+      return rms ? launch_fixup_t<kEpiQKV, kRMSNorm>(h, T, pairs, stream, p)
+                 : launch_fixup_t<kEpiQKV, kLayerNorm>(h, T, pairs, stream, p);
+    case kEpiSwiGLU:
+      return rms ? launch_fixup_t<kEpiSwiGLU, kRMSNorm>(h, T, pairs, stream, p)
+                 : launch_fixup_t<kEpiSwiGLU, kLayerNorm>(h, T, pairs, stream, p);
+    default:
+      return rms ? launch_fixup_t<kEpiGELU, kRMSNorm>(h, T, pairs, stream, p)
+                 : launch_fixup_t<kEpiGELU, kLayerNorm>(h, T, pairs, stream, p);
+  }
+}
+
 fnl_status launch_k1(fnl_handle* h, const Call& c, float2* stats, cudaStream_t stream) {
   const int nvec = c.K / 8;
   const int v = (nvec + fnl::kK1Threads - 1) / fnl::kK1Threads;
@@ -656,12 +693,11 @@ fnl_status plan_kernel(fnl_handle* h, const Call& c, Kern kern, int cls_req, Pla
                             (c.op == Op::SwiGLU ? (c.I + 255) / 256 : (c.N + fnl::k4::BN - 1) / fnl::k4::BN);
     q.grid = 2 * static_cast<int>(std::min<long long>(pairs_max, tiles));
     // Stream-K form: the whole waves stay whole tiles, and the (tile, 32-wide
-    // k-block) units of the tiles left over are dealt evenly over all pairs.
-    // Measured on B200 it lost to the plain forms (70B QKV at M = 256: 187 us
-    // against 85 us for the 128x256 stream-K kernel; M = 2048: 472 against 395
-    // us with whole tiles): the last pair to arrive at a split tile reads the
-    // others' 128 x 512 fp32 partial sums back through L2. So it is a tuner
-    // candidate and a forced path, not the default.
+    // k-block) units of the tiles left over are dealt evenly over all pairs;
+    // the fix-up kernel adds the split tiles' partial sums. Measured on B200:
+    // 70B QKV at M = 2048 (2.16 waves) 348 us against 396 with whole tiles; at
+    // M = 256 (20 tiles, all split) 90 us against 86 for the 128x256 stream-K
+    // kernel; with a last wave more than half full, whole tiles win.
     const long long nkb4 = (c.K + fnl::k4::BK - 1) / fnl::k4::BK;
     if (kern == Kern::K4S) {
       if (tiles * nkb4 < pairs_max)
@@ -751,7 +787,13 @@ fnl_status default_plan(fnl_handle* h, const Call& c, Plan* pl) {
   const double t_w = 1.6 * waves(tiles_w, max_ctas);
   const int pairs = h->opt.max_ctas == 0 ? resident_pairs(h) : 0;
   const double t_p = pairs > 0 ? 1.45 * waves(tiles_p, pairs) : 1e30;
-  if (t_p <= t_w && t_p <= t_n) return plan_kernel(h, c, Kern::K4, -1, pl);
+  // The pair kernel's stream-K form once there is a whole wave: the leftover
+  // tiles' units spread over all pairs, at about half a tile's time of extra
+  // cost (partial-sum stores, the fix-up kernel; 0.1-0.6 measured on B200 at
+  // the prefill shapes: 70B QKV at M = 2048, 2.16 waves, 396 -> 348 us)
+  const double t_ps = pairs > 0 && tiles_p >= pairs ? 1.45 * (static_cast<double>(tiles_p) / pairs + 0.5) : 1e30;
+  const double t_pair = std::min(t_p, t_ps);
+  if (t_pair <= t_w && t_pair <= t_n) return plan_kernel(h, c, t_ps < t_p ? Kern::K4S : Kern::K4, -1, pl);
   return plan_kernel(h, c, t_w <= t_n ? Kern::K2W : Kern::K2, -1, pl);
 }
 
@@ -855,7 +897,13 @@ fnl_status launch_plan(fnl_handle* h, const Call& c, const Plan& q) {
   // streams its first weight tiles before griddepcontrol.wait and touches
   // activations, statistics, workspace and outputs only after it.
   const bool pdl = true;
-  if (nonorm) return dispatch_residual(h, small, wide, pair, q.grid, q.threads, q.smem, pdl, c.stream, mx, mw, p);
+  // the pair kernel's stream-K form: its split tiles are finished by the fix-up kernel
+  const bool fixup = pair && q.sk != 0;
+  if (nonorm) {
+    st = dispatch_residual(h, small, wide, pair, q.grid, q.threads, q.smem, pdl, c.stream, mx, mw, p);
+    if (st == FNL_OK && fixup) st = launch_fixup(h, fnl::kEpiResidual, fnl::kNoNorm, q.T, q.grid / 2, c.stream, p);
+    return st;
+  }
   if (c.fp8) {
     if ((st = launch_fp8_prepass(h, c, reinterpret_cast<float4*>(stats), q8, c.stream)) != FNL_OK) return st;
     return dispatch_fp8(h, epi_of(c), q.grid, q.threads, q.smem, pdl, c.stream, mx, mr, mw, p);
@@ -866,15 +914,20 @@ fnl_status launch_plan(fnl_handle* h, const Call& c, const Plan& q) {
   const int epi = c.op == Op::QKV ? fnl::kEpiQKV : (c.op == Op::SwiGLU ? fnl::kEpiSwiGLU : fnl::kEpiGELU);
   switch (epi) {
     case fnl::kEpiQKV:
-      return dispatch_gemm<fnl::kEpiQKV>(h, small, rms, q.grid, q.threads, q.smem, pdl, c.stream, mx, mr, mw, p, wide,
-                                         pair);
+      st = dispatch_gemm<fnl::kEpiQKV>(h, small, rms, q.grid, q.threads, q.smem, pdl, c.stream, mx, mr, mw, p, wide,
+                                       pair);
+      break;
     case fnl::kEpiSwiGLU:
-      return dispatch_gemm<fnl::kEpiSwiGLU>(h, small, rms, q.grid, q.threads, q.smem, pdl, c.stream, mx, mr, mw, p,
-                                            wide, pair);
+      st = dispatch_gemm<fnl::kEpiSwiGLU>(h, small, rms, q.grid, q.threads, q.smem, pdl, c.stream, mx, mr, mw, p,
+                                          wide, pair);
+      break;
     default:
-      return dispatch_gemm<fnl::kEpiGELU>(h, small, rms, q.grid, q.threads, q.smem, pdl, c.stream, mx, mr, mw, p, wide,
-                                          pair);
+      st = dispatch_gemm<fnl::kEpiGELU>(h, small, rms, q.grid, q.threads, q.smem, pdl, c.stream, mx, mr, mw, p, wide,
+                                        pair);
   }
+  if (st == FNL_OK && fixup)
+    st = launch_fixup(h, epi, rms ? fnl::kRMSNorm : fnl::kLayerNorm, q.T, q.grid / 2, c.stream, p);
+  return st;
 }
 
 // ------------------------------------------------------------------ tuner

@@ -46,9 +46,14 @@
 //
 // Work split: each pair takes whole tiles in turn, or, when the tiles fill the
 // pairs' waves poorly (70B QKV at M = 256: 20 tiles for 74 pairs; M = 2048: 2.2
-// waves), stream-K: the (tile, k-block) units are dealt evenly over the pairs
-// and a tile shared by several pairs is summed by the last to arrive (see the
-// epilogue).
+// waves), stream-K: the (tile, k-block) units are dealt evenly over the pairs.
+// A pair that holds only part of a tile's k-blocks stores its fp32 partial sums
+// in a slot and moves on; the fix-up kernel k6_pair_fixup, launched right after,
+// adds each split tile's slots in slot order and runs the epilogue, spread over
+// the whole GPU. (Summed inside this kernel by the last pair to arrive, the
+// gather of up to 5 x 256 KB of partial sums per CTA through L2 ran on 128
+// threads of one pair and held that pair's next segment: 70B QKV at M = 256
+// took 187 us, against 85 us for the 128 x 256 stream-K kernel.)
 #pragma once
 
 #include "common.cuh"
@@ -98,10 +103,9 @@ constexpr int GROUP_M = 8;         // pair rows (of 256 tokens) sharing a W tile
 struct Ctrl {
   uint64_t full_w[MAX_OST], conv[MAX_OST], empty[MAX_OST];   // operand ring
   uint64_t raw_full[MAX_RST], raw_empty[MAX_RST];            // raw ring
-  uint64_t tfull, tempty, sfull[2], efree[2], drain, esync;
+  uint64_t tfull, tempty, sfull[2], efree[2], drain;
   uint32_t tmem_base;
   int abort_flag;
-  int last_flag;   // stream-K: this CTA arrived last at the current partial tile
   float rs[2][CONV_GROUPS][BM];   // RMSNorm: per segment buffer, per converter group, sum of h^2 per row
 };
 constexpr int SMEM_BYTES = RINGS_BYTES + VEC_BYTES + static_cast<int>(sizeof(Ctrl)) + 1024;
@@ -245,9 +249,7 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
       mbar_init(&ctrl->efree[b], NUM_EPI_WARPS);
     }
     mbar_init(&ctrl->drain, 1);
-    mbar_init(&ctrl->esync, NUM_EPI_WARPS * EPI_SHARES);   // every epilogue share of this CTA
     ctrl->abort_flag = 0;
-    ctrl->last_flag = 0;
     fence_mbar_init();
   }
   if (warp == WARP_TMA && lane == 0) {
@@ -277,12 +279,8 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
   // start on the next segment. Every taking warp of both CTAs arrives on the
   // even CTA's tempty.
   // A segment that is only part of its tile's k-blocks (stream-K, nseg > 1)
-  // first stores this CTA's 128 rows of partial sums (fp32 [128][512], and the
-  // rows' partial sums of h^2) in its slot; one thread's acquire-release arrival
-  // on the tile half's counter then elects the CTA that arrives last, which sums
-  // the nseg slots in slot order (its own from TMEM), so the result does not
-  // depend on the arrival order, runs the epilogue and resets the counter.
-  uint32_t esync_phase = 0;
+  // stores this CTA's 128 rows of partial sums (fp32 [128][512], and the rows'
+  // partial sums of h^2) in its slot instead; k6_pair_fixup finishes the tile.
   auto epilogue_share = [&](int i, int t, int slot, int nseg, int j) -> bool {
     const int q32 = (warp & 3) * 32;
     const int row_local = q32 + lane;
@@ -313,12 +311,11 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
     // TMEM column of 16-column chunk cc: the gate and up halves for SwiGLU
     constexpr int NCH = EPI == kEpiSwiGLU ? 16 : BN / 16;
     const bool partial = nseg > 1;
-    // slot sl of this tile half: 128 rows x 512 fp32 partial sums, 128 partial sums of h^2
-    const size_t half0 = static_cast<size_t>(partial ? segs0.sk_tile(t) : 0) * p.max_seg * 2 + rank;
-    auto part_row = [&](int sl) { return p.part + ((half0 + static_cast<size_t>(sl) * 2) * BM + row_local) * 512; };
-    bool last = true;
     if (partial) {
-      float* own = part_row(slot);
+      // slot `slot` of this tile half: 128 rows x 512 fp32 partial sums, 128 partial sums of h^2
+      const size_t half =
+          (static_cast<size_t>(segs0.sk_tile(t)) * p.max_seg + static_cast<size_t>(slot)) * 2 + rank;
+      float* own = p.part + (half * BM + row_local) * 512;
 #pragma unroll 1
       for (int cc = j; cc < NCH; cc += EPI_SHARES) {
         uint32_t a0[16];
@@ -339,71 +336,17 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
             *reinterpret_cast<uint4*>(own + cc * 16 + e) = make_uint4(a0[e], a0[e + 1], a0[e + 2], a0[e + 3]);
         }
       }
-      if (NORM == kRMSNorm && j == 0) p.part_ss[(half0 + static_cast<size_t>(slot) * 2) * BM + row_local] = ssum;
-      // every share of this CTA has stored its part; then the arrival (one thread), then its result
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctrl->esync);
-      if (!warp_wait(&ctrl->esync, esync_phase, abortf, p.status, kStatusWaitDrain, p.wait_ns)) {
-        if (lane == 0) abort_pair();
-        return false;
-      }
-      esync_phase ^= 1u;
-      if (j == 0 && (warp & 3) == 0 && lane == 0) {
-        unsigned* cnt = p.counters + static_cast<size_t>(segs0.sk_tile(t)) * 2 + rank;
-        const unsigned old = atom_add_acq_rel_gpu(cnt, 1u);
-        const int is_last = old == static_cast<unsigned>(nseg - 1) ? 1 : 0;
-        ctrl->last_flag = is_last;
-        if (is_last) *cnt = 0u;   // no other CTA touches it again in this launch
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctrl->esync);
-      if (!warp_wait(&ctrl->esync, esync_phase, abortf, p.status, kStatusWaitDrain, p.wait_ns)) {
-        if (lane == 0) abort_pair();
-        return false;
-      }
-      esync_phase ^= 1u;
-      last = ctrl->last_flag != 0;
-    }
-    if (last) {
+      if (NORM == kRMSNorm && j == 0) p.part_ss[half * BM + row_local] = ssum;
+    } else {
       float scale = 1.f;
-      if (NORM == kRMSNorm) {
-        float tot = ssum;
-        if (partial) {
-          tot = 0.f;
-          for (int sl = 0; sl < nseg; ++sl)
-            tot += sl == slot ? ssum : __ldcg(p.part_ss + (half0 + static_cast<size_t>(sl) * 2) * BM + row_local);
-        }
-        scale = 1.f / sqrtf(tot / static_cast<float>(K) + p.eps);
-      }
+      if (NORM == kRMSNorm) scale = 1.f / sqrtf(ssum / static_cast<float>(K) + p.eps);
       if (NORM == kRMSNorm && j == 0 && nb == 0 && row_ok && p.rstd_out != nullptr) p.rstd_out[m] = scale;
-      // 16 columns at TMEM column `col`: this CTA's own value, plus (partial) the other slots in slot order
       auto gather16 = [&](int col, float (&v)[16]) {
         uint32_t a0[16];
         tmem_ld16(tbase + col, a0);
         tmem_ld_wait();
-        if (!partial) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(a0[e]);
-          return;
-        }
-#pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = 0.f;
-        for (int sl = 0; sl < nseg; ++sl) {
-          if (sl == slot) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] += __uint_as_float(a0[e]);
-          } else {
-            const float* src = part_row(sl) + col;
-#pragma unroll
-            for (int e = 0; e < 16; e += 4) {
-              const float4 w = __ldcg(reinterpret_cast<const float4*>(src + e));
-              v[e] += w.x;
-              v[e + 1] += w.y;
-              v[e + 2] += w.z;
-              v[e + 3] += w.w;
-            }
-          }
-        }
+        for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(a0[e]);
       };
       // 16-column chunks: few registers held, so the converter warps can take shares without spilling
       if (EPI == kEpiSwiGLU) {
@@ -809,6 +752,98 @@ __global__ void __launch_bounds__(k4::NUM_THREADS, 1)
   if (warp == WARP_MMA) {
     tc_fence_after();
     tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- K6
+// Fix-up of the pair kernel's split tiles (its stream-K form), launched right
+// after it as its programmatic dependent. For split tile ts (tile sk_full + ts
+// of the pair raster) the nseg pairs that held its k-blocks each stored, per
+// CTA half and slot, 128 rows x 512 fp32 partial sums and the rows' 128
+// partial sums of h^2. One CTA per (split tile, half, 16-row group); each
+// thread adds the slots of its 8-column chunks in slot order (the result does
+// not depend on which pair finished first) and applies the op's epilogue as
+// the pair kernel does: the RMSNorm scale from the summed h^2, then bias and
+// the QKV split, SwiGLU, GELU or the residual add. The partial sums were
+// written just before, so they are read through L2 (ld.global.cg).
+namespace k6 {
+constexpr int ROWS = 16;                  // rows of a tile half per CTA
+constexpr int GROUPS = k4::BM / ROWS;     // 8 CTAs per tile half
+constexpr int THREADS = 256;
+}  // namespace k6
+
+template <int EPI, int NORM>
+__global__ void __launch_bounds__(k6::THREADS) k6_pair_fixup(const OpParams p, int G) {
+  using namespace k4;
+  pdl_wait();   // every slot of the pair kernel is stored and visible
+  pdl_launch_dependents();
+  const int M = p.M, K = p.K;
+  const int num_m2 = (M + 2 * BM - 1) / (2 * BM);
+  const int num_n = (EPI == kEpiSwiGLU) ? (p.I + 255) / 256 : (p.N + BN - 1) / BN;
+  const int nkb = (K + BK - 1) / BK;
+  const int full = p.sk_full;
+  const long long U = static_cast<long long>(num_m2 * num_n - full) * nkb;
+  const int ts = blockIdx.x / (2 * k6::GROUPS);
+  const int rank = (blockIdx.x / k6::GROUPS) & 1;
+  const int rg = blockIdx.x % k6::GROUPS;
+  const int first = unit_owner_fast(static_cast<long long>(ts) * nkb, G, U);
+  const int last = unit_owner_fast(static_cast<long long>(ts + 1) * nkb - 1, G, U);
+  const int nseg = last - first + 1;
+  if (nseg < 2) return;   // one pair held the whole tile and ran its epilogue
+  int mb2, nb;
+  tile_coords(full + ts, num_m2, num_n, mb2, nb);
+  const size_t half0 = static_cast<size_t>(ts) * p.max_seg * 2 + rank;
+  // 8-column chunks per row (SwiGLU: gate chunks, each with the matching up chunk)
+  constexpr int CH = EPI == kEpiSwiGLU ? 32 : 64;
+  constexpr int ITEMS = k6::ROWS * CH / k6::THREADS;
+#pragma unroll
+  for (int it = 0; it < ITEMS; ++it) {
+    const int idx = threadIdx.x + it * k6::THREADS;
+    const int row_local = rg * k6::ROWS + idx / CH;
+    const int ch = idx % CH;
+    const int m = mb2 * 2 * BM + rank * BM + row_local;
+    if (m >= M) continue;
+    float scale = 1.f;
+    if (NORM == kRMSNorm) {
+      float tot = 0.f;
+      for (int sl = 0; sl < nseg; ++sl)
+        tot += __ldcg(p.part_ss + (half0 + static_cast<size_t>(sl) * 2) * BM + row_local);
+      scale = 1.f / sqrtf(tot / static_cast<float>(K) + p.eps);
+      if (nb == 0 && ch == 0 && p.rstd_out != nullptr) p.rstd_out[m] = scale;
+    }
+    auto sum8 = [&](int col, float (&v)[8]) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = 0.f;
+      for (int sl = 0; sl < nseg; ++sl) {
+        const float* src = p.part + ((half0 + static_cast<size_t>(sl) * 2) * BM + row_local) * 512 + col;
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(src));
+        const float4 b = __ldcg(reinterpret_cast<const float4*>(src + 4));
+        v[0] += a.x;
+        v[1] += a.y;
+        v[2] += a.z;
+        v[3] += a.w;
+        v[4] += b.x;
+        v[5] += b.y;
+        v[6] += b.z;
+        v[7] += b.w;
+      }
+    };
+    if (EPI == kEpiSwiGLU) {
+      const int jj = nb * 256 + ch * 8;
+      if (jj < p.I) {
+        float g[8], u[8];
+        sum8(ch * 8, g);
+        sum8(256 + ch * 8, u);
+        store_swiglu8(p, m, jj, g, u, scale);
+      }
+    } else {
+      const int n = nb * BN + ch * 8;
+      if (n < p.N) {
+        float a[8];
+        sum8(ch * 8, a);
+        store_out8<EPI>(p, m, n, a, scale);
+      }
+    }
   }
 }
 
