@@ -373,6 +373,9 @@ def _roofline(w, per_launch_ms, bound):
     return achieved, pk["bf16_tflops_sustained"], "TFLOP/s", f"{pk_src} bf16_tflops_sustained"
 
 
+SETTLE_S = 1.0   # untimed seconds of the step loop between the warm-up steps and the timed steps
+
+
 def _sustain(bed, g, seconds):
     """Keep replaying g for `seconds` (clock record of short timed regions)."""
     t_end = time.time() + seconds
@@ -403,7 +406,10 @@ def bench_fnl(w, steps, warmup, world, rank, local, tune=True, path="auto"):
 
     sampler = ClockSampler(local)
     sampler.start()
-    time.sleep(0.3)
+    # the same step loop for SETTLE_S more, untimed, so that the timed steps run at the
+    # clock the GPU holds under continuous load (a long prefill batch, a serving loop)
+    # instead of its first power-cap transient; it also covers the sampler's start
+    _sustain(bed, g_full, SETTLE_S)
     barrier(world)
     torch.cuda.synchronize()
     t_wall0 = time.time()
@@ -476,7 +482,8 @@ def bench_fnl(w, steps, warmup, world, rank, local, tune=True, path="auto"):
                    **({"seqs": len(w.seq_lens)} if w.seq_lens else {}),
                    "l2": f"inputs larger than L2: {R} rotating copies of W/x/residual "
                          f"({R * bed.per_copy / 1e6:.0f} MB vs L2 {bed.l2 / 1e6:.0f} MB)",
-                   "timing": f"CUDA graph replays of {R} calls, CUDA events on the launch stream",
+                   "timing": f"CUDA graph replays of {R} calls, CUDA events on the launch stream; "
+                             f"after the warm-up steps the same loop runs {SETTLE_S} s more untimed (steady clock)",
                    "plan": bed.plan,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "tflops": round(w.flops() * steps * world / (ms_max / 1e3) / 1e12, 3),
@@ -513,7 +520,7 @@ def sweep_entry(w, local, min_ms=100.0, tune=True):
     n = max(1, int(np.ceil(min_ms / max(one * bed.R, 1e-3))))
     sampler = ClockSampler(local)
     sampler.start()
-    time.sleep(0.2)
+    _sustain(bed, g, SETTLE_S / 2)   # steady clock, as for the headline
     t0 = time.time()
     ms = bed.timed([g] * n)
     t1 = time.time()
