@@ -319,14 +319,16 @@ def test_pair_kernel_row_tails(cuda_device, M, op, norm):
 
 
 # Pair kernel, stream-K form (forced): few tiles for the 74 pairs, so the (tile,
-# k-block) units are dealt over all pairs and each tile is summed from several
-# pairs' partial sums (K not a multiple of the 32-wide k-block in two cases).
+# k-block) units are dealt over all pairs and the fix-up kernel sums each tile
+# from several pairs' partial sums (K not a multiple of the 32-wide k-block in
+# two cases); every epilogue with each norm.
 STREAM_K_CASES = [
     ("qkv", "rmsnorm", 300, 2048, dict(Hq=6, Hkv=2, D=128, bias_out=True)),
     ("qkv", "layernorm", 513, 2000, dict(Hq=4, Hkv=2, D=128)),
     ("swiglu", "rmsnorm", 260, 1536, dict(I=600, bias_out=True)),
     ("swiglu", "layernorm", 256, 4096, dict(I=256)),   # one tile over every pair
     ("gelu", "layernorm", 256, 2600, dict(N=1000, bias_in=True, bias_out=True)),
+    ("gelu", "rmsnorm", 300, 1024, dict(N=1000, bias_out=True)),
     ("residual", "none", 384, 2048, dict(N=704, bias_out=True)),
 ]
 
@@ -337,7 +339,7 @@ def test_pair_kernel_stream_k(cuda_device, op, norm, M, K, kw):
     w, inputs = synthetic.make_custom(op, norm, M, K, seed=M + K, **kw)
     _, got = run_and_check(h, w, inputs)
     assert "stream-K" in h.last_plan(), h.last_plan()
-    # the slot-order sum makes the result independent of which pair arrives last
+    # the slot-order sum makes the result independent of which pair finishes first
     _, again = run_and_check(h, w, inputs)
     for k, v in got.items():
         if v is not None:
