@@ -93,7 +93,9 @@ class Handle:
     no stream synchronisation, on later calls up to that size). path forces a
     kernel: "auto" (by M), "splitk" (small-M kernel, stream-K form), "cluster"
     (small-M kernel, cluster form), "tile" (128x256 tiles), "wide" (128x512
-    tiles), "pair" (256x512 tiles on CTA pairs). max_ctas caps the grid (0 = all SMs). precision: "default" (split
+    tiles), "pair" (256x512 tiles on CTA pairs), "pair_sk" (the pair kernel's
+    stream-K form, its split tiles finished by the fix-up kernel). max_ctas
+    caps the grid (0 = all SMs). precision: "default" (split
     hi + lo operand for SwiGLU only), "split", "single". wait_ns: limit of the
     kernels' main-loop waits (0 = 4 s). debug_stall_calls: fault injection for
     tests of the status path (the next that-many calls withhold one weight copy,
