@@ -704,11 +704,13 @@ fnl_status plan_kernel(fnl_handle* h, const Call& c, Kern kern, int cls_req, Pla
         return fail(h, FNL_ERR_UNSUPPORTED, "the pair kernel's stream-K form needs a unit per pair");
       const long long full = (tiles / pairs_max) * pairs_max;
       if (2 * (tiles - full) > kMaxTiles) return fail(h, FNL_ERR_UNSUPPORTED, "too many W tiles");
-      q.sk = 1;
-      q.sk_full = static_cast<int>(full);
-      q.T = static_cast<int>(tiles - full);   // the split tiles (partial-sum slots, counters)
-      q.grid = 2 * pairs_max;
-      q.max_seg = max_segments(q.T, static_cast<int>(nkb4), pairs_max);
+      if (full < tiles) {   // (whole waves only: nothing to split, the plain form)
+        q.sk = 1;
+        q.sk_full = static_cast<int>(full);
+        q.T = static_cast<int>(tiles - full);   // the split tiles (partial-sum slots)
+        q.grid = 2 * pairs_max;
+        q.max_seg = max_segments(q.T, static_cast<int>(nkb4), pairs_max);
+      }
     }
     q.cls = 2;
     q.smem = fnl::k4::SMEM_BYTES;
@@ -898,7 +900,7 @@ fnl_status launch_plan(fnl_handle* h, const Call& c, const Plan& q) {
   // activations, statistics, workspace and outputs only after it.
   const bool pdl = true;
   // the pair kernel's stream-K form: its split tiles are finished by the fix-up kernel
-  const bool fixup = pair && q.sk != 0;
+  const bool fixup = pair && q.sk != 0 && q.T > 0;
   if (nonorm) {
     st = dispatch_residual(h, small, wide, pair, q.grid, q.threads, q.smem, pdl, c.stream, mx, mw, p);
     if (st == FNL_OK && fixup) st = launch_fixup(h, fnl::kEpiResidual, fnl::kNoNorm, q.T, q.grid / 2, c.stream, p);
