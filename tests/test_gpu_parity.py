@@ -347,6 +347,16 @@ def test_pair_kernel_stream_k(cuda_device, op, norm, M, K, kw):
     h.close()
 
 
+def test_pair_kernel_stream_k_without_split_tiles(cuda_device):
+    """The stream-K form forced on 74 tiles (37 row pairs x 2 column tiles):
+    whole waves only on a B200's 74 resident pairs, so nothing is split and the
+    plan is the plain form (no fix-up launch); every element against the oracle."""
+    h = fnl.Handle(0, path="pair_sk")
+    w, inputs = synthetic.make_custom("qkv", "rmsnorm", 37 * 256, 256, Hq=6, Hkv=1, D=128, bias_out=True, seed=9)
+    run_and_check(h, w, inputs)
+    h.close()
+
+
 @pytest.mark.parametrize("kind", ["whole tiles", "stream-K", "whole waves + stream-K"])
 def test_pair_kernel_repeat_full_compare(cuda_device, kind):
     """Every row against the oracle, and bitwise-equal repeats, with the
