@@ -101,7 +101,7 @@ typedef enum {
   FNL_PATH_TILE_PAIR_SPLIT = 6 /* the pair kernel's stream-K form: whole waves of tiles as above, the tiles left
                                   over dealt to all pairs as (tile, k-block) units; a fix-up kernel launched
                                   after it adds each split tile's partial sums in a fixed order and runs the
-                                  epilogue (a candidate of the shape tuner) */
+                                  epilogue (AUTO takes it when the last wave is less than about half full) */
 } fnl_path;
 
 /* How the normalised activation a is rounded for the bf16 tensor cores.
