@@ -50,3 +50,15 @@ def test_units_per_step_are_the_bound_quantity():
             assert unit == "GB/s" and per_step == pytest.approx(w.algorithmic_bytes() / 1e9)
         else:
             assert unit == "TFLOP/s" and per_step == pytest.approx(w.flops() / 1e12)
+
+
+def test_roofline_denominators_are_the_measured_peaks():
+    pk, src = bench.peaks()
+    w = WL["c5_70b_rms_qkv_ragged"]
+    achieved, peak, unit, _ = bench._roofline(w, 10.0, "tensor")   # 10 ms per launch
+    assert peak == pk["bf16_tflops_sustained"] and unit == "TFLOP/s"
+    assert achieved == pytest.approx(w.flops() / 1e-2 / 1e12)
+    w = WL["c2_decode_rms_qkv"]
+    achieved, peak, unit, _ = bench._roofline(w, 0.02, "hbm")      # 20 us per launch
+    assert peak == pk["hbm_gbs"] and unit == "GB/s"
+    assert achieved == pytest.approx(w.algorithmic_bytes() / 2e-5 / 1e9)
